@@ -1,0 +1,413 @@
+"""Benchmark of the whole quantisation path on one layer per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1]
+
+One step = the whole hot path over one seeded synthetic layer, q_proj-like by default (W bf16
+[5120, 5120], X bf16 [8192 tokens, 5120] generated as 16 chunks of 512, group 128, damping
+0.01 * mean(diag H)):
+  H = X^T X (SYRK) -> imatrix -> damping + Cholesky chain -> GPTQ sweep (codes, scales, qerr)
+  -> Bf16TrilDiagF32 encode of H -> decode.
+Metric: GPTQ-int4 weights/s = N*K / step time (whole job, all ranks).  Inputs are resident in
+HBM; L2 is flushed (a 256 MiB write) between timed steps.  `e2e` repeats the measurement through
+the same C ABI calls with the inputs in pinned host memory: their H2D copies and the D2H copy of
+the results (codes, scales, encoded H, qerr) are inside its timed region.
+
+Under torchrun every rank quantises its own independent layer (weak scaling, no collective in
+the data path); times are the max over ranks.  `--impl reference` times the fp64 CPU oracle
+on a bounded sample of the same workload instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.path is None or not os.path.exists(self.path):
+            return out
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return out
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        busy = [v for v in sm if v > 0]
+        out.update(sm_mhz=statistics.median(busy) if busy else None, sm_max_mhz=max(mx) if mx else None,
+                   reasons=sorted(reasons), samples=len(rows))
+        return out
+
+
+# ------------------------------------------------------------------------------------ our arm
+
+class Layer:
+    """Device buffers of one layer and the calls of one step, all through the C ABI binding."""
+
+    def __init__(self, hq, cfg, device):
+        self.hq = hq
+        self.cfg = cfg
+        self.dev = device
+        N, K, G = cfg.N, cfg.K, cfg.group
+        self.X = wl.make_activations(cfg, device)
+        self.W = wl.make_weights(cfg, device)
+        self.H = torch.zeros((K, K), dtype=torch.float32, device=device)
+        self.imp = torch.empty(K, dtype=torch.float32, device=device)
+        self.codes, self.scales = hq.gptq_outputs(N, K, G, device)
+        self.ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(N, K, G), device)
+        self.tril = torch.empty(hq.hq_bf16tril_bytes(K), dtype=torch.uint8, device=device)
+        self.Hfull = torch.empty((K, K), dtype=torch.float32, device=device)
+        self.qerr = torch.zeros(1, dtype=torch.float64, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step(self, X=None, W=None, stage_events=None):
+        hq, cfg = self.hq, self.cfg
+        X = self.X if X is None else X
+        W = self.W if W is None else W
+        ev = stage_events
+        if ev is not None:
+            ev[0].record()
+        self.H.zero_()
+        hq.hq_hessian_accumulate(self.H, X, dev_status=self.status)
+        if ev is not None:
+            ev[1].record()
+        hq.hq_imatrix(self.H, cfg.T, self.imp)
+        hq.hq_gptq_quantize(W, self.H, cfg.group, cfg.damp, self.codes, self.scales, self.ws,
+                            imp=self.imp if cfg.use_imatrix else None, want_qerr=False, qerr_dev=self.qerr)
+        if ev is not None:
+            ev[2].record()
+        hq.hq_hessian_pack_bf16tril(self.H, self.tril)
+        if ev is not None:
+            ev[3].record()
+        hq.hq_hessian_unpack_bf16tril(self.tril, cfg.K, self.Hfull)
+        if ev is not None:
+            ev[4].record()
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, rank, world, local_rank):
+    import post_weight_quantization_tcgen05_b200 as hq
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = wl.CONFIGS[args.config]
+    layer = Layer(hq, cfg, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, each bracketed by events, L2 flushed between steps
+    n_ev = 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    launches0 = hq.hq_debug_launch_count()
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            layer.step(stage_events=evs[k])
+        torch.cuda.synchronize()
+    _barrier(world)
+    launches = (hq.hq_debug_launch_count() - launches0) // max(args.steps, 1)
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    syrk_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    gptq_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    enc_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    dec_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    total_ms = _max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    weights = cfg.N * cfg.K
+    value = weights * world * args.steps / (total_ms / 1e3)
+
+    # ---- e2e: same calls, inputs from pinned host memory, results copied back
+    e2e = None if args.no_e2e else measure_e2e(args, layer, flush, world)
+    peaks = _peaks()
+    syrk_flop = cfg.T * cfg.K * (cfg.K + 1)
+    syrk_avg_s = statistics.mean(syrk_ms) / 1e3
+    syrk_tflops = syrk_flop / syrk_avg_s / 1e12
+    enc_bytes = 2 * cfg.K * (cfg.K + 1) + hq.hq_bf16tril_bytes(cfg.K)   # H lower triangle read + payload
+    dec_bytes = hq.hq_bf16tril_bytes(cfg.K) + 4 * cfg.K * cfg.K
+    clocks = clk.summary()
+    return_line = build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops,
+                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        return_line["cpu_baseline"] = cpu_baseline(cfg, layer)
+    return return_line
+
+
+def measure_e2e(args, layer, flush, world):
+    cfg = layer.cfg
+    weights = cfg.N * cfg.K
+    Xh = layer.X.cpu().pin_memory()
+    Wh = layer.W.cpu().pin_memory()
+    Xd = torch.empty_like(layer.X)
+    Wd = torch.empty_like(layer.W)
+    codes_h = torch.empty(layer.codes.shape, dtype=layer.codes.dtype).pin_memory()
+    scales_h = torch.empty(layer.scales.shape, dtype=layer.scales.dtype).pin_memory()
+    tril_h = torch.empty(layer.tril.shape, dtype=layer.tril.dtype).pin_memory()
+    qerr_h = torch.empty(1, dtype=torch.float64).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(2):
+        Xd.copy_(Xh, non_blocking=True)
+        Wd.copy_(Wh, non_blocking=True)
+        layer.step(Xd, Wd)
+    torch.cuda.synchronize()
+    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    _barrier(world)
+    for k in range(e2e_steps):
+        flush.fill_(k & 0xFF)
+        e_start[k].record()
+        Xd.copy_(Xh, non_blocking=True)
+        Wd.copy_(Wh, non_blocking=True)
+        layer.step(Xd, Wd)
+        codes_h.copy_(layer.codes, non_blocking=True)
+        scales_h.copy_(layer.scales, non_blocking=True)
+        tril_h.copy_(layer.tril, non_blocking=True)
+        qerr_h.copy_(layer.qerr, non_blocking=True)
+        e_end[k].record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    e2e_ms = _max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_start, e_end)), world) / e2e_steps
+    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+    d2h = (codes_h.numel() * codes_h.element_size() + scales_h.numel() * scales_h.element_size() +
+           tril_h.numel() * tril_h.element_size() + 8)
+    return {"value": weights * world / (e2e_ms / 1e3), "unit": "weights/s", "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops, enc_bytes,
+               dec_bytes, peaks, e2e, launches, clocks):
+    line = {
+        "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
+        "value": value,
+        "unit": "weights/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 in, fp32 compute (tcgen05 bf16 SYRK, tf32 trailing update)",
+        "data": "synthetic (seeded; shapes and distributions of the q_proj-like layer)",
+        "config": {"workload": f"{cfg.name}: W bf16 [{cfg.N}, {cfg.K}], X bf16 [{cfg.T}, {cfg.K}] "
+                               f"({cfg.n_chunks} chunks of {cfg.chunk}), group {cfg.group}, damp {cfg.damp}",
+                   "layers_per_gpu": 1, "l2": "flushed between timed steps (256 MiB write)"},
+        "stages_ms": {"syrk": statistics.mean(syrk_ms), "imatrix+factor+sweep": statistics.mean(gptq_ms),
+                      "tril_encode": statistics.mean(enc_ms), "tril_decode": statistics.mean(dec_ms)},
+        "xtx_tflops": syrk_tflops,
+        "codec_gbs": {"encode": enc_bytes / (statistics.mean(enc_ms) / 1e3) / 1e9,
+                      "decode": dec_bytes / (statistics.mean(dec_ms) / 1e3) / 1e9},
+        "roofline": {"kernel": "umma_gemm_kernel<kSyrkBF16> (X^T X)", "bound": "tensor",
+                     "achieved": syrk_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": syrk_tflops / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": peaks["source"] + " bf16 dense burst"},
+        "e2e": e2e,
+        "gpu_launches": int(launches) * args.steps,
+        "gpu_launches_per_step": int(launches),
+        "clocks": clocks,
+    }
+    return line
+
+
+# ------------------------------------------------------------------------------------ oracle
+
+def _blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(cfg, X, W, rows: int):
+    """Times the oracle on one layer: full Hessian, factorisation and codec, sweep on `rows`
+    rows; returns (estimated seconds for the whole layer, details)."""
+    import oracle
+    t0 = time.perf_counter()
+    H = oracle.hessian(X)
+    t1 = time.perf_counter()
+    Hd, _ = oracle.damp_hessian(H, cfg.damp)
+    U = oracle.upper_factor_of_inverse(Hd)
+    t2 = time.perf_counter()
+    codes, scales, _ = oracle.gptq_sweep(W[:rows], U, cfg.group)
+    oracle.qerr(W[:rows], codes, scales, cfg.group)
+    t3 = time.perf_counter()
+    buf = oracle.bf16tril_encode(H.astype(np.float32))
+    oracle.bf16tril_decode(buf, cfg.K)
+    t4 = time.perf_counter()
+    sweep_full = (t3 - t2) * cfg.N / rows
+    est = (t1 - t0) + (t2 - t1) + sweep_full + (t4 - t3)
+    return est, {"syrk_s": t1 - t0, "factor_s": t2 - t1, "sweep_s_sample": t3 - t2, "codec_s": t4 - t3}
+
+
+def cpu_baseline(cfg, layer=None, rows: int = 32):
+    if layer is not None:
+        X = layer.X.double().cpu().numpy()
+        W = layer.W.double().cpu().numpy()
+    else:
+        X = wl.make_activations(cfg, "cpu").double().numpy()
+        W = wl.make_weights(cfg, "cpu").double().numpy()
+    est, det = oracle_sample(cfg, X, W, rows)
+    return {"value": cfg.N * cfg.K / est, "unit": "weights/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"full fp64 Hessian of X [{cfg.T}, {cfg.K}], full factorisation and codec, sweep of "
+                       f"{rows} of {cfg.N} rows scaled to all rows (rows are independent)"),
+            "stages_s": det}
+
+
+def run_reference(args):
+    cfg = wl.CONFIGS[args.config]
+    X = wl.make_activations(cfg, "cpu").double().numpy()
+    W = wl.make_weights(cfg, "cpu").double().numpy()
+    rows = 8
+    for _ in range(args.warmup):
+        oracle_sample(cfg, X, W, rows)
+    ests = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        est, _ = oracle_sample(cfg, X, W, rows)
+        ests.append(est)
+    wall = time.perf_counter() - t0
+    value = cfg.N * cfg.K / statistics.mean(ests)
+    cores = _blas_threads()
+    sample = (f"per step: full fp64 Hessian of X [{cfg.T}, {cfg.K}], full factorisation and codec, sweep of "
+              f"{rows} of {cfg.N} rows scaled to all rows")
+    return {
+        "impl": "reference",
+        "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
+        "value": value, "unit": "weights/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(ests) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": f"{cfg.name}: W [{cfg.N}, {cfg.K}], X [{cfg.T}, {cfg.K}], group {cfg.group}"},
+        "cpu_baseline": {"value": value, "unit": "weights/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

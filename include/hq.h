@@ -1,0 +1,154 @@
+/*
+ * hq.h -- C ABI of libhq.so: Hessian-aware int4 weight quantisation (GPTQ) of one linear
+ * layer on an NVIDIA B200 (sm_100a), and the Bf16TrilDiagF32 Hessian codec.
+ *
+ * Sources of the operations (page title, section):
+ *   [calib] "hipfire-calib-data" dataset card -- "Hessian storage: Bf16TrilDiagF32
+ *           (quant_type 130)"; "REQUIRED: project to PSD before Cholesky"; "The fix".
+ *   [gptq]  ork-driver wiki "Exp 2026-08-18 GPTQ Int4" -- experiment summary (GPTQ sweep,
+ *           Cholesky-based Hessian inverse, uniform symmetric int4 [-8,7] with a
+ *           per-(row,group) scale, dequant w = code*scale), the qerr definition, the
+ *           test_offline_load notes (optional qerr output, byte-identical codes).
+ *   [imat]  AtomicChat Qwen3.8-27B GGUF card -- "The importance matrix" (statistics are
+ *           sums over chunks; importance = mean squared activation per channel).
+ *
+ * Conventions for every entry point:
+ *   - Array pointers are DEVICE pointers owned by the caller unless a parameter says
+ *     "host".  The library allocates no memory and keeps no state between calls; a caller
+ *     that runs calls concurrently gives each its own workspace.
+ *   - Matrices are row-major and densely packed (leading dimension = column count).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it.
+ *   - Invalid arguments are refused with HQ_ERR_INVALID (or HQ_ERR_UNSUPPORTED for a
+ *     well-formed shape this build does not handle) BEFORE anything is launched; nothing
+ *     is ever silently substituted.  On any error the contents of outputs are undefined.
+ *   - All kernels run on the device that is current when the call is made.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* hq_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_INVALID = 1,     /* bad pointer, size, dtype or parameter value */
+  HQ_ERR_UNSUPPORTED = 2, /* a shape this build refuses (e.g. K not a multiple of 128) */
+  HQ_ERR_NOT_PD = 3,      /* damped Hessian not positive definite (Cholesky pivot <= 0) */
+  HQ_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired; outputs undefined */
+  HQ_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  HQ_ERR_WORKSPACE = 6    /* workspace NULL, misaligned (256 B) or smaller than required */
+} hq_status;
+
+typedef enum { HQ_F32 = 0, HQ_BF16 = 1 } hq_dtype;
+
+/* Human-readable name of a status code (static storage). */
+const char* hq_status_string(int status);
+
+/* ABI version of this header (incremented on any incompatible change). */
+int hq_abi_version(void);
+
+/*
+ * H += X^T X  -- calibration Hessian accumulation ([calib] "Hessian storage": full
+ * Hessians XX^T with X laid out [channels, tokens]; [imat]: the statistic is a sum over
+ * chunks, so a corpus is fed chunk by chunk into the same H).
+ *   H      : fp32 [K, K], read-modify-write of the LOWER triangle including the diagonal
+ *            (element (i, j), i >= j).  The strict upper triangle is never read or written.
+ *   X      : [T, K] tokens x channels, dtype x_dtype (HQ_BF16 or HQ_F32).  Products are
+ *            exact (bf16*bf16 or fp32*fp32) and accumulated in fp32.
+ *   T >= 0 (T == 0 is a no-op), K >= 1.
+ *   dev_status : optional device int; if non-NULL a kernel that hits a bounded-wait timeout
+ *            stores HQ_ERR_TIMEOUT there (the caller zeroes it beforehand).
+ * Asynchronous: returns after enqueueing.  H must not alias X.
+ */
+hq_status hq_hessian_accumulate(float* H, const void* X, int x_dtype, int64_t T, int64_t K,
+                                int* dev_status, hq_stream_t stream);
+
+/*
+ * imp[k] = H[k, k] / tokens  -- importance vector = mean squared activation per channel
+ * ([gptq] qerr paragraph: diag(H)[k] = sum_t a_k^2, the imatrix is its mean).
+ *   H fp32 [K, K] (diagonal read), imp fp32 [K] out.  tokens >= 1.  Asynchronous.
+ */
+hq_status hq_imatrix(const float* H, int64_t K, int64_t tokens, float* imp, hq_stream_t stream);
+
+/* Bytes of workspace hq_gptq_quantize needs for this shape (0 if the shape is invalid). */
+size_t hq_gptq_workspace_bytes(int64_t N, int64_t K, int64_t group);
+
+/*
+ * GPTQ int4 quantisation of one layer ([gptq] experiment summary):
+ *   lambda = damp * mean(diag H); U = upper Cholesky factor of (H + lambda I)^-1;
+ *   columns j = 0..K-1 in order, for every row n:
+ *     at a group start: s = fp32(max |Wc[n, j:j+group]| / 7) from the current weights;
+ *     c = clamp(rint(Wc[n,j] / s), -8, 7) (s == 0 -> c = 0); q = c * s;
+ *     e = (Wc[n,j] - q) / U[j,j];  Wc[n,k] -= e * U[j,k] for k > j.
+ *   qerr = sqrt(sum imp[k] (W[n,k] - q[n,k])^2 / sum imp[k] W[n,k]^2) over the ORIGINAL W,
+ *   imp = 1 when NULL ([gptq] qerr definition).
+ * Arguments:
+ *   W      : [N, K] row-major, dtype w_dtype (HQ_BF16 or HQ_F32); not modified.
+ *   H      : fp32 [K, K] undamped Hessian; only the lower triangle incl. diagonal is read;
+ *            not modified.
+ *   group  : group size along K; must divide K and be a multiple of 32.
+ *   K      : a multiple of 128.  N >= 1.
+ *   damp   : > 0 and finite; mean(diag H) must be > 0.
+ *   imp    : optional fp32 [K] importance (NULL -> all ones); only affects qerr.
+ *   codes  : uint8 [N, K/2] out; byte (n, p) = (c[n,2p] & 0xF) | (c[n,2p+1] & 0xF) << 4,
+ *            4-bit two's complement (the even column in the low nibble).
+ *   scales : fp32 [N, K/group] out, row-major.
+ *   qerr_out : optional HOST double* (NULL -> not returned).
+ *   qerr_dev : optional DEVICE double* (NULL -> not written); written asynchronously.
+ *   workspace : device buffer of at least hq_gptq_workspace_bytes(N, K, group) bytes,
+ *            256-byte aligned, owned by the caller, not shared with a concurrent call.
+ * The call synchronises `stream` once at its end to read the factorisation status, and
+ * returns HQ_ERR_NOT_PD if a Cholesky pivot was not positive.  codes and scales do not
+ * depend on whether qerr is requested, and are identical run to run.
+ */
+hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
+                           int64_t group, float damp, const float* imp, uint8_t* codes,
+                           float* scales, double* qerr_out, double* qerr_dev, void* workspace,
+                           size_t workspace_bytes, hq_stream_t stream);
+
+/* Bytes of workspace hq_rtn_quantize needs (0 if the shape is invalid). */
+size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group);
+
+/*
+ * Round-to-nearest int4 with the same quantiser and no error feedback (ork's "crude
+ * symmetric absmax/7 rounding", [gptq] experiment summary): s = fp32(max|W[n,group]|/7),
+ * c = clamp(rint(W/s), -8, 7).  Same argument meanings and output layouts as
+ * hq_gptq_quantize.  Synchronises `stream` only when qerr_out != NULL.
+ */
+hq_status hq_rtn_quantize(const void* W, int w_dtype, int64_t N, int64_t K, int64_t group,
+                          const float* imp, uint8_t* codes, float* scales, double* qerr_out,
+                          double* qerr_dev, void* workspace, size_t workspace_bytes,
+                          hq_stream_t stream);
+
+/* Bf16TrilDiagF32 payload size: K*4 + K*(K-1)/2*2 bytes ([calib] "Hessian storage"). */
+size_t hq_bf16tril_bytes(int64_t K);
+
+/*
+ * Bf16TrilDiagF32 encode ([calib] "Hessian storage: Bf16TrilDiagF32 (quant_type 130)"):
+ *   out[0 : 4K)            = H[i,i] as little-endian fp32, i = 0..K-1;
+ *   out[4K + 2*(i(i-1)/2 + j)] = (fp32 bits of H[i,j]) >> 16 as little-endian u16, i > j
+ *                            (bf16 by truncation, not rounding).
+ *   H fp32 [K, K] (diagonal and strict lower triangle read), out hq_bf16tril_bytes(K) bytes.
+ *   K >= 1.  Asynchronous.  Bit-exact by definition.
+ */
+hq_status hq_hessian_pack_bf16tril(const float* H, int64_t K, uint8_t* out, hq_stream_t stream);
+
+/*
+ * Bf16TrilDiagF32 decode, "mirrored on read": H[i,i] = diagonal; H[i,j] = H[j,i] =
+ * fp32(bits << 16) for i > j.  in: hq_bf16tril_bytes(K) bytes; H_full fp32 [K, K] out (both
+ * triangles written).  K >= 1.  Asynchronous.
+ */
+hq_status hq_hessian_unpack_bf16tril(const uint8_t* in, int64_t K, float* H_full,
+                                     hq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

@@ -1,0 +1,51 @@
+/*
+ * hq_debug.h -- stage-level entry points of libhq.so for parity tests and profiling.
+ * They run single stages of the path that hq.h composes, so each stage can be compared
+ * with the oracle on its own.  Same conventions as hq.h (device pointers, caller-owned
+ * memory, refusal before launch, asynchronous unless stated).
+ */
+#ifndef HQ_DEBUG_H
+#define HQ_DEBUG_H
+
+#include "hq.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * The damping + factorisation stage of hq_gptq_quantize alone: writes U^T (fp32 [K, K],
+ * row-major; U^T[c, j] = U[j, c] for c >= j, zero above the diagonal) where U is the upper
+ * Cholesky factor of (H + damp * mean(diag H) I)^-1 ([gptq] experiment summary, "Cholesky-
+ * based Hessian inverse").  Uses hq_gptq_workspace_bytes(1, K, 128) bytes of workspace.
+ * Synchronises `stream` and returns HQ_ERR_NOT_PD / HQ_ERR_INVALID like hq_gptq_quantize.
+ */
+hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, void* workspace,
+                          size_t workspace_bytes, hq_stream_t stream);
+
+/*
+ * hq_gptq_quantize with an explicit choice of the trailing-update kernel:
+ * update_impl 0 = tcgen05 tf32 tensor-core kernel (the default path), 1 = fp32 CUDA-core
+ * kernel (reference for the tensor-core one).
+ */
+hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
+                                      int64_t group, float damp, const float* imp, uint8_t* codes,
+                                      float* scales, double* qerr_out, double* qerr_dev, void* workspace,
+                                      size_t workspace_bytes, int update_impl, hq_stream_t stream);
+
+/*
+ * hq_hessian_accumulate with an explicit kernel choice: impl 0 = automatic (tcgen05 for
+ * eligible bf16 inputs), 1 = fp32 CUDA-core kernel for every input.
+ */
+hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype, int64_t T, int64_t K,
+                                           int* dev_status, int impl, hq_stream_t stream);
+
+/* Number of kernels libhq.so has launched in this process so far (all devices, all
+ * threads).  A statistic for profiling; never reset. */
+uint64_t hq_debug_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_DEBUG_H */

@@ -59,6 +59,7 @@ __all__ = [
     "upper_factor_by_reversal",
     "gptq_sweep",
     "gptq_quantize",
+    "gptq_sweep_forced",
     "rtn_quantize",
     "dequantize",
     "qerr",
@@ -203,6 +204,43 @@ def gptq_sweep(W, U, group: int):
         codes[:, j] = c
         E[:, j] = e
     return codes, scales, E
+
+
+def gptq_sweep_forced(W, U, group: int, forced_codes):
+    """The same sweep with every code decision replaced by `forced_codes` (teacher forcing).
+
+    Used to compare another implementation's scales and errors on ITS OWN code trajectory:
+    once two implementations round one near-tie differently, the error feedback moves every
+    later weight of that row, so plain element-wise comparison of later scales is meaningless.
+    Besides (scales, errors) it returns, for every column, the code the unforced rule would
+    pick from the same current weight, and the ratio w / s that rule rounds.
+    Returns (scales fp32 [N, K/group], errors fp64 [N, K], free_codes int8 [N, K],
+    ratios fp32 [N, K]).
+    """
+    Wc = np.array(W, dtype=np.float64, copy=True)
+    U = np.asarray(U, dtype=np.float64)
+    C = np.asarray(forced_codes).astype(np.float64)
+    N, K = Wc.shape
+    if K % group:
+        raise ValueError("group must divide K")
+    scales = np.zeros((N, K // group), dtype=np.float32)
+    E = np.zeros((N, K), dtype=np.float64)
+    free = np.zeros((N, K), dtype=np.int8)
+    ratios = np.zeros((N, K), dtype=np.float32)
+    for j in range(K):
+        g = j // group
+        if j % group == 0:
+            scales[:, g] = _group_scale(np.max(np.abs(Wc[:, j:j + group]), axis=1))
+        s = scales[:, g]
+        free[:, j] = _round_code(Wc[:, j], s)
+        safe = np.where(s > 0, s, np.float32(1.0))
+        ratios[:, j] = np.where(s > 0, (Wc[:, j].astype(np.float32) / safe).astype(np.float32), 0.0)
+        q = C[:, j] * s.astype(np.float64)
+        e = (Wc[:, j] - q) / U[j, j]
+        if j + 1 < K:
+            Wc[:, j + 1:] -= np.outer(e, U[j, j + 1:])
+        E[:, j] = e
+    return scales, E, free, ratios
 
 
 def gptq_quantize(W, H, group: int, damp: float):

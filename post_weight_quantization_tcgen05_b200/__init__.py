@@ -1,0 +1,205 @@
+"""Python binding of libhq.so: GPTQ int4 weight quantisation and the Bf16TrilDiagF32 codec
+on NVIDIA B200 (sm_100a).
+
+Argument marshalling only: every function checks tensor dtypes, shapes and devices, turns
+them into raw pointers and sizes, and calls the C entry point of the same name (declared in
+include/hq.h and include/hq_debug.h).  Every step of the computation runs in the library's
+CUDA kernels.  Importing this package fails loudly when libhq.so has not been built
+(``python post_weight_quantization_tcgen05_b200/build.py``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhq.so")
+
+HQ_OK = 0
+HQ_ERR_INVALID = 1
+HQ_ERR_UNSUPPORTED = 2
+HQ_ERR_NOT_PD = 3
+HQ_ERR_TIMEOUT = 4
+HQ_ERR_CUDA = 5
+HQ_ERR_WORKSPACE = 6
+HQ_F32 = 0
+HQ_BF16 = 1
+
+_DTYPE = {torch.float32: HQ_F32, torch.bfloat16: HQ_BF16}
+
+
+class HQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libhq.so not found at {_LIB_PATH}; build it with "
+                      "`python post_weight_quantization_tcgen05_b200/build.py`")
+
+lib = ctypes.CDLL(_LIB_PATH)
+
+_vp, _i64, _int, _f, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "hq_status_string": (ctypes.c_char_p, [_int]),
+    "hq_abi_version": (_int, []),
+    "hq_hessian_accumulate": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp]),
+    "hq_imatrix": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "hq_gptq_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "hq_gptq_quantize": (_int, [_vp, _int, _i64, _i64, _vp, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hq_rtn_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "hq_rtn_quantize": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hq_bf16tril_bytes": (_sz, [_i64]),
+    "hq_hessian_pack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
+    "hq_hessian_unpack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
+    "hq_debug_factor": (_int, [_vp, _i64, _f, _vp, _vp, _sz, _vp]),
+    "hq_debug_gptq_quantize_impl": (_int, [_vp, _int, _i64, _i64, _vp, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                           _int, _vp]),
+    "hq_debug_hessian_accumulate_impl": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _int, _vp]),
+    "hq_debug_launch_count": (ctypes.c_uint64, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def status_string(status: int) -> str:
+    return lib.hq_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != HQ_OK:
+        raise HQError(status, where)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype(t) -> int:
+    if t.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return _DTYPE[t.dtype]
+
+
+# --------------------------------------------------------------------------- entry points
+
+def hq_abi_version() -> int:
+    return lib.hq_abi_version()
+
+
+def hq_debug_launch_count() -> int:
+    return int(lib.hq_debug_launch_count())
+
+
+def hq_hessian_accumulate(H, X, dev_status=None, stream=None) -> None:
+    """H (fp32 [K, K]) += X^T X on the lower triangle; X [T, K] bf16 or fp32."""
+    T, K = X.shape
+    if H.dtype != torch.float32 or tuple(H.shape) != (K, K):
+        raise ValueError("H must be fp32 [K, K]")
+    _check(lib.hq_hessian_accumulate(_ptr(H), _ptr(X), _dtype(X), T, K, _ptr(dev_status), _stream(stream)),
+           "hq_hessian_accumulate")
+
+
+def hq_debug_hessian_accumulate_impl(H, X, impl: int, dev_status=None, stream=None) -> None:
+    T, K = X.shape
+    _check(lib.hq_debug_hessian_accumulate_impl(_ptr(H), _ptr(X), _dtype(X), T, K, _ptr(dev_status), int(impl),
+                                                _stream(stream)), "hq_debug_hessian_accumulate_impl")
+
+
+def hq_imatrix(H, tokens: int, imp, stream=None) -> None:
+    K = H.shape[0]
+    _check(lib.hq_imatrix(_ptr(H), K, int(tokens), _ptr(imp), _stream(stream)), "hq_imatrix")
+
+
+def hq_gptq_workspace_bytes(N: int, K: int, group: int) -> int:
+    return int(lib.hq_gptq_workspace_bytes(N, K, group))
+
+
+def hq_rtn_workspace_bytes(N: int, K: int, group: int) -> int:
+    return int(lib.hq_rtn_workspace_bytes(N, K, group))
+
+
+def hq_gptq_quantize(W, H, group: int, damp: float, codes, scales, workspace, imp=None, want_qerr: bool = True,
+                     qerr_dev=None, stream=None):
+    """GPTQ int4 of W [N, K] against the undamped fp32 H; returns qerr (host) if requested."""
+    N, K = W.shape
+    q = ctypes.c_double(float("nan"))
+    st = lib.hq_gptq_quantize(_ptr(W), _dtype(W), N, K, _ptr(H), int(group), float(damp), _ptr(imp), _ptr(codes),
+                              _ptr(scales), ctypes.byref(q) if want_qerr else None, _ptr(qerr_dev), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hq_gptq_quantize")
+    return q.value if want_qerr else None
+
+
+def hq_debug_gptq_quantize_impl(W, H, group: int, damp: float, codes, scales, workspace, update_impl: int, imp=None,
+                                want_qerr: bool = True, qerr_dev=None, stream=None):
+    N, K = W.shape
+    q = ctypes.c_double(float("nan"))
+    st = lib.hq_debug_gptq_quantize_impl(_ptr(W), _dtype(W), N, K, _ptr(H), int(group), float(damp), _ptr(imp),
+                                         _ptr(codes), _ptr(scales), ctypes.byref(q) if want_qerr else None,
+                                         _ptr(qerr_dev), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         int(update_impl), _stream(stream))
+    _check(st, "hq_debug_gptq_quantize_impl")
+    return q.value if want_qerr else None
+
+
+def hq_rtn_quantize(W, group: int, codes, scales, workspace, imp=None, want_qerr: bool = True, qerr_dev=None,
+                    stream=None):
+    N, K = W.shape
+    q = ctypes.c_double(float("nan"))
+    st = lib.hq_rtn_quantize(_ptr(W), _dtype(W), N, K, int(group), _ptr(imp), _ptr(codes), _ptr(scales),
+                             ctypes.byref(q) if want_qerr else None, _ptr(qerr_dev), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hq_rtn_quantize")
+    return q.value if want_qerr else None
+
+
+def hq_debug_factor(H, damp: float, Ut_out, workspace, stream=None) -> None:
+    K = H.shape[0]
+    _check(lib.hq_debug_factor(_ptr(H), K, float(damp), _ptr(Ut_out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)), "hq_debug_factor")
+
+
+def hq_bf16tril_bytes(K: int) -> int:
+    return int(lib.hq_bf16tril_bytes(K))
+
+
+def hq_hessian_pack_bf16tril(H, out, stream=None) -> None:
+    K = H.shape[0]
+    _check(lib.hq_hessian_pack_bf16tril(_ptr(H), K, _ptr(out), _stream(stream)), "hq_hessian_pack_bf16tril")
+
+
+def hq_hessian_unpack_bf16tril(inp, K: int, H_full, stream=None) -> None:
+    _check(lib.hq_hessian_unpack_bf16tril(_ptr(inp), K, _ptr(H_full), _stream(stream)), "hq_hessian_unpack_bf16tril")
+
+
+# --------------------------------------------------------------------------- allocation helpers
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A uint8 device buffer of nbytes (torch's caching allocator returns 512-byte aligned blocks)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def gptq_outputs(N: int, K: int, group: int, device="cuda"):
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((N, K // group), dtype=torch.float32, device=device)
+    return codes, scales

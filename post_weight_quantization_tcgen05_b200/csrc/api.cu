@@ -1,0 +1,193 @@
+// The C ABI of libhq.so (include/hq.h, include/hq_debug.h): argument validation, workspace
+// carving and stage orchestration.  Every computation happens in the kernels of the other
+// translation units; this file only checks arguments and enqueues work.
+#include <math.h>
+#include <string.h>
+
+#include "../../include/hq.h"
+#include "../../include/hq_debug.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hq {
+uint64_t& launch_counter() {
+  static uint64_t n = 0;
+  return n;
+}
+}  // namespace hq
+
+using namespace hq;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+bool valid_dtype(int d) { return d == HQ_F32 || d == HQ_BF16; }
+
+hq_status finish_sync(cudaStream_t s, const WsHeader* dev_hdr, double* qerr_out) {
+  WsHeader h{};
+  HQ_CUDA_TRY(cudaMemcpyAsync(&h, dev_hdr, sizeof(WsHeader), cudaMemcpyDeviceToHost, s));
+  HQ_CUDA_TRY(cudaStreamSynchronize(s));
+  if (h.status == HQ_ERR_TIMEOUT) return HQ_ERR_TIMEOUT;
+  if (h.info == -1) return HQ_ERR_INVALID;
+  if (h.info > 0) return HQ_ERR_NOT_PD;
+  if (qerr_out != nullptr) *qerr_out = h.qerr;
+  return HQ_OK;
+}
+
+hq_status check_gptq_args(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
+                          uint8_t* codes, float* scales) {
+  if (W == nullptr || H == nullptr || codes == nullptr || scales == nullptr) return HQ_ERR_INVALID;
+  if (!valid_dtype(w_dtype)) return HQ_ERR_INVALID;
+  if (N < 1 || K < 1 || group < 1) return HQ_ERR_INVALID;
+  if (!(damp > 0.f) || !isfinite(damp)) return HQ_ERR_INVALID;
+  if (K % group != 0) return HQ_ERR_INVALID;
+  if (!gptq_shape_ok(N, K, group)) return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+
+hq_status gptq_common(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
+                      const float* imp, uint8_t* codes, float* scales, double* qerr_out, double* qerr_dev,
+                      void* workspace, size_t workspace_bytes, int update_impl, cudaStream_t s) {
+  hq_status st = check_gptq_args(W, w_dtype, N, K, H, group, damp, codes, scales);
+  if (st != HQ_OK) return st;
+  const GptqLayout L = gptq_layout(N, K, group);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.total) return HQ_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = launch_gptq(W, w_dtype, N, K, H, group, damp, imp, codes, scales, qerr_dev, ws, update_impl, s);
+  if (st != HQ_OK) return st;
+  return finish_sync(s, reinterpret_cast<const WsHeader*>(ws + L.header), qerr_out);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hq_status_string(int status) {
+  switch (status) {
+    case HQ_OK: return "HQ_OK";
+    case HQ_ERR_INVALID: return "HQ_ERR_INVALID";
+    case HQ_ERR_UNSUPPORTED: return "HQ_ERR_UNSUPPORTED";
+    case HQ_ERR_NOT_PD: return "HQ_ERR_NOT_PD";
+    case HQ_ERR_TIMEOUT: return "HQ_ERR_TIMEOUT";
+    case HQ_ERR_CUDA: return "HQ_ERR_CUDA";
+    case HQ_ERR_WORKSPACE: return "HQ_ERR_WORKSPACE";
+    default: return "HQ_ERR_UNKNOWN";
+  }
+}
+
+int hq_abi_version(void) { return kAbiVersion; }
+
+uint64_t hq_debug_launch_count(void) { return __atomic_load_n(&launch_counter(), __ATOMIC_RELAXED); }
+
+hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype, int64_t T, int64_t K,
+                                           int* dev_status, int impl, hq_stream_t stream) {
+  if (H == nullptr || K < 1 || T < 0 || !valid_dtype(x_dtype) || (impl != 0 && impl != 1)) return HQ_ERR_INVALID;
+  if (T > 0 && X == nullptr) return HQ_ERR_INVALID;
+  if (T == 0) return HQ_OK;
+  if (K > (int64_t(1) << 20) || T > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (impl == 0 && syrk_tc_eligible(X, x_dtype, T, K)) return launch_syrk_tc(H, X, T, K, dev_status, s);
+  return launch_syrk_simt(H, X, x_dtype, T, K, s);
+}
+
+hq_status hq_hessian_accumulate(float* H, const void* X, int x_dtype, int64_t T, int64_t K, int* dev_status,
+                                hq_stream_t stream) {
+  return hq_debug_hessian_accumulate_impl(H, X, x_dtype, T, K, dev_status, 0, stream);
+}
+
+__global__ void imatrix_kernel(const float* __restrict__ H, int64_t K, double inv_tokens, float* __restrict__ imp) {
+  for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < K;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    imp[k] = static_cast<float>(static_cast<double>(H[k * K + k]) * inv_tokens);
+}
+
+hq_status hq_imatrix(const float* H, int64_t K, int64_t tokens, float* imp, hq_stream_t stream) {
+  if (H == nullptr || imp == nullptr || K < 1 || tokens < 1) return HQ_ERR_INVALID;
+  const int grid = static_cast<int>(ceil_div(K, 256) < 1024 ? ceil_div(K, 256) : 1024);
+  imatrix_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(H, K, 1.0 / static_cast<double>(tokens), imp);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
+}
+
+size_t hq_gptq_workspace_bytes(int64_t N, int64_t K, int64_t group) {
+  if (!gptq_shape_ok(N, K, group)) return 0;
+  return gptq_layout(N, K, group).total;
+}
+
+hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group,
+                           float damp, const float* imp, uint8_t* codes, float* scales, double* qerr_out,
+                           double* qerr_dev, void* workspace, size_t workspace_bytes, hq_stream_t stream) {
+  return gptq_common(W, w_dtype, N, K, H, group, damp, imp, codes, scales, qerr_out, qerr_dev, workspace,
+                     workspace_bytes, 0, static_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
+                                      int64_t group, float damp, const float* imp, uint8_t* codes, float* scales,
+                                      double* qerr_out, double* qerr_dev, void* workspace, size_t workspace_bytes,
+                                      int update_impl, hq_stream_t stream) {
+  if (update_impl != 0 && update_impl != 1) return HQ_ERR_INVALID;
+  return gptq_common(W, w_dtype, N, K, H, group, damp, imp, codes, scales, qerr_out, qerr_dev, workspace,
+                     workspace_bytes, update_impl, static_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, void* workspace,
+                          size_t workspace_bytes, hq_stream_t stream) {
+  if (H == nullptr || Ut_out == nullptr) return HQ_ERR_INVALID;
+  if (!(damp > 0.f) || !isfinite(damp)) return HQ_ERR_INVALID;
+  if (!gptq_shape_ok(1, K, 128)) return HQ_ERR_UNSUPPORTED;
+  const GptqLayout L = gptq_layout(1, K, 128);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.total) return HQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
+  float* A = reinterpret_cast<float*>(ws + L.a);
+  hq_status st = launch_factor(H, K, damp, A, reinterpret_cast<float*>(ws + L.x), reinterpret_cast<float*>(ws + L.t),
+                               reinterpret_cast<float*>(ws + L.dinv), &hdr->lam, &hdr->info, A, s);
+  if (st != HQ_OK) return st;
+  HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, A, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  return finish_sync(s, hdr, nullptr);
+}
+
+size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group) {
+  if (N < 1 || K < 2 || group < 2 || group % 2 != 0 || K % group != 0) return 0;
+  return rtn_workspace(N, K, group);
+}
+
+hq_status hq_rtn_quantize(const void* W, int w_dtype, int64_t N, int64_t K, int64_t group, const float* imp,
+                          uint8_t* codes, float* scales, double* qerr_out, double* qerr_dev, void* workspace,
+                          size_t workspace_bytes, hq_stream_t stream) {
+  if (W == nullptr || codes == nullptr || scales == nullptr || !valid_dtype(w_dtype)) return HQ_ERR_INVALID;
+  if (N < 1 || K < 2 || group < 2 || K % group != 0) return HQ_ERR_INVALID;
+  if (group % 2 != 0) return HQ_ERR_UNSUPPORTED;
+  const size_t need = rtn_workspace(N, K, group);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need) return HQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  hq_status st = launch_rtn(W, w_dtype, N, K, group, imp, codes, scales, qerr_dev, ws, s);
+  if (st != HQ_OK) return st;
+  if (qerr_out == nullptr) return HQ_OK;
+  return finish_sync(s, reinterpret_cast<const WsHeader*>(ws), qerr_out);
+}
+
+size_t hq_bf16tril_bytes(int64_t K) {
+  if (K < 1) return 0;
+  return static_cast<size_t>(K) * 4 + static_cast<size_t>(K) * (K - 1) / 2 * 2;
+}
+
+hq_status hq_hessian_pack_bf16tril(const float* H, int64_t K, uint8_t* out, hq_stream_t stream) {
+  if (H == nullptr || out == nullptr || K < 1) return HQ_ERR_INVALID;
+  if (!aligned(out, 16) || !aligned(H, 4)) return HQ_ERR_INVALID;
+  if (K > (int64_t(1) << 20)) return HQ_ERR_UNSUPPORTED;
+  return launch_tril_encode(H, K, out, static_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_hessian_unpack_bf16tril(const uint8_t* in, int64_t K, float* H_full, hq_stream_t stream) {
+  if (in == nullptr || H_full == nullptr || K < 1) return HQ_ERR_INVALID;
+  if (!aligned(in, 16) || !aligned(H_full, 4)) return HQ_ERR_INVALID;
+  if (K > (int64_t(1) << 20)) return HQ_ERR_UNSUPPORTED;
+  return launch_tril_decode(in, K, H_full, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

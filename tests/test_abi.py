@@ -1,0 +1,99 @@
+"""The C ABI without a GPU: libhq.so loads, exports every function include/*.h declares,
+and refuses invalid arguments before launching anything.  Size queries are checked against
+the page formulas."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in ("hq.h", "hq_debug.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(hq_[a-z0-9_]+)\s*\(", src, re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def hq():
+    import post_weight_quantization_tcgen05_b200 as m
+    return m
+
+
+def test_every_declared_symbol_is_exported(hq):
+    names = _declared_functions()
+    assert len(names) >= 14
+    for n in sorted(names):
+        assert hasattr(hq.lib, n), n
+        assert n in hq._SIGS, f"binding lacks {n}"
+
+
+def test_version_and_status_strings(hq):
+    assert hq.hq_abi_version() == 1
+    assert hq.status_string(0) == "HQ_OK"
+    assert hq.status_string(3) == "HQ_ERR_NOT_PD"
+    assert hq.status_string(99) == "HQ_ERR_UNKNOWN"
+
+
+def test_bf16tril_bytes_matches_page_formula(hq):
+    import oracle
+    for K in (1, 2, 3, 128, 5120, 6144, 17408):
+        assert hq.hq_bf16tril_bytes(K) == oracle.bf16tril_bytes(K)
+    assert hq.hq_bf16tril_bytes(0) == 0
+
+
+def test_workspace_queries(hq):
+    assert hq.hq_gptq_workspace_bytes(64, 128, 32) > 0
+    assert hq.hq_gptq_workspace_bytes(64, 100, 32) == 0      # K not a multiple of 128
+    assert hq.hq_gptq_workspace_bytes(64, 128, 48) == 0      # group not a multiple of 32
+    assert hq.hq_gptq_workspace_bytes(0, 128, 32) == 0
+    assert hq.hq_gptq_workspace_bytes(64, 384, 96) == 0      # 96 straddles 128-column blocks
+    big = hq.hq_gptq_workspace_bytes(5120, 17408, 128)
+    assert big >= 2 * 17408 * 17408 * 4 + 5120 * 17408 * 4
+    assert hq.hq_rtn_workspace_bytes(64, 128, 32) > 0
+    assert hq.hq_rtn_workspace_bytes(64, 128, 3) == 0
+
+
+def test_invalid_arguments_refused_before_launch(hq):
+    L = hq.lib
+    fake = ctypes.c_void_p(256)  # never dereferenced: refusals happen on the host
+    # NULL pointers
+    assert L.hq_hessian_accumulate(None, fake, 1, 8, 8, None, None) == hq.HQ_ERR_INVALID
+    assert L.hq_hessian_accumulate(fake, None, 1, 8, 8, None, None) == hq.HQ_ERR_INVALID
+    # bad dtype, bad sizes
+    assert L.hq_hessian_accumulate(fake, fake, 7, 8, 8, None, None) == hq.HQ_ERR_INVALID
+    assert L.hq_hessian_accumulate(fake, fake, 1, -1, 8, None, None) == hq.HQ_ERR_INVALID
+    assert L.hq_hessian_accumulate(fake, fake, 1, 8, 0, None, None) == hq.HQ_ERR_INVALID
+    # T == 0 is a no-op that launches nothing
+    assert L.hq_hessian_accumulate(fake, None, 1, 0, 8, None, None) == hq.HQ_OK
+    args = dict(W=fake, dt=1, N=64, K=128, H=fake, group=32, damp=0.01, imp=None, codes=fake, scales=fake,
+                qo=None, qd=None, ws=ctypes.c_void_p(1 << 20), wsb=1 << 40, s=None)
+
+    def gq(**kw):
+        a = dict(args, **kw)
+        return L.hq_gptq_quantize(a["W"], a["dt"], a["N"], a["K"], a["H"], a["group"], a["damp"], a["imp"],
+                                  a["codes"], a["scales"], a["qo"], a["qd"], a["ws"], a["wsb"], a["s"])
+
+    assert gq(W=None) == hq.HQ_ERR_INVALID
+    assert gq(dt=5) == hq.HQ_ERR_INVALID
+    assert gq(damp=0.0) == hq.HQ_ERR_INVALID
+    assert gq(damp=float("nan")) == hq.HQ_ERR_INVALID
+    assert gq(group=48) == hq.HQ_ERR_INVALID            # does not divide K
+    assert gq(K=100, group=50) == hq.HQ_ERR_UNSUPPORTED  # K not a multiple of 128
+    assert gq(K=384, group=96) == hq.HQ_ERR_UNSUPPORTED
+    assert gq(ws=None) == hq.HQ_ERR_WORKSPACE
+    assert gq(wsb=16) == hq.HQ_ERR_WORKSPACE
+    assert gq(ws=ctypes.c_void_p((1 << 20) + 8)) == hq.HQ_ERR_WORKSPACE  # misaligned
+    assert L.hq_rtn_quantize(fake, 1, 64, 128, 3, None, fake, fake, None, None, fake, 1 << 30, None) == hq.HQ_ERR_INVALID
+    assert L.hq_rtn_quantize(fake, 1, 64, 128, 32, None, fake, fake, None, None, None, 1 << 30, None) == hq.HQ_ERR_WORKSPACE
+    assert L.hq_hessian_pack_bf16tril(fake, 0, fake, None) == hq.HQ_ERR_INVALID
+    assert L.hq_hessian_pack_bf16tril(fake, 8, ctypes.c_void_p(258), None) == hq.HQ_ERR_INVALID  # out not 16-B aligned
+    assert L.hq_hessian_unpack_bf16tril(None, 8, fake, None) == hq.HQ_ERR_INVALID
+    assert L.hq_imatrix(fake, 8, 0, fake, None) == hq.HQ_ERR_INVALID

@@ -1,0 +1,315 @@
+"""GPU parity of each stage against the oracle on small and ragged shapes (all through the
+C ABI).  Inputs are seeded; the oracle always sees the same bytes the GPU sees, and never
+anything the CUDA path produced."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from gpu_helpers import (H_REL_FRO, LOSS_REL, QERR_REL, check_gptq_parity, rel_fro, to_np64, unpack_codes)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hq():
+    import post_weight_quantization_tcgen05_b200 as m
+    return m
+
+
+def _gen(seed, device="cuda"):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+# ----------------------------------------------------------------------------- codec
+
+def _random_h(K, seed):
+    g = _gen(seed)
+    H = torch.randn((K, K), generator=g, device="cuda") * torch.exp(3 * torch.randn((K, K), generator=g, device="cuda"))
+    if K >= 4:
+        bits = H.view(torch.int32)
+        bits[1, 0] = 0x7F800000       # +inf
+        bits[2, 0] = 0x7FC00001       # NaN
+        bits[2, 1] = 0x7F800001       # NaN whose payload sits in the low half
+        bits[3, 0] = 0x00000001       # smallest denormal
+        bits[3, 1] = -0x80000000      # -0
+        bits[3, 2] = 0x3F808001       # 1.0000153: truncation, not rounding
+    return H
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 5, 64, 127, 128, 129, 1000, 2049])
+def test_codec_encode_bit_exact(hq, cuda_device, K):
+    H = _random_h(K, 100 + K)
+    out = torch.full((hq.hq_bf16tril_bytes(K),), 0xAB, dtype=torch.uint8, device="cuda")
+    hq.hq_hessian_pack_bf16tril(H, out)
+    torch.cuda.synchronize()
+    ref = oracle.bf16tril_encode(H.cpu().numpy())
+    assert out.cpu().numpy().tobytes() == ref
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 64, 129, 1000, 2049])
+def test_codec_decode_bit_exact(hq, cuda_device, K):
+    nb = hq.hq_bf16tril_bytes(K)
+    g = _gen(200 + K)
+    buf = torch.randint(0, 256, (nb,), generator=g, device="cuda", dtype=torch.int32).to(torch.uint8)
+    Hf = torch.full((K, K), 7.0, device="cuda")
+    hq.hq_hessian_unpack_bf16tril(buf, K, Hf)
+    torch.cuda.synchronize()
+    ref = oracle.bf16tril_decode(buf.cpu().numpy().tobytes(), K)
+    assert np.array_equal(Hf.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+# ----------------------------------------------------------------------------- SYRK
+
+def _syrk_check(hq, X, impl, chunks=1):
+    T, K = X.shape
+    H = torch.triu(torch.full((K, K), -123.0, device="cuda"), 1)  # sentinel above the diagonal
+    bounds = np.linspace(0, T, chunks + 1).astype(int)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        hq.hq_debug_hessian_accumulate_impl(H, X[a:b].contiguous(), impl)
+    torch.cuda.synchronize()
+    ref = oracle.hessian(to_np64(X))
+    Hn = to_np64(H)
+    lo = np.tril(np.ones((K, K), bool))
+    assert np.all(Hn[~lo] == -123.0), "strict upper triangle must not be touched"
+    err = rel_fro(Hn[lo], ref[lo])
+    assert err <= H_REL_FRO, err
+    return err
+
+
+@pytest.mark.parametrize("T,K", [(512, 128), (1, 64), (33, 7), (300, 200)])
+def test_syrk_fp32_simt(hq, cuda_device, T, K):
+    cfg = wl.small_config(wl.CONFIGS[0], N=1, K=K, T=T)
+    X = wl.make_activations(cfg, "cuda")
+    _syrk_check(hq, X, impl=0)
+
+
+@pytest.mark.parametrize("T,K", [(64, 128), (1, 128), (100, 256), (4096, 384), (777, 1000), (129, 1032), (2048, 640)])
+def test_syrk_bf16_tensor_core(hq, cuda_device, T, K):
+    cfg = wl.small_config(wl.CONFIGS[1], N=1, K=K, T=T)
+    X = wl.make_activations(cfg, "cuda")
+    _syrk_check(hq, X, impl=0)
+
+
+def test_syrk_bf16_chunked_and_simt_agree(hq, cuda_device):
+    cfg = wl.small_config(wl.CONFIGS[1], N=1, K=512, T=3000)
+    X = wl.make_activations(cfg, "cuda")
+    _syrk_check(hq, X, impl=0, chunks=5)
+    _syrk_check(hq, X, impl=1, chunks=2)
+
+
+# ----------------------------------------------------------------------------- factorisation
+
+def _spd(K, seed, corr=0.7):
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((K, 2 * K))
+    H = A @ A.T / (2 * K)
+    H = (1 - corr) * np.diag(np.diag(H)) + corr * H
+    d = np.exp(rng.standard_normal(K))
+    return (H * np.outer(d, d)).astype(np.float32)
+
+
+@pytest.mark.parametrize("K", [128, 256, 640])
+def test_factor_upper_cholesky_of_inverse(hq, cuda_device, K):
+    H = _spd(K, K)
+    Hd = torch.from_numpy(H).cuda()
+    ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(1, K, 128))
+    Ut = torch.empty((K, K), device="cuda")
+    hq.hq_debug_factor(Hd, 0.01, Ut, ws)
+    Hdamp, _ = oracle.damp_hessian(H.astype(np.float64), 0.01)
+    U = oracle.upper_factor_of_inverse(Hdamp)
+    Ug = to_np64(Ut).T
+    assert np.array_equal(Ug, np.triu(Ug))
+    assert rel_fro(Ug, U) < 2e-4
+    I = Ug @ Hdamp @ Ug.T
+    assert np.abs(I - np.eye(K)).max() < 5e-3
+
+
+def test_factor_not_positive_definite(hq, cuda_device):
+    K = 128
+    H = np.eye(K, dtype=np.float32) * 5
+    H[K // 2, K // 2] = -1.0
+    ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(1, K, 128))
+    Ut = torch.empty((K, K), device="cuda")
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_debug_factor(torch.from_numpy(H).cuda(), 0.01, Ut, ws)
+    assert e.value.status == hq.HQ_ERR_NOT_PD
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_debug_factor(torch.from_numpy(-np.eye(K, dtype=np.float32)).cuda(), 0.01, Ut, ws)
+    assert e.value.status == hq.HQ_ERR_INVALID
+
+
+# ----------------------------------------------------------------------------- GPTQ
+
+def _run_gptq(hq, W, H, group, damp=0.01, imp=None, impl=0):
+    N, K = W.shape
+    codes, scales = hq.gptq_outputs(N, K, group)
+    ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(N, K, group))
+    q = hq.hq_debug_gptq_quantize_impl(W, H, group, damp, codes, scales, ws, impl, imp=imp)
+    torch.cuda.synchronize()
+    return unpack_codes(codes), scales.cpu().numpy(), q
+
+
+def _compare_gptq(W, H64, group, codes_g, scales_g, qerr_g, imp=None, damp=0.01, what=""):
+    Wn = to_np64(W)
+    Hd, _ = oracle.damp_hessian(H64, damp)
+    U = oracle.upper_factor_of_inverse(Hd)
+    rc, rs = check_gptq_parity(Wn, U, group, codes_g, scales_g, what)
+    r = {"codes": rc, "scales": rs}
+    q_ref = oracle.qerr(Wn, r["codes"], r["scales"], group, imp)
+    assert abs(qerr_g - q_ref) <= QERR_REL * q_ref + 1e-12, (qerr_g, q_ref)
+    l_ref = oracle.layer_loss(Wn, r["codes"], r["scales"], group, H64)
+    l_gpu = oracle.layer_loss(Wn, codes_g, scales_g, group, H64)
+    assert abs(l_gpu - l_ref) <= LOSS_REL * l_ref + 1e-12, (l_gpu, l_ref)
+    # the GPU's own qerr equals the oracle's qerr of the GPU's codes (checks the reduction)
+    q_of_gpu = oracle.qerr(Wn, codes_g, scales_g, group, imp)
+    assert abs(qerr_g - q_of_gpu) <= 1e-6 * max(q_of_gpu, 1e-12)
+    return r
+
+
+def test_gptq_tiny_layer_pipeline(hq, cuda_device):
+    """The tiny configuration end to end: SYRK on the GPU, then GPTQ; the oracle runs its own
+    fp64 path from the same X and W."""
+    cfg = wl.CONFIGS[0]
+    X = wl.make_activations(cfg, "cuda")
+    W = wl.make_weights(cfg, "cuda")
+    H = torch.zeros((cfg.K, cfg.K), device="cuda")
+    hq.hq_hessian_accumulate(H, X)
+    codes, scales, q = _run_gptq(hq, W, H, cfg.group, cfg.damp)
+    H64 = oracle.hessian(to_np64(X))
+    _compare_gptq(W, H64, cfg.group, codes, scales, q, what="tiny")
+
+
+@pytest.mark.parametrize("impl", [0, 1])
+@pytest.mark.parametrize("N,K,group,wdt", [(64, 128, 32, "f32"), (33, 256, 64, "f32"), (1, 384, 128, "bf16"),
+                                            (200, 512, 256, "bf16"), (130, 640, 128, "f32")])
+def test_gptq_stage_correlated(hq, cuda_device, N, K, group, wdt, impl):
+    """Strong compensation (low-rank correlated activations), ragged N, all group kinds,
+    both trailing-update kernels; H given as the oracle's own fp32 Hessian."""
+    cfg = wl.correlated_config(N, K, T=2 * K, group=group, seed=N + K)
+    X = wl.make_activations(cfg, "cpu")
+    H64 = oracle.hessian(X.double().numpy())
+    H32 = H64.astype(np.float32)
+    W = wl.make_weights(cfg, "cpu", N=N, K=K).to(wl.torch_dtype(wdt)).cuda()
+    codes, scales, q = _run_gptq(hq, W, torch.from_numpy(H32).cuda(), group, impl=impl)
+    _compare_gptq(W, H32.astype(np.float64), group, codes, scales, q, what=f"corr N={N} K={K} g={group}")
+
+
+def test_gptq_diagonal_hessian_equals_rtn(hq, cuda_device):
+    N, K, G = 96, 256, 32
+    rng = np.random.default_rng(5)
+    W = torch.from_numpy(rng.uniform(-1, 1, (N, K)).astype(np.float32)).cuda()
+    H = torch.from_numpy(np.diag(np.exp(rng.standard_normal(K))).astype(np.float32)).cuda()
+    c1, s1, q1 = _run_gptq(hq, W, H, G)
+    codes, scales = hq.gptq_outputs(N, K, G)
+    ws = hq.alloc_workspace(hq.hq_rtn_workspace_bytes(N, K, G))
+    q2 = hq.hq_rtn_quantize(W, G, codes, scales, ws)
+    c2, s2 = unpack_codes(codes), scales.cpu().numpy()
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2) and abs(q1 - q2) <= 1e-12 * q2
+    cr, sr = oracle.rtn_quantize(W.cpu().numpy(), G)
+    assert np.array_equal(c2, cr) and np.array_equal(s2, sr)
+    assert abs(q2 - oracle.qerr(W.cpu().numpy(), cr, sr, G)) < 1e-12
+
+
+def test_gptq_outputs_independent_of_qerr_request_and_deterministic(hq, cuda_device):
+    cfg = wl.correlated_config(160, 384, T=768, group=128, seed=3)
+    X = wl.make_activations(cfg, "cpu")
+    H = torch.from_numpy(oracle.hessian(X.double().numpy()).astype(np.float32)).cuda()
+    W = wl.make_weights(cfg, "cuda", N=160, K=384)
+    N, K, G = 160, 384, 128
+    ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(N, K, G))
+    outs = []
+    for want in (True, False, True):
+        codes, scales = hq.gptq_outputs(N, K, G)
+        qd = torch.zeros(1, dtype=torch.float64, device="cuda")
+        q = hq.hq_gptq_quantize(W, H, G, 0.01, codes, scales, ws, want_qerr=want, qerr_dev=qd)
+        torch.cuda.synchronize()
+        outs.append((codes.cpu().numpy().tobytes(), scales.cpu().numpy().tobytes(), q, qd.item()))
+    assert outs[0][0] == outs[1][0] == outs[2][0]
+    assert outs[0][1] == outs[1][1] == outs[2][1]
+    assert outs[1][2] is None and outs[0][2] == outs[2][2] == outs[0][3] == outs[1][3]
+
+
+def test_gptq_importance_moves_qerr_and_scale_cancels(hq, cuda_device):
+    cfg = wl.correlated_config(64, 256, T=512, group=64, seed=9)
+    X = wl.make_activations(cfg, "cpu")
+    H64 = oracle.hessian(X.double().numpy())
+    H = torch.from_numpy(H64.astype(np.float32)).cuda()
+    W = wl.make_weights(cfg, "cuda", N=64, K=256)
+    imp = torch.empty(256, device="cuda")
+    hq.hq_imatrix(H, 512, imp)
+    torch.cuda.synchronize()
+    assert np.allclose(imp.cpu().numpy(), oracle.imatrix(H.cpu().numpy().astype(np.float64), 512), rtol=1e-6)
+    c0, s0, q0 = _run_gptq(hq, W, H, 64)
+    c1, s1, q1 = _run_gptq(hq, W, H, 64, imp=imp)
+    c2, s2, q2 = _run_gptq(hq, W, H, 64, imp=imp * 1024)
+    assert np.array_equal(c0, c1) and np.array_equal(c1, c2)
+    assert q0 != q1
+    assert abs(q1 - q2) <= 1e-12 * q1
+    assert abs(q1 - oracle.qerr(to_np64(W), c1, s1, 64, imp.cpu().numpy())) <= 1e-6 * q1
+
+
+def test_gptq_hessian_power_of_two_scaling_is_bit_exact(hq, cuda_device):
+    cfg = wl.correlated_config(96, 384, T=768, group=128, seed=4)
+    X = wl.make_activations(cfg, "cpu")
+    H = torch.from_numpy(oracle.hessian(X.double().numpy()).astype(np.float32)).cuda()
+    W = wl.make_weights(cfg, "cuda", N=96, K=384)
+    a = _run_gptq(hq, W, H, 128)
+    b = _run_gptq(hq, W, H * 4.0, 128)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_gptq_row_permutation(hq, cuda_device):
+    cfg = wl.correlated_config(100, 256, T=512, group=128, seed=6)
+    X = wl.make_activations(cfg, "cpu")
+    H = torch.from_numpy(oracle.hessian(X.double().numpy()).astype(np.float32)).cuda()
+    W = wl.make_weights(cfg, "cuda", N=100, K=256)
+    perm = torch.randperm(100, generator=_gen(1, "cpu")).cuda()
+    a = _run_gptq(hq, W, H, 128)
+    b = _run_gptq(hq, W[perm].contiguous(), H, 128)
+    p = perm.cpu().numpy()
+    assert np.array_equal(a[0][p], b[0]) and np.array_equal(a[1][p], b[1])
+
+
+def test_gptq_exact_grid_recovered(hq, cuda_device):
+    N, K, G = 64, 256, 32
+    rng = np.random.default_rng(11)
+    codes = rng.integers(-7, 8, (N, K))
+    codes[:, ::G] = 7
+    W = torch.from_numpy((codes * 2.0 ** -4).astype(np.float32)).cuda()
+    cfg = wl.correlated_config(N, K, T=512, group=G, seed=12)
+    X = wl.make_activations(cfg, "cpu")
+    H = torch.from_numpy(oracle.hessian(X.double().numpy()).astype(np.float32)).cuda()
+    c, s, q = _run_gptq(hq, W, H, G)
+    assert np.array_equal(c, codes) and q == 0.0
+
+
+def test_gptq_not_pd_reported(hq, cuda_device):
+    K, N = 128, 8
+    H = np.eye(K, dtype=np.float32) * 5
+    H[3, 3] = -1.0
+    W = torch.ones((N, K), device="cuda")
+    with pytest.raises(hq.HQError) as e:
+        _run_gptq(hq, W, torch.from_numpy(H).cuda(), 32)
+    assert e.value.status == hq.HQ_ERR_NOT_PD
+
+
+# ----------------------------------------------------------------------------- RTN
+
+@pytest.mark.parametrize("N,K,G", [(1, 2, 2), (37, 96, 32), (256, 4096, 128), (64, 4096, 4096)])
+def test_rtn_bit_exact(hq, cuda_device, N, K, G):
+    rng = np.random.default_rng(N * K)
+    Wn = rng.uniform(-1, 1, (N, K)).astype(np.float32)
+    W = torch.from_numpy(Wn).cuda()
+    codes, scales = hq.gptq_outputs(N, K, G)
+    ws = hq.alloc_workspace(hq.hq_rtn_workspace_bytes(N, K, G))
+    q = hq.hq_rtn_quantize(W, G, codes, scales, ws)
+    cr, sr = oracle.rtn_quantize(Wn, G)
+    assert np.array_equal(unpack_codes(codes), cr)
+    assert np.array_equal(scales.cpu().numpy(), sr)
+    qr = oracle.qerr(Wn, cr, sr, G)
+    assert abs(q - qr) <= 1e-12 * max(qr, 1e-300) + 1e-15

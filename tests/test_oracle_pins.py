@@ -346,6 +346,23 @@ def test_gptq_k4_bruteforce():
     assert lg.sum() <= lr.sum()
 
 
+def test_forced_sweep_reproduces_free_sweep_and_keeps_loss_identity():
+    rng = np.random.default_rng(17)
+    N, K, G = 16, 128, 32
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    Hd, _ = O.damp_hessian(_spd(K, rng, corr=0.9), 0.01)
+    U = O.upper_factor_of_inverse(Hd)
+    codes, scales, E = O.gptq_sweep(W, U, G)
+    s2, E2, free, ratios = O.gptq_sweep_forced(W, U, G, codes)
+    assert np.array_equal(s2, scales) and np.array_equal(E2, E) and np.array_equal(free, codes)
+    # forcing other codes: D = E U still holds, so tr(D H' D^T) = sum e^2 for ANY codes
+    other = np.clip(codes + rng.integers(-1, 2, codes.shape), -8, 7)
+    s3, E3, free3, _ = O.gptq_sweep_forced(W, U, G, other)
+    D = W - O.dequantize(other, s3, G)
+    assert abs(float(np.sum((D @ Hd) * D)) - float(np.sum(E3 ** 2))) / float(np.sum(E3 ** 2)) < 1e-9
+    assert not np.array_equal(free3, other)
+
+
 def test_gptq_scale_invariance_of_hessian():
     rng = np.random.default_rng(12)
     N, K, G = 16, 128, 32
