@@ -24,9 +24,9 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
                           size_t workspace_bytes, hq_stream_t stream);
 
 /*
- * hq_gptq_quantize with an explicit choice of the trailing-update kernel:
- * update_impl 0 = tcgen05 tf32 tensor-core kernel (the default path), 1 = fp32 CUDA-core
- * kernel (reference for the tensor-core one).
+ * hq_gptq_quantize with an explicit choice of the lazy-update kernel:
+ * update_impl 0 = tcgen05 tensor cores in 3xTF32 (the default path), 1 = fp32 CUDA cores
+ * (reference for the tensor-core one), 2 = tcgen05 tensor cores in plain tf32.
  */
 hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
                                       int64_t group, float damp, const float* imp, uint8_t* codes,
@@ -39,6 +39,17 @@ hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int
  */
 hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype, int64_t T, int64_t K,
                                            int* dev_status, int impl, hq_stream_t stream);
+
+/*
+ * The tensor-core fp32 GEMM used by the factorisation and the GPTQ lazy updates:
+ *   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]
+ * for m < M, n < N (if `lower`, only elements with m >= n are written).  split3 = 1 selects
+ * 3xTF32 (about fp32 accuracy), 0 plain tf32.  A and B 16-byte aligned, lda and ldb
+ * multiples of 4.  No counterpart on the pages: a building block of the path.
+ */
+hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
+                             const float* B, int64_t ldb, float alpha, float beta, int lower, int split3,
+                             hq_stream_t stream);
 
 /* Number of kernels libhq.so has launched in this process so far (all devices, all
  * threads).  A statistic for profiling; never reset. */

@@ -60,6 +60,7 @@ _SIGS = {
                                            _int, _vp]),
     "hq_debug_hessian_accumulate_impl": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _int, _vp]),
     "hq_debug_launch_count": (ctypes.c_uint64, []),
+    "hq_debug_tf32_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _f, _f, _int, _int, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -177,6 +178,15 @@ def hq_debug_factor(H, damp: float, Ut_out, workspace, stream=None) -> None:
     K = H.shape[0]
     _check(lib.hq_debug_factor(_ptr(H), K, float(damp), _ptr(Ut_out), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)), "hq_debug_factor")
+
+
+def hq_debug_tf32_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, split3=True, stream=None) -> None:
+    """C = beta C + alpha A B^T (fp32 row-major views, tensor cores)."""
+    M, Kred = A.shape
+    N = B.shape[0]
+    _check(lib.hq_debug_tf32_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
+                                  float(alpha), float(beta), int(bool(lower)), int(bool(split3)), _stream(stream)),
+           "hq_debug_tf32_gemm")
 
 
 def hq_bf16tril_bytes(K: int) -> int:

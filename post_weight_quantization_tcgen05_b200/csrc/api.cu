@@ -126,7 +126,7 @@ hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int
                                       int64_t group, float damp, const float* imp, uint8_t* codes, float* scales,
                                       double* qerr_out, double* qerr_dev, void* workspace, size_t workspace_bytes,
                                       int update_impl, hq_stream_t stream) {
-  if (update_impl != 0 && update_impl != 1) return HQ_ERR_INVALID;
+  if (update_impl < 0 || update_impl > 2) return HQ_ERR_INVALID;
   return gptq_common(W, w_dtype, N, K, H, group, damp, imp, codes, scales, qerr_out, qerr_dev, workspace,
                      workspace_bytes, update_impl, static_cast<cudaStream_t>(stream));
 }
@@ -143,11 +143,34 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
   float* A = reinterpret_cast<float*>(ws + L.a);
-  hq_status st = launch_factor(H, K, damp, A, reinterpret_cast<float*>(ws + L.x), reinterpret_cast<float*>(ws + L.t),
-                               reinterpret_cast<float*>(ws + L.dinv), &hdr->lam, &hdr->info, A, s);
+  hq_status st = launch_factor(H, K, damp, A, reinterpret_cast<float*>(ws + L.x), reinterpret_cast<float*>(ws + L.xt),
+                               reinterpret_cast<float*>(ws + L.t), &hdr->lam, &hdr->info, &hdr->status, A,
+                               reinterpret_cast<float*>(ws + L.t), s);
   if (st != HQ_OK) return st;
   HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, A, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return finish_sync(s, hdr, nullptr);
+}
+
+hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
+                             const float* B, int64_t ldb, float alpha, float beta, int lower, int split3,
+                             hq_stream_t stream) {
+  if (C == nullptr || A == nullptr || B == nullptr || M < 0 || N < 0 || Kred < 1) return HQ_ERR_INVALID;
+  if (ldc < N || lda < Kred || ldb < Kred) return HQ_ERR_INVALID;
+  Tf32Gemm g{};
+  g.C = C;
+  g.ldc = ldc;
+  g.M = M;
+  g.N = N;
+  g.Kred = Kred;
+  g.A = A;
+  g.lda = lda;
+  g.B = B;
+  g.ldb = ldb;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.lower = lower ? 1 : 0;
+  g.split3 = split3 != 0;
+  return tf32_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
 size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group) {

@@ -5,21 +5,32 @@
 // U, the upper Cholesky factor of (H + lambda I)^-1, is reached through the index reversal J:
 // with M = J (H + lambda I) J = L L^T (L lower), U = J L^-1 J.  By uniqueness of the Cholesky
 // factor this is the same U as Cholesky -> inverse -> Cholesky of the inverse, at half the
-// flops.  Steps (all fp32 on the device):
+// flops.  Only X = L^-1 is ever needed, so the factorisation and the inversion are one
+// recursion on M:
+//
+//   chol_inv([A11 .; A21 A22]):  X11 = chol_inv(A11)
+//                                T   = A21 X11^T          (= L21)
+//                                A22 = A22 - T T^T        (Schur complement, lower part)
+//                                X22 = chol_inv(A22)
+//                                Y^T = X11^T T^T          (Y = T X11)
+//                                X21 = -X22 Y
+//
+// Every product takes both operands K-major (row-major [rows, contraction]), so X^T is kept
+// next to X (leaves write both, X21^T is copied by a tiled transpose).  The products run on the
+// tensor cores in 3xTF32 (gemm_tf32.cuh).  Leaves are 128 x 128 blocks factored and inverted by
+// one CTA (chol_inv_leaf_kernel).  Steps:
 //   1. lambda = damp * mean(diag H)            (fp64 reduction, one CTA)
 //   2. A = J (H + lambda I) J, lower triangle  (tiled transpose; H's lower triangle is read)
-//   3. A = L, blocked right-looking Cholesky   (64-wide panels: diagonal block in one CTA,
-//      which also inverts it; panel solve by the inverted block; trailing update)
-//   4. X = L^-1, recursive halving             (diagonal blocks from step 3, off-diagonal
-//      blocks X21 = -X22 (L21 X11))
-//   5. U^T = J X^T J written row-major         (U^T[c, j] = X[K-1-j, K-1-c], c >= j)
-// A device flag `info` receives the first failing pivot (1-based) and stops later kernels.
+//   3. X = L^-1 and X^T by the recursion above
+//   4. U = J X J and U^T = J X^T J, both row-major (180-degree rotated copies)
+// A device flag `info` receives the first failing pivot (1-based, in M's order) and stops
+// every later kernel.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace hq {
 
-constexpr int NB = 64;
+constexpr int kLeaf = 128;
 
 // ------------------------------------------------------------------------- 1. lambda
 
@@ -78,247 +89,256 @@ __global__ void __launch_bounds__(256) reverse_damp_kernel(const float* __restri
   }
 }
 
-// ------------------------------------------------------------------------- 3. Cholesky
+// ------------------------------------------------------------------------- 3a. leaf
 
-// Factor the NB x NB diagonal block at (p, p) in shared memory, write L11 (upper part zeroed)
-// back into A and its inverse into Dinv[p].
-__global__ void __launch_bounds__(256) potrf_diag_kernel(float* __restrict__ A, int64_t K, int p,
-                                                         float* __restrict__ Dinv, int* __restrict__ info) {
+// Lower 4 x 4 tiles of the 128 x 128 leaf, enumerated row by row: 32 * 33 / 2 = 528 tiles;
+// thread t owns tiles t, t + 256 and t + 512, so a warp's tiles lie in one band of rows.
+__device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
+  int r = static_cast<int>((sqrtf(8.f * idx + 1.f) - 1.f) * 0.5f);
+  while (r * (r + 1) / 2 > idx) --r;
+  while ((r + 1) * (r + 2) / 2 <= idx) ++r;
+  ti = r;
+  tj = idx - r * (r + 1) / 2;
+}
+
+// Factor the 128 x 128 lower block at A as L D L^T (unit L) by right-looking elimination, and
+// at the same time eliminate Y = L^-1 (unit lower); writes X = D^-1/2 Y = (L D^1/2)^-1, the
+// inverse of the Cholesky factor, with zeros above the diagonal.  Every element lives in a
+// register of the thread that owns its tile; step k publishes column k of the Schur
+// complement and row k of Y through double-buffered shared memory (one barrier per step).
+__global__ void __launch_bounds__(256, 1) chol_inv_leaf_kernel(const float* __restrict__ A, int64_t lda,
+                                                               float* __restrict__ X, float* __restrict__ XT,
+                                                               int64_t ldx, int* __restrict__ info, int diag_off) {
   if (*info != 0) return;
-  __shared__ float S[NB][NB + 1];
-  __shared__ float X[NB][NB + 1];
-  __shared__ int bad;
-  const int64_t o = static_cast<int64_t>(p) * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    S[r][c] = (c <= r) ? A[(o + r) * K + o + c] : 0.f;
+  __shared__ float colbuf[2][kLeaf];
+  __shared__ float yrow[2][kLeaf];
+  __shared__ float dbuf[kLeaf];
+  const int t = threadIdx.x;
+  int ti[3], tj[3];
+  bool own[3];
+  float v[3][16], y[3][16];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    const int idx = t + 256 * q;
+    own[q] = idx < 528;
+    leaf_tile(own[q] ? idx : 0, ti[q], tj[q]);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int i = 4 * ti[q] + r, j = 4 * tj[q] + c;
+        v[q][r * 4 + c] = (own[q] && j <= i) ? A[i * lda + j] : 0.f;
+        y[q][r * 4 + c] = (own[q] && i == j) ? 1.f : 0.f;
+      }
   }
-  if (threadIdx.x == 0) bad = 0;
+  if (t < kLeaf) {
+    yrow[0][t] = 0.f;
+    yrow[1][t] = 0.f;
+  }
   __syncthreads();
-  for (int k = 0; k < NB; ++k) {
-    if (threadIdx.x == 0) {
-      const float d = S[k][k];
-      if (!(d > 0.f) || !isfinite(d)) {
-        bad = 1;
-        atomicCAS(info, 0, static_cast<int>(o + k + 1));
-      } else {
-        S[k][k] = sqrtf(d);
+
+  for (int k = 0; k < kLeaf; ++k) {
+    const int buf = k & 1, kt = k >> 2, kc = k & 3;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      if (!own[q]) continue;
+      if (tj[q] == kt) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float x = v[q][r * 4];
+#pragma unroll
+          for (int c = 1; c < 4; ++c) x = (c == kc) ? v[q][r * 4 + c] : x;
+          colbuf[buf][4 * ti[q] + r] = x;
+        }
+      }
+      if (ti[q] == kt) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float x = y[q][c];
+#pragma unroll
+          for (int r = 1; r < 4; ++r) x = (r == kc) ? y[q][r * 4 + c] : x;
+          yrow[buf][4 * tj[q] + c] = x;
+        }
       }
     }
     __syncthreads();
-    if (bad) return;
-    const float lkk = S[k][k];
-    for (int i = k + 1 + threadIdx.x; i < NB; i += blockDim.x) S[i][k] = S[i][k] / lkk;
-    __syncthreads();
-    const int m = NB - k - 1;
-    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
-      const int i = k + 1 + e / m, j = k + 1 + e % m;
-      if (j <= i) S[i][j] = fmaf(-S[i][k], S[j][k], S[i][j]);
+    const float d = colbuf[buf][k];
+    if (!(d > 0.f) || !isfinite(d)) {
+      if (t == 0) atomicCAS(info, 0, diag_off + k + 1);
+      return;  // uniform: every thread read the same pivot
     }
-    __syncthreads();
-  }
-  // inverse of the lower-triangular block, one column per thread (forward substitution)
-  if (threadIdx.x < NB) {
-    const int j = threadIdx.x;
-    for (int i = 0; i < j; ++i) X[i][j] = 0.f;
-    X[j][j] = 1.f / S[j][j];
-    for (int i = j + 1; i < NB; ++i) {
-      float acc = 0.f;
-      for (int k = j; k < i; ++k) acc = fmaf(S[i][k], X[k][j], acc);
-      X[i][j] = -acc / S[i][i];
+    const float inv_d = 1.f / d;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      if (!own[q]) continue;
+      const int i0 = 4 * ti[q], j0 = 4 * tj[q];
+      if (i0 + 3 <= k) continue;  // every row of the tile is at or above the pivot
+      float a[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) a[r] = (i0 + r > k) ? colbuf[buf][i0 + r] * inv_d : 0.f;  // L[i][k]
+      if (j0 + 3 > k) {
+        // Schur update S[i][j] -= S[i][k] S[j][k] / d_k  for i, j > k
+        float b[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) b[c] = (j0 + c > k) ? colbuf[buf][j0 + c] : 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v[q][r * 4 + c] = fmaf(-a[r], b[c], v[q][r * 4 + c]);
+      }
+      if (j0 <= k) {
+        // elimination of Y: Y[i][j] -= L[i][k] Y[k][j]  for i > k, j <= k
+        float yb[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) yb[c] = yrow[buf][j0 + c];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) y[q][r * 4 + c] = fmaf(-a[r], yb[c], y[q][r * 4 + c]);
+      }
     }
   }
+  // X[i][j] = Y[i][j] / sqrt(d_i)
+#pragma unroll
+  for (int q = 0; q < 3; ++q)
+    if (own[q] && ti[q] == tj[q])
+#pragma unroll
+      for (int r = 0; r < 4; ++r) dbuf[4 * ti[q] + r] = v[q][r * 4 + r];
   __syncthreads();
-  float* D = Dinv + static_cast<int64_t>(p) * NB * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    A[(o + r) * K + o + c] = (c <= r) ? S[r][c] : 0.f;
-    D[e] = X[r][c];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    if (!own[q]) continue;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float sc = 1.f / sqrtf(dbuf[4 * ti[q] + r]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) y[q][r * 4 + c] *= sc;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i = 4 * ti[q] + r;
+      *reinterpret_cast<float4*>(X + static_cast<int64_t>(i) * ldx + 4 * tj[q]) =
+          make_float4(y[q][r * 4 + 0], y[q][r * 4 + 1], y[q][r * 4 + 2], y[q][r * 4 + 3]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = 4 * tj[q] + c;
+      *reinterpret_cast<float4*>(XT + static_cast<int64_t>(j) * ldx + 4 * ti[q]) =
+          make_float4(y[q][0 * 4 + c], y[q][1 * 4 + c], y[q][2 * 4 + c], y[q][3 * 4 + c]);
+    }
   }
 }
 
-// L21 = A21 * L11^-T = A21 * Dinv^T for the NB-row slab per CTA below the diagonal block.
-__global__ void __launch_bounds__(256) trsm_panel_kernel(float* __restrict__ A, int64_t K, int p,
-                                                         const float* __restrict__ Dinv,
-                                                         const int* __restrict__ info) {
-  if (*info != 0) return;
-  __shared__ float As[NB][NB + 1];
-  __shared__ float Ds[NB][NB + 1];
-  const int64_t o = static_cast<int64_t>(p) * NB;
-  const int64_t r0 = o + NB + static_cast<int64_t>(blockIdx.x) * NB;
-  const float* D = Dinv + static_cast<int64_t>(p) * NB * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    As[r][c] = (r0 + r < K) ? A[(r0 + r) * K + o + c] : 0.f;
-    Ds[r][c] = D[e];
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, j = e % NB;
-    if (r0 + r >= K) continue;
-    float acc = 0.f;
-    for (int k = 0; k <= j; ++k) acc = fmaf(As[r][k], Ds[j][k], acc);  // Dinv lower: k <= j
-    A[(r0 + r) * K + o + j] = acc;
-  }
-}
+// ------------------------------------------------------------------------- 3b. recursion
 
-// ------------------------------------------------------------------------- CUDA-core GEMM
-
-// C[m, n] = beta * C[m, n] + alpha * sum_k A(m, k) B(k, n), with A(m, k) = A[m*sam + k*sak]
-// and B(k, n) = B[k*sbk + n*sbn].  lower_only: only tiles/elements with m >= n (row and
-// column indices offset by diag_off: element kept when m + diag_off >= n).
-struct SimtGemm {
-  const float* A;
-  int64_t sam, sak;
-  const float* B;
-  int64_t sbk, sbn;
-  float* C;
-  int64_t ldc;
-  int M, N, Kc;
-  float alpha, beta;
-  int lower_only;
+struct FactorCtx {
+  float* A;
+  float* X;
+  float* XT;
+  int64_t K;
+  int* info;
+  int* status;
+  cudaStream_t s;
 };
 
-__global__ void __launch_bounds__(256) gemm_simt_kernel(SimtGemm g, const int* __restrict__ info) {
-  if (info != nullptr && *info != 0) return;
-  const int tiles_n = (g.N + 63) / 64;
-  const int tm = blockIdx.x / tiles_n, tn = blockIdx.x % tiles_n;
-  if (g.lower_only && tn > tm) return;
-  const int m0 = tm * 64, n0 = tn * 64;
-  __shared__ float As[16][64];
-  __shared__ float Bs[16][64];
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < g.Kc; k0 += 16) {
-    for (int e = threadIdx.x; e < 16 * 64; e += 256) {
-      const int kk = e / 64, c = e % 64;
-      const int k = k0 + kk;
-      As[kk][c] = (k < g.Kc && m0 + c < g.M) ? g.A[(m0 + c) * g.sam + k * g.sak] : 0.f;
-      Bs[kk][c] = (k < g.Kc && n0 + c < g.N) ? g.B[k * g.sbk + (n0 + c) * g.sbn] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a[u] = As[kk][ty + 16 * u];
-        b[u] = Bs[kk][tx + 16 * u];
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int m = m0 + ty + 16 * u;
-    if (m >= g.M) continue;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int n = n0 + tx + 16 * v;
-      if (n >= g.N || (g.lower_only && n > m)) continue;
-      float* c = g.C + static_cast<int64_t>(m) * g.ldc + n;
-      *c = (g.beta == 0.f ? 0.f : g.beta * *c) + g.alpha * acc[u][v];
-    }
-  }
+static hq_status gemm(const FactorCtx& c, float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
+                      const float* B, int64_t ldb, float alpha, float beta, bool lower) {
+  Tf32Gemm g{};
+  g.C = C;
+  g.ldc = ldc;
+  g.M = M;
+  g.N = N;
+  g.Kred = Kred;
+  g.A = A;
+  g.lda = lda;
+  g.B = B;
+  g.ldb = ldb;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.lower = lower ? 1 : 0;
+  g.split3 = true;
+  g.skip = c.info;
+  g.status = c.status;
+  return tf32_gemm(g, c.s);
 }
 
-static hq_status gemm_simt(const SimtGemm& g, const int* info, cudaStream_t s) {
-  if (g.M <= 0 || g.N <= 0) return HQ_OK;
-  const int64_t tiles = ceil_div(g.M, 64) * ceil_div(g.N, 64);
-  gemm_simt_kernel<<<static_cast<unsigned>(tiles), 256, 0, s>>>(g, info);
+// dst[j][i] = src[i][j] for an R x C block (32 x 32 tiles through shared memory).
+__global__ void __launch_bounds__(256) transpose_kernel(const float* __restrict__ src, int64_t lds, int64_t R,
+                                                        int64_t C, float* __restrict__ dst, int64_t ldd,
+                                                        const int* __restrict__ info) {
+  if (*info != 0) return;
+  __shared__ float t[32][33];
+  const int64_t tiles_c = (C + 31) / 32;
+  const int64_t r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
+  for (int i = ty; i < 32; i += 8)
+    if (r0 + i < R && c0 + tx < C) t[i][tx] = src[(r0 + i) * lds + c0 + tx];
+  __syncthreads();
+  for (int j = ty; j < 32; j += 8)
+    if (c0 + j < C && r0 + tx < R) dst[(c0 + j) * ldd + r0 + tx] = t[tx][j];
+}
+
+// X = L^-1 and X^T for the n x n block of A at (off, off); `tmp` has room for the temporaries
+// of this level and all levels below (2 * n2 * n1 floats here, a quarter of that below...).
+static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, float* tmp) {
+  const int64_t K = c.K;
+  if (n == kLeaf) {
+    chol_inv_leaf_kernel<<<1, 256, 0, c.s>>>(c.A + off * K + off, K, c.X + off * K + off, c.XT + off * K + off, K,
+                                             c.info, static_cast<int>(off));
+    HQ_LAUNCH_CHECK();
+    return HQ_OK;
+  }
+  const int64_t n1 = (n / kLeaf / 2) * kLeaf, n2 = n - n1;
+  float* T = tmp;             // n2 x n1: L21
+  float* YT = tmp + n2 * n1;  // n1 x n2: (L21 X11)^T
+  float* rest = YT + n2 * n1;
+  const float* A21 = c.A + (off + n1) * K + off;
+  float* A22 = c.A + (off + n1) * K + off + n1;
+  const float* X11 = c.X + off * K + off;
+  const float* XT11 = c.XT + off * K + off;
+  float* X21 = c.X + (off + n1) * K + off;
+  const float* X22 = c.X + (off + n1) * K + off + n1;
+  float* XT12 = c.XT + off * K + off + n1;
+  const int in1 = static_cast<int>(n1), in2 = static_cast<int>(n2);
+  hq_status st = chol_inv(c, off, n1, rest);
+  if (st != HQ_OK) return st;
+  st = gemm(c, T, n1, in2, in1, in1, A21, K, X11, K, 1.f, 0.f, false);     // T = A21 X11^T
+  if (st != HQ_OK) return st;
+  st = gemm(c, A22, K, in2, in2, in1, T, n1, T, n1, -1.f, 1.f, true);      // A22 -= T T^T
+  if (st != HQ_OK) return st;
+  st = chol_inv(c, off + n1, n2, rest);
+  if (st != HQ_OK) return st;
+  st = gemm(c, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.f, 0.f, false);    // Y^T = X11^T T^T
+  if (st != HQ_OK) return st;
+  st = gemm(c, X21, K, in2, in1, in2, X22, K, YT, n2, -1.f, 0.f, false);   // X21 = -X22 Y
+  if (st != HQ_OK) return st;
+  const int64_t tiles = ceil_div(n2, 32) * ceil_div(n1, 32);
+  transpose_kernel<<<static_cast<unsigned>(tiles), 256, 0, c.s>>>(X21, K, n2, n1, XT12, K, c.info);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
 }
 
-// ------------------------------------------------------------------------- 4. L^-1
+// ------------------------------------------------------------------------- 4. U, U^T
 
-static hq_status invert_lower_rec(const float* L, float* X, float* T, int64_t K, int64_t off, int64_t n,
-                                  const float* Dinv, const int* info, cudaStream_t s) {
-  if (n == NB) {
-    // X block = Dinv[off / NB]
-    HQ_CUDA_TRY(cudaMemcpy2DAsync(X + off * K + off, K * sizeof(float), Dinv + (off / NB) * NB * NB,
-                                  NB * sizeof(float), NB * sizeof(float), NB, cudaMemcpyDeviceToDevice, s));
-    return HQ_OK;
-  }
-  const int64_t nblk = n / NB;
-  const int64_t n1 = (nblk / 2) * NB, n2 = n - n1;
-  hq_status st = invert_lower_rec(L, X, T, K, off, n1, Dinv, info, s);
-  if (st != HQ_OK) return st;
-  st = invert_lower_rec(L, X, T, K, off + n1, n2, Dinv, info, s);
-  if (st != HQ_OK) return st;
-  // T = L21 X11   (n2 x n1)
-  SimtGemm g1{};
-  g1.A = L + (off + n1) * K + off;
-  g1.sam = K;
-  g1.sak = 1;
-  g1.B = X + off * K + off;
-  g1.sbk = K;
-  g1.sbn = 1;
-  g1.C = T;
-  g1.ldc = n1;
-  g1.M = static_cast<int>(n2);
-  g1.N = static_cast<int>(n1);
-  g1.Kc = static_cast<int>(n1);
-  g1.alpha = 1.f;
-  g1.beta = 0.f;
-  st = gemm_simt(g1, info, s);
-  if (st != HQ_OK) return st;
-  // X21 = -X22 T  (n2 x n1)
-  SimtGemm g2{};
-  g2.A = X + (off + n1) * K + off + n1;
-  g2.sam = K;
-  g2.sak = 1;
-  g2.B = T;
-  g2.sbk = n1;
-  g2.sbn = 1;
-  g2.C = X + (off + n1) * K + off;
-  g2.ldc = K;
-  g2.M = static_cast<int>(n2);
-  g2.N = static_cast<int>(n1);
-  g2.Kc = static_cast<int>(n2);
-  g2.alpha = -1.f;
-  g2.beta = 0.f;
-  return gemm_simt(g2, info, s);
-}
-
-// ------------------------------------------------------------------------- 5. U^T
-
-// Ut[c][j] = X[K-1-j][K-1-c] for c >= j, 0 above the diagonal.  32 x 32 tiles via smem.
-__global__ void __launch_bounds__(256) anti_transpose_kernel(const float* __restrict__ X, int64_t K,
-                                                             float* __restrict__ Ut, const int* __restrict__ info) {
+// U[j][c] = X[K-1-j][K-1-c] and U^T[j][c] = X^T[K-1-j][K-1-c]: 180-degree rotations (U upper,
+// U^T lower, zeros elsewhere because X and X^T hold zeros there).
+__global__ void rotate_kernel(const float* __restrict__ X, const float* __restrict__ XT, int64_t K,
+                              float* __restrict__ U, float* __restrict__ Ut, const int* __restrict__ info) {
   if (*info != 0) return;
-  __shared__ float t[32][33];
-  const int64_t tiles = (K + 31) / 32;
-  const int64_t tc = blockIdx.x / tiles, tj = blockIdx.x % tiles;
-  const int64_t c0 = tc * 32, j0 = tj * 32;
-  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
-  // source rows K-1-j (j in tile), columns K-1-c (c in tile)
-  for (int jj = ty; jj < 32; jj += 8) {
-    const int64_t j = j0 + jj, c = c0 + tx;
-    float v = 0.f;
-    if (j < K && c < K && c >= j) v = X[(K - 1 - j) * K + (K - 1 - c)];
-    t[jj][tx] = v;  // t[j][c]
-  }
-  __syncthreads();
-  for (int cc = ty; cc < 32; cc += 8) {
-    const int64_t c = c0 + cc, j = j0 + tx;
-    if (c < K && j < K) Ut[c * K + j] = t[tx][cc];
+  const int64_t n = K * K;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t src = n - 1 - e;  // (K-1-j)*K + (K-1-c) for e = j*K + c
+    U[e] = X[src];
+    Ut[e] = XT[src];
   }
 }
 
 // ------------------------------------------------------------------------- driver
 
-size_t factor_workspace_floats(int64_t K) {
-  // A (K^2), X (K^2), T (K^2/4), Dinv (K * NB)
-  return static_cast<size_t>(K) * K * 2 + static_cast<size_t>(K / 2) * (K - K / 2 + NB) + static_cast<size_t>(K) * NB;
-}
-
-hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* X, float* T, float* Dinv,
-                        double* lam, int* info, float* Ut, cudaStream_t s) {
+hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* X, float* XT, float* T, double* lam,
+                        int* info, int* status, float* Ut, float* U, cudaStream_t s) {
+  if (K % kLeaf != 0) return HQ_ERR_UNSUPPORTED;
   damp_stats_kernel<<<1, 1024, 0, s>>>(H, K, damp, lam, info);
   HQ_LAUNCH_CHECK();
   {
@@ -326,41 +346,14 @@ hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* 
     reverse_damp_kernel<<<static_cast<unsigned>(nb * (nb + 1) / 2), 256, 0, s>>>(H, K, lam, A, info);
     HQ_LAUNCH_CHECK();
   }
-  const int np = static_cast<int>(K / NB);
-  for (int p = 0; p < np; ++p) {
-    potrf_diag_kernel<<<1, 256, 0, s>>>(A, K, p, Dinv, info);
-    HQ_LAUNCH_CHECK();
-    const int rows_below = static_cast<int>(K - static_cast<int64_t>(p + 1) * NB);
-    if (rows_below <= 0) break;
-    trsm_panel_kernel<<<static_cast<unsigned>(ceil_div(rows_below, NB)), 256, 0, s>>>(A, K, p, Dinv, info);
-    HQ_LAUNCH_CHECK();
-    SimtGemm g{};
-    const int64_t o = static_cast<int64_t>(p + 1) * NB;
-    g.A = A + o * K + p * NB;  // L21 rows (o.., panel cols)
-    g.sam = K;
-    g.sak = 1;
-    g.B = A + o * K + p * NB;  // B(k, n) = L21[n][k]
-    g.sbk = 1;
-    g.sbn = K;
-    g.C = A + o * K + o;
-    g.ldc = K;
-    g.M = rows_below;
-    g.N = rows_below;
-    g.Kc = NB;
-    g.alpha = -1.f;
-    g.beta = 1.f;
-    g.lower_only = 1;
-    hq_status st = gemm_simt(g, info, s);
-    if (st != HQ_OK) return st;
-  }
   HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(float), s));
-  hq_status st = invert_lower_rec(A, X, T, K, 0, K, Dinv, info, s);
+  HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(float), s));
+  FactorCtx c{A, X, XT, K, info, status, s};
+  hq_status st = chol_inv(c, 0, K, T);
   if (st != HQ_OK) return st;
-  {
-    const int64_t nt = ceil_div(K, 32);
-    anti_transpose_kernel<<<static_cast<unsigned>(nt * nt), 256, 0, s>>>(X, K, Ut, info);
-    HQ_LAUNCH_CHECK();
-  }
+  const int64_t grid = ceil_div(K * K, 4 * 256) < 148 * 32 ? ceil_div(K * K, 4 * 256) : 148 * 32;
+  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, U, Ut, info);
+  HQ_LAUNCH_CHECK();
   return HQ_OK;
 }
 

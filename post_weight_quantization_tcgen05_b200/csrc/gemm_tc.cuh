@@ -239,14 +239,7 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t src = tmem + lane_off + static_cast<uint32_t>(acc * kGemmBN + h * 128);
-#pragma unroll
-        for (int c = 0; c < 128; c += 16) {
-          float v[16];
-          ptx::tmem_ld16(src + c, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) sum[c + i] += v[i];
-        }
+        ptx::tmem_add128(tmem + lane_off + static_cast<uint32_t>(acc * kGemmBN + h * 128), sum);
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&acce[acc]);

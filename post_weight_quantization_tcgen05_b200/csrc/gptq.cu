@@ -2,35 +2,45 @@
 // experiment summary: error-feedback sweep, uniform symmetric int4 [-8, 7], per-(row, group)
 // scale absmax/7, dequant w = code * scale; qerr definition in the same page).
 //
-// The sweep walks K in 128-column blocks.  For each block:
-//   * sweep_block_kernel: the sequential part.  Four lanes share one row (lane l owns the
-//     columns 4m + l of the block, 32 fp32 values in registers); the 128 x 128 diagonal block
-//     of U sits in shared memory.  Per column j: group scale at a group start (4-lane absmax),
-//     broadcast of w_j from its owner lane, code c = clamp(rint(w_j / s), -8, 7), error
-//     e = (w_j - c s) / U[j, j], and the in-block feedback w_k -= e U[j, k] for k > j.  It
-//     writes the block's errors (fp32, row-major [N, 128]), the packed int4 codes, the scales
-//     and fp64 partial sums of the qerr numerator and denominator over the ORIGINAL weights.
-//   * the lazy trailing update W[:, J+128:] -= Err * U[J:J+128, J+128:], a dense contraction
-//     run on the tensor cores (tcgen05 kind::tf32, gemm_tc.cuh) with B = U^T row-major.
+// The sweep walks K in 128-column blocks grouped into panels of P columns (P = 512, or a
+// multiple of the group size when groups are wider than a block).  Per block:
+//   * sweep_block_kernel: the sequential part.  Four lanes share a row; lane l holds the
+//     row's columns l, l+4, l+8, ... as 32 "slots" in registers.  The columns are visited in
+//     rounds of four: at the end of a round every lane shifts its slots down by one, so the
+//     column being quantised is always slot 0 of lane (j mod 4), a compile-time lane inside the
+//     4-way unrolled round, and the loop body stays small enough for the instruction cache.
+//     Per column j: group scale at a group start (4-lane absmax), broadcast of w_j, code
+//     c = clamp(rint(w_j / s), -8, 7), error e = (w_j - c s) / U[j, j], and the feedback
+//     w_k -= e U[j, k] for k > j, with U's row j pre-permuted in shared memory so that each
+//     lane reads its 32 values with eight aligned 16-byte loads.  It writes the block's
+//     errors into the panel's error buffer, the packed int4 codes, the scales and fp64 partial
+//     sums of the qerr numerator and denominator over the ORIGINAL weights.
+//   * inner lazy update of the rest of the panel, W[:, b+128 : panel end] -= Err_b U[b, ...]
+//     (contraction 128; the panel's N x P working weights stay in L2);
+// and after the panel the outer lazy update W[:, panel end:] -= Err_panel U[panel, ...] with
+// contraction P.  Both updates are dense contractions on the tensor cores (gemm_tf32.cuh, by
+// default 3xTF32) with B = U^T row-major.  Blocking only reorders exact sums: every column
+// still receives the feedback of every earlier column before it is quantised.
 // U^T comes from factor.cu.  The working copy of W is fp32 in the workspace.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
-#include "gemm_tc.cuh"
 #include "kernels.cuh"
-#include "tmap.cuh"
 
 namespace hq {
 
-constexpr int kBlk = 128;       // sweep block width
-constexpr int kRowsPerCta = 32;  // 4 warps x 8 rows (4 lanes per row)
+constexpr int kBlk = 128;        // sweep block width
+constexpr int kRowsPerCta = 32;  // 4 warps x 8 rows, 4 lanes per row
+constexpr int kSweepThreads = 128;
 
 struct SweepArgs {
   float* Wf;
   int64_t N, K;
-  const float* Ut;
+  const float* U;    // U row-major (upper triangular)
   int group;
-  float* Err;
+  float* Err;        // panel error buffer [N, P]
+  int64_t err_ld;    // P
+  int err_col;       // column of this block inside the panel buffer
   uint8_t* codes;
   float* scales;
   const void* W;
@@ -44,40 +54,62 @@ __device__ __forceinline__ float load_w(const void* W, int dt, int64_t idx) {
   return dt == HQ_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(W)[idx]) : static_cast<const float*>(W)[idx];
 }
 
-__device__ __forceinline__ float quant_code(float w, float s) {
+// c = clamp(rint(w / s), -8, 7) with w / s the IEEE fp32 quotient.  w * (1/s) is within a
+// couple of ulps of the quotient, so it rounds the same way unless it lies within 1e-5 of a
+// half-integer; only then is the exact division taken.
+__device__ __forceinline__ float quant_code(float w, float s, float rs) {
   if (!(s > 0.f)) return 0.f;
-  float c = rintf(__fdiv_rn(w, s));
-  return fminf(fmaxf(c, -8.f), 7.f);
+  float q = w * rs;
+  const float a = fabsf(q);
+  if (fabsf(a - floorf(a) - 0.5f) < 1e-5f) q = __fdiv_rn(w, s);
+  return fminf(fmaxf(rintf(q), -8.f), 7.f);
 }
 
 // GS: group size when it is 32, 64 or 128 (scales computed inside the block), or 0 when the
 // group spans several blocks (scale computed at the group's first block from Wf).
 template <int GS>
-__global__ void __launch_bounds__(128) sweep_block_kernel(SweepArgs a, int j0) {
+__global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a, int j0) {
   if (*a.info != 0) return;
+  constexpr int LD = kBlk + 1;  // padded row of the staging buffer
   extern __shared__ float sm[];
-  float* Us = sm;                                    // [128][129]: Us[j][k] = U[j0+j][j0+k]
-  float* err_s = Us + kBlk * (kBlk + 1);             // [32][128]
-  float* scl_s = err_s + kRowsPerCta * kBlk;         // [32][4]
-  int8_t* code_s = reinterpret_cast<int8_t*>(scl_s + kRowsPerCta * 4);  // [32][128]
+  float* Ur = sm;                                  // [128 j][4 lanes][32 slots], see below
+  float* stage = Ur + kBlk * kBlk;                 // [32][129]: weights in, errors out
+  float* scl_s = stage + kRowsPerCta * LD;         // [32][4]
+  float* inv_diag = scl_s + kRowsPerCta * 4;       // [128]: 1 / U[j][j]
+  int8_t* code_s = reinterpret_cast<int8_t*>(inv_diag + kBlk);  // [32][128]
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, l = lane & 3, rg = lane >> 2;
-  const int rl = warp * 8 + rg;  // row within the CTA
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + rl;
+  const int warp = tid >> 5, lane = tid & 31, l = lane & 3;
+  const int rl = warp * 8 + (lane >> 2);  // row within the CTA
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  const int64_t row = r0 + rl;
   const bool valid = row < a.N;
   const int64_t K = a.K;
 
-  for (int e = tid; e < kBlk * kBlk; e += blockDim.x) {
-    const int k = e / kBlk, j = e % kBlk;
-    Us[j * (kBlk + 1) + k] = (k >= j) ? a.Ut[(j0 + k) * K + j0 + j] : 0.f;
+  // Ur[j][l][m] = U[j0 + j][j0 + 4 * (j / 4 + m) + l], zero past the block: the U values lane
+  // l needs at column j, relative to the round of j.
+  for (int e = tid; e < kBlk * kBlk; e += kSweepThreads) {
+    const int j = e >> 7, rem = e & 127, ll = rem >> 5, m = rem & 31;
+    const int col = 4 * ((j >> 2) + m) + ll;
+    Ur[e] = col < kBlk ? a.U[(j0 + j) * K + j0 + col] : 0.f;
   }
+  // weights: coalesced 512-byte rows into the staging buffer
+  for (int r = warp; r < kRowsPerCta; r += 4) {
+    const float4 v = (r0 + r < a.N) ? reinterpret_cast<const float4*>(a.Wf + (r0 + r) * K + j0)[lane]
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    float* d = stage + r * LD + 4 * lane;
+    d[0] = v.x;
+    d[1] = v.y;
+    d[2] = v.z;
+    d[3] = v.w;
+  }
+  __syncthreads();
+  for (int j = tid; j < kBlk; j += kSweepThreads) inv_diag[j] = __frcp_rn(a.U[(j0 + j) * K + j0 + j]);
   float w[32];
-  const float* wrow = a.Wf + row * K + j0;
 #pragma unroll
-  for (int m = 0; m < 32; ++m) w[m] = valid ? wrow[4 * m + l] : 0.f;
+  for (int m = 0; m < 32; ++m) w[m] = stage[rl * LD + 4 * m + l];
 
-  float s = 0.f;
+  float s = 0.f, rs = 0.f;
   if (GS == 0) {
     const int G = a.group;
     const int64_t g = j0 / G;
@@ -92,67 +124,84 @@ __global__ void __launch_bounds__(128) sweep_block_kernel(SweepArgs a, int j0) {
     } else {
       s = valid ? a.scales[row * (K / G) + g] : 0.f;
     }
+    rs = __frcp_rn(s);
     if (l == 0) scl_s[rl * 4] = s;
   }
   __syncthreads();
 
+  float* err_row = stage + rl * LD;
+  int8_t* code_row = code_s + rl * kBlk;
+  const int src_base = lane & ~3;
+#pragma unroll 1
+  for (int R = 0; R < kBlk / 4; ++R) {
 #pragma unroll
-  for (int j = 0; j < kBlk; ++j) {
-    if (GS != 0 && (j % (GS == 0 ? 1 : GS)) == 0) {
-      float am = 0.f;
+    for (int jr = 0; jr < 4; ++jr) {
+      const int j = 4 * R + jr;
+      if (GS != 0 && jr == 0 && (R % ((GS == 0 ? 4 : GS) / 4)) == 0) {
+        float am = 0.f;
 #pragma unroll
-      for (int m = j / 4; m < (j + GS) / 4; ++m) am = fmaxf(am, fabsf(w[m]));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      s = __fdiv_rn(am, 7.f);
-      if (l == 0) scl_s[rl * 4 + j / (GS == 0 ? 1 : GS)] = s;
+        for (int m = 0; m < (GS == 0 ? 4 : GS) / 4; ++m) am = fmaxf(am, fabsf(w[m]));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        s = __fdiv_rn(am, 7.f);
+        rs = __frcp_rn(s);
+        if (l == 0) scl_s[rl * 4 + j / (GS == 0 ? 4 : GS)] = s;
+      }
+      const float wj = __shfl_sync(0xffffffffu, w[0], src_base | jr);
+      const float c = quant_code(wj, s, rs);
+      const float d = fmaf(-c, s, wj);
+      const float e = d * inv_diag[j];
+      if (l == jr) {
+        err_row[j] = e;
+        code_row[j] = static_cast<int8_t>(c);
+      }
+      const float4* u4 = reinterpret_cast<const float4*>(Ur + (j * 4 + l) * 32);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 u = u4[q];
+        if (q > 0 || l > jr) w[4 * q] = fmaf(-e, u.x, w[4 * q]);
+        w[4 * q + 1] = fmaf(-e, u.y, w[4 * q + 1]);
+        w[4 * q + 2] = fmaf(-e, u.z, w[4 * q + 2]);
+        w[4 * q + 3] = fmaf(-e, u.w, w[4 * q + 3]);
+      }
     }
-    const float wj = __shfl_sync(0xffffffffu, w[j / 4], (lane & ~3) | (j & 3));
-    const float c = quant_code(wj, s);
-    const float d = fmaf(-c, s, wj);
-    const float e = __fdiv_rn(d, Us[j * (kBlk + 1) + j]);
-    if (l == (j & 3)) {
-      err_s[rl * kBlk + j] = e;
-      code_s[rl * kBlk + j] = static_cast<int8_t>(c);
-    }
-    const float* urow = Us + j * (kBlk + 1);
 #pragma unroll
-    for (int m = j / 4; m < 32; ++m) w[m] = fmaf(-e, urow[4 * m + l], w[m]);
+    for (int m = 0; m < 31; ++m) w[m] = w[m + 1];
+    w[31] = 0.f;
   }
   __syncthreads();
 
-  // errors -> Err [N, 128], codes -> packed bytes, scales, qerr partials
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
-  for (int e = tid; e < kRowsPerCta * kBlk; e += blockDim.x) {
-    const int r = e / kBlk, k = e % kBlk;
-    if (r0 + r < a.N) a.Err[(r0 + r) * kBlk + k] = err_s[r * kBlk + k];
-  }
-  for (int e = tid; e < kRowsPerCta * (kBlk / 2); e += blockDim.x) {
-    const int r = e / (kBlk / 2), p = e % (kBlk / 2);
-    if (r0 + r < a.N) {
-      const int lo = code_s[r * kBlk + 2 * p] & 0xF, hi = code_s[r * kBlk + 2 * p + 1] & 0xF;
-      a.codes[(r0 + r) * (K / 2) + j0 / 2 + p] = static_cast<uint8_t>(lo | (hi << 4));
-    }
+  // errors -> panel buffer (coalesced rows), codes -> packed bytes, scales, qerr partials
+  for (int r = warp; r < kRowsPerCta; r += 4) {
+    if (r0 + r >= a.N) break;
+    const float* src = stage + r * LD + 4 * lane;
+    reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = make_float4(src[0], src[1], src[2], src[3]);
+    // lane writes bytes 2*lane, 2*lane+1 of the row's 64 code bytes
+    const int8_t* cs = code_s + r * kBlk + 4 * lane;
+    const uint32_t b0 = (cs[0] & 0xF) | ((cs[1] & 0xF) << 4);
+    const uint32_t b1 = (cs[2] & 0xF) | ((cs[3] & 0xF) << 4);
+    reinterpret_cast<uint16_t*>(a.codes + (r0 + r) * (K / 2) + j0 / 2)[lane] = static_cast<uint16_t>(b0 | (b1 << 8));
   }
   if (GS != 0) {
     constexpr int ng = (GS == 0) ? 1 : kBlk / GS;
-    for (int e = tid; e < kRowsPerCta * ng; e += blockDim.x) {
-      const int r = e / ng, g = e % ng;
-      if (r0 + r < a.N) a.scales[(r0 + r) * (K / (GS == 0 ? 1 : GS)) + j0 / (GS == 0 ? 1 : GS) + g] = scl_s[r * 4 + g];
-    }
+    if (valid && l == 0)
+#pragma unroll
+      for (int g = 0; g < ng; ++g) a.scales[row * (K / (GS == 0 ? 1 : GS)) + j0 / (GS == 0 ? 1 : GS) + g] = scl_s[rl * 4 + g];
   }
   double num = 0.0, den = 0.0;
-  for (int e = tid; e < kRowsPerCta * kBlk; e += blockDim.x) {
-    const int r = e / kBlk, k = e % kBlk;
-    if (r0 + r >= a.N) continue;
-    const double wo = static_cast<double>(load_w(a.W, a.w_dtype, (r0 + r) * K + j0 + k));
-    const double sc = static_cast<double>(GS != 0 ? scl_s[r * 4 + k / (GS == 0 ? 1 : GS)] : scl_s[r * 4]);
-    const double q = static_cast<double>(code_s[r * kBlk + k]) * sc;
-    const double im = a.imp != nullptr ? static_cast<double>(a.imp[j0 + k]) : 1.0;
-    num += im * (wo - q) * (wo - q);
-    den += im * wo * wo;
+  for (int r = warp; r < kRowsPerCta; r += 4) {
+    if (r0 + r >= a.N) break;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int k = 4 * lane + i;
+      const double wo = static_cast<double>(load_w(a.W, a.w_dtype, (r0 + r) * K + j0 + k));
+      const double sc = static_cast<double>(GS != 0 ? scl_s[r * 4 + k / (GS == 0 ? 1 : GS)] : scl_s[r * 4]);
+      const double q = static_cast<double>(code_s[r * kBlk + k]) * sc;
+      const double im = a.imp != nullptr ? static_cast<double>(a.imp[j0 + k]) : 1.0;
+      num += im * (wo - q) * (wo - q);
+      den += im * wo * wo;
+    }
   }
-  // deterministic CTA reduction: warp shuffles, then the four warp sums in order
   for (int off = 16; off > 0; off >>= 1) {
     num += __shfl_down_sync(0xffffffffu, num, off);
     den += __shfl_down_sync(0xffffffffu, den, off);
@@ -170,8 +219,8 @@ __global__ void __launch_bounds__(128) sweep_block_kernel(SweepArgs a, int j0) {
   }
 }
 
-constexpr size_t kSweepSmem = (kBlk * (kBlk + 1) + kRowsPerCta * kBlk + kRowsPerCta * 4) * sizeof(float) +
-                              kRowsPerCta * kBlk;
+constexpr size_t kSweepSmem =
+    (kBlk * kBlk + kRowsPerCta * (kBlk + 1) + kRowsPerCta * 4 + kBlk) * sizeof(float) + kRowsPerCta * kBlk;
 
 __global__ void w_prep_kernel(const void* __restrict__ W, int dt, int64_t n, float* __restrict__ Wf) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
@@ -222,10 +271,19 @@ bool gptq_shape_ok(int64_t N, int64_t K, int64_t group) {
   return true;
 }
 
-GptqLayout gptq_layout(int64_t N, int64_t K, int64_t /*group*/) {
+// Panel width of the two-level update: 512 columns, or a multiple of a group wider than a
+// block so that every group lies inside one panel.
+static int64_t panel_width(int64_t K, int64_t group) {
+  const int64_t base = group > kBlk ? group : kBlk;
+  int64_t P = base * ((512 / base) > 1 ? (512 / base) : 1);
+  return P < K ? P : K;
+}
+
+GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   GptqLayout L{};
   const size_t al = 256;
   L.sweep_grid = static_cast<int>(ceil_div(N, kRowsPerCta));
+  const int64_t P = panel_width(K, group);
   size_t off = 0;
   L.header = off;
   off = round_up(off + sizeof(WsHeader), al);
@@ -234,21 +292,23 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t /*group*/) {
   L.wf = off;
   off = round_up(off + static_cast<size_t>(N) * K * sizeof(float), al);
   L.err = off;
-  off = round_up(off + static_cast<size_t>(N) * kBlk * sizeof(float), al);
+  off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
   L.a = off;
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
   L.x = off;
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  L.xt = off;
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
   L.t = off;
-  off = round_up(off + static_cast<size_t>(K / 2) * (K - K / 2 + 64) * sizeof(float), al);
-  L.dinv = off;
-  off = round_up(off + static_cast<size_t>(K) * 64 * sizeof(float), al);
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
   L.total = off;
   return L;
 }
 
-static hq_status launch_update_simt(float* Wf, int64_t N, int64_t K, int j0, const float* Err, const float* Ut,
-                                    const int* info, cudaStream_t s);
+// W[:, c0 : c0+ncols] -= E[:, 0:kred] * U[k0 : k0+kred, c0 : c0+ncols]   (E row stride lde)
+static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
+                              int64_t lde, int64_t k0, int64_t kred, const float* Ut, const int* info, int* status,
+                              cudaStream_t s);
 
 hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
                       const float* imp, uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws,
@@ -260,13 +320,14 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   float* Err = reinterpret_cast<float*>(ws + L.err);
   float* A = reinterpret_cast<float*>(ws + L.a);
   float* X = reinterpret_cast<float*>(ws + L.x);
+  float* XT = reinterpret_cast<float*>(ws + L.xt);
   float* T = reinterpret_cast<float*>(ws + L.t);
-  float* Dinv = reinterpret_cast<float*>(ws + L.dinv);
   HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
 
-  hq_status st = launch_factor(H, K, damp, A, X, T, Dinv, &hdr->lam, &hdr->info, /*Ut=*/A, s);
+  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, /*Ut=*/A, /*U=*/T, s);
   if (st != HQ_OK) return st;
   const float* Ut = A;
+  const float* U = T;
 
   {
     const int64_t n = N * K;
@@ -275,13 +336,15 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
     HQ_LAUNCH_CHECK();
   }
 
+  const int64_t P = panel_width(K, group);
   SweepArgs a{};
   a.Wf = Wf;
   a.N = N;
   a.K = K;
-  a.Ut = Ut;
+  a.U = U;
   a.group = static_cast<int>(group);
   a.Err = Err;
+  a.err_ld = P;
   a.codes = codes;
   a.scales = scales;
   a.W = W;
@@ -299,55 +362,33 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   }
   HQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSweepSmem)));
 
-  CUtensorMap mapE, mapU;
-  if (update_impl == 0) {
-    if (!make_tmap_2d(&mapE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Err, kBlk, static_cast<uint64_t>(N), kBlk * 4, 32, 128))
-      return HQ_ERR_CUDA;
-    if (!make_tmap_2d(&mapU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ut, static_cast<uint64_t>(K), static_cast<uint64_t>(K),
-                      static_cast<uint64_t>(K) * 4, 32, 256))
-      return HQ_ERR_CUDA;
-    HQ_CUDA_TRY(cudaFuncSetAttribute(umma_gemm_kernel<GemmMode::kUpdateTF32>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes));
-  }
-
-  const int nblk = static_cast<int>(K / kBlk);
-  for (int b = 0; b < nblk; ++b) {
-    const int j0 = b * kBlk;
-    kern<<<L.sweep_grid, 128, kSweepSmem, s>>>(a, j0);
-    HQ_LAUNCH_CHECK();
-    const int64_t ncols = K - j0 - kBlk;
-    if (ncols <= 0) continue;
-    if (update_impl == 0) {
-      GemmArgs g{};
-      g.C = Wf;
-      g.ldc = K;
-      g.M = static_cast<int>(N);
-      g.Ncols = static_cast<int>(ncols);
-      g.Kred = kBlk;
-      g.col0 = j0 + kBlk;
-      g.b_x0 = j0;
-      g.b_y0 = j0 + kBlk;
-      g.tiles_n = static_cast<int>(ceil_div(ncols, kGemmBN));
-      g.skip = &hdr->info;
-      g.status = &hdr->status;
-      const int64_t ctas = ceil_div(N, kGemmBM) * g.tiles_n;
-      umma_gemm_kernel<GemmMode::kUpdateTF32><<<static_cast<unsigned>(ctas), gemm_threads(GemmMode::kUpdateTF32), kGemmSmemBytes, s>>>(
-          mapE, mapU, g);
+  for (int64_t p0 = 0; p0 < K; p0 += P) {
+    const int64_t p1 = (p0 + P < K) ? p0 + P : K;
+    for (int64_t j0 = p0; j0 < p1; j0 += kBlk) {
+      a.err_col = static_cast<int>(j0 - p0);
+      kern<<<L.sweep_grid, kSweepThreads, kSweepSmem, s>>>(a, static_cast<int>(j0));
       HQ_LAUNCH_CHECK();
-    } else {
-      st = launch_update_simt(Wf, N, K, j0, Err, Ut, &hdr->info, s);
+      const int64_t j1 = j0 + kBlk;
+      if (j1 < p1) {  // inner update of the rest of the panel
+        st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), P, j0, kBlk, Ut, &hdr->info,
+                          &hdr->status, s);
+        if (st != HQ_OK) return st;
+      }
+    }
+    if (p1 < K) {  // outer update of everything right of the panel
+      st = sweep_update(update_impl, Wf, N, K, p1, K - p1, Err, P, p0, p1 - p0, Ut, &hdr->info, &hdr->status, s);
       if (st != HQ_OK) return st;
     }
   }
-  return launch_qerr_finalize(partials, static_cast<int64_t>(nblk) * L.sweep_grid, hdr, qerr_dev, s);
+  return launch_qerr_finalize(partials, static_cast<int64_t>(K / kBlk) * L.sweep_grid, hdr, qerr_dev, s);
 }
 
-// CUDA-core fp32 version of the trailing update (cross-check of the tensor-core kernel).
-__global__ void __launch_bounds__(256) update_simt_kernel(float* __restrict__ Wf, int64_t N, int64_t K, int j0,
-                                                          const float* __restrict__ Err,
-                                                          const float* __restrict__ Ut, const int* __restrict__ info) {
+// CUDA-core fp32 version of the lazy update (cross-check of the tensor-core kernel).
+__global__ void __launch_bounds__(256) update_simt_kernel(float* __restrict__ C, int64_t ldc, int64_t M,
+                                                          int64_t ncols, const float* __restrict__ E, int64_t lde,
+                                                          const float* __restrict__ B, int64_t ldb, int64_t kred,
+                                                          const int* __restrict__ info) {
   if (*info != 0) return;
-  const int64_t ncols = K - j0 - kBlk;
   const int64_t tiles_n = (ncols + 63) / 64;
   const int64_t tm = blockIdx.x / tiles_n, tn = blockIdx.x % tiles_n;
   const int64_t m0 = tm * 64, n0 = tn * 64;
@@ -355,11 +396,12 @@ __global__ void __launch_bounds__(256) update_simt_kernel(float* __restrict__ Wf
   __shared__ float Bs[16][64];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   float acc[4][4] = {};
-  for (int k0 = 0; k0 < kBlk; k0 += 16) {
+  for (int64_t k0 = 0; k0 < kred; k0 += 16) {
     for (int e = threadIdx.x; e < 16 * 64; e += 256) {
       const int kk = e % 16, c = e / 16;
-      As[kk][c] = (m0 + c < N) ? Err[(m0 + c) * kBlk + k0 + kk] : 0.f;
-      Bs[kk][c] = (n0 + c < ncols) ? Ut[(j0 + kBlk + n0 + c) * K + j0 + k0 + kk] : 0.f;
+      const bool kin = k0 + kk < kred;
+      As[kk][c] = (kin && m0 + c < M) ? E[(m0 + c) * lde + k0 + kk] : 0.f;
+      Bs[kk][c] = (kin && n0 + c < ncols) ? B[(n0 + c) * ldb + k0 + kk] : 0.f;
     }
     __syncthreads();
 #pragma unroll
@@ -373,22 +415,41 @@ __global__ void __launch_bounds__(256) update_simt_kernel(float* __restrict__ Wf
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int64_t m = m0 + ty + 16 * u;
-    if (m >= N) continue;
+    if (m >= M) continue;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int64_t n = n0 + tx + 16 * v;
-      if (n < ncols) Wf[m * K + j0 + kBlk + n] -= acc[u][v];
+      if (n < ncols) C[m * ldc + n] -= acc[u][v];
     }
   }
 }
 
-static hq_status launch_update_simt(float* Wf, int64_t N, int64_t K, int j0, const float* Err, const float* Ut,
-                                    const int* info, cudaStream_t s) {
-  const int64_t ncols = K - j0 - kBlk;
-  const int64_t ctas = ceil_div(N, 64) * ceil_div(ncols, 64);
-  update_simt_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(Wf, N, K, j0, Err, Ut, info);
-  HQ_LAUNCH_CHECK();
-  return HQ_OK;
+static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
+                              int64_t lde, int64_t k0, int64_t kred, const float* Ut, const int* info, int* status,
+                              cudaStream_t s) {
+  const float* B = Ut + c0 * K + k0;  // B(n, k) = U^T[c0 + n][k0 + k] = U[k0 + k][c0 + n]
+  if (impl == 1) {
+    const int64_t ctas = ceil_div(N, 64) * ceil_div(ncols, 64);
+    update_simt_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(Wf + c0, K, N, ncols, E, lde, B, K, kred, info);
+    HQ_LAUNCH_CHECK();
+    return HQ_OK;
+  }
+  Tf32Gemm g{};
+  g.C = Wf + c0;
+  g.ldc = K;
+  g.M = static_cast<int>(N);
+  g.N = static_cast<int>(ncols);
+  g.Kred = static_cast<int>(kred);
+  g.A = E;
+  g.lda = lde;
+  g.B = B;
+  g.ldb = K;
+  g.alpha = -1.f;
+  g.beta = 1.f;
+  g.split3 = (impl == 0);
+  g.skip = info;
+  g.status = status;
+  return tf32_gemm(g, s);
 }
 
 }  // namespace hq

@@ -17,14 +17,31 @@ hq_status launch_syrk_simt(float* H, const void* X, int x_dtype, int64_t T, int6
 hq_status launch_tril_encode(const float* H, int64_t K, uint8_t* out, cudaStream_t s);
 hq_status launch_tril_decode(const uint8_t* in, int64_t K, float* H, cudaStream_t s);
 
-// factor.cu
-size_t factor_workspace_floats(int64_t K);
-hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* X, float* T, float* Dinv,
-                        double* lam, int* info, float* Ut, cudaStream_t s);
+// gemm_tf32.cu: C = beta C + alpha A B^T on the tensor cores (kind::tf32)
+struct Tf32Gemm {
+  float* C;
+  int64_t ldc;
+  int M, N, Kred;
+  const float* A;  // A(m, k) = A[m * lda + k]
+  int64_t lda;
+  const float* B;  // B(n, k) = B[n * ldb + k]
+  int64_t ldb;
+  float alpha, beta;
+  int lower, row0, col0;  // write only row0 + m >= col0 + n when lower
+  bool split3;            // 3xTF32 (about fp32 accuracy) instead of 1xTF32
+  const int* skip;
+  int* status;
+};
+hq_status tf32_gemm(const Tf32Gemm& g, cudaStream_t s);
 
-// sweep.cu
+// factor.cu: U (row-major, upper) and U^T (row-major, lower) of the damped Hessian; A, X, XT
+// and T are K x K fp32 scratch (U^T may alias A, U may alias T).
+hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* X, float* XT, float* T, double* lam,
+                        int* info, int* status, float* Ut, float* U, cudaStream_t s);
+
+// gptq.cu
 struct GptqLayout {
-  size_t header, partials, wf, err, a, x, t, dinv, total;
+  size_t header, partials, wf, err, a, x, xt, t, total;
   int sweep_grid;
 };
 // Device-side header at the start of the GPTQ / RTN workspace.

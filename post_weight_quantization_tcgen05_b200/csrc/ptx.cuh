@@ -142,6 +142,39 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 32 consecutive 32-bit columns without waiting; pair with tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Adds 128 consecutive TMEM columns of this thread's lane into acc[0..127]: four x32 loads in
+// flight, one wait.
+__device__ __forceinline__ void tmem_add128(uint32_t taddr, float (&acc)[128]) {
+  uint32_t r0[32], r1[32], r2[32], r3[32];
+  tmem_ld32_nowait(taddr, r0);
+  tmem_ld32_nowait(taddr + 32, r1);
+  tmem_ld32_nowait(taddr + 64, r2);
+  tmem_ld32_nowait(taddr + 96, r3);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    acc[i] += __uint_as_float(r0[i]);
+    acc[32 + i] += __uint_as_float(r1[i]);
+    acc[64 + i] += __uint_as_float(r2[i]);
+    acc[96 + i] += __uint_as_float(r3[i]);
+  }
+}
+
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading- and stride-
 // dimension byte offsets (all >> 4), version 1 at bit 46, 128-byte swizzle (2) at bit 61.
 // Tiles are 1024-byte aligned so the base-offset field stays 0.

@@ -113,7 +113,7 @@ def _spd(K, seed, corr=0.7):
     return (H * np.outer(d, d)).astype(np.float32)
 
 
-@pytest.mark.parametrize("K", [128, 256, 640])
+@pytest.mark.parametrize("K", [128, 256, 640, 1152])
 def test_factor_upper_cholesky_of_inverse(hq, cuda_device, K):
     H = _spd(K, K)
     Hd = torch.from_numpy(H).cuda()
@@ -184,7 +184,7 @@ def test_gptq_tiny_layer_pipeline(hq, cuda_device):
     _compare_gptq(W, H64, cfg.group, codes, scales, q, what="tiny")
 
 
-@pytest.mark.parametrize("impl", [0, 1])
+@pytest.mark.parametrize("impl", [0, 1, 2])
 @pytest.mark.parametrize("N,K,group,wdt", [(64, 128, 32, "f32"), (33, 256, 64, "f32"), (1, 384, 128, "bf16"),
                                             (200, 512, 256, "bf16"), (130, 640, 128, "f32")])
 def test_gptq_stage_correlated(hq, cuda_device, N, K, group, wdt, impl):
@@ -313,3 +313,31 @@ def test_rtn_bit_exact(hq, cuda_device, N, K, G):
     assert np.array_equal(scales.cpu().numpy(), sr)
     qr = oracle.qerr(Wn, cr, sr, G)
     assert abs(q - qr) <= 1e-12 * max(qr, 1e-300) + 1e-15
+
+
+# ----------------------------------------------------------------------------- tf32 GEMM
+
+@pytest.mark.parametrize("split3", [True, False])
+@pytest.mark.parametrize("M,N,Kred,lower", [(128, 128, 32, False), (300, 200, 100, False), (5120, 384, 128, False),
+                                             (640, 640, 512, True), (1, 7, 4, False)])
+def test_tf32_gemm_against_fp64(hq, cuda_device, M, N, Kred, lower, split3):
+    g = _gen(M * 7 + N)
+    kp = (Kred + 3) // 4 * 4
+    A = torch.zeros((M, kp), device="cuda")
+    B = torch.zeros((N, kp), device="cuda")
+    A[:, :Kred] = torch.randn((M, Kred), generator=g, device="cuda")
+    B[:, :Kred] = torch.randn((N, Kred), generator=g, device="cuda")
+    C0 = torch.randn((M, N), generator=g, device="cuda")
+    C = C0.clone()
+    hq.lib.hq_debug_tf32_gemm(C.data_ptr(), N, M, N, Kred, A.data_ptr(), kp, B.data_ptr(), kp, -1.0, 1.0,
+                              int(lower), int(split3), None)
+    torch.cuda.synchronize()
+    ref = C0.double() - A[:, :Kred].double() @ B[:, :Kred].double().T
+    got = C.double()
+    if lower:
+        mask = torch.ones((M, N), dtype=torch.bool, device="cuda").tril()
+        assert torch.equal(got[~mask], C0.double()[~mask])
+        got, ref = got[mask], ref[mask]
+    err = ((got - ref).norm() / ref.norm()).item()
+    # 3xTF32: about 2^-21 per product; plain tf32 (mantissa truncated to 10 bits): about 2^-10
+    assert err < (2e-6 if split3 else 2e-3), err
