@@ -227,20 +227,52 @@ __global__ void __launch_bounds__(Tf32Cfg<SPLIT3>::kThreads, 1)
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (ok) {
-      // warp q writes rows q, q+4, ...: lane = 16-byte chunk, coalesced 512-byte rows
-      for (int rr = q; rr < Cfg::BM; rr += 4) {
-        const int m = m0 + rr;
-        if (m >= args.M) break;
-        const float4 v = tile[rr * 32 + (lane ^ (rr & 7))];
-        float* crow = args.C + static_cast<int64_t>(m) * args.ldc;
-        const float vv[4] = {v.x, v.y, v.z, v.w};
+      // warp q writes rows q, q+4, ...: lane = 16-byte chunk of a coalesced 512-byte row.
+      // Eight rows per batch so that the loads of C are all in flight before any store.
+      const bool full_tile = (m0 + Cfg::BM <= args.M) && (n0 + Cfg::BN <= args.N) && !args.lower &&
+                             ((reinterpret_cast<uintptr_t>(args.C) & 15) == 0) && (args.ldc % 4 == 0);
+      const int n = n0 + 4 * lane;
+      for (int rb = 0; rb < Cfg::BM / 4; rb += 8) {
+        float4 old[8];
+        if (args.beta != 0.f) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int n = n0 + 4 * lane + i;
-          if (n >= args.N) continue;
-          if (args.lower && args.row0 + m < args.col0 + n) continue;
-          const float old = (args.beta != 0.f) ? crow[n] : 0.f;
-          crow[n] = args.beta * old + args.alpha * vv[i];
+          for (int u = 0; u < 8; ++u) {
+            const int m = m0 + q + 4 * (rb + u);
+            old[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (full_tile) {
+              old[u] = *reinterpret_cast<const float4*>(args.C + static_cast<int64_t>(m) * args.ldc + n);
+            } else if (m < args.M) {
+              const float* cr = args.C + static_cast<int64_t>(m) * args.ldc;
+              if (n + 0 < args.N) old[u].x = cr[n + 0];
+              if (n + 1 < args.N) old[u].y = cr[n + 1];
+              if (n + 2 < args.N) old[u].z = cr[n + 2];
+              if (n + 3 < args.N) old[u].w = cr[n + 3];
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int rr = q + 4 * (rb + u);
+          const int m = m0 + rr;
+          const float4 v = tile[rr * 32 + (lane ^ (rr & 7))];
+          float4 o;
+          if (args.beta != 0.f) {
+            o.x = fmaf(args.alpha, v.x, args.beta * old[u].x);
+            o.y = fmaf(args.alpha, v.y, args.beta * old[u].y);
+            o.z = fmaf(args.alpha, v.z, args.beta * old[u].z);
+            o.w = fmaf(args.alpha, v.w, args.beta * old[u].w);
+          } else {
+            o = make_float4(args.alpha * v.x, args.alpha * v.y, args.alpha * v.z, args.alpha * v.w);
+          }
+          if (full_tile) {
+            *reinterpret_cast<float4*>(args.C + static_cast<int64_t>(m) * args.ldc + n) = o;
+          } else if (m < args.M) {
+            float* cr = args.C + static_cast<int64_t>(m) * args.ldc;
+            const float ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (n + i < args.N && !(args.lower && args.row0 + m < args.col0 + n + i)) cr[n + i] = ov[i];
+          }
         }
       }
     }

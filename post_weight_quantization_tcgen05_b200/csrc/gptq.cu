@@ -4,15 +4,16 @@
 //
 // The sweep walks K in 128-column blocks grouped into panels of P columns (P = 512, or a
 // multiple of the group size when groups are wider than a block).  Per block:
-//   * sweep_block_kernel: the sequential part.  Four lanes share a row; lane l holds the
-//     row's columns l, l+4, l+8, ... as 32 "slots" in registers.  The columns are visited in
-//     rounds of four: at the end of a round every lane shifts its slots down by one, so the
-//     column being quantised is always slot 0 of lane (j mod 4), a compile-time lane inside the
-//     4-way unrolled round, and the loop body stays small enough for the instruction cache.
-//     Per column j: group scale at a group start (4-lane absmax), broadcast of w_j, code
-//     c = clamp(rint(w_j / s), -8, 7), error e = (w_j - c s) / U[j, j], and the feedback
-//     w_k -= e U[j, k] for k > j, with U's row j pre-permuted in shared memory so that each
-//     lane reads its 32 values with eight aligned 16-byte loads.  It writes the block's
+//   * sweep_block_kernel: the sequential part.  A group of eight lanes carries two rows;
+//     lane l holds columns l, l+8, l+16, ... of both rows as 16 "slots" each, in registers.
+//     The columns are visited in rounds of eight: at the end of a round every lane shifts its
+//     slots down by one, so the column being quantised is always slot 0 of lane (j mod 8), a
+//     compile-time lane inside the 8-way unrolled round, and the loop body stays small enough
+//     for the instruction cache.  Per column j and row: group scale at a group start (8-lane
+//     absmax), broadcast of w_j, code c = clamp(rint(w_j / s), -8, 7), error
+//     e = (w_j - c s) / U[j, j], and the feedback w_k -= e U[j, k] for k > j.  U's row j is
+//     pre-permuted (and XOR-swizzled against bank conflicts) in shared memory so that each
+//     lane reads its 16 values with four 16-byte loads, used for both of its rows.  It writes the block's
 //     errors into the panel's error buffer, the packed int4 codes, the scales and fp64 partial
 //     sums of the qerr numerator and denominator over the ORIGINAL weights.
 //   * inner lazy update of the rest of the panel, W[:, b+128 : panel end] -= Err_b U[b, ...]
@@ -30,7 +31,9 @@
 namespace hq {
 
 constexpr int kBlk = 128;        // sweep block width
-constexpr int kRowsPerCta = 32;  // 4 warps x 8 rows, 4 lanes per row
+constexpr int kLanesPerRow = 8;
+constexpr int kSlots = kBlk / kLanesPerRow;  // 16 columns per lane
+constexpr int kRowsPerCta = 32;              // 4 warps x 4 lane groups x 2 rows
 constexpr int kSweepThreads = 128;
 
 struct SweepArgs {
@@ -56,45 +59,59 @@ __device__ __forceinline__ float load_w(const void* W, int dt, int64_t idx) {
 
 // c = clamp(rint(w / s), -8, 7) with w / s the IEEE fp32 quotient.  w * (1/s) is within a
 // couple of ulps of the quotient, so it rounds the same way unless it lies within 1e-5 of a
-// half-integer; only then is the exact division taken.
+// half-integer; only then is the exact division taken.  Rounding to nearest-even uses the
+// 1.5 * 2^23 shift (exact for |q| < 2^22; larger values are clamped anyway).
 __device__ __forceinline__ float quant_code(float w, float s, float rs) {
   if (!(s > 0.f)) return 0.f;
+  constexpr float kShift = 12582912.f;
   float q = w * rs;
-  const float a = fabsf(q);
-  if (fabsf(a - floorf(a) - 0.5f) < 1e-5f) q = __fdiv_rn(w, s);
-  return fminf(fmaxf(rintf(q), -8.f), 7.f);
+  float r = (q + kShift) - kShift;
+  if (fabsf(q - r) > 0.5f - 1e-5f) r = rintf(__fdiv_rn(w, s));
+  return fminf(fmaxf(r, -8.f), 7.f);
 }
 
 // GS: group size when it is 32, 64 or 128 (scales computed inside the block), or 0 when the
 // group spans several blocks (scale computed at the group's first block from Wf).
+// Offset (in floats) of chunk q (4 floats) of lane l's 16 U values for column j.  The XOR
+// keeps the eight lanes of a quarter-warp on eight different 16-byte bank groups.
+__device__ __forceinline__ int ur_off(int j, int l, int q) { return (j * kLanesPerRow + l) * kSlots + 4 * (q ^ (l >> 1)); }
+
 template <int GS>
 __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a, int j0) {
   if (*a.info != 0) return;
   constexpr int LD = kBlk + 1;  // padded row of the staging buffer
+  constexpr int kGS = (GS == 0 ? kLanesPerRow : GS) / kLanesPerRow;  // slots per group
   extern __shared__ float sm[];
-  float* Ur = sm;                                  // [128 j][4 lanes][32 slots], see below
+  float* Ur = sm;                                  // [128 j][8 lanes][16 slots], swizzled
   float* stage = Ur + kBlk * kBlk;                 // [32][129]: weights in, errors out
   float* scl_s = stage + kRowsPerCta * LD;         // [32][4]
   float* inv_diag = scl_s + kRowsPerCta * 4;       // [128]: 1 / U[j][j]
   int8_t* code_s = reinterpret_cast<int8_t*>(inv_diag + kBlk);  // [32][128]
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, l = lane & 3;
-  const int rl = warp * 8 + (lane >> 2);  // row within the CTA
+  const int warp = tid >> 5, lane = tid & 31, l = lane & (kLanesPerRow - 1);
+  const int rl0 = warp * (32 / kLanesPerRow) + lane / kLanesPerRow;  // rows rl0 and rl0 + 16
+  const int rl1 = rl0 + kRowsPerCta / 2;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
-  const int64_t row = r0 + rl;
-  const bool valid = row < a.N;
   const int64_t K = a.K;
 
-  // Ur[j][l][m] = U[j0 + j][j0 + 4 * (j / 4 + m) + l], zero past the block: the U values lane
-  // l needs at column j, relative to the round of j.
-  for (int e = tid; e < kBlk * kBlk; e += kSweepThreads) {
-    const int j = e >> 7, rem = e & 127, ll = rem >> 5, m = rem & 31;
-    const int col = 4 * ((j >> 2) + m) + ll;
-    Ur[e] = col < kBlk ? a.U[(j0 + j) * K + j0 + col] : 0.f;
+  // Ur: U[j0 + j][j0 + 8 * (j / 8 + m) + l] for slot m of lane l, zero past the block.
+  for (int e = tid; e < kBlk * kBlk; e += kSweepThreads) Ur[e] = 0.f;
+  __syncthreads();
+#pragma unroll 4
+  for (int e = tid; e < kBlk * (kBlk / 4); e += kSweepThreads) {
+    const int j = e >> 5, q4 = e & 31;  // row j, columns 4 q4 .. 4 q4 + 3
+    const float4 u = reinterpret_cast<const float4*>(a.U + (j0 + j) * K + j0)[q4];
+    const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int col = 4 * q4 + i;
+      const int m = col / kLanesPerRow - j / kLanesPerRow;
+      if (m >= 0) Ur[ur_off(j, col % kLanesPerRow, m >> 2) + (m & 3)] = uv[i];
+    }
   }
   // weights: coalesced 512-byte rows into the staging buffer
-  for (int r = warp; r < kRowsPerCta; r += 4) {
+  for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
     const float4 v = (r0 + r < a.N) ? reinterpret_cast<const float4*>(a.Wf + (r0 + r) * K + j0)[lane]
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
     float* d = stage + r * LD + 4 * lane;
@@ -105,74 +122,123 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
   }
   __syncthreads();
   for (int j = tid; j < kBlk; j += kSweepThreads) inv_diag[j] = __frcp_rn(a.U[(j0 + j) * K + j0 + j]);
-  float w[32];
+  float w0[kSlots], w1[kSlots];
 #pragma unroll
-  for (int m = 0; m < 32; ++m) w[m] = stage[rl * LD + 4 * m + l];
+  for (int m = 0; m < kSlots; ++m) {
+    w0[m] = stage[rl0 * LD + kLanesPerRow * m + l];
+    w1[m] = stage[rl1 * LD + kLanesPerRow * m + l];
+  }
 
-  float s = 0.f, rs = 0.f;
+  float s0 = 0.f, rs0 = 0.f, s1 = 0.f, rs1 = 0.f;
   if (GS == 0) {
+    // the group spans several blocks: its scale is taken at its first block from the current
+    // weights of all its columns, and read back in the later blocks
     const int G = a.group;
     const int64_t g = j0 / G;
-    if (j0 % G == 0) {
-      float am = 0.f;
-      if (valid)
-        for (int i = l; i < G; i += 4) am = fmaxf(am, fabsf(a.Wf[row * K + j0 + i]));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      s = __fdiv_rn(am, 7.f);
-      if (valid && l == 0) a.scales[row * (K / G) + g] = s;
-    } else {
-      s = valid ? a.scales[row * (K / G) + g] : 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int rl = h ? rl1 : rl0;
+      const int64_t row = r0 + rl;
+      const bool valid = row < a.N;
+      float sc;
+      if (j0 % G == 0) {
+        float am = 0.f;
+        if (valid)
+          for (int i = l; i < G; i += kLanesPerRow) am = fmaxf(am, fabsf(a.Wf[row * K + j0 + i]));
+#pragma unroll
+        for (int x = 1; x < kLanesPerRow; x <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, x));
+        sc = __fdiv_rn(am, 7.f);
+        if (valid && l == 0) a.scales[row * (K / G) + g] = sc;
+      } else {
+        sc = valid ? a.scales[row * (K / G) + g] : 0.f;
+      }
+      if (l == 0) scl_s[rl * 4] = sc;
+      if (h) {
+        s1 = sc;
+        rs1 = __frcp_rn(sc);
+      } else {
+        s0 = sc;
+        rs0 = __frcp_rn(sc);
+      }
     }
-    rs = __frcp_rn(s);
-    if (l == 0) scl_s[rl * 4] = s;
   }
   __syncthreads();
 
-  float* err_row = stage + rl * LD;
-  int8_t* code_row = code_s + rl * kBlk;
-  const int src_base = lane & ~3;
+  float* err0 = stage + rl0 * LD;
+  float* err1 = stage + rl1 * LD;
+  int8_t* code0 = code_s + rl0 * kBlk;
+  int8_t* code1 = code_s + rl1 * kBlk;
+  const int src_base = lane & ~(kLanesPerRow - 1);
 #pragma unroll 1
-  for (int R = 0; R < kBlk / 4; ++R) {
+  for (int R = 0; R < kSlots; ++R) {
 #pragma unroll
-    for (int jr = 0; jr < 4; ++jr) {
-      const int j = 4 * R + jr;
-      if (GS != 0 && jr == 0 && (R % ((GS == 0 ? 4 : GS) / 4)) == 0) {
-        float am = 0.f;
+    for (int jr = 0; jr < kLanesPerRow; ++jr) {
+      const int j = kLanesPerRow * R + jr;
+      if (GS != 0 && jr == 0 && (R % kGS) == 0) {
+        float am0 = 0.f, am1 = 0.f;
 #pragma unroll
-        for (int m = 0; m < (GS == 0 ? 4 : GS) / 4; ++m) am = fmaxf(am, fabsf(w[m]));
-        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-        s = __fdiv_rn(am, 7.f);
-        rs = __frcp_rn(s);
-        if (l == 0) scl_s[rl * 4 + j / (GS == 0 ? 4 : GS)] = s;
+        for (int m = 0; m < kGS; ++m) {
+          am0 = fmaxf(am0, fabsf(w0[m]));
+          am1 = fmaxf(am1, fabsf(w1[m]));
+        }
+#pragma unroll
+        for (int x = 1; x < kLanesPerRow; x <<= 1) {
+          am0 = fmaxf(am0, __shfl_xor_sync(0xffffffffu, am0, x));
+          am1 = fmaxf(am1, __shfl_xor_sync(0xffffffffu, am1, x));
+        }
+        s0 = __fdiv_rn(am0, 7.f);
+        s1 = __fdiv_rn(am1, 7.f);
+        rs0 = __frcp_rn(s0);
+        rs1 = __frcp_rn(s1);
+        if (l == 0) {
+          scl_s[rl0 * 4 + j / (GS == 0 ? 1 : GS)] = s0;
+          scl_s[rl1 * 4 + j / (GS == 0 ? 1 : GS)] = s1;
+        }
       }
-      const float wj = __shfl_sync(0xffffffffu, w[0], src_base | jr);
-      const float c = quant_code(wj, s, rs);
-      const float d = fmaf(-c, s, wj);
-      const float e = d * inv_diag[j];
+      float u[kSlots];
+#pragma unroll
+      for (int q = 0; q < kSlots / 4; ++q) {
+        const float4 t = *reinterpret_cast<const float4*>(Ur + ur_off(j, l, q));
+        u[4 * q] = t.x;
+        u[4 * q + 1] = t.y;
+        u[4 * q + 2] = t.z;
+        u[4 * q + 3] = t.w;
+      }
+      const float idg = inv_diag[j];
+      const float wj0 = __shfl_sync(0xffffffffu, w0[0], src_base | jr);
+      const float wj1 = __shfl_sync(0xffffffffu, w1[0], src_base | jr);
+      const float c0 = quant_code(wj0, s0, rs0);
+      const float c1 = quant_code(wj1, s1, rs1);
+      const float e0 = fmaf(-c0, s0, wj0) * idg;
+      const float e1 = fmaf(-c1, s1, wj1) * idg;
       if (l == jr) {
-        err_row[j] = e;
-        code_row[j] = static_cast<int8_t>(c);
+        err0[j] = e0;
+        err1[j] = e1;
+        code0[j] = static_cast<int8_t>(c0);
+        code1[j] = static_cast<int8_t>(c1);
       }
-      const float4* u4 = reinterpret_cast<const float4*>(Ur + (j * 4 + l) * 32);
+      if (l > jr) {
+        w0[0] = fmaf(-e0, u[0], w0[0]);
+        w1[0] = fmaf(-e1, u[0], w1[0]);
+      }
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 u = u4[q];
-        if (q > 0 || l > jr) w[4 * q] = fmaf(-e, u.x, w[4 * q]);
-        w[4 * q + 1] = fmaf(-e, u.y, w[4 * q + 1]);
-        w[4 * q + 2] = fmaf(-e, u.z, w[4 * q + 2]);
-        w[4 * q + 3] = fmaf(-e, u.w, w[4 * q + 3]);
+      for (int m = 1; m < kSlots; ++m) {
+        w0[m] = fmaf(-e0, u[m], w0[m]);
+        w1[m] = fmaf(-e1, u[m], w1[m]);
       }
     }
 #pragma unroll
-    for (int m = 0; m < 31; ++m) w[m] = w[m + 1];
-    w[31] = 0.f;
+    for (int m = 0; m < kSlots - 1; ++m) {
+      w0[m] = w0[m + 1];
+      w1[m] = w1[m + 1];
+    }
+    w0[kSlots - 1] = 0.f;
+    w1[kSlots - 1] = 0.f;
   }
   __syncthreads();
 
   // errors -> panel buffer (coalesced rows), codes -> packed bytes, scales, qerr partials
-  for (int r = warp; r < kRowsPerCta; r += 4) {
+  for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
     if (r0 + r >= a.N) break;
     const float* src = stage + r * LD + 4 * lane;
     reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = make_float4(src[0], src[1], src[2], src[3]);
@@ -184,12 +250,13 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
   }
   if (GS != 0) {
     constexpr int ng = (GS == 0) ? 1 : kBlk / GS;
-    if (valid && l == 0)
-#pragma unroll
-      for (int g = 0; g < ng; ++g) a.scales[row * (K / (GS == 0 ? 1 : GS)) + j0 / (GS == 0 ? 1 : GS) + g] = scl_s[rl * 4 + g];
+    for (int e = tid; e < kRowsPerCta * ng; e += kSweepThreads) {
+      const int r = e / ng, g = e % ng;
+      if (r0 + r < a.N) a.scales[(r0 + r) * (K / (GS == 0 ? 1 : GS)) + j0 / (GS == 0 ? 1 : GS) + g] = scl_s[r * 4 + g];
+    }
   }
   double num = 0.0, den = 0.0;
-  for (int r = warp; r < kRowsPerCta; r += 4) {
+  for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
     if (r0 + r >= a.N) break;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -206,16 +273,21 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
     num += __shfl_down_sync(0xffffffffu, num, off);
     den += __shfl_down_sync(0xffffffffu, den, off);
   }
-  __shared__ double red[4][2];
+  __shared__ double red[kSweepThreads / 32][2];
   if (lane == 0) {
     red[warp][0] = num;
     red[warp][1] = den;
   }
   __syncthreads();
   if (tid == 0) {
+    double sn = 0.0, sd = 0.0;
+    for (int wq = 0; wq < kSweepThreads / 32; ++wq) {
+      sn += red[wq][0];
+      sd += red[wq][1];
+    }
     double* p = a.partials + (static_cast<int64_t>(j0 / kBlk) * gridDim.x + blockIdx.x) * 2;
-    p[0] = red[0][0] + red[1][0] + red[2][0] + red[3][0];
-    p[1] = red[0][1] + red[1][1] + red[2][1] + red[3][1];
+    p[0] = sn;
+    p[1] = sd;
   }
 }
 
