@@ -91,8 +91,16 @@ __global__ void __launch_bounds__(256) reverse_damp_kernel(const float* __restri
 
 // ------------------------------------------------------------------------- 3a. leaf
 
-// Lower 4 x 4 tiles of the 128 x 128 leaf, enumerated row by row: 32 * 33 / 2 = 528 tiles;
-// thread t owns tiles t, t + 256 and t + 512, so a warp's tiles lie in one band of rows.
+// Factor the 128 x 128 lower block at A as L D L^T (unit L) by right-looking elimination, and
+// at the same time eliminate Y = L^-1 (unit lower); writes X = D^-1/2 Y = (L D^1/2)^-1, the
+// inverse of the Cholesky factor (zeros above the diagonal), and X^T.  The lower triangle is
+// cut into 528 tiles of 4 x 4; thread t of 512 owns tile t (and t + 512) of both S and Y, in
+// registers.  Step k publishes column k of the Schur complement and row k of Y through
+// double-buffered shared memory (one barrier per step); every thread then updates its tiles.
+constexpr int kLB = kLeaf;      // 128
+constexpr int kLeafThreads = 512;
+constexpr int kLeafTiles = 528;  // 32 * 33 / 2
+
 __device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
   int r = static_cast<int>((sqrtf(8.f * idx + 1.f) - 1.f) * 0.5f);
   while (r * (r + 1) / 2 > idx) --r;
@@ -101,26 +109,22 @@ __device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
   tj = idx - r * (r + 1) / 2;
 }
 
-// Factor the 128 x 128 lower block at A as L D L^T (unit L) by right-looking elimination, and
-// at the same time eliminate Y = L^-1 (unit lower); writes X = D^-1/2 Y = (L D^1/2)^-1, the
-// inverse of the Cholesky factor, with zeros above the diagonal.  Every element lives in a
-// register of the thread that owns its tile; step k publishes column k of the Schur
-// complement and row k of Y through double-buffered shared memory (one barrier per step).
-__global__ void __launch_bounds__(256, 1) chol_inv_leaf_kernel(const float* __restrict__ A, int64_t lda,
-                                                               float* __restrict__ X, float* __restrict__ XT,
-                                                               int64_t ldx, int* __restrict__ info, int diag_off) {
+__global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const float* __restrict__ A, int64_t lda,
+                                                                         float* __restrict__ X, float* __restrict__ XT,
+                                                                         int64_t ldx, int* __restrict__ info,
+                                                                         int diag_off) {
   if (*info != 0) return;
-  __shared__ float colbuf[2][kLeaf];
-  __shared__ float yrow[2][kLeaf];
-  __shared__ float dbuf[kLeaf];
+  __shared__ __align__(16) float colbuf[2][kLB];
+  __shared__ __align__(16) float yrow[2][kLB];
+  __shared__ float dbuf[kLB];
   const int t = threadIdx.x;
-  int ti[3], tj[3];
-  bool own[3];
-  float v[3][16], y[3][16];
+  int ti[2], tj[2];
+  bool own[2];
+  float v[2][16], y[2][16];
 #pragma unroll
-  for (int q = 0; q < 3; ++q) {
-    const int idx = t + 256 * q;
-    own[q] = idx < 528;
+  for (int q = 0; q < 2; ++q) {
+    const int idx = t + kLeafThreads * q;
+    own[q] = idx < kLeafTiles;
     leaf_tile(own[q] ? idx : 0, ti[q], tj[q]);
 #pragma unroll
     for (int r = 0; r < 4; ++r)
@@ -131,16 +135,16 @@ __global__ void __launch_bounds__(256, 1) chol_inv_leaf_kernel(const float* __re
         y[q][r * 4 + c] = (own[q] && i == j) ? 1.f : 0.f;
       }
   }
-  if (t < kLeaf) {
+  if (t < kLB) {
     yrow[0][t] = 0.f;
     yrow[1][t] = 0.f;
   }
   __syncthreads();
 
-  for (int k = 0; k < kLeaf; ++k) {
+  for (int k = 0; k < kLB; ++k) {
     const int buf = k & 1, kt = k >> 2, kc = k & 3;
 #pragma unroll
-    for (int q = 0; q < 3; ++q) {
+    for (int q = 0; q < 2; ++q) {
       if (!own[q]) continue;
       if (tj[q] == kt) {
 #pragma unroll
@@ -169,18 +173,22 @@ __global__ void __launch_bounds__(256, 1) chol_inv_leaf_kernel(const float* __re
     }
     const float inv_d = 1.f / d;
 #pragma unroll
-    for (int q = 0; q < 3; ++q) {
+    for (int q = 0; q < 2; ++q) {
       if (!own[q]) continue;
       const int i0 = 4 * ti[q], j0 = 4 * tj[q];
       if (i0 + 3 <= k) continue;  // every row of the tile is at or above the pivot
-      float a[4];
+      const float4 a4 = *reinterpret_cast<const float4*>(&colbuf[buf][i0]);
+      float a[4] = {a4.x * inv_d, a4.y * inv_d, a4.z * inv_d, a4.w * inv_d};  // L[i][k]
 #pragma unroll
-      for (int r = 0; r < 4; ++r) a[r] = (i0 + r > k) ? colbuf[buf][i0 + r] * inv_d : 0.f;  // L[i][k]
+      for (int r = 0; r < 4; ++r)
+        if (i0 + r <= k) a[r] = 0.f;
       if (j0 + 3 > k) {
         // Schur update S[i][j] -= S[i][k] S[j][k] / d_k  for i, j > k
-        float b[4];
+        const float4 b4 = *reinterpret_cast<const float4*>(&colbuf[buf][j0]);
+        float b[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) b[c] = (j0 + c > k) ? colbuf[buf][j0 + c] : 0.f;
+        for (int c = 0; c < 4; ++c)
+          if (j0 + c <= k) b[c] = 0.f;
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -188,29 +196,28 @@ __global__ void __launch_bounds__(256, 1) chol_inv_leaf_kernel(const float* __re
       }
       if (j0 <= k) {
         // elimination of Y: Y[i][j] -= L[i][k] Y[k][j]  for i > k, j <= k
-        float yb[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) yb[c] = yrow[buf][j0 + c];
+        const float4 yb = *reinterpret_cast<const float4*>(&yrow[buf][j0]);
+        const float ybv[4] = {yb.x, yb.y, yb.z, yb.w};
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) y[q][r * 4 + c] = fmaf(-a[r], yb[c], y[q][r * 4 + c]);
+          for (int c = 0; c < 4; ++c) y[q][r * 4 + c] = fmaf(-a[r], ybv[c], y[q][r * 4 + c]);
       }
     }
   }
   // X[i][j] = Y[i][j] / sqrt(d_i)
 #pragma unroll
-  for (int q = 0; q < 3; ++q)
+  for (int q = 0; q < 2; ++q)
     if (own[q] && ti[q] == tj[q])
 #pragma unroll
       for (int r = 0; r < 4; ++r) dbuf[4 * ti[q] + r] = v[q][r * 4 + r];
   __syncthreads();
 #pragma unroll
-  for (int q = 0; q < 3; ++q) {
+  for (int q = 0; q < 2; ++q) {
     if (!own[q]) continue;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float sc = 1.f / sqrtf(dbuf[4 * ti[q] + r]);
+      const float sc = __fdiv_rn(1.f, sqrtf(dbuf[4 * ti[q] + r]));
 #pragma unroll
       for (int c = 0; c < 4; ++c) y[q][r * 4 + c] *= sc;
     }
@@ -283,8 +290,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const float* __restrict_
 static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, float* tmp) {
   const int64_t K = c.K;
   if (n == kLeaf) {
-    chol_inv_leaf_kernel<<<1, 256, 0, c.s>>>(c.A + off * K + off, K, c.X + off * K + off, c.XT + off * K + off, K,
-                                             c.info, static_cast<int>(off));
+    chol_inv_leaf_kernel<<<1, kLeafThreads, 0, c.s>>>(c.A + off * K + off, K, c.X + off * K + off,
+                                                      c.XT + off * K + off, K, c.info, static_cast<int>(off));
     HQ_LAUNCH_CHECK();
     return HQ_OK;
   }
