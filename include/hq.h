@@ -14,8 +14,9 @@
  *
  * Conventions for every entry point:
  *   - Array pointers are DEVICE pointers owned by the caller unless a parameter says
- *     "host".  The library allocates no memory and keeps no state between calls; a caller
- *     that runs calls concurrently gives each its own workspace.
+ *     "host".  The library allocates no memory; a caller that runs calls concurrently gives
+ *     each its own workspace.  (hq_rtn_quantize_noalloc instead uses one fixed scratch array
+ *     that is part of the library's device image.)
  *   - Matrices are row-major and densely packed (leading dimension = column count).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it.
  *   - Invalid arguments are refused with HQ_ERR_INVALID (or HQ_ERR_UNSUPPORTED for a
@@ -125,6 +126,29 @@ hq_status hq_rtn_quantize(const void* W, int w_dtype, int64_t N, int64_t K, int6
                           const float* imp, uint8_t* codes, float* scales, double* qerr_out,
                           double* qerr_dev, void* workspace, size_t workspace_bytes,
                           hq_stream_t stream);
+
+/*
+ * hq_rtn_quantize without a workspace, for callers that cannot hand the library scratch memory
+ * when they quantise: an application that has already reserved all device memory for its own
+ * pool, a service that forbids allocation after start-up, a plugin living under another
+ * framework's allocator.  The pages have no counterpart to this entry point; it is a deployment
+ * convenience.  Same arguments, results and output layouts as hq_rtn_quantize, minus
+ * `workspace` / `workspace_bytes`.
+ *   - Scratch (qerr partial sums, status) lives in one fixed array in the library's device
+ *     memory: HQ_RTN_NOALLOC_MAX_GROUPS * 16 + 256 bytes (16 MiB + 256 B), held on every GPU
+ *     that loads the library until the process exits.  N * (K / group) above
+ *     HQ_RTN_NOALLOC_MAX_GROUPS is refused with HQ_ERR_UNSUPPORTED before any launch.
+ *   - The call allocates nothing (no cudaMalloc, no allocating library routine).  The first
+ *     call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ *     device current; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last call's contents; each
+ *     call re-initialises what it needs.  Calls whose GPU work overlaps (different streams,
+ *     different host threads) race on it: serialise them.
+ */
+#define HQ_RTN_NOALLOC_MAX_GROUPS 1048576
+hq_status hq_rtn_quantize_noalloc(const void* W, int w_dtype, int64_t N, int64_t K, int64_t group,
+                                  const float* imp, uint8_t* codes, float* scales, double* qerr_out,
+                                  double* qerr_dev, hq_stream_t stream);
 
 /* Bf16TrilDiagF32 payload size: K*4 + K*(K-1)/2*2 bytes ([calib] "Hessian storage"). */
 size_t hq_bf16tril_bytes(int64_t K);

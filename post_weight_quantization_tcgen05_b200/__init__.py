@@ -52,6 +52,7 @@ _SIGS = {
     "hq_gptq_quantize": (_int, [_vp, _int, _i64, _i64, _vp, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hq_rtn_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "hq_rtn_quantize": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hq_rtn_quantize_noalloc": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "hq_bf16tril_bytes": (_sz, [_i64]),
     "hq_hessian_pack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
     "hq_hessian_unpack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
@@ -171,6 +172,17 @@ def hq_rtn_quantize(W, group: int, codes, scales, workspace, imp=None, want_qerr
                              ctypes.byref(q) if want_qerr else None, _ptr(qerr_dev), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hq_rtn_quantize")
+    return q.value if want_qerr else None
+
+
+def hq_rtn_quantize_noalloc(W, group: int, codes, scales, imp=None, want_qerr: bool = True, qerr_dev=None,
+                            stream=None):
+    """hq_rtn_quantize with the library's own fixed scratch instead of a workspace."""
+    N, K = W.shape
+    q = ctypes.c_double(float("nan"))
+    st = lib.hq_rtn_quantize_noalloc(_ptr(W), _dtype(W), N, K, int(group), _ptr(imp), _ptr(codes), _ptr(scales),
+                                     ctypes.byref(q) if want_qerr else None, _ptr(qerr_dev), _stream(stream))
+    _check(st, "hq_rtn_quantize_noalloc")
     return q.value if want_qerr else None
 
 
