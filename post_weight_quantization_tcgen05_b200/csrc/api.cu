@@ -142,12 +142,13 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
-  float* A = reinterpret_cast<float*>(ws + L.a);
-  hq_status st = launch_factor(H, K, damp, A, reinterpret_cast<float*>(ws + L.x), reinterpret_cast<float*>(ws + L.xt),
-                               reinterpret_cast<float*>(ws + L.t), &hdr->lam, &hdr->info, &hdr->status, A,
-                               reinterpret_cast<float*>(ws + L.t), s);
+  float* Ut = nullptr;
+  float* U = nullptr;
+  hq_status st = launch_factor(H, K, damp, reinterpret_cast<double*>(ws + L.a), reinterpret_cast<double*>(ws + L.x),
+                               reinterpret_cast<double*>(ws + L.xt), reinterpret_cast<double*>(ws + L.t), &hdr->lam,
+                               &hdr->info, &hdr->status, &Ut, &U, s);
   if (st != HQ_OK) return st;
-  HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, A, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, Ut, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return finish_sync(s, hdr, nullptr);
 }
 

@@ -20,7 +20,7 @@
 // tensor cores in 3xTF32 (gemm_tf32.cuh).  Leaves are 128 x 128 blocks factored and inverted by
 // one CTA (chol_inv_leaf_kernel).  Steps:
 //   1. lambda = damp * mean(diag H)            (fp64 reduction, one CTA)
-//   2. A = J (H + lambda I) J, lower triangle  (tiled transpose; H's lower triangle is read)
+//   2. A = J (H + lambda I) J in fp64, lower triangle (tiled transpose of H's lower triangle)
 //   3. X = L^-1 and X^T by the recursion above
 //   4. U = J X J and U^T = J X^T J, both row-major (180-degree rotated copies)
 // A device flag `info` receives the first failing pivot (1-based, in M's order) and stops
@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(1024) damp_stats_kernel(const float* __restric
 // ------------------------------------------------------------------------- 2. reverse + damp
 
 __global__ void __launch_bounds__(256) reverse_damp_kernel(const float* __restrict__ H, int64_t K,
-                                                           const double* __restrict__ lam, float* __restrict__ A,
+                                                           const double* __restrict__ lam, double* __restrict__ A,
                                                            const int* __restrict__ info) {
   if (*info != 0) return;
   __shared__ float t[32][33];
@@ -78,13 +78,13 @@ __global__ void __launch_bounds__(256) reverse_damp_kernel(const float* __restri
   for (int i = ty; i < 32; i += 8) {
     const int64_t a = a0 + i, b = b0 + tx;
     if (a >= K || b >= K) continue;
-    float v;
+    double v;
     if (a > b)
-      v = t[tx][i];
+      v = static_cast<double>(t[tx][i]);
     else if (a == b)
-      v = static_cast<float>(static_cast<double>(t[tx][i]) + l);
+      v = static_cast<double>(t[tx][i]) + l;
     else
-      v = 0.f;
+      v = 0.0;
     A[a * K + b] = v;
   }
 }
@@ -93,12 +93,12 @@ __global__ void __launch_bounds__(256) reverse_damp_kernel(const float* __restri
 
 // Factor the 128 x 128 lower block at A as L D L^T (unit L) by right-looking elimination, and
 // at the same time eliminate Y = L^-1 (unit lower); writes X = D^-1/2 Y = (L D^1/2)^-1, the
-// inverse of the Cholesky factor (zeros above the diagonal), and X^T.  The lower triangle is
-// cut into 528 tiles of 4 x 4; thread t of 512 owns tile t (and t + 512) of both S and Y, in
-// registers.  Step k publishes column k of the Schur complement and row k of Y through
+// inverse of the Cholesky factor (zeros above the diagonal), and X^T.  fp64.  The lower
+// triangle is cut into 528 tiles of 4 x 4; thread t of 288 owns tiles t and t + 288 of both S
+// and Y, in registers.  Step k publishes column k of the Schur complement and row k of Y through
 // double-buffered shared memory (one barrier per step); every thread then updates its tiles.
 constexpr int kLB = kLeaf;      // 128
-constexpr int kLeafThreads = 512;
+constexpr int kLeafThreads = 288;
 constexpr int kLeafTiles = 528;  // 32 * 33 / 2
 
 __device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
@@ -109,18 +109,18 @@ __device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
   tj = idx - r * (r + 1) / 2;
 }
 
-__global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const float* __restrict__ A, int64_t lda,
-                                                                         float* __restrict__ X, float* __restrict__ XT,
-                                                                         int64_t ldx, int* __restrict__ info,
-                                                                         int diag_off) {
+__global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const double* __restrict__ A, int64_t lda,
+                                                                         double* __restrict__ X,
+                                                                         double* __restrict__ XT, int64_t ldx,
+                                                                         int* __restrict__ info, int diag_off) {
   if (*info != 0) return;
-  __shared__ __align__(16) float colbuf[2][kLB];
-  __shared__ __align__(16) float yrow[2][kLB];
-  __shared__ float dbuf[kLB];
+  __shared__ __align__(16) double colbuf[2][kLB];
+  __shared__ __align__(16) double yrow[2][kLB];
+  __shared__ double dbuf[kLB];
   const int t = threadIdx.x;
   int ti[2], tj[2];
   bool own[2];
-  float v[2][16], y[2][16];
+  double v[2][16], y[2][16];
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int idx = t + kLeafThreads * q;
@@ -131,13 +131,13 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const fl
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int i = 4 * ti[q] + r, j = 4 * tj[q] + c;
-        v[q][r * 4 + c] = (own[q] && j <= i) ? A[i * lda + j] : 0.f;
-        y[q][r * 4 + c] = (own[q] && i == j) ? 1.f : 0.f;
+        v[q][r * 4 + c] = (own[q] && j <= i) ? A[i * lda + j] : 0.0;
+        y[q][r * 4 + c] = (own[q] && i == j) ? 1.0 : 0.0;
       }
   }
   if (t < kLB) {
-    yrow[0][t] = 0.f;
-    yrow[1][t] = 0.f;
+    yrow[0][t] = 0.0;
+    yrow[1][t] = 0.0;
   }
   __syncthreads();
 
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const fl
       if (tj[q] == kt) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          float x = v[q][r * 4];
+          double x = v[q][r * 4];
 #pragma unroll
           for (int c = 1; c < 4; ++c) x = (c == kc) ? v[q][r * 4 + c] : x;
           colbuf[buf][4 * ti[q] + r] = x;
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const fl
       if (ti[q] == kt) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float x = y[q][c];
+          double x = y[q][c];
 #pragma unroll
           for (int r = 1; r < 4; ++r) x = (r == kc) ? y[q][r * 4 + c] : x;
           yrow[buf][4 * tj[q] + c] = x;
@@ -166,42 +166,39 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const fl
       }
     }
     __syncthreads();
-    const float d = colbuf[buf][k];
-    if (!(d > 0.f) || !isfinite(d)) {
+    const double d = colbuf[buf][k];
+    if (!(d > 0.0) || !isfinite(d)) {
       if (t == 0) atomicCAS(info, 0, diag_off + k + 1);
       return;  // uniform: every thread read the same pivot
     }
-    const float inv_d = 1.f / d;
+    const double inv_d = 1.0 / d;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       if (!own[q]) continue;
       const int i0 = 4 * ti[q], j0 = 4 * tj[q];
       if (i0 + 3 <= k) continue;  // every row of the tile is at or above the pivot
-      const float4 a4 = *reinterpret_cast<const float4*>(&colbuf[buf][i0]);
-      float a[4] = {a4.x * inv_d, a4.y * inv_d, a4.z * inv_d, a4.w * inv_d};  // L[i][k]
+      double a[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-        if (i0 + r <= k) a[r] = 0.f;
+      for (int r = 0; r < 4; ++r) a[r] = (i0 + r > k) ? colbuf[buf][i0 + r] * inv_d : 0.0;  // L[i][k]
       if (j0 + 3 > k) {
         // Schur update S[i][j] -= S[i][k] S[j][k] / d_k  for i, j > k
-        const float4 b4 = *reinterpret_cast<const float4*>(&colbuf[buf][j0]);
-        float b[4] = {b4.x, b4.y, b4.z, b4.w};
+        double b[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (j0 + c <= k) b[c] = 0.f;
+        for (int c = 0; c < 4; ++c) b[c] = (j0 + c > k) ? colbuf[buf][j0 + c] : 0.0;
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) v[q][r * 4 + c] = fmaf(-a[r], b[c], v[q][r * 4 + c]);
+          for (int c = 0; c < 4; ++c) v[q][r * 4 + c] = fma(-a[r], b[c], v[q][r * 4 + c]);
       }
       if (j0 <= k) {
         // elimination of Y: Y[i][j] -= L[i][k] Y[k][j]  for i > k, j <= k
-        const float4 yb = *reinterpret_cast<const float4*>(&yrow[buf][j0]);
-        const float ybv[4] = {yb.x, yb.y, yb.z, yb.w};
+        double yb[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) yb[c] = yrow[buf][j0 + c];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) y[q][r * 4 + c] = fmaf(-a[r], ybv[c], y[q][r * 4 + c]);
+          for (int c = 0; c < 4; ++c) y[q][r * 4 + c] = fma(-a[r], yb[c], y[q][r * 4 + c]);
       }
     }
   }
@@ -217,21 +214,21 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const fl
     if (!own[q]) continue;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float sc = __fdiv_rn(1.f, sqrtf(dbuf[4 * ti[q] + r]));
+      const double sc = 1.0 / sqrt(dbuf[4 * ti[q] + r]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) y[q][r * 4 + c] *= sc;
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int i = 4 * ti[q] + r;
-      *reinterpret_cast<float4*>(X + static_cast<int64_t>(i) * ldx + 4 * tj[q]) =
-          make_float4(y[q][r * 4 + 0], y[q][r * 4 + 1], y[q][r * 4 + 2], y[q][r * 4 + 3]);
+      double* xr = X + static_cast<int64_t>(4 * ti[q] + r) * ldx + 4 * tj[q];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) xr[c] = y[q][r * 4 + c];
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int j = 4 * tj[q] + c;
-      *reinterpret_cast<float4*>(XT + static_cast<int64_t>(j) * ldx + 4 * ti[q]) =
-          make_float4(y[q][0 * 4 + c], y[q][1 * 4 + c], y[q][2 * 4 + c], y[q][3 * 4 + c]);
+      double* xr = XT + static_cast<int64_t>(4 * tj[q] + c) * ldx + 4 * ti[q];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) xr[r] = y[q][r * 4 + c];
     }
   }
 }
@@ -239,18 +236,18 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const fl
 // ------------------------------------------------------------------------- 3b. recursion
 
 struct FactorCtx {
-  float* A;
-  float* X;
-  float* XT;
+  double* A;
+  double* X;
+  double* XT;
   int64_t K;
   int* info;
   int* status;
   cudaStream_t s;
 };
 
-static hq_status gemm(const FactorCtx& c, float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
-                      const float* B, int64_t ldb, float alpha, float beta, bool lower) {
-  Tf32Gemm g{};
+static hq_status gemm(const FactorCtx& c, double* C, int64_t ldc, int M, int N, int Kred, const double* A,
+                      int64_t lda, const double* B, int64_t ldb, double alpha, double beta, bool lower) {
+  F64Gemm g{};
   g.C = C;
   g.ldc = ldc;
   g.M = M;
@@ -263,18 +260,16 @@ static hq_status gemm(const FactorCtx& c, float* C, int64_t ldc, int M, int N, i
   g.alpha = alpha;
   g.beta = beta;
   g.lower = lower ? 1 : 0;
-  g.split3 = true;
   g.skip = c.info;
-  g.status = c.status;
-  return tf32_gemm(g, c.s);
+  return f64_gemm(g, c.s);
 }
 
 // dst[j][i] = src[i][j] for an R x C block (32 x 32 tiles through shared memory).
-__global__ void __launch_bounds__(256) transpose_kernel(const float* __restrict__ src, int64_t lds, int64_t R,
-                                                        int64_t C, float* __restrict__ dst, int64_t ldd,
+__global__ void __launch_bounds__(256) transpose_kernel(const double* __restrict__ src, int64_t lds, int64_t R,
+                                                        int64_t C, double* __restrict__ dst, int64_t ldd,
                                                         const int* __restrict__ info) {
   if (*info != 0) return;
-  __shared__ float t[32][33];
+  __shared__ double t[32][33];
   const int64_t tiles_c = (C + 31) / 32;
   const int64_t r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
   const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
@@ -286,8 +281,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const float* __restrict_
 }
 
 // X = L^-1 and X^T for the n x n block of A at (off, off); `tmp` has room for the temporaries
-// of this level and all levels below (2 * n2 * n1 floats here, a quarter of that below...).
-static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, float* tmp) {
+// of this level and all levels below (2 * n2 * n1 here, about a quarter of that per level below).
+static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tmp) {
   const int64_t K = c.K;
   if (n == kLeaf) {
     chol_inv_leaf_kernel<<<1, kLeafThreads, 0, c.s>>>(c.A + off * K + off, K, c.X + off * K + off,
@@ -296,28 +291,28 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, float* tmp
     return HQ_OK;
   }
   const int64_t n1 = (n / kLeaf / 2) * kLeaf, n2 = n - n1;
-  float* T = tmp;             // n2 x n1: L21
-  float* YT = tmp + n2 * n1;  // n1 x n2: (L21 X11)^T
-  float* rest = YT + n2 * n1;
-  const float* A21 = c.A + (off + n1) * K + off;
-  float* A22 = c.A + (off + n1) * K + off + n1;
-  const float* X11 = c.X + off * K + off;
-  const float* XT11 = c.XT + off * K + off;
-  float* X21 = c.X + (off + n1) * K + off;
-  const float* X22 = c.X + (off + n1) * K + off + n1;
-  float* XT12 = c.XT + off * K + off + n1;
+  double* T = tmp;             // n2 x n1: L21
+  double* YT = tmp + n2 * n1;  // n1 x n2: (L21 X11)^T
+  double* rest = YT + n2 * n1;
+  const double* A21 = c.A + (off + n1) * K + off;
+  double* A22 = c.A + (off + n1) * K + off + n1;
+  const double* X11 = c.X + off * K + off;
+  const double* XT11 = c.XT + off * K + off;
+  double* X21 = c.X + (off + n1) * K + off;
+  const double* X22 = c.X + (off + n1) * K + off + n1;
+  double* XT12 = c.XT + off * K + off + n1;
   const int in1 = static_cast<int>(n1), in2 = static_cast<int>(n2);
   hq_status st = chol_inv(c, off, n1, rest);
   if (st != HQ_OK) return st;
-  st = gemm(c, T, n1, in2, in1, in1, A21, K, X11, K, 1.f, 0.f, false);     // T = A21 X11^T
+  st = gemm(c, T, n1, in2, in1, in1, A21, K, X11, K, 1.0, 0.0, false);     // T = A21 X11^T
   if (st != HQ_OK) return st;
-  st = gemm(c, A22, K, in2, in2, in1, T, n1, T, n1, -1.f, 1.f, true);      // A22 -= T T^T
+  st = gemm(c, A22, K, in2, in2, in1, T, n1, T, n1, -1.0, 1.0, true);      // A22 -= T T^T
   if (st != HQ_OK) return st;
   st = chol_inv(c, off + n1, n2, rest);
   if (st != HQ_OK) return st;
-  st = gemm(c, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.f, 0.f, false);    // Y^T = X11^T T^T
+  st = gemm(c, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.0, 0.0, false);    // Y^T = X11^T T^T
   if (st != HQ_OK) return st;
-  st = gemm(c, X21, K, in2, in1, in2, X22, K, YT, n2, -1.f, 0.f, false);   // X21 = -X22 Y
+  st = gemm(c, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false);   // X21 = -X22 Y
   if (st != HQ_OK) return st;
   const int64_t tiles = ceil_div(n2, 32) * ceil_div(n1, 32);
   transpose_kernel<<<static_cast<unsigned>(tiles), 256, 0, c.s>>>(X21, K, n2, n1, XT12, K, c.info);
@@ -327,24 +322,25 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, float* tmp
 
 // ------------------------------------------------------------------------- 4. U, U^T
 
-// U[j][c] = X[K-1-j][K-1-c] and U^T[j][c] = X^T[K-1-j][K-1-c]: 180-degree rotations (U upper,
-// U^T lower, zeros elsewhere because X and X^T hold zeros there).
-__global__ void rotate_kernel(const float* __restrict__ X, const float* __restrict__ XT, int64_t K,
+// U[j][c] = X[K-1-j][K-1-c] and U^T[j][c] = X^T[K-1-j][K-1-c], rounded to fp32: 180-degree
+// rotations (U upper, U^T lower, zeros elsewhere because X and X^T hold zeros there).
+__global__ void rotate_kernel(const double* __restrict__ X, const double* __restrict__ XT, int64_t K,
                               float* __restrict__ U, float* __restrict__ Ut, const int* __restrict__ info) {
   if (*info != 0) return;
   const int64_t n = K * K;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t src = n - 1 - e;  // (K-1-j)*K + (K-1-c) for e = j*K + c
-    U[e] = X[src];
-    Ut[e] = XT[src];
+    U[e] = static_cast<float>(X[src]);
+    Ut[e] = static_cast<float>(XT[src]);
   }
 }
 
 // ------------------------------------------------------------------------- driver
 
-hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* X, float* XT, float* T, double* lam,
-                        int* info, int* status, float* Ut, float* U, cudaStream_t s) {
+hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
+                        double* lam, int* info, int* status, float** Ut, float** U, cudaStream_t s) {
+  (void)status;
   if (K % kLeaf != 0) return HQ_ERR_UNSUPPORTED;
   damp_stats_kernel<<<1, 1024, 0, s>>>(H, K, damp, lam, info);
   HQ_LAUNCH_CHECK();
@@ -353,13 +349,16 @@ hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* 
     reverse_damp_kernel<<<static_cast<unsigned>(nb * (nb + 1) / 2), 256, 0, s>>>(H, K, lam, A, info);
     HQ_LAUNCH_CHECK();
   }
-  HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(float), s));
-  HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(float), s));
+  HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(double), s));
+  HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(double), s));
   FactorCtx c{A, X, XT, K, info, status, s};
   hq_status st = chol_inv(c, 0, K, T);
   if (st != HQ_OK) return st;
+  // A is dead now: U^T and U (fp32) go into its storage
+  *Ut = reinterpret_cast<float*>(A);
+  *U = reinterpret_cast<float*>(A) + K * K;
   const int64_t grid = ceil_div(K * K, 4 * 256) < 148 * 32 ? ceil_div(K * K, 4 * 256) : 148 * 32;
-  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, U, Ut, info);
+  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, *U, *Ut, info);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
 }

@@ -365,14 +365,14 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   off = round_up(off + static_cast<size_t>(N) * K * sizeof(float), al);
   L.err = off;
   off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
-  L.a = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  L.a = off;  // fp64 A, later U^T and U in fp32
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.x = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.xt = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.t = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.total = off;
   return L;
 }
@@ -390,16 +390,16 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   double* partials = reinterpret_cast<double*>(ws + L.partials);
   float* Wf = reinterpret_cast<float*>(ws + L.wf);
   float* Err = reinterpret_cast<float*>(ws + L.err);
-  float* A = reinterpret_cast<float*>(ws + L.a);
-  float* X = reinterpret_cast<float*>(ws + L.x);
-  float* XT = reinterpret_cast<float*>(ws + L.xt);
-  float* T = reinterpret_cast<float*>(ws + L.t);
+  double* A = reinterpret_cast<double*>(ws + L.a);
+  double* X = reinterpret_cast<double*>(ws + L.x);
+  double* XT = reinterpret_cast<double*>(ws + L.xt);
+  double* T = reinterpret_cast<double*>(ws + L.t);
   HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
 
-  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, /*Ut=*/A, /*U=*/T, s);
+  float* Ut = nullptr;
+  float* U = nullptr;
+  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, s);
   if (st != HQ_OK) return st;
-  const float* Ut = A;
-  const float* U = T;
 
   {
     const int64_t n = N * K;

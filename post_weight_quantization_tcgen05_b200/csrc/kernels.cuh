@@ -34,10 +34,26 @@ struct Tf32Gemm {
 };
 hq_status tf32_gemm(const Tf32Gemm& g, cudaStream_t s);
 
-// factor.cu: U (row-major, upper) and U^T (row-major, lower) of the damped Hessian; A, X, XT
-// and T are K x K fp32 scratch (U^T may alias A, U may alias T).
-hq_status launch_factor(const float* H, int64_t K, float damp, float* A, float* X, float* XT, float* T, double* lam,
-                        int* info, int* status, float* Ut, float* U, cudaStream_t s);
+// gemm_f64.cu: C = beta C + alpha A B^T in fp64 on the CUDA cores
+struct F64Gemm {
+  double* C;
+  int64_t ldc;
+  int M, N, Kred;
+  const double* A;  // A(m, k) = A[m * lda + k]
+  int64_t lda;
+  const double* B;  // B(n, k) = B[n * ldb + k]
+  int64_t ldb;
+  double alpha, beta;
+  int lower, row0, col0;
+  const int* skip;
+};
+hq_status f64_gemm(const F64Gemm& g, cudaStream_t s);
+
+// factor.cu: U (row-major, upper) and U^T (row-major, lower) of the damped Hessian, in fp32,
+// from an fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; U and U^T are written into
+// the first and second halves of A's storage once A is no longer needed.
+hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
+                        double* lam, int* info, int* status, float** Ut, float** U, cudaStream_t s);
 
 // gptq.cu
 struct GptqLayout {
