@@ -41,7 +41,7 @@ hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype,
                                            int* dev_status, int impl, hq_stream_t stream);
 
 /*
- * The tensor-core fp32 GEMM used by the factorisation and the GPTQ lazy updates:
+ * The tensor-core fp32 GEMM used by the GPTQ lazy updates:
  *   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]
  * for m < M, n < N (if `lower`, only elements with m >= n are written).  split3 = 1 selects
  * 3xTF32 (about fp32 accuracy), 0 plain tf32.  A and B 16-byte aligned, lda and ldb
@@ -50,6 +50,29 @@ hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype,
 hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
                              const float* B, int64_t ldb, float alpha, float beta, int lower, int split3,
                              hq_stream_t stream);
+
+/*
+ * The fp64 GEMM of the factorisation (fp64 tensor cores, mma.sync m8n8k4):
+ *   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]
+ * for m < M, n < N (if `lower`, M == N and only elements with m >= n are written).
+ * tri declares a triangular operand whose zeros the kernel skips (the result is the same
+ * when the operand really is zero there): 0 none, 1 A upper (A[m][k] = 0 for k < m),
+ * 2 A lower (A[m][k] = 0 for k > m), 3 B lower (B[n][k] = 0 for k > n).
+ * Kred a multiple of 16; A, B 16-byte aligned, lda and ldb even.  `scratch` (scratch_elems doubles, may be
+ * NULL) lets the kernel split the contraction when the problem has few output tiles; the
+ * partial sums are added in a fixed order, so results are identical run to run.
+ * No counterpart on the pages: a building block of the path.
+ */
+hq_status hq_debug_f64_gemm(double* C, int64_t ldc, int M, int N, int Kred, const double* A, int64_t lda,
+                            const double* B, int64_t ldb, double alpha, double beta, int lower, int tri,
+                            double* scratch, int64_t scratch_elems, hq_stream_t stream);
+
+/*
+ * out[i] = 1 / d[i] (fp64) by the reciprocal the factorisation's leaf kernel uses for its pivots
+ * (hardware approximation refined by two Newton-Raphson steps), for d[i] positive, normal and
+ * finite (other inputs give unspecified values).  n >= 0.  No counterpart on the pages.
+ */
+hq_status hq_debug_rcp_f64(const double* d, double* out, int64_t n, hq_stream_t stream);
 
 /* Number of kernels libhq.so has launched in this process so far (all devices, all
  * threads).  A statistic for profiling; never reset. */

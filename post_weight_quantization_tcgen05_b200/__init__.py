@@ -43,6 +43,8 @@ if not os.path.exists(_LIB_PATH):
 lib = ctypes.CDLL(_LIB_PATH)
 
 _vp, _i64, _int, _f, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_dbl = ctypes.c_double
+
 _SIGS = {
     "hq_status_string": (ctypes.c_char_p, [_int]),
     "hq_abi_version": (_int, []),
@@ -62,6 +64,9 @@ _SIGS = {
     "hq_debug_hessian_accumulate_impl": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _int, _vp]),
     "hq_debug_launch_count": (ctypes.c_uint64, []),
     "hq_debug_tf32_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _f, _f, _int, _int, _vp]),
+    "hq_debug_rcp_f64": (_int, [_vp, _vp, _i64, _vp]),
+    "hq_debug_f64_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _dbl, _dbl, _int, _int, _vp,
+                                 _i64, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -199,6 +204,20 @@ def hq_debug_tf32_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, split3=True, s
     _check(lib.hq_debug_tf32_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
                                   float(alpha), float(beta), int(bool(lower)), int(bool(split3)), _stream(stream)),
            "hq_debug_tf32_gemm")
+
+
+def hq_debug_rcp_f64(d, out, stream=None) -> None:
+    """out = 1 / d (fp64) by the factorisation leaf's pivot reciprocal."""
+    _check(lib.hq_debug_rcp_f64(_ptr(d), _ptr(out), d.numel(), _stream(stream)), "hq_debug_rcp_f64")
+
+
+def hq_debug_f64_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, tri=0, scratch=None, stream=None) -> None:
+    """C = beta C + alpha A B^T (fp64 row-major views, fp64 tensor cores); tri declares a triangular operand."""
+    M, Kred = A.shape
+    N = B.shape[0]
+    _check(lib.hq_debug_f64_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
+                                 float(alpha), float(beta), int(bool(lower)), int(tri), _ptr(scratch),
+                                 0 if scratch is None else scratch.numel(), _stream(stream)), "hq_debug_f64_gemm")
 
 
 def hq_bf16tril_bytes(K: int) -> int:

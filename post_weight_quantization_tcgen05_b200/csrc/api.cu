@@ -152,6 +152,39 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
   return finish_sync(s, hdr, nullptr);
 }
 
+hq_status hq_debug_rcp_f64(const double* d, double* out, int64_t n, hq_stream_t stream) {
+  if (n < 0 || (n > 0 && (d == nullptr || out == nullptr))) return HQ_ERR_INVALID;
+  return launch_rcp_nr(d, out, n, static_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_debug_f64_gemm(double* C, int64_t ldc, int M, int N, int Kred, const double* A, int64_t lda,
+                            const double* B, int64_t ldb, double alpha, double beta, int lower, int tri,
+                            double* scratch, int64_t scratch_elems, hq_stream_t stream) {
+  if (C == nullptr || A == nullptr || B == nullptr || M < 0 || N < 0 || Kred < 1) return HQ_ERR_INVALID;
+  if (ldc < N || lda < Kred || ldb < Kred || tri < kTriNone || tri > kTriBLower || scratch_elems < 0)
+    return HQ_ERR_INVALID;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 8) || lda % 2 != 0 || ldb % 2 != 0) return HQ_ERR_INVALID;
+  if (Kred % 16 != 0 || (lower && M != N)) return HQ_ERR_UNSUPPORTED;
+  F64Gemm g{};
+  g.C = C;
+  g.ldc = ldc;
+  g.M = M;
+  g.N = N;
+  g.Kred = Kred;
+  g.A = A;
+  g.lda = lda;
+  g.B = B;
+  g.ldb = ldb;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.lower = lower ? 1 : 0;
+  g.tri = tri;
+  g.scratch = scratch;
+  g.scratch_elems = scratch == nullptr ? 0 : scratch_elems;
+  g.skip = nullptr;
+  return f64_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
 hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
                              const float* B, int64_t ldb, float alpha, float beta, int lower, int split3,
                              hq_stream_t stream) {

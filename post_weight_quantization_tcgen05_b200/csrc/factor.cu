@@ -16,9 +16,10 @@
 //                                X21 = -X22 Y
 //
 // Every product takes both operands K-major (row-major [rows, contraction]), so X^T is kept
-// next to X (leaves write both, X21^T is copied by a tiled transpose).  The products run on the
-// tensor cores in 3xTF32 (gemm_tf32.cuh).  Leaves are 128 x 128 blocks factored and inverted by
-// one CTA (chol_inv_leaf_kernel).  Steps:
+// next to X (leaves write both, X21^T is copied by a tiled transpose).  Everything runs in fp64
+// (gemm_f64.cu for the products; each declares its triangular operand so that tiles skip the
+// zero part of the contraction).  Leaves are 64 x 64 blocks factored and inverted by one CTA
+// (chol_inv_leaf_kernel).  Steps:
 //   1. lambda = damp * mean(diag H)            (fp64 reduction, one CTA)
 //   2. A = J (H + lambda I) J in fp64, lower triangle (tiled transpose of H's lower triangle)
 //   3. X = L^-1 and X^T by the recursion above
@@ -30,7 +31,7 @@
 
 namespace hq {
 
-constexpr int kLeaf = 128;
+constexpr int kLeaf = 64;
 
 // ------------------------------------------------------------------------- 1. lambda
 
@@ -91,15 +92,49 @@ __global__ void __launch_bounds__(256) reverse_damp_kernel(const float* __restri
 
 // ------------------------------------------------------------------------- 3a. leaf
 
-// Factor the 128 x 128 lower block at A as L D L^T (unit L) by right-looking elimination, and
+// 1 / d for d > 0 (normal, finite): the hardware approximation (rcp.approx.ftz.f64) refined by
+// two Newton-Raphson steps for the reciprocal, r <- r + r (1 - d r), each of which squares the
+// relative error; within 2 ulp of the correctly rounded quotient.  About a third of the latency
+// of the IEEE division, which sits on the leaf's critical path once per pivot.
+__device__ __forceinline__ double rcp_nr(double d) {
+  double r;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(r) : "d"(d));
+  double e = fma(-d, r, 1.0);
+  r = fma(r, e, r);
+  e = fma(-d, r, 1.0);
+  return fma(r, e, r);
+}
+
+__global__ void rcp_nr_kernel(const double* __restrict__ d, double* __restrict__ out, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = rcp_nr(d[i]);
+}
+
+hq_status launch_rcp_nr(const double* d, double* out, int64_t n, cudaStream_t s) {
+  if (n <= 0) return HQ_OK;
+  const int64_t grid = ceil_div(n, 256) < 148 * 16 ? ceil_div(n, 256) : 148 * 16;
+  rcp_nr_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(d, out, n);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
+}
+
+// Factor the 64 x 64 lower block at A as L D L^T (unit L) by right-looking elimination, and
 // at the same time eliminate Y = L^-1 (unit lower); writes X = D^-1/2 Y = (L D^1/2)^-1, the
 // inverse of the Cholesky factor (zeros above the diagonal), and X^T.  fp64.  The lower
-// triangle is cut into 528 tiles of 4 x 4; thread t of 288 owns tiles t and t + 288 of both S
-// and Y, in registers.  Step k publishes column k of the Schur complement and row k of Y through
-// double-buffered shared memory (one barrier per step); every thread then updates its tiles.
-constexpr int kLB = kLeaf;      // 128
-constexpr int kLeafThreads = 288;
-constexpr int kLeafTiles = 528;  // 32 * 33 / 2
+// triangle of the leaf is cut into 136 tiles of 4 x 4; thread t < 136 owns tile t of both S and
+// Y, in registers.  Before step k, the owners publish column k of the Schur complement (with
+// zeros at rows <= k), row k of Y (zeros right of k) and 1 / d_k through double-buffered shared
+// memory; one barrier per step.  Because of those zeros every thread applies the same rank-1
+// update to all 32 of its elements without masks (the part of a tile the step does not touch
+// gets a zero factor).  Only the elements step k + 1 publishes (one column of the S tile, one
+// row of the Y tile) are updated before the barrier; the rest of step k's update is applied
+// after it, while step k + 1's shared-memory loads are in flight.  The step loop is unrolled by
+// four so that positions inside a tile are compile-time register indices.  Pivots are checked
+// once at the end (a bad pivot only produces values that are then discarded).
+constexpr int kLB = kLeaf;                                 // 64
+constexpr int kLeafTiles = (kLB / 4) * (kLB / 4 + 1) / 2;  // 136
+constexpr int kLeafThreads = 160;                          // 5 warps, one tile per thread
 
 __device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
   int r = static_cast<int>((sqrtf(8.f * idx + 1.f) - 1.f) * 0.5f);
@@ -116,120 +151,134 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
   if (*info != 0) return;
   __shared__ __align__(16) double colbuf[2][kLB];
   __shared__ __align__(16) double yrow[2][kLB];
+  __shared__ double pinv[2];
   __shared__ double dbuf[kLB];
+  __shared__ int bad;
   const int t = threadIdx.x;
-  int ti[2], tj[2];
-  bool own[2];
-  double v[2][16], y[2][16];
+  const bool own = t < kLeafTiles;
+  int ti, tj;
+  leaf_tile(own ? t : 0, ti, tj);
+  const int i0 = 4 * ti, j0 = 4 * tj;
+  double v[16], y[16];
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int idx = t + kLeafThreads * q;
-    own[q] = idx < kLeafTiles;
-    leaf_tile(own[q] ? idx : 0, ti[q], tj[q]);
+  for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int i = 4 * ti[q] + r, j = 4 * tj[q] + c;
-        v[q][r * 4 + c] = (own[q] && j <= i) ? A[i * lda + j] : 0.0;
-        y[q][r * 4 + c] = (own[q] && i == j) ? 1.0 : 0.0;
-      }
-  }
+    for (int c = 0; c < 4; ++c) {
+      v[r * 4 + c] = (own && j0 + c <= i0 + r) ? A[(i0 + r) * lda + j0 + c] : 0.0;
+      y[r * 4 + c] = (own && i0 + r == j0 + c) ? 1.0 : 0.0;
+    }
   if (t < kLB) {
-    yrow[0][t] = 0.0;
-    yrow[1][t] = 0.0;
+    colbuf[0][t] = colbuf[1][t] = 0.0;
+    yrow[0][t] = yrow[1][t] = 0.0;
+  }
+  if (t == 0) bad = kLB;
+  __syncthreads();
+  // publish column 0 (rows > 0), row 0 of Y and 1 / d_0
+  if (own && tj == 0) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) colbuf[0][i0 + r] = (ti > 0 || r > 0) ? v[r * 4] : 0.0;
+  }
+  if (own && ti == 0) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) yrow[0][j0 + c] = y[c];
+    pinv[0] = rcp_nr(v[0]);
   }
   __syncthreads();
 
-  for (int k = 0; k < kLB; ++k) {
-    const int buf = k & 1, kt = k >> 2, kc = k & 3;
+  // factors of the previous step, whose update is finished at the start of this one
+  double pa[4] = {0.0, 0.0, 0.0, 0.0}, pb[4] = {0.0, 0.0, 0.0, 0.0}, pyb[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int kt = 0; kt < kLB / 4; ++kt) {
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (!own[q]) continue;
-      if (tj[q] == kt) {
+    for (int kc = 0; kc < 4; ++kc) {
+      const int buf = kc & 1;  // == k & 1
+      const bool last = (kt == kLB / 4 - 1) && kc == 3;
+      // step k - 1's update, except column kc of S and row kc of Y (done before its barrier)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          double x = v[q][r * 4];
+      for (int r = 0; r < 4; ++r)
 #pragma unroll
-          for (int c = 1; c < 4; ++c) x = (c == kc) ? v[q][r * 4 + c] : x;
-          colbuf[buf][4 * ti[q] + r] = x;
-        }
+        for (int c = 0; c < 4; ++c)
+          if (c != kc) v[r * 4 + c] = fma(-pa[r], pb[c], v[r * 4 + c]);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (r == kc) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) y[r * 4 + c] = fma(-pa[r], pyb[c], y[r * 4 + c]);
       }
-      if (ti[q] == kt) {
+      if (last) break;  // pivot 63 updates nothing: no row lies below it
+      const double inv_d = pinv[buf];
+      const double2 ca0 = *reinterpret_cast<const double2*>(&colbuf[buf][i0]);
+      const double2 ca1 = *reinterpret_cast<const double2*>(&colbuf[buf][i0 + 2]);
+      const double2 cb0 = *reinterpret_cast<const double2*>(&colbuf[buf][j0]);
+      const double2 cb1 = *reinterpret_cast<const double2*>(&colbuf[buf][j0 + 2]);
+      const double2 yb0 = *reinterpret_cast<const double2*>(&yrow[buf][j0]);
+      const double2 yb1 = *reinterpret_cast<const double2*>(&yrow[buf][j0 + 2]);
+      // L[i][k] (zero at and above the pivot), S[j][k] (zero at and left of it), Y[k][j]
+      const double a[4] = {ca0.x * inv_d, ca0.y * inv_d, ca1.x * inv_d, ca1.y * inv_d};
+      const double b[4] = {cb0.x, cb0.y, cb1.x, cb1.y};
+      const double yb[4] = {yb0.x, yb0.y, yb1.x, yb1.y};
+
+      // elements published for step k + 1: column k + 1 of S, row k + 1 of Y, d_{k+1}
+      const int ktn = (kc == 3) ? kt + 1 : kt;
+      const int cn = (kc + 1) & 3;
+      const int nb = buf ^ 1;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          double x = y[q][c];
+      for (int r = 0; r < 4; ++r) v[r * 4 + cn] = fma(-a[r], b[cn], v[r * 4 + cn]);
 #pragma unroll
-          for (int r = 1; r < 4; ++r) x = (r == kc) ? y[q][r * 4 + c] : x;
-          yrow[buf][4 * tj[q] + c] = x;
-        }
+      for (int c = 0; c < 4; ++c) y[cn * 4 + c] = fma(-a[cn], yb[c], y[cn * 4 + c]);
+      if (own && tj == ktn) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) colbuf[nb][i0 + r] = (ti > ktn || r > cn) ? v[r * 4 + cn] : 0.0;
+        // a new tile column: the last row of the previous diagonal tile still holds a value in
+        // this buffer (published two steps ago)
+        if (cn == 0 && ti == ktn) colbuf[nb][i0 - 1] = 0.0;
       }
-    }
-    __syncthreads();
-    const double d = colbuf[buf][k];
-    if (!(d > 0.0) || !isfinite(d)) {
-      if (t == 0) atomicCAS(info, 0, diag_off + k + 1);
-      return;  // uniform: every thread read the same pivot
-    }
-    const double inv_d = 1.0 / d;
+      if (own && ti == ktn) {
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (!own[q]) continue;
-      const int i0 = 4 * ti[q], j0 = 4 * tj[q];
-      if (i0 + 3 <= k) continue;  // every row of the tile is at or above the pivot
-      double a[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) a[r] = (i0 + r > k) ? colbuf[buf][i0 + r] * inv_d : 0.0;  // L[i][k]
-      if (j0 + 3 > k) {
-        // Schur update S[i][j] -= S[i][k] S[j][k] / d_k  for i, j > k
-        double b[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) b[c] = (j0 + c > k) ? colbuf[buf][j0 + c] : 0.0;
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) v[q][r * 4 + c] = fma(-a[r], b[c], v[q][r * 4 + c]);
+        for (int c = 0; c < 4; ++c) yrow[nb][j0 + c] = y[cn * 4 + c];
+        if (tj == ktn) pinv[nb] = rcp_nr(v[cn * 4 + cn]);
       }
-      if (j0 <= k) {
-        // elimination of Y: Y[i][j] -= L[i][k] Y[k][j]  for i > k, j <= k
-        double yb[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) yb[c] = yrow[buf][j0 + c];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) y[q][r * 4 + c] = fma(-a[r], yb[c], y[q][r * 4 + c]);
+      for (int r = 0; r < 4; ++r) {
+        pa[r] = a[r];
+        pb[r] = b[r];
+        pyb[r] = yb[r];
       }
+      __syncthreads();
     }
   }
+  // pivots d_i (the diagonal of S when it was eliminated); the first bad one fails the leaf
+  if (own && ti == tj) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const double d = v[r * 4 + r];
+      dbuf[i0 + r] = d;
+      if (!(d >= 2.2250738585072014e-308) || !isfinite(d)) atomicMin(&bad, i0 + r);  // not normal, > 0
+    }
+  }
+  __syncthreads();
+  if (bad < kLB) {
+    if (t == 0) atomicCAS(info, 0, diag_off + bad + 1);
+    return;
+  }
+  if (!own) return;
   // X[i][j] = Y[i][j] / sqrt(d_i)
 #pragma unroll
-  for (int q = 0; q < 2; ++q)
-    if (own[q] && ti[q] == tj[q])
+  for (int r = 0; r < 4; ++r) {
+    const double sc = 1.0 / sqrt(dbuf[i0 + r]);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) dbuf[4 * ti[q] + r] = v[q][r * 4 + r];
-  __syncthreads();
+    for (int c = 0; c < 4; ++c) y[r * 4 + c] *= sc;
+  }
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    if (!own[q]) continue;
+  for (int r = 0; r < 4; ++r) {
+    double* xr = X + static_cast<int64_t>(i0 + r) * ldx + j0;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const double sc = 1.0 / sqrt(dbuf[4 * ti[q] + r]);
+    for (int c = 0; c < 4; ++c) xr[c] = y[r * 4 + c];
+  }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) y[q][r * 4 + c] *= sc;
-    }
+  for (int c = 0; c < 4; ++c) {
+    double* xr = XT + static_cast<int64_t>(j0 + c) * ldx + i0;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      double* xr = X + static_cast<int64_t>(4 * ti[q] + r) * ldx + 4 * tj[q];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) xr[c] = y[q][r * 4 + c];
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      double* xr = XT + static_cast<int64_t>(4 * tj[q] + c) * ldx + 4 * ti[q];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) xr[r] = y[q][r * 4 + c];
-    }
+    for (int r = 0; r < 4; ++r) xr[r] = y[r * 4 + c];
   }
 }
 
@@ -239,14 +288,17 @@ struct FactorCtx {
   double* A;
   double* X;
   double* XT;
+  double* tmp_end;  // end of the temporaries region
   int64_t K;
   int* info;
   int* status;
   cudaStream_t s;
 };
 
-static hq_status gemm(const FactorCtx& c, double* C, int64_t ldc, int M, int N, int Kred, const double* A,
-                      int64_t lda, const double* B, int64_t ldb, double alpha, double beta, bool lower) {
+// `scratch` (up to the end of the temporaries) receives split-K partial tiles.
+static hq_status gemm(const FactorCtx& c, double* scratch, double* C, int64_t ldc, int M, int N, int Kred,
+                      const double* A, int64_t lda, const double* B, int64_t ldb, double alpha, double beta,
+                      bool lower, int tri) {
   F64Gemm g{};
   g.C = C;
   g.ldc = ldc;
@@ -260,6 +312,9 @@ static hq_status gemm(const FactorCtx& c, double* C, int64_t ldc, int M, int N, 
   g.alpha = alpha;
   g.beta = beta;
   g.lower = lower ? 1 : 0;
+  g.tri = tri;
+  g.scratch = scratch;
+  g.scratch_elems = c.tmp_end - scratch;
   g.skip = c.info;
   return f64_gemm(g, c.s);
 }
@@ -304,15 +359,15 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
   const int in1 = static_cast<int>(n1), in2 = static_cast<int>(n2);
   hq_status st = chol_inv(c, off, n1, rest);
   if (st != HQ_OK) return st;
-  st = gemm(c, T, n1, in2, in1, in1, A21, K, X11, K, 1.0, 0.0, false);     // T = A21 X11^T
+  st = gemm(c, rest, T, n1, in2, in1, in1, A21, K, X11, K, 1.0, 0.0, false, kTriBLower);  // T = A21 X11^T
   if (st != HQ_OK) return st;
-  st = gemm(c, A22, K, in2, in2, in1, T, n1, T, n1, -1.0, 1.0, true);      // A22 -= T T^T
+  st = gemm(c, rest, A22, K, in2, in2, in1, T, n1, T, n1, -1.0, 1.0, true, kTriNone);     // A22 -= T T^T
   if (st != HQ_OK) return st;
   st = chol_inv(c, off + n1, n2, rest);
   if (st != HQ_OK) return st;
-  st = gemm(c, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.0, 0.0, false);    // Y^T = X11^T T^T
+  st = gemm(c, rest, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.0, 0.0, false, kTriAUpper); // Y^T = X11^T T^T
   if (st != HQ_OK) return st;
-  st = gemm(c, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false);   // X21 = -X22 Y
+  st = gemm(c, rest, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false, kTriALower); // X21 = -X22 Y
   if (st != HQ_OK) return st;
   const int64_t tiles = ceil_div(n2, 32) * ceil_div(n1, 32);
   transpose_kernel<<<static_cast<unsigned>(tiles), 256, 0, c.s>>>(X21, K, n2, n1, XT12, K, c.info);
@@ -351,7 +406,7 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   }
   HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(double), s));
   HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(double), s));
-  FactorCtx c{A, X, XT, K, info, status, s};
+  FactorCtx c{A, X, XT, T + K * K, K, info, status, s};
   hq_status st = chol_inv(c, 0, K, T);
   if (st != HQ_OK) return st;
   // A is dead now: U^T and U (fp32) go into its storage

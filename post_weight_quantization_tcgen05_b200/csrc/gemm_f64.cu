@@ -1,103 +1,261 @@
-// fp64 GEMM on the CUDA cores for the factorisation:
+// fp64 GEMM for the factorisation, on the fp64 tensor cores (mma.sync m8n8k4 .f64):
 //
 //   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]    m < M, n < N
 //
-// (both operands K-major, optionally only the lower part row0 + m >= col0 + n written).
+// (both operands K-major; optionally only the lower part m >= n written; a triangular operand
+// can be declared so that each tile skips the part of the contraction where it is zero).
 // The damped Hessians of strongly correlated layers have condition numbers around 1e6, and the
 // Schur-complement updates of the Cholesky recursion cancel a large common component, so the
 // factorisation runs in fp64 end to end (fp32 loses about kappa * 6e-8 there, which measurably
-// changes GPTQ codes).  128 x 128 tiles per CTA, 256 threads with 8 x 8 outputs each, k-chunks
-// of 16 staged through shared memory (transposed to k-major), with the next chunk's global loads
-// in flight while the current one is multiplied.
+// changes GPTQ codes).  The fp64 MMA rounds like an fp64 FMA chain; on B200 it sustains about
+// 37 TFLOP/s against about 33 for CUDA-core DFMA, with a fraction of the issue slots.
+//
+// Design: BT x BT output tiles (BT = 128: 8 warps of 32 x 64; BT = 64: 4 warps of 32 x 32).
+// Operands stream through a 4-stage cp.async ring of [BT rows][16 k] slices; element (r, k) of a
+// slice sits at r * 16 + (k ^ ((r & 3) << 2)), so that a fragment load (8 rows x 4 consecutive
+// k) touches distinct banks in each half-warp, and 16-byte pairs stay contiguous for cp.async.
+// Tiles are launched most expensive first (their contraction length depends on the triangular
+// operand).  When a problem has too few tiles to fill the GPU, the contraction is split over
+// CTAs that write partial tiles to scratch, and a second kernel adds the partials in a fixed
+// order (so results do not depend on scheduling).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace hq {
+namespace {
 
-constexpr int kDT = 128;  // tile
-constexpr int kDK = 16;   // k-chunk
-constexpr int kDP = kDT + 2;  // padded smem row (doubles)
+constexpr int kDK = 16;  // k per stage
+constexpr int kStages = 4;
+constexpr int kSMs = 148;
 
-__global__ void __launch_bounds__(256) f64_gemm_kernel(F64Gemm g) {
+template <int BT>
+struct F64Cfg {
+  static constexpr int kWarpsM = BT == 128 ? 4 : 2;
+  static constexpr int kWarpsN = 2;
+  static constexpr int kThreads = 32 * kWarpsM * kWarpsN;
+  static constexpr int kWM = BT / kWarpsM;  // warp tile rows (32)
+  static constexpr int kWN = BT / kWarpsN;  // warp tile cols (64 or 32)
+  static constexpr int kFM = kWM / 8;       // 8 x 8 MMA tiles per warp tile, rows
+  static constexpr int kFN = kWN / 8;       // ... cols
+  static constexpr int kStageElems = 2 * BT * kDK;
+  static constexpr int kSmemBytes = kStages * kStageElems * static_cast<int>(sizeof(double));
+  static constexpr int kPairs = BT * kDK / 2 / kThreads;  // 16-byte copies per operand per stage per thread
+};
+
+__device__ __forceinline__ void cp_async16(double* smem, const double* gmem, bool valid) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 16 : 0;  // 0: nothing read, the destination is zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// D (8 x 8) += A (8 x 4) B (4 x 8): lane (g = lane / 4, t = lane % 4) holds A[g][t], B[t][g] and
+// D[g][2t], D[g][2t + 1].
+__device__ __forceinline__ void dmma(double& d0, double& d1, double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ int swz(int r, int k) { return r * kDK + (k ^ ((r & 3) << 2)); }
+
+// Tile t of the launch order -> (tile row, tile column).
+__device__ __forceinline__ void tile_of(const F64Gemm& g, int BT, int t, int& mt, int& nt) {
+  const int tm = (g.M + BT - 1) / BT, tn = (g.N + BT - 1) / BT;
+  if (g.lower) {  // lower tiles only, row by row (all of equal cost)
+    int r = static_cast<int>((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+    while (r * (r + 1) / 2 > t) --r;
+    while ((r + 1) * (r + 2) / 2 <= t) ++r;
+    mt = r;
+    nt = t - r * (r + 1) / 2;
+    return;
+  }
+  switch (g.tri) {
+    case kTriBLower:  // contraction length grows with the column tile
+      nt = tn - 1 - t / tm;
+      mt = t % tm;
+      break;
+    case kTriALower:  // grows with the row tile
+      mt = tm - 1 - t / tn;
+      nt = t % tn;
+      break;
+    default:  // kTriAUpper shrinks with the row tile; kTriNone is uniform
+      mt = t / tn;
+      nt = t % tn;
+      break;
+  }
+}
+
+template <int BT>
+__global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm g, int splits) {
+  using Cfg = F64Cfg<BT>;
+  extern __shared__ __align__(16) double smem[];
   if (g.skip != nullptr && *g.skip != 0) return;
-  const int tiles_n = (g.N + kDT - 1) / kDT;
-  const int m0 = (blockIdx.x / tiles_n) * kDT, n0 = (blockIdx.x % tiles_n) * kDT;
-  if (g.lower && g.row0 + m0 + kDT - 1 < g.col0 + n0) return;
-  __shared__ __align__(16) double As[kDK][kDP];
-  __shared__ __align__(16) double Bs[kDK][kDP];
-  const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;  // output rows ty*8.., columns tx*8..
-  // loader: each thread brings 8 doubles of A and 8 of B per chunk: rows lr, lr+64, k quad lk
-  const int lr = tid >> 2, lk = (tid & 3) * 4;
-  double ra[2][4], rb[2][4];
-  auto load = [&](int k0) {
+  const int t = blockIdx.x / splits, sp = blockIdx.x % splits;
+  int mt, nt;
+  tile_of(g, BT, t, mt, nt);
+  const int m0 = mt * BT, n0 = nt * BT;
+  // contraction range of this tile (a triangular operand is zero outside it), slice aligned
+  int kbeg = 0, kend = g.Kred;
+  if (g.tri == kTriAUpper) kbeg = m0;                 // A[m][k] = 0 for k < m
+  if (g.tri == kTriALower) kend = min(kend, m0 + BT);  // A[m][k] = 0 for k > m
+  if (g.tri == kTriBLower) kend = min(kend, n0 + BT);  // B[n][k] = 0 for k > n
+  const int nch_all = kend > kbeg ? (kend - kbeg) / kDK : 0;
+  const int base = nch_all / splits, rem = nch_all % splits;
+  const int nch = base + (sp < rem ? 1 : 0);
+  const int kfirst = kbeg + (sp * base + min(sp, rem)) * kDK;
+
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int wm0 = (warp / Cfg::kWarpsN) * Cfg::kWM, wn0 = (warp % Cfg::kWarpsN) * Cfg::kWN;
+  const int fg = lane / 4, ft = lane % 4;
+
+  // loader: 16-byte pair p = tid + threads * u of a slice is row p / 8, k 2 * (p % 8)
+  auto load_stage = [&](int stage, int k0) {
+    double* As = smem + stage * Cfg::kStageElems;
+    double* Bs = As + BT * kDK;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = lr + 64 * h;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int k = k0 + lk + u;
-        ra[h][u] = (m0 + r < g.M && k < g.Kred) ? g.A[static_cast<int64_t>(m0 + r) * g.lda + k] : 0.0;
-        rb[h][u] = (n0 + r < g.N && k < g.Kred) ? g.B[static_cast<int64_t>(n0 + r) * g.ldb + k] : 0.0;
-      }
+    for (int u = 0; u < Cfg::kPairs; ++u) {
+      const int p = tid + Cfg::kThreads * u;
+      const int r = p / 8, k = 2 * (p % 8);
+      const int dst = swz(r, k);
+      const bool va = m0 + r < g.M, vb = n0 + r < g.N;
+      cp_async16(As + dst, g.A + static_cast<int64_t>(va ? m0 + r : m0) * g.lda + k0 + k, va);
+      cp_async16(Bs + dst, g.B + static_cast<int64_t>(vb ? n0 + r : n0) * g.ldb + k0 + k, vb);
     }
   };
-  double acc[8][8];
+
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < nch) load_stage(s, kfirst + s * kDK);
+    cp_async_commit();
+  }
+  double acc[Cfg::kFM][Cfg::kFN][2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-  load(0);
-  for (int k0 = 0; k0 < g.Kred; k0 += kDK) {
-    __syncthreads();
+  for (int i = 0; i < Cfg::kFM; ++i)
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+    for (int j = 0; j < Cfg::kFN; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+
+  for (int c = 0; c < nch; ++c) {
+    cp_async_wait<kStages - 2>();  // slice c has landed (this thread's part)
+    __syncthreads();               // ... everyone's; and slice c - 1 is no longer read
+    {
+      const int cn = c + kStages - 1;
+      if (cn < nch) load_stage(cn % kStages, kfirst + cn * kDK);
+      cp_async_commit();
+    }
+    const double* As = smem + (c % kStages) * Cfg::kStageElems;
+    const double* Bs = As + BT * kDK;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        As[lk + u][lr + 64 * h] = ra[h][u];
-        Bs[lk + u][lr + 64 * h] = rb[h][u];
-      }
-    __syncthreads();
-    if (k0 + kDK < g.Kred) load(k0 + kDK);
+    for (int k4 = 0; k4 < kDK; k4 += 4) {
+      double a[Cfg::kFM], b[Cfg::kFN];
 #pragma unroll
-    for (int k = 0; k < kDK; ++k) {
-      double a[8], b[8];
+      for (int i = 0; i < Cfg::kFM; ++i) a[i] = As[swz(wm0 + 8 * i + fg, k4 + ft)];
 #pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        const double2 av = *reinterpret_cast<const double2*>(&As[k][ty * 8 + i]);
-        const double2 bv = *reinterpret_cast<const double2*>(&Bs[k][tx * 8 + i]);
-        a[i] = av.x;
-        a[i + 1] = av.y;
-        b[i] = bv.x;
-        b[i + 1] = bv.y;
-      }
+      for (int j = 0; j < Cfg::kFN; ++j) b[j] = Bs[swz(wn0 + 8 * j + fg, k4 + ft)];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < Cfg::kFM; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < Cfg::kFN; ++j) dmma(acc[i][j][0], acc[i][j][1], a[i], b[j]);
     }
   }
+  cp_async_wait<0>();
+
+  // lane holds C rows wm0 + 8 i + fg, columns wn0 + 8 j + 2 ft + {0, 1}
+  const int64_t MN = static_cast<int64_t>(g.M) * g.N;
+  double* P = splits > 1 ? g.scratch + sp * MN : nullptr;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int m = m0 + ty * 8 + i;
+  for (int i = 0; i < Cfg::kFM; ++i) {
+    const int m = m0 + wm0 + 8 * i + fg;
     if (m >= g.M) continue;
-    double* crow = g.C + static_cast<int64_t>(m) * g.ldc;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int n = n0 + tx * 8 + j;
-      if (n >= g.N || (g.lower && g.row0 + m < g.col0 + n)) continue;
-      crow[n] = (g.beta != 0.0 ? g.beta * crow[n] : 0.0) + g.alpha * acc[i][j];
+    for (int j = 0; j < Cfg::kFN; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = n0 + wn0 + 8 * j + 2 * ft + h;
+        if (n >= g.N) continue;
+        if (P != nullptr) {
+          P[static_cast<int64_t>(m) * g.N + n] = acc[i][j][h];
+        } else if (!(g.lower && m < n)) {
+          double* cp = g.C + static_cast<int64_t>(m) * g.ldc + n;
+          *cp = (g.beta != 0.0 ? g.beta * *cp : 0.0) + g.alpha * acc[i][j][h];
+        }
+      }
     }
   }
 }
 
+// C = beta C + alpha * (sum of the partial tiles, split 0 first).
+__global__ void __launch_bounds__(256) f64_splitk_reduce_kernel(F64Gemm g, int splits) {
+  if (g.skip != nullptr && *g.skip != 0) return;
+  const int64_t MN = static_cast<int64_t>(g.M) * g.N;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < MN;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int m = static_cast<int>(e / g.N), n = static_cast<int>(e % g.N);
+    if (g.lower && m < n) continue;
+    double sum = 0.0;
+    for (int s = 0; s < splits; ++s) sum += g.scratch[s * MN + e];
+    double* c = g.C + static_cast<int64_t>(m) * g.ldc + n;
+    *c = (g.beta != 0.0 ? g.beta * *c : 0.0) + g.alpha * sum;
+  }
+}
+
+template <int BT>
+int64_t tile_count(const F64Gemm& g) {
+  const int64_t tm = ceil_div(g.M, BT), tn = ceil_div(g.N, BT);
+  return g.lower ? tm * (tm + 1) / 2 : tm * tn;
+}
+
+template <int BT>
+hq_status launch_f64(const F64Gemm& g, int64_t tiles, int splits, cudaStream_t s) {
+  using Cfg = F64Cfg<BT>;
+  const int64_t ctas = tiles * splits;
+  if (ctas > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
+  HQ_CUDA_TRY(cudaFuncSetAttribute(f64_gemm_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   Cfg::kSmemBytes));
+  f64_gemm_kernel<BT><<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmemBytes, s>>>(g, splits);
+  HQ_LAUNCH_CHECK();
+  if (splits > 1) {
+    const int64_t MN = static_cast<int64_t>(g.M) * g.N;
+    const int64_t grid = std::min<int64_t>(ceil_div(MN, 256), kSMs * 8);
+    f64_splitk_reduce_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(g, splits);
+    HQ_LAUNCH_CHECK();
+  }
+  return HQ_OK;
+}
+
+// Number of contraction splits: at least `target_ctas` CTAs where possible, every split at
+// least four slices long, all partial tiles within the scratch.
+int choose_splits(const F64Gemm& g, int64_t tiles, int64_t target_ctas) {
+  if (g.scratch == nullptr || tiles >= target_ctas) return 1;
+  const int64_t avg_chunks = (g.Kred / kDK) / (g.tri != kTriNone ? 2 : 1);
+  int64_t sp = ceil_div(target_ctas, tiles);
+  sp = std::min<int64_t>(sp, std::max<int64_t>(1, avg_chunks / 4));
+  sp = std::min<int64_t>(sp, 16);
+  const int64_t MN = static_cast<int64_t>(g.M) * g.N;
+  sp = std::min<int64_t>(sp, g.scratch_elems / MN);
+  return static_cast<int>(std::max<int64_t>(sp, 1));
+}
+
+}  // namespace
+
 hq_status f64_gemm(const F64Gemm& g, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0) return HQ_OK;
-  const int64_t tiles = ceil_div(g.M, kDT) * ceil_div(g.N, kDT);
-  if (tiles > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
-  f64_gemm_kernel<<<static_cast<unsigned>(tiles), 256, 0, s>>>(g);
-  HQ_LAUNCH_CHECK();
-  return HQ_OK;
+  if (g.Kred % kDK != 0 || (g.lower && g.M != g.N)) return HQ_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(g.A) | reinterpret_cast<uintptr_t>(g.B)) % 16 != 0 || g.lda % 2 != 0 ||
+      g.ldb % 2 != 0)
+    return HQ_ERR_UNSUPPORTED;
+  // 128-wide tiles (one CTA per SM) when they fill the SMs at least once, else 64-wide (up to
+  // three per SM), split along the contraction when even those are too few
+  const int64_t t128 = tile_count<128>(g);
+  if (t128 >= kSMs) return launch_f64<128>(g, t128, 1, s);
+  const int64_t t64 = tile_count<64>(g);
+  return launch_f64<64>(g, t64, choose_splits(g, t64, 2 * kSMs), s);
 }
 
 }  // namespace hq

@@ -35,19 +35,26 @@ struct Tf32Gemm {
 hq_status tf32_gemm(const Tf32Gemm& g, cudaStream_t s);
 
 // gemm_f64.cu: C = beta C + alpha A B^T in fp64 on the CUDA cores
+enum F64Tri { kTriNone = 0, kTriAUpper = 1, kTriALower = 2, kTriBLower = 3 };
 struct F64Gemm {
   double* C;
   int64_t ldc;
-  int M, N, Kred;
+  int M, N, Kred;   // Kred a multiple of 16
   const double* A;  // A(m, k) = A[m * lda + k]
   int64_t lda;
   const double* B;  // B(n, k) = B[n * ldb + k]
   int64_t ldb;
   double alpha, beta;
-  int lower, row0, col0;
+  int lower;        // write only m >= n (M == N)
+  int tri;          // F64Tri: which operand is triangular (zero outside its triangle)
+  double* scratch;  // room for split-K partial tiles (may be NULL: no split)
+  int64_t scratch_elems;
   const int* skip;
 };
 hq_status f64_gemm(const F64Gemm& g, cudaStream_t s);
+
+// factor.cu: out[i] = 1 / d[i] by the leaf's Newton-Raphson reciprocal (for tests)
+hq_status launch_rcp_nr(const double* d, double* out, int64_t n, cudaStream_t s);
 
 // factor.cu: U (row-major, upper) and U^T (row-major, lower) of the damped Hessian, in fp32,
 // from an fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; U and U^T are written into

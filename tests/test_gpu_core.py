@@ -317,6 +317,57 @@ def test_rtn_bit_exact(hq, cuda_device, N, K, G):
 
 # ----------------------------------------------------------------------------- tf32 GEMM
 
+def test_leaf_pivot_reciprocal_within_two_ulp(hq, cuda_device):
+    """The leaf's Newton-Raphson reciprocal against the correctly rounded fp64 quotient, over
+    pivots spanning the normal range (log-uniform magnitudes)."""
+    g = _gen(77)
+    e = torch.rand(1 << 20, generator=g, device="cuda", dtype=torch.float64) * 1200.0 - 600.0
+    m = 1.0 + torch.rand(1 << 20, generator=g, device="cuda", dtype=torch.float64)
+    d = m * torch.exp2(e.round())
+    out = torch.empty_like(d)
+    hq.hq_debug_rcp_f64(d, out)
+    ref = 1.0 / d
+    torch.cuda.synchronize()
+    ulp = (ref.abs() * 2.0 ** -52)
+    err = ((out - ref).abs() / ulp).max().item()
+    assert err <= 2.0, err
+
+
+@pytest.mark.parametrize("M,N,Kred,lower,tri,split", [
+    (64, 64, 64, False, 0, False), (200, 136, 48, False, 0, True), (320, 192, 128, False, 3, True),
+    (1280, 1280, 1280, False, 1, True), (1280, 1280, 1280, False, 2, True), (1280, 1280, 1280, True, 0, True),
+    (2560, 2560, 2560, True, 0, False), (2560, 1280, 2560, False, 3, False)])
+def test_f64_gemm_against_fp64(hq, cuda_device, M, N, Kred, lower, tri, split):
+    """The factorisation's fp64 GEMM against torch's fp64 matmul, with its triangular-operand
+    skipping (on operands that are zero there), the lower mask and the split-K path (which
+    must also be bit-identical run to run)."""
+    g = _gen(M * 5 + N + tri)
+    A = torch.randn((M, Kred), generator=g, device="cuda", dtype=torch.float64)
+    B = torch.randn((N, Kred), generator=g, device="cuda", dtype=torch.float64)
+    if tri == 1:
+        A = A.triu()
+    elif tri == 2:
+        A = A.tril()
+    elif tri == 3:
+        B = B.tril()
+    C0 = torch.randn((M, N), generator=g, device="cuda", dtype=torch.float64)
+    scratch = torch.empty(16 * M * N, device="cuda", dtype=torch.float64) if split else None
+    C = C0.clone()
+    hq.hq_debug_f64_gemm(C, A, B, alpha=-1.0, beta=1.0, lower=lower, tri=tri, scratch=scratch)
+    C2 = C0.clone()
+    hq.hq_debug_f64_gemm(C2, A, B, alpha=-1.0, beta=1.0, lower=lower, tri=tri, scratch=scratch)
+    torch.cuda.synchronize()
+    assert torch.equal(C, C2)
+    ref = C0 - A @ B.T
+    got = C
+    if lower:
+        mask = torch.ones((M, N), dtype=torch.bool, device="cuda").tril()
+        assert torch.equal(got[~mask], C0[~mask])
+        got, ref = got[mask], ref[mask]
+    err = ((got - ref).norm() / ref.norm()).item()
+    assert err < 1e-13, err
+
+
 @pytest.mark.parametrize("split3", [True, False])
 @pytest.mark.parametrize("M,N,Kred,lower", [(128, 128, 32, False), (300, 200, 100, False), (5120, 384, 128, False),
                                              (640, 640, 512, True), (1, 7, 4, False)])
