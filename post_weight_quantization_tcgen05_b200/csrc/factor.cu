@@ -18,7 +18,7 @@
 // Every product takes both operands K-major (row-major [rows, contraction]), so X^T is kept
 // next to X (leaves write both, X21^T is copied by a tiled transpose).  Everything runs in fp64
 // (gemm_f64.cu for the products; each declares its triangular operand so that tiles skip the
-// zero part of the contraction).  Leaves are 64 x 64 blocks factored and inverted by one CTA
+// zero part of the contraction).  Leaves are 128 x 128 blocks factored and inverted by one CTA
 // (chol_inv_leaf_kernel).  Steps:
 //   1. lambda = damp * mean(diag H)            (fp64 reduction, one CTA)
 //   2. A = J (H + lambda I) J in fp64, lower triangle (tiled transpose of H's lower triangle)
@@ -31,7 +31,7 @@
 
 namespace hq {
 
-constexpr int kLeaf = 64;
+constexpr int kLeaf = 128;
 
 // ------------------------------------------------------------------------- 1. lambda
 
@@ -119,29 +119,98 @@ hq_status launch_rcp_nr(const double* d, double* out, int64_t n, cudaStream_t s)
   return HQ_OK;
 }
 
-// Factor the 64 x 64 lower block at A as L D L^T (unit L) by right-looking elimination, and
-// at the same time eliminate Y = L^-1 (unit lower); writes X = D^-1/2 Y = (L D^1/2)^-1, the
-// inverse of the Cholesky factor (zeros above the diagonal), and X^T.  fp64.  The lower
-// triangle of the leaf is cut into 136 tiles of 4 x 4; thread t < 136 owns tile t of both S and
-// Y, in registers.  Before step k, the owners publish column k of the Schur complement (with
-// zeros at rows <= k), row k of Y (zeros right of k) and 1 / d_k through double-buffered shared
-// memory; one barrier per step.  Because of those zeros every thread applies the same rank-1
-// update to all 32 of its elements without masks (the part of a tile the step does not touch
-// gets a zero factor).  Only the elements step k + 1 publishes (one column of the S tile, one
-// row of the Y tile) are updated before the barrier; the rest of step k's update is applied
-// after it, while step k + 1's shared-memory loads are in flight.  The step loop is unrolled by
-// four so that positions inside a tile are compile-time register indices.  Pivots are checked
-// once at the end (a bad pivot only produces values that are then discarded).
-constexpr int kLB = kLeaf;                                 // 64
-constexpr int kLeafTiles = (kLB / 4) * (kLB / 4 + 1) / 2;  // 136
-constexpr int kLeafThreads = 160;                          // 5 warps, one tile per thread
+// L D L^T of a symmetric 4 x 4 block given by its lower part s (row-major 4 x 4; only
+// s[r][c], c <= r, read): pivots d, the strict lower part m of L^-1 (m10 m20 m30 m21 m31 m32)
+// and w = S^-1 (row-major 4 x 4, both triangles).
+__device__ __forceinline__ void ldl4_inverse(const double (&s)[16], double (&d)[4], double (&m)[6],
+                                             double (&w)[16]) {
+  d[0] = s[0];
+  const double r0 = rcp_nr(d[0]);
+  const double l10 = s[4] * r0, l20 = s[8] * r0, l30 = s[12] * r0;
+  d[1] = fma(-l10, s[4], s[5]);
+  const double r1 = rcp_nr(d[1]);
+  const double t21 = fma(-l20, s[4], s[9]), t31 = fma(-l30, s[4], s[13]);
+  const double l21 = t21 * r1, l31 = t31 * r1;
+  d[2] = fma(-l21, t21, fma(-l20, s[8], s[10]));
+  const double r2 = rcp_nr(d[2]);
+  const double t32 = fma(-l31, t21, fma(-l30, s[8], s[14]));
+  const double l32 = t32 * r2;
+  d[3] = fma(-l32, t32, fma(-l31, t31, fma(-l30, s[12], s[15])));
+  const double r3 = rcp_nr(d[3]);
+  // M = L^-1 (unit lower)
+  const double m10 = -l10, m21 = -l21, m32 = -l32;
+  const double m20 = -fma(l21, m10, l20);
+  const double m31 = -fma(l32, m21, l31);
+  const double m30 = -fma(l32, m20, fma(l31, m10, l30));
+  m[0] = m10; m[1] = m20; m[2] = m30; m[3] = m21; m[4] = m31; m[5] = m32;
+  // W = M^T D^-1 M: W[a][b] = sum_{k >= max(a, b)} M[k][a] M[k][b] / d_k
+  const double w33 = r3, w32 = r3 * m32, w31 = r3 * m31, w30 = r3 * m30;
+  const double q2 = r2 * m21, q3 = r3 * m32;  // reused products
+  const double w22 = fma(q3, m32, r2);
+  const double w21 = fma(q3, m31, q2);
+  const double w20 = fma(q3, m30, r2 * m20);
+  const double w11 = fma(r3 * m31, m31, fma(q2, m21, r1));
+  const double w10 = fma(r3 * m31, m30, fma(q2, m20, r1 * m10));
+  const double w00 = fma(r3 * m30, m30, fma(r2 * m20, m20, fma(r1 * m10, m10, r0)));
+  w[0] = w00; w[1] = w10; w[2] = w20; w[3] = w30;
+  w[4] = w10; w[5] = w11; w[6] = w21; w[7] = w31;
+  w[8] = w20; w[9] = w21; w[10] = w22; w[11] = w32;
+  w[12] = w30; w[13] = w31; w[14] = w32; w[15] = w33;
+}
 
-__device__ __forceinline__ void leaf_tile(int idx, int& ti, int& tj) {
-  int r = static_cast<int>((sqrtf(8.f * idx + 1.f) - 1.f) * 0.5f);
-  while (r * (r + 1) / 2 > idx) --r;
-  while ((r + 1) * (r + 2) / 2 <= idx) ++r;
-  ti = r;
-  tj = idx - r * (r + 1) / 2;
+// X = L^-1 and X^T for the 128 x 128 lower block at A, where A = L L^T (Cholesky), by blocked
+// right-looking elimination with 4 x 4 pivot blocks, in one CTA of 16 warps.  fp64.  The Schur
+// complement S and Y (the block elimination of the identity) live in shared memory as the 136
+// lower 8 x 8 tiles of each; warp I owns tile row I of both.  Block step kt (pivot block
+// B = rows/columns 4kt .. 4kt+3), with the panel P = S[:, B] read with zeros at rows <= 4kt+3
+// and W = S_BB^-1 = L_B^-T D_B^-1 L_B^-1 (computed in the previous step):
+//   warp I computes G_I = P_I W (one fp64 MMA) and then updates its tiles, one fp64 MMA
+//   (m8n8k4) per 8 x 8 tile:  S[I][J] -= G_I P_J^T (right of B),  Y[I][J] -= G_I Y[B][J] (left);
+//   the warp owning the next pivot block's diagonal tile updates that tile first and computes
+//   the next W (and keeps D_B, L_B^-1) while the others go on; one barrier per block step.
+// Rows of Y in block B are final once B is eliminated, up to L_B^-1 and D_B^-1/2:
+// X[B][j] = D_B^-1/2 L_B^-1 Y[B][j], applied at the end.  Pivots (the entries of D) are checked
+// at the end (a bad pivot only produces values that are then discarded).
+constexpr int kLB = kLeaf;                    // 128
+constexpr int kLT = kLB / 8;                  // 16 tile rows, one per warp
+constexpr int kLTiles = kLT * (kLT + 1) / 2;  // 136
+constexpr int kLeafThreads = 32 * kLT;
+constexpr size_t kLeafSmem = (2 * kLTiles * 64 + 2 * 16 + kLB + (kLB / 4) * 6) * sizeof(double);
+
+// Element (r, c) of lower tile (I, J): tiles row by row, 64 doubles each, the two 4-column
+// halves of rows 2, 3, 6, 7 swapped (fragment loads of 8 rows x 4 columns and of 4 rows x 8
+// columns then hit distinct banks in each half-warp; 16-byte pairs stay contiguous).
+__device__ __forceinline__ int lt_idx(int I, int J, int r, int c) {
+  return (I * (I + 1) / 2 + J) * 64 + r * 8 + (c ^ (((r >> 1) & 1) << 2));
+}
+
+// D (8 x 8) += A (8 x 4) B (4 x 8): lane (g = lane / 4, t = lane % 4) holds A[g][t], B[t][g] and
+// D[g][2t], D[g][2t + 1].
+__device__ __forceinline__ void dmma_leaf(double& d0, double& d1, double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+      : "+d"(d0), "+d"(d1)
+      : "d"(a), "d"(b));
+}
+
+// W, D, L^-1 of pivot block `blk` (rows 4 blk .. 4 blk + 3) from S in shared memory (every lane
+// of the calling warp computes them; lane 0 stores).
+__device__ __forceinline__ void leaf_block_inverse(const double* Ssm, int blk, double* wdst, double* dsm,
+                                                   double* msm, int lane) {
+  const int JB = blk >> 1, h = blk & 1;
+  double sd[16], d[4], m[6], w[16];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) sd[r * 4 + c] = (c <= r) ? Ssm[lt_idx(JB, JB, 4 * h + r, 4 * h + c)] : 0.0;
+  ldl4_inverse(sd, d, m, w);
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) wdst[q] = w[q];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dsm[4 * blk + q] = d[q];
+#pragma unroll
+    for (int q = 0; q < 6; ++q) msm[blk * 6 + q] = m[q];
+  }
 }
 
 __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const double* __restrict__ A, int64_t lda,
@@ -149,136 +218,163 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
                                                                          double* __restrict__ XT, int64_t ldx,
                                                                          int* __restrict__ info, int diag_off) {
   if (*info != 0) return;
-  __shared__ __align__(16) double colbuf[2][kLB];
-  __shared__ __align__(16) double yrow[2][kLB];
-  __shared__ double pinv[2];
-  __shared__ double dbuf[kLB];
+  extern __shared__ __align__(16) double lsm[];
+  double* Ssm = lsm;                 // S tiles (later X)
+  double* Ysm = Ssm + kLTiles * 64;  // Y tiles
+  double* wsm = Ysm + kLTiles * 64;  // W of the current and of the next block, 4 x 4 each
+  double* dsm = wsm + 2 * 16;        // pivots
+  double* msm = dsm + kLB;           // strict lower part of L_B^-1 per block (6 each)
   __shared__ int bad;
-  const int t = threadIdx.x;
-  const bool own = t < kLeafTiles;
-  int ti, tj;
-  leaf_tile(own ? t : 0, ti, tj);
-  const int i0 = 4 * ti, j0 = 4 * tj;
-  double v[16], y[16];
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int fg = lane / 4, ft = lane % 4;
+
+  // S = lower part of A, Y = I (all loads of a thread in flight together)
+#pragma unroll 1
+  for (int u0 = 0; u0 < kLB * kLB / kLeafThreads; u0 += 16) {
+    double vals[16];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      v[r * 4 + c] = (own && j0 + c <= i0 + r) ? A[(i0 + r) * lda + j0 + c] : 0.0;
-      y[r * 4 + c] = (own && i0 + r == j0 + c) ? 1.0 : 0.0;
+    for (int u = 0; u < 16; ++u) {
+      const int e = tid + kLeafThreads * (u0 + u), i = e / kLB, j = e % kLB;
+      vals[u] = (j <= i) ? A[static_cast<int64_t>(i) * lda + j] : 0.0;
     }
-  if (t < kLB) {
-    colbuf[0][t] = colbuf[1][t] = 0.0;
-    yrow[0][t] = yrow[1][t] = 0.0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int e = tid + kLeafThreads * (u0 + u), i = e / kLB, j = e % kLB;
+      if (j / 8 > i / 8) continue;  // tile above the diagonal: not stored
+      Ssm[lt_idx(i / 8, j / 8, i % 8, j % 8)] = vals[u];
+      Ysm[lt_idx(i / 8, j / 8, i % 8, j % 8)] = (i == j) ? 1.0 : 0.0;
+    }
   }
-  if (t == 0) bad = kLB;
+  if (tid == 0) bad = kLB;
   __syncthreads();
-  // publish column 0 (rows > 0), row 0 of Y and 1 / d_0
-  if (own && tj == 0) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) colbuf[0][i0 + r] = (ti > 0 || r > 0) ? v[r * 4] : 0.0;
-  }
-  if (own && ti == 0) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) yrow[0][j0 + c] = y[c];
-    pinv[0] = rcp_nr(v[0]);
-  }
+  if (warp == 0) leaf_block_inverse(Ssm, 0, wsm, dsm, msm, lane);
   __syncthreads();
 
-  // factors of the previous step, whose update is finished at the start of this one
-  double pa[4] = {0.0, 0.0, 0.0, 0.0}, pb[4] = {0.0, 0.0, 0.0, 0.0}, pyb[4] = {0.0, 0.0, 0.0, 0.0};
+  const int I = warp;
   for (int kt = 0; kt < kLB / 4; ++kt) {
-#pragma unroll
-    for (int kc = 0; kc < 4; ++kc) {
-      const int buf = kc & 1;  // == k & 1
-      const bool last = (kt == kLB / 4 - 1) && kc == 3;
-      // step k - 1's update, except column kc of S and row kc of Y (done before its barrier)
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c != kc) v[r * 4 + c] = fma(-pa[r], pb[c], v[r * 4 + c]);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (r == kc) continue;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) y[r * 4 + c] = fma(-pa[r], pyb[c], y[r * 4 + c]);
+    const int JB = kt >> 1, h = kt & 1;
+    const int J0 = JB + h;        // first tile row / column with an element beyond the pivot block
+    const int lim = 4 * kt + 3;   // rows <= lim have no part in the update
+    const int JBn = (kt + 1) >> 1;  // diagonal tile of the next pivot block
+    if (I >= J0) {
+      // -G_I = -P_I W: A = P_I (8 x 4, zero at rows <= lim), B = W padded to 4 x 8
+      double a;
+      {
+        const double p = (8 * I + fg > lim) ? Ssm[lt_idx(I, JB, fg, 4 * h + ft)] : 0.0;
+        const double wv = (fg < 4) ? wsm[(kt & 1) * 16 + ft * 4 + fg] : 0.0;  // W[t][g]
+        double g0 = 0.0, g1 = 0.0;
+        dmma_leaf(g0, g1, p, wv);
+        const int src = 4 * fg + (ft >> 1);  // lane holding G[g][t]
+        const double x0 = __shfl_sync(0xffffffffu, g0, src), x1 = __shfl_sync(0xffffffffu, g1, src);
+        a = -((ft & 1) ? x1 : x0);
       }
-      if (last) break;  // pivot 63 updates nothing: no row lies below it
-      const double inv_d = pinv[buf];
-      const double2 ca0 = *reinterpret_cast<const double2*>(&colbuf[buf][i0]);
-      const double2 ca1 = *reinterpret_cast<const double2*>(&colbuf[buf][i0 + 2]);
-      const double2 cb0 = *reinterpret_cast<const double2*>(&colbuf[buf][j0]);
-      const double2 cb1 = *reinterpret_cast<const double2*>(&colbuf[buf][j0 + 2]);
-      const double2 yb0 = *reinterpret_cast<const double2*>(&yrow[buf][j0]);
-      const double2 yb1 = *reinterpret_cast<const double2*>(&yrow[buf][j0 + 2]);
-      // L[i][k] (zero at and above the pivot), S[j][k] (zero at and left of it), Y[k][j]
-      const double a[4] = {ca0.x * inv_d, ca0.y * inv_d, ca1.x * inv_d, ca1.y * inv_d};
-      const double b[4] = {cb0.x, cb0.y, cb1.x, cb1.y};
-      const double yb[4] = {yb0.x, yb0.y, yb1.x, yb1.y};
-
-      // elements published for step k + 1: column k + 1 of S, row k + 1 of Y, d_{k+1}
-      const int ktn = (kc == 3) ? kt + 1 : kt;
-      const int cn = (kc + 1) & 3;
-      const int nb = buf ^ 1;
+      // S[I][J] -= G_I P_J^T for J0 <= J <= I.  The next pivot block's diagonal tile is
+      // (J0, J0) (J0 == JBn): its warp has no other S tile and computes the next W right after.
+      // Tiles go four at a time: loads, then MMAs, then stores.
+      const bool next_w = (I == JBn) && (kt + 1 < kLB / 4);
+      for (int J1 = J0; J1 <= I; J1 += 4) {
+        double b[4];
+        double2 cv[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) v[r * 4 + cn] = fma(-a[r], b[cn], v[r * 4 + cn]);
+        for (int u = 0; u < 4; ++u) {
+          const int J = J1 + u;
+          b[u] = 0.0;
+          cv[u] = make_double2(0.0, 0.0);
+          if (J > I) continue;
+          b[u] = (8 * J + fg > lim) ? Ssm[lt_idx(J, JB, fg, 4 * h + ft)] : 0.0;  // P_J[g][t]
+          cv[u] = *reinterpret_cast<const double2*>(&Ssm[lt_idx(I, J, fg, 2 * ft)]);
+        }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) y[cn * 4 + c] = fma(-a[cn], yb[c], y[cn * 4 + c]);
-      if (own && tj == ktn) {
+        for (int u = 0; u < 4; ++u) dmma_leaf(cv[u].x, cv[u].y, a, b[u]);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) colbuf[nb][i0 + r] = (ti > ktn || r > cn) ? v[r * 4 + cn] : 0.0;
-        // a new tile column: the last row of the previous diagonal tile still holds a value in
-        // this buffer (published two steps ago)
-        if (cn == 0 && ti == ktn) colbuf[nb][i0 - 1] = 0.0;
+        for (int u = 0; u < 4; ++u) {
+          const int J = J1 + u;
+          if (J <= I && !(J == JB && h == 0 && ft < 2))  // B's own columns stay
+            *reinterpret_cast<double2*>(&Ssm[lt_idx(I, J, fg, 2 * ft)]) = cv[u];
+        }
       }
-      if (own && ti == ktn) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) yrow[nb][j0 + c] = y[cn * 4 + c];
-        if (tj == ktn) pinv[nb] = rcp_nr(v[cn * 4 + cn]);
+      if (next_w) {
+        __syncwarp();
+        leaf_block_inverse(Ssm, kt + 1, wsm + ((kt + 1) & 1) * 16, dsm, msm, lane);
       }
+      // Y[I][J] -= G_I Y[B][J] for J <= JB
+      for (int J1 = 0; J1 <= JB; J1 += 4) {
+        double b[4];
+        double2 cv[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        pa[r] = a[r];
-        pb[r] = b[r];
-        pyb[r] = yb[r];
+        for (int u = 0; u < 4; ++u) {
+          const int J = J1 + u;
+          b[u] = 0.0;
+          cv[u] = make_double2(0.0, 0.0);
+          if (J > JB) continue;
+          b[u] = Ysm[lt_idx(JB, J, 4 * h + ft, fg)];  // Y[B][8J + g], row t
+          cv[u] = *reinterpret_cast<const double2*>(&Ysm[lt_idx(I, J, fg, 2 * ft)]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dmma_leaf(cv[u].x, cv[u].y, a, b[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int J = J1 + u;
+          if (J <= JB && !(I == JB && h == 0 && fg < 4))  // B's own rows stay
+            *reinterpret_cast<double2*>(&Ysm[lt_idx(I, J, fg, 2 * ft)]) = cv[u];
+        }
       }
-      __syncthreads();
     }
+    __syncthreads();
   }
-  // pivots d_i (the diagonal of S when it was eliminated); the first bad one fails the leaf
-  if (own && ti == tj) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const double d = v[r * 4 + r];
-      dbuf[i0 + r] = d;
-      if (!(d >= 2.2250738585072014e-308) || !isfinite(d)) atomicMin(&bad, i0 + r);  // not normal, > 0
-    }
+  // pivots; the first bad one fails the leaf
+  if (tid < kLB) {
+    const double dd = dsm[tid];
+    if (!(dd >= 2.2250738585072014e-308) || !isfinite(dd)) atomicMin(&bad, tid);  // not normal, > 0
   }
   __syncthreads();
   if (bad < kLB) {
-    if (t == 0) atomicCAS(info, 0, diag_off + bad + 1);
+    if (tid == 0) atomicCAS(info, 0, diag_off + bad + 1);
     return;
   }
-  if (!own) return;
-  // X[i][j] = Y[i][j] / sqrt(d_i)
+  // X tile (I, J) = C_I Y tile (I, J), with C_I = diag(D_b^-1/2 L_b^-1, D_b'^-1/2 L_b'^-1) the
+  // block-diagonal 8 x 8 matrix of tile row I's two pivot blocks (two fp64 MMAs per tile);
+  // written to X (row-major) and X^T straight from the fragments.  Elements above the diagonal
+  // come out zero, as X and X^T already hold there.
+  double* csm = Ssm;  // (S is no longer needed) row i: the 4 coefficients of its block's row
+  {
+    const int i = tid;  // row i of the leaf, block i / 4, row r = i % 4 of that block
+    if (i < kLB) {
+      const double dl = dsm[i];
+      double mv[6];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const double sc = 1.0 / sqrt(dbuf[i0 + r]);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) y[r * 4 + c] *= sc;
+      for (int q = 0; q < 6; ++q) mv[q] = msm[(i / 4) * 6 + q];
+      const int r = i % 4;
+      const double sc = 1.0 / sqrt(dl);
+      // row r of L_b^-1: (m10 m20 m30 m21 m31 m32) = M[1][0] M[2][0] M[3][0] M[2][1] M[3][1] M[3][2]
+      const double c0 = r == 0 ? 1.0 : (r == 1 ? mv[0] : (r == 2 ? mv[1] : mv[2]));
+      const double c1 = r == 1 ? 1.0 : (r == 2 ? mv[3] : (r == 3 ? mv[4] : 0.0));
+      const double c2 = r == 2 ? 1.0 : (r == 3 ? mv[5] : 0.0);
+      const double c3 = r == 3 ? 1.0 : 0.0;
+      csm[i * 4 + 0] = c0 * sc;
+      csm[i * 4 + 1] = c1 * sc;
+      csm[i * 4 + 2] = c2 * sc;
+      csm[i * 4 + 3] = c3 * sc;
+    }
+    __syncthreads();
   }
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    double* xr = X + static_cast<int64_t>(i0 + r) * ldx + j0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) xr[c] = y[r * 4 + c];
-  }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    double* xr = XT + static_cast<int64_t>(j0 + c) * ldx + i0;
-#pragma unroll
-    for (int r = 0; r < 4; ++r) xr[r] = y[r * 4 + c];
+  for (int T = warp; T < kLTiles; T += kLT) {
+    int TI = static_cast<int>((sqrtf(8.f * T + 1.f) - 1.f) * 0.5f);
+    if (TI * (TI + 1) / 2 > T) --TI;
+    if ((TI + 1) * (TI + 2) / 2 <= T) ++TI;
+    const int TJ = T - TI * (TI + 1) / 2;
+    // k = 0..3 (rows 0..3 of the Y tile) feed output rows 0..3; k = 4..7 feed rows 4..7
+    const double a0 = (fg < 4) ? csm[(8 * TI + fg) * 4 + ft] : 0.0;
+    const double a1 = (fg >= 4) ? csm[(8 * TI + fg) * 4 + ft] : 0.0;
+    const double b0 = Ysm[lt_idx(TI, TJ, ft, fg)];      // Y[8TI + t][8TJ + g]
+    const double b1 = Ysm[lt_idx(TI, TJ, 4 + ft, fg)];  // Y[8TI + 4 + t][8TJ + g]
+    double x0 = 0.0, x1 = 0.0;
+    dmma_leaf(x0, x1, a0, b0);
+    dmma_leaf(x0, x1, a1, b1);
+    const int i = 8 * TI + fg, j = 8 * TJ + 2 * ft;
+    *reinterpret_cast<double2*>(&X[static_cast<int64_t>(i) * ldx + j]) = make_double2(x0, x1);
+    XT[static_cast<int64_t>(j) * ldx + i] = x0;
+    XT[static_cast<int64_t>(j + 1) * ldx + i] = x1;
   }
 }
 
@@ -340,7 +436,7 @@ __global__ void __launch_bounds__(256) transpose_kernel(const double* __restrict
 static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tmp) {
   const int64_t K = c.K;
   if (n == kLeaf) {
-    chol_inv_leaf_kernel<<<1, kLeafThreads, 0, c.s>>>(c.A + off * K + off, K, c.X + off * K + off,
+    chol_inv_leaf_kernel<<<1, kLeafThreads, kLeafSmem, c.s>>>(c.A + off * K + off, K, c.X + off * K + off,
                                                       c.XT + off * K + off, K, c.info, static_cast<int>(off));
     HQ_LAUNCH_CHECK();
     return HQ_OK;
@@ -397,6 +493,8 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
                         double* lam, int* info, int* status, float** Ut, float** U, cudaStream_t s) {
   (void)status;
   if (K % kLeaf != 0) return HQ_ERR_UNSUPPORTED;
+  HQ_CUDA_TRY(cudaFuncSetAttribute(chol_inv_leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(kLeafSmem)));
   damp_stats_kernel<<<1, 1024, 0, s>>>(H, K, damp, lam, info);
   HQ_LAUNCH_CHECK();
   {
