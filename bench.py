@@ -179,21 +179,27 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
+    for w in range(args.warmup):
+        if w == args.warmup - 1:  # creates the timing events of the dominant kernel before the timed region
+            hq.hq_debug_timing_start([DOMINANT])
         layer.step()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, each bracketed by events, L2 flushed between steps
+    # ---- timed region: K steps, each bracketed by events, L2 flushed between steps; the library
+    #      records events around every launch of the dominant kernel on its own stream
     n_ev = 5
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     launches0 = hq.hq_debug_launch_count()
     _barrier(world)
     torch.cuda.synchronize()
+    hq.hq_debug_timing_start([DOMINANT])
     with ClockSampler(local_rank) as clk:
         for k in range(args.steps):
             flush.fill_(k & 0xFF)
             layer.step(stage_events=evs[k])
         torch.cuda.synchronize()
+    hq.hq_debug_timing_stop()
+    dom = hq.hq_debug_timing_read(DOMINANT)
     _barrier(world)
     launches = (hq.hq_debug_launch_count() - launches0) // max(args.steps, 1)
     step_ms = [e[0].elapsed_time(e[4]) for e in evs]
@@ -208,6 +214,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- e2e: same calls, inputs from pinned host memory, results copied back
     e2e = None if args.no_e2e else measure_e2e(args, layer, flush, world)
+    # ---- per-kernel breakdown (outside the timed region: events around every launch)
+    kernels = kernel_breakdown(hq, layer, flush)
     peaks = _peaks()
     syrk_flop = cfg.T * cfg.K * (cfg.K + 1)
     syrk_avg_s = statistics.mean(syrk_ms) / 1e3
@@ -216,10 +224,76 @@ def run_ours(args, rank, world, local_rank):
     dec_bytes = hq.hq_bf16tril_bytes(cfg.K) + 4 * cfg.K * cfg.K
     clocks = clk.summary()
     return_line = build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops,
-                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks)
+                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks, dom, kernels,
+                             fp64_mma_peak(hq))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         return_line["cpu_baseline"] = cpu_baseline(cfg, layer)
     return return_line
+
+
+# The kernel with the largest share of a step (ncu launch list of this benchmark) and the others
+# reported in the breakdown, with the unit of their algorithmic work.
+DOMINANT = "f64_gemm_128"
+KERNEL_NAMES = {"f64_gemm_128": ("f64_gemm_kernel<128>", "TFLOP/s"),
+                "f64_gemm_64": ("f64_gemm_kernel<64> + split-K reduce", "TFLOP/s"),
+                "leaf": ("chol_inv_leaf_kernel", "TFLOP/s"),
+                "sweep": ("sweep_block_kernel", "GB/s"),
+                "tf32_gemm": ("tf32_gemm_kernel (3xTF32 lazy updates)", "TFLOP/s"),
+                "syrk": ("umma_gemm_kernel<kSyrkBF16>", "TFLOP/s")}
+# fp64 tensor-core peak: no measured figure exists for fp64, so the measured bf16 burst is scaled
+# by NVIDIA's nominal dense ratio for B200 (fp64 tensor 37 TFLOP/s : bf16 2250 TFLOP/s)
+FP64_OVER_BF16 = 37.0 / 2250.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "f64_gemm_kernel_128_q_proj.md")
+KERNEL_SOURCE = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "csrc", "gemm_f64.cu")
+
+
+def kernel_breakdown(hq, layer, flush, steps: int = 2):
+    """Per kernel class: device time and achieved rate over `steps` steps, every launch timed."""
+    hq.hq_debug_timing_start(list(KERNEL_NAMES))
+    layer.step()  # creates the events
+    torch.cuda.synchronize()
+    hq.hq_debug_timing_start(list(KERNEL_NAMES))
+    for k in range(steps):
+        flush.fill_(k & 0xFF)
+        layer.step()
+    torch.cuda.synchronize()
+    hq.hq_debug_timing_stop()
+    out = {}
+    for cls, (name, unit) in KERNEL_NAMES.items():
+        ms, work, n = hq.hq_debug_timing_read(cls)
+        if n == 0:
+            continue
+        scale = 1e12 if unit == "TFLOP/s" else 1e9
+        out[cls] = {"kernel": name, "ms_per_step": ms / steps, "launches_per_step": n / steps,
+                    "achieved": work / (ms / 1e3) / scale, "unit": unit}
+    return out
+
+
+def fp64_mma_peak(hq):
+    """fp64 MMA rate of a kernel doing nothing else (context for the fp64 roofline)."""
+    try:
+        return hq.hq_debug_fp64_mma_rate()
+    except Exception:
+        return None
+
+
+def profiled_traffic():
+    """dram bytes per launch of the dominant kernel from the committed ncu summary, or None when
+    the kernel's source has changed since that capture."""
+    import hashlib
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    with open(KERNEL_SOURCE, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    vals = {}
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha256")):
+                k, v = line.strip().split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != sha or "traffic_bytes_per_launch" not in vals:
+        return None
+    return float(vals["traffic_bytes_per_launch"])
 
 
 def measure_e2e(args, layer, flush, world):
@@ -264,7 +338,19 @@ def measure_e2e(args, layer, flush, world):
 
 
 def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops, enc_bytes,
-               dec_bytes, peaks, e2e, launches, clocks):
+               dec_bytes, peaks, e2e, launches, clocks, dom, kernels, fp64_peak_measured):
+    dom_ms, dom_flop, dom_n = dom
+    achieved = dom_flop / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
+    peak = peaks["bf16_tflops"] * FP64_OVER_BF16
+    roofline = {"kernel": KERNEL_NAMES[DOMINANT][0] + " (fp64 MMA, factorisation products)", "bound": "tensor",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak if achieved is not None else None, "traffic": profiled_traffic(),
+                "launches_per_step": dom_n / max(args.steps, 1), "ms_per_step": dom_ms / max(args.steps, 1),
+                "peak_source": (f"{peaks['source']} bf16 dense burst {peaks['bf16_tflops']} TFLOP/s x nominal "
+                                f"fp64-tensor/bf16 ratio 37/2250"),
+                "fp64_mma_rate_measured": fp64_peak_measured,
+                "frac_of_measured_fp64_mma": (achieved / fp64_peak_measured
+                                              if achieved is not None and fp64_peak_measured else None)}
     line = {
         "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
         "value": value,
@@ -276,7 +362,7 @@ def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, d
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 in, fp32 compute (tcgen05 bf16 SYRK, tf32 trailing update)",
+        "dtype": "bf16 in; bf16 tcgen05 SYRK (fp32 accumulate), fp64 factorisation, fp32 sweep, 3xTF32 updates",
         "data": "synthetic (seeded; shapes and distributions of the q_proj-like layer)",
         "config": {"workload": f"{cfg.name}: W bf16 [{cfg.N}, {cfg.K}], X bf16 [{cfg.T}, {cfg.K}] "
                                f"({cfg.n_chunks} chunks of {cfg.chunk}), group {cfg.group}, damp {cfg.damp}",
@@ -286,10 +372,12 @@ def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, d
         "xtx_tflops": syrk_tflops,
         "codec_gbs": {"encode": enc_bytes / (statistics.mean(enc_ms) / 1e3) / 1e9,
                       "decode": dec_bytes / (statistics.mean(dec_ms) / 1e3) / 1e9},
-        "roofline": {"kernel": "umma_gemm_kernel<kSyrkBF16> (X^T X)", "bound": "tensor",
-                     "achieved": syrk_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": syrk_tflops / peaks["bf16_tflops"], "traffic": None,
-                     "peak_source": peaks["source"] + " bf16 dense burst"},
+        "roofline": roofline,
+        "kernels": kernels,
+        "syrk_roofline": {"kernel": "umma_gemm_kernel<kSyrkBF16> (X^T X)", "bound": "tensor",
+                          "achieved": syrk_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": syrk_tflops / peaks["bf16_tflops"],
+                          "peak_source": peaks["source"] + " bf16 dense burst"},
         "e2e": e2e,
         "gpu_launches": int(launches) * args.steps,
         "gpu_launches_per_step": int(launches),

@@ -74,6 +74,32 @@ hq_status hq_debug_f64_gemm(double* C, int64_t ldc, int M, int N, int Kred, cons
  */
 hq_status hq_debug_rcp_f64(const double* d, double* out, int64_t n, hq_stream_t stream);
 
+/*
+ * Event timing of kernel classes, for profiling from the caller's side.  While a class's bit
+ * is set in class_mask, every launch of that class records a CUDA event pair on its own
+ * stream, with the launch's algorithmic work: 0 = fp64 GEMM, 128-wide tiles (flops);
+ * 1 = fp64 GEMM, 64-wide tiles, including its split-K reduction (flops); 2 = factorisation
+ * leaf (flops of a 128 x 128 Cholesky and triangular inverse); 3 = GPTQ block sweep (bytes);
+ * 4 = tf32 lazy-update GEMM (flops of the product); 5 = tcgen05 SYRK (flops).
+ * hq_debug_timing_start clears the records and sets the mask; hq_debug_timing_read
+ * synchronises the recorded events and returns the sum of durations (ms), of work and the
+ * number of launches of one class; hq_debug_timing_stop clears the mask.  Events are created
+ * on first use and kept.  One process-wide record: not for concurrent use.  No counterpart
+ * on the pages.
+ */
+hq_status hq_debug_timing_start(int class_mask);
+hq_status hq_debug_timing_stop(void);
+hq_status hq_debug_timing_read(int kernel_class, double* ms_total, double* work_total, int64_t* launches);
+
+/*
+ * fp64 MMA (mma.sync m8n8k4 .f64) rate in TFLOP/s of a kernel that does nothing else (8
+ * independent accumulators per warp, two CTAs of 256 threads per SM), timed with CUDA events
+ * on `stream`; synchronises it.  `scratch`: device buffer of at least 296 * 256 * 8 bytes.
+ * Returns a negative value on failure.  Context for the fp64 GEMM's roofline; no counterpart
+ * on the pages.
+ */
+double hq_debug_fp64_mma_rate(void* scratch, int64_t scratch_bytes, hq_stream_t stream);
+
 /* Number of kernels libhq.so has launched in this process so far (all devices, all
  * threads).  A statistic for profiling; never reset. */
 uint64_t hq_debug_launch_count(void);

@@ -65,6 +65,10 @@ _SIGS = {
     "hq_debug_launch_count": (ctypes.c_uint64, []),
     "hq_debug_tf32_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _f, _f, _int, _int, _vp]),
     "hq_debug_rcp_f64": (_int, [_vp, _vp, _i64, _vp]),
+    "hq_debug_fp64_mma_rate": (ctypes.c_double, [_vp, _i64, _vp]),
+    "hq_debug_timing_start": (_int, [_int]),
+    "hq_debug_timing_stop": (_int, []),
+    "hq_debug_timing_read": (_int, [_int, _vp, _vp, _vp]),
     "hq_debug_f64_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _dbl, _dbl, _int, _int, _vp,
                                  _i64, _vp]),
 }
@@ -204,6 +208,38 @@ def hq_debug_tf32_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, split3=True, s
     _check(lib.hq_debug_tf32_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
                                   float(alpha), float(beta), int(bool(lower)), int(bool(split3)), _stream(stream)),
            "hq_debug_tf32_gemm")
+
+
+def hq_debug_fp64_mma_rate(stream=None) -> float:
+    """Measured fp64 MMA rate (TFLOP/s) of a kernel that does nothing else."""
+    scratch = torch.empty(296 * 256, dtype=torch.float64, device="cuda")
+    r = lib.hq_debug_fp64_mma_rate(_ptr(scratch), scratch.numel() * 8, _stream(stream))
+    if r < 0:
+        raise HQError(HQ_ERR_CUDA, "hq_debug_fp64_mma_rate")
+    return float(r)
+
+
+TIMING_CLASSES = {"f64_gemm_128": 0, "f64_gemm_64": 1, "leaf": 2, "sweep": 3, "tf32_gemm": 4, "syrk": 5}
+
+
+def hq_debug_timing_start(classes) -> None:
+    """Start event timing of the named kernel classes (see TIMING_CLASSES)."""
+    mask = 0
+    for c in classes:
+        mask |= 1 << TIMING_CLASSES[c]
+    _check(lib.hq_debug_timing_start(mask), "hq_debug_timing_start")
+
+
+def hq_debug_timing_stop() -> None:
+    _check(lib.hq_debug_timing_stop(), "hq_debug_timing_stop")
+
+
+def hq_debug_timing_read(cls: str):
+    """(total ms, total work, launches) recorded for one kernel class."""
+    ms, work, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_int64()
+    _check(lib.hq_debug_timing_read(TIMING_CLASSES[cls], ctypes.byref(ms), ctypes.byref(work), ctypes.byref(n)),
+           "hq_debug_timing_read")
+    return ms.value, work.value, n.value
 
 
 def hq_debug_rcp_f64(d, out, stream=None) -> None:

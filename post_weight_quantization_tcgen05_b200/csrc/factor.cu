@@ -436,9 +436,11 @@ __global__ void __launch_bounds__(256) transpose_kernel(const double* __restrict
 static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tmp) {
   const int64_t K = c.K;
   if (n == kLeaf) {
+    const int tm = timer_start(kTimeLeaf, c.s);
     chol_inv_leaf_kernel<<<1, kLeafThreads, kLeafSmem, c.s>>>(c.A + off * K + off, K, c.X + off * K + off,
                                                       c.XT + off * K + off, K, c.info, static_cast<int>(off));
     HQ_LAUNCH_CHECK();
+    timer_stop(tm, 2.0 * kLeaf * kLeaf * kLeaf / 3.0, c.s);  // Cholesky n^3/3 + triangular inverse n^3/3
     return HQ_OK;
   }
   const int64_t n1 = (n / kLeaf / 2) * kLeaf, n2 = n - n1;

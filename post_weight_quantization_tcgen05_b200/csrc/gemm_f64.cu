@@ -211,6 +211,22 @@ int64_t tile_count(const F64Gemm& g) {
   return g.lower ? tm * (tm + 1) / 2 : tm * tn;
 }
 
+// Algorithmic flops of a product: 2 per multiply-add that a triangular operand does not zero
+// (for `lower`, only the written elements count).
+double f64_gemm_flops(const F64Gemm& g) {
+  const double M = g.M, N = g.N, K = g.Kred;
+  auto tri_sum = [K](double n) {  // sum_{i < n} min(i + 1, K)
+    return n <= K ? n * (n + 1) / 2 : K * (K + 1) / 2 + (n - K) * K;
+  };
+  if (g.lower) return 2.0 * M * (M + 1) / 2 * K;
+  switch (g.tri) {
+    case kTriBLower: return 2.0 * M * tri_sum(N);
+    case kTriALower: return 2.0 * N * tri_sum(M);
+    case kTriAUpper: return 2.0 * N * (M <= K ? M * K - M * (M - 1) / 2 : K * (K + 1) / 2);  // sum max(K - m, 0)
+    default: return 2.0 * M * N * K;
+  }
+}
+
 template <int BT>
 hq_status launch_f64(const F64Gemm& g, int64_t tiles, int splits, cudaStream_t s) {
   using Cfg = F64Cfg<BT>;
@@ -218,6 +234,7 @@ hq_status launch_f64(const F64Gemm& g, int64_t tiles, int splits, cudaStream_t s
   if (ctas > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
   HQ_CUDA_TRY(cudaFuncSetAttribute(f64_gemm_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    Cfg::kSmemBytes));
+  const int tm = timer_start(BT == 128 ? kTimeF64Gemm128 : kTimeF64Gemm64, s);
   f64_gemm_kernel<BT><<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmemBytes, s>>>(g, splits);
   HQ_LAUNCH_CHECK();
   if (splits > 1) {
@@ -226,6 +243,7 @@ hq_status launch_f64(const F64Gemm& g, int64_t tiles, int splits, cudaStream_t s
     f64_splitk_reduce_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(g, splits);
     HQ_LAUNCH_CHECK();
   }
+  timer_stop(tm, f64_gemm_flops(g), s);
   return HQ_OK;
 }
 
@@ -258,4 +276,50 @@ hq_status f64_gemm(const F64Gemm& g, cudaStream_t s) {
   return launch_f64<64>(g, t64, choose_splits(g, t64, 2 * kSMs), s);
 }
 
+// fp64 MMA issue rate with nothing else in the way: each warp runs 8 independent accumulator
+// chains (the operands are registers; one store per thread at the end).
+__global__ void __launch_bounds__(256) fp64_mma_rate_kernel(double* out, int iters) {
+  double c0[8], c1[8];
+  const double a = 1.0 + threadIdx.x * 1e-9, b = 0.999999;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c0[i] = c1[i] = i * 1e-3;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dmma(c0[i], c1[i], a, b);
+  }
+  double acc = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc += c0[i] + c1[i];
+  out[blockIdx.x * blockDim.x + threadIdx.x] = acc;
+}
+
 }  // namespace hq
+
+using namespace hq;
+
+extern "C" double hq_debug_fp64_mma_rate(void* scratch, int64_t scratch_bytes, hq_stream_t stream) {
+  constexpr int kBlocks = 2 * kSMs, kThreads = 256, kIters = 20000;
+  if (scratch == nullptr || scratch_bytes < static_cast<int64_t>(kBlocks) * kThreads * 8) return -1.0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* out = static_cast<double*>(scratch);
+  fp64_mma_rate_kernel<<<kBlocks, kThreads, 0, s>>>(out, 100);  // warm-up
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) != cudaSuccess) return -1.0;
+  if (cudaEventCreate(&e1) != cudaSuccess) {
+    cudaEventDestroy(e0);
+    return -1.0;
+  }
+  cudaEventRecord(e0, s);
+  fp64_mma_rate_kernel<<<kBlocks, kThreads, 0, s>>>(out, kIters);
+  cudaEventRecord(e1, s);
+  float ms = 0.f;
+  const bool ok = cudaEventSynchronize(e1) == cudaSuccess && cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess;
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (!ok || ms <= 0.f) {
+    (void)cudaGetLastError();
+    return -1.0;
+  }
+  const double flops = 2.0 * 256 * 8 * static_cast<double>(kIters) * kBlocks * (kThreads / 32);
+  return flops / (ms * 1e-3) / 1e12;
+}

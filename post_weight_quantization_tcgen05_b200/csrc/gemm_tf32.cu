@@ -12,8 +12,10 @@ static hq_status launch_tf32(const CUtensorMap& ma, const CUtensorMap& mb, const
   using Cfg = Tf32Cfg<SPLIT3>;
   auto kern = tf32_gemm_kernel<SPLIT3>;
   HQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+  const int tm = timer_start(kTimeTf32Gemm, s);
   kern<<<tiles, Cfg::kThreads, Cfg::kSmemBytes, s>>>(ma, mb, a);
   HQ_LAUNCH_CHECK();
+  timer_stop(tm, 2.0 * a.M * a.N * static_cast<double>(a.Kred), s);  // the product's flops
   return HQ_OK;
 }
 

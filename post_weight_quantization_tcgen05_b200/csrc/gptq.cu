@@ -438,8 +438,13 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
     const int64_t p1 = (p0 + P < K) ? p0 + P : K;
     for (int64_t j0 = p0; j0 < p1; j0 += kBlk) {
       a.err_col = static_cast<int>(j0 - p0);
+      const int tm = timer_start(kTimeSweep, s);
       kern<<<L.sweep_grid, kSweepThreads, kSweepSmem, s>>>(a, static_cast<int>(j0));
       HQ_LAUNCH_CHECK();
+      // bytes: the block of working weights in, its errors out (fp32), the block of U^T, packed
+      // codes and the block's scales out
+      timer_stop(tm, static_cast<double>(N) * kBlk * 8.0 + kBlk * kBlk * 4.0 + N * (kBlk / 2.0) +
+                         N * (static_cast<double>(kBlk) / group) * 4.0, s);
       const int64_t j1 = j0 + kBlk;
       if (j1 < p1) {  // inner update of the rest of the panel
         st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), P, j0, kBlk, Ut, &hdr->info,

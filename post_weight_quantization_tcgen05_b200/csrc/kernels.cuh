@@ -34,7 +34,21 @@ struct Tf32Gemm {
 };
 hq_status tf32_gemm(const Tf32Gemm& g, cudaStream_t s);
 
-// gemm_f64.cu: C = beta C + alpha A B^T in fp64 on the CUDA cores
+// timing.cu: optional event timing of kernel classes (hq_debug_timing_*).  timer_start returns
+// -1 (and records nothing) unless the class is being timed; `work` is the launch's algorithmic
+// flops or bytes.
+enum TimerClass {
+  kTimeF64Gemm128 = 0,  // f64_gemm_kernel, 128-wide tiles (flops)
+  kTimeF64Gemm64 = 1,   // f64_gemm_kernel, 64-wide tiles, with its split-K reduction (flops)
+  kTimeLeaf = 2,        // chol_inv_leaf_kernel (flops of Cholesky + triangular inverse)
+  kTimeSweep = 3,       // sweep_block_kernel (bytes)
+  kTimeTf32Gemm = 4,    // tf32_gemm_kernel (flops of the product, not of its 3 passes)
+  kTimeSyrk = 5,        // tcgen05 SYRK (flops)
+};
+int timer_start(int cls, cudaStream_t s);
+void timer_stop(int idx, double work, cudaStream_t s);
+
+// gemm_f64.cu: C = beta C + alpha A B^T in fp64 on the fp64 tensor cores
 enum F64Tri { kTriNone = 0, kTriAUpper = 1, kTriALower = 2, kTriBLower = 3 };
 struct F64Gemm {
   double* C;

@@ -117,8 +117,10 @@ hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev
   a.Ncols = static_cast<int>(K);
   a.Kred = static_cast<int>(T);
   a.status = dev_status;
+  const int tm = timer_start(kTimeSyrk, s);
   umma_gemm_kernel<GemmMode::kSyrkBF16><<<static_cast<unsigned>(tiles), gemm_threads(GemmMode::kSyrkBF16), kGemmSmemBytes, s>>>(map, map, a);
   HQ_LAUNCH_CHECK();
+  timer_stop(tm, static_cast<double>(T) * K * (K + 1), s);  // 2 flops x T x K (K + 1) / 2 lower entries
   return HQ_OK;
 }
 

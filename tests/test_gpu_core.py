@@ -392,3 +392,26 @@ def test_tf32_gemm_against_fp64(hq, cuda_device, M, N, Kred, lower, split3):
     err = ((got - ref).norm() / ref.norm()).item()
     # 3xTF32: about 2^-21 per product; plain tf32 (mantissa truncated to 10 bits): about 2^-10
     assert err < (2e-6 if split3 else 2e-3), err
+
+
+def test_kernel_timing_records_every_launch(hq, cuda_device):
+    """The event timing of kernel classes sees each factorisation leaf once per 128 columns
+    and the algorithmic work it reports is the stated formula."""
+    K = 512
+    g = _gen(5)
+    X = torch.randn((1024, K), generator=g, device="cuda")
+    H = torch.zeros((K, K), device="cuda")
+    hq.hq_hessian_accumulate(H, X)
+    ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(1, K, 128))
+    Ut = torch.empty((K, K), device="cuda")
+    hq.hq_debug_timing_start(["leaf", "f64_gemm_128", "f64_gemm_64"])
+    hq.hq_debug_factor(H, 0.01, Ut, ws)
+    hq.hq_debug_timing_stop()
+    ms, work, n = hq.hq_debug_timing_read("leaf")
+    assert n == K // 128 and ms > 0.0
+    assert work == pytest.approx(n * 2.0 * 128 ** 3 / 3.0)
+    ms64, work64, n64 = hq.hq_debug_timing_read("f64_gemm_64")
+    assert n64 > 0 and ms64 > 0.0 and work64 > 0.0
+    # nothing is recorded once timing is stopped
+    hq.hq_debug_factor(H, 0.01, Ut, ws)
+    assert hq.hq_debug_timing_read("leaf")[2] == n
