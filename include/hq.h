@@ -105,7 +105,10 @@ size_t hq_gptq_workspace_bytes(int64_t N, int64_t K, int64_t group);
  *   workspace : device buffer of at least hq_gptq_workspace_bytes(N, K, group) bytes,
  *            256-byte aligned, owned by the caller, not shared with a concurrent call.
  * The call synchronises `stream` once at its end to read the factorisation status, and
- * returns HQ_ERR_NOT_PD if a Cholesky pivot was not positive.  codes and scales do not
+ * returns HQ_ERR_NOT_PD if a Cholesky pivot was not positive.  Part of the factorisation runs
+ * on a second stream that the library creates once per host thread and device (with a few
+ * events, kept for the thread's lifetime); it is joined back into `stream` before the call's
+ * later work, so ordering on `stream` is as if everything ran there.  codes and scales do not
  * depend on whether qerr is requested, and are identical run to run.
  */
 hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,

@@ -26,6 +26,8 @@
 //   4. U = J X J and U^T = J X^T J, both row-major (180-degree rotated copies)
 // A device flag `info` receives the first failing pivot (1-based, in M's order) and stops
 // every later kernel.
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -380,6 +382,32 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
 
 // ------------------------------------------------------------------------- 3b. recursion
 
+// A second stream per (host thread, device) for the work off the recursion's critical path,
+// and a pool of events for the dependencies between the two streams (created on first use,
+// kept for the thread's lifetime).
+struct SideStream {
+  cudaStream_t s2 = nullptr;
+  std::vector<cudaEvent_t> ev;
+  size_t used = 0;
+  ~SideStream() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    if (s2 != nullptr) cudaStreamDestroy(s2);
+  }
+};
+
+static hq_status side_stream(SideStream** out) {
+  constexpr int kMaxDevices = 64;
+  thread_local SideStream pool[kMaxDevices];
+  int dev = -1;
+  HQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
+  SideStream& ss = pool[dev];
+  if (ss.s2 == nullptr) HQ_CUDA_TRY(cudaStreamCreateWithFlags(&ss.s2, cudaStreamNonBlocking));
+  ss.used = 0;
+  *out = &ss;
+  return HQ_OK;
+}
+
 struct FactorCtx {
   double* A;
   double* X;
@@ -388,13 +416,27 @@ struct FactorCtx {
   int64_t K;
   int* info;
   int* status;
-  cudaStream_t s;
+  cudaStream_t s;   // the caller's stream: the critical path
+  SideStream* side;  // s2: Y^T products and transposes
 };
 
-// `scratch` (up to the end of the temporaries) receives split-K partial tiles.
-static hq_status gemm(const FactorCtx& c, double* scratch, double* C, int64_t ldc, int M, int N, int Kred,
-                      const double* A, int64_t lda, const double* B, int64_t ldb, double alpha, double beta,
-                      bool lower, int tri) {
+// `from` -> `to`: work enqueued on `to` from now on waits for everything enqueued on `from` so far.
+static hq_status stream_dep(SideStream* ss, cudaStream_t from, cudaStream_t to) {
+  if (ss->used == ss->ev.size()) {
+    cudaEvent_t e;
+    HQ_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    ss->ev.push_back(e);
+  }
+  cudaEvent_t e = ss->ev[ss->used++];
+  HQ_CUDA_TRY(cudaEventRecord(e, from));
+  HQ_CUDA_TRY(cudaStreamWaitEvent(to, e, 0));
+  return HQ_OK;
+}
+
+// `scratch` (up to the end of the temporaries; NULL: no split) receives split-K partial tiles.
+static hq_status gemm(const FactorCtx& c, cudaStream_t s, double* scratch, double* C, int64_t ldc, int M, int N,
+                      int Kred, const double* A, int64_t lda, const double* B, int64_t ldb, double alpha,
+                      double beta, bool lower, int tri) {
   F64Gemm g{};
   g.C = C;
   g.ldc = ldc;
@@ -410,9 +452,9 @@ static hq_status gemm(const FactorCtx& c, double* scratch, double* C, int64_t ld
   g.lower = lower ? 1 : 0;
   g.tri = tri;
   g.scratch = scratch;
-  g.scratch_elems = c.tmp_end - scratch;
+  g.scratch_elems = scratch == nullptr ? 0 : c.tmp_end - scratch;
   g.skip = c.info;
-  return f64_gemm(g, c.s);
+  return f64_gemm(g, s);
 }
 
 // dst[j][i] = src[i][j] for an R x C block (32 x 32 tiles through shared memory).
@@ -433,6 +475,10 @@ __global__ void __launch_bounds__(256) transpose_kernel(const double* __restrict
 
 // X = L^-1 and X^T for the n x n block of A at (off, off); `tmp` has room for the temporaries
 // of this level and all levels below (2 * n2 * n1 here, about a quarter of that per level below).
+// Critical path on c.s: left half, T, the Schur update, right half, X21.  Y^T (needs only T and
+// the left half) and the transpose of X21 run on the side stream, overlapping the right half's
+// leaves and small products; they take no split-K scratch (the region beyond this level's
+// temporaries belongs to the right half meanwhile).
 static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tmp) {
   const int64_t K = c.K;
   if (n == kLeaf) {
@@ -455,20 +501,27 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
   const double* X22 = c.X + (off + n1) * K + off + n1;
   double* XT12 = c.XT + off * K + off + n1;
   const int in1 = static_cast<int>(n1), in2 = static_cast<int>(n2);
+  cudaStream_t s2 = c.side->s2;
   hq_status st = chol_inv(c, off, n1, rest);
   if (st != HQ_OK) return st;
-  st = gemm(c, rest, T, n1, in2, in1, in1, A21, K, X11, K, 1.0, 0.0, false, kTriBLower);  // T = A21 X11^T
+  st = gemm(c, c.s, rest, T, n1, in2, in1, in1, A21, K, X11, K, 1.0, 0.0, false, kTriBLower);  // T = A21 X11^T
   if (st != HQ_OK) return st;
-  st = gemm(c, rest, A22, K, in2, in2, in1, T, n1, T, n1, -1.0, 1.0, true, kTriNone);     // A22 -= T T^T
+  st = stream_dep(c.side, c.s, s2);
+  if (st != HQ_OK) return st;
+  st = gemm(c, s2, nullptr, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.0, 0.0, false, kTriAUpper);  // Y^T = X11^T T^T
+  if (st != HQ_OK) return st;
+  st = gemm(c, c.s, rest, A22, K, in2, in2, in1, T, n1, T, n1, -1.0, 1.0, true, kTriNone);       // A22 -= T T^T
   if (st != HQ_OK) return st;
   st = chol_inv(c, off + n1, n2, rest);
   if (st != HQ_OK) return st;
-  st = gemm(c, rest, YT, n2, in1, in2, in1, XT11, K, T, n1, 1.0, 0.0, false, kTriAUpper); // Y^T = X11^T T^T
+  st = stream_dep(c.side, s2, c.s);  // Y^T
   if (st != HQ_OK) return st;
-  st = gemm(c, rest, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false, kTriALower); // X21 = -X22 Y
+  st = gemm(c, c.s, rest, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false, kTriALower);  // X21 = -X22 Y
+  if (st != HQ_OK) return st;
+  st = stream_dep(c.side, c.s, s2);
   if (st != HQ_OK) return st;
   const int64_t tiles = ceil_div(n2, 32) * ceil_div(n1, 32);
-  transpose_kernel<<<static_cast<unsigned>(tiles), 256, 0, c.s>>>(X21, K, n2, n1, XT12, K, c.info);
+  transpose_kernel<<<static_cast<unsigned>(tiles), 256, 0, s2>>>(X21, K, n2, n1, XT12, K, c.info);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
 }
@@ -506,9 +559,17 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   }
   HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(double), s));
   HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(double), s));
-  FactorCtx c{A, X, XT, T + K * K, K, info, status, s};
-  hq_status st = chol_inv(c, 0, K, T);
+  SideStream* side = nullptr;
+  hq_status st = side_stream(&side);
   if (st != HQ_OK) return st;
+  FactorCtx c{A, X, XT, T + K * K, K, info, status, s, side};
+  st = stream_dep(side, s, side->s2);  // the side stream starts after everything before this call
+  if (st != HQ_OK) return st;
+  st = chol_inv(c, 0, K, T);
+  // the caller's stream waits for the side stream's last work, also when enqueueing failed midway
+  const hq_status st_join = stream_dep(side, side->s2, s);
+  if (st != HQ_OK) return st;
+  if (st_join != HQ_OK) return st_join;
   // A is dead now: U^T and U (fp32) go into its storage
   *Ut = reinterpret_cast<float*>(A);
   *U = reinterpret_cast<float*>(A) + K * K;
