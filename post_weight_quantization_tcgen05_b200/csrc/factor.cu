@@ -530,22 +530,32 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
 
 // U[j][c] = X[K-1-j][K-1-c] and U^T[j][c] = X^T[K-1-j][K-1-c], rounded to fp32: 180-degree
 // rotations (U upper, U^T lower, zeros elsewhere because X and X^T hold zeros there).
+// With Ut_hi != NULL, also the strict lower part of U^T as a tf32 part (low 13 mantissa bits
+// cleared) plus the exact fp32 remainder, the operands of the 3xTF32 lazy updates.
 __global__ void rotate_kernel(const double* __restrict__ X, const double* __restrict__ XT, int64_t K,
-                              float* __restrict__ U, float* __restrict__ Ut, const int* __restrict__ info) {
+                              float* __restrict__ U, float* __restrict__ Ut, float* __restrict__ Ut_hi,
+                              float* __restrict__ Ut_lo, const int* __restrict__ info) {
   if (*info != 0) return;
   const int64_t n = K * K;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t src = n - 1 - e;  // (K-1-j)*K + (K-1-c) for e = j*K + c
     U[e] = static_cast<float>(X[src]);
-    Ut[e] = static_cast<float>(XT[src]);
+    const float ut = static_cast<float>(XT[src]);
+    Ut[e] = ut;
+    if (Ut_hi != nullptr && e % K < e / K) {
+      const float hi = __uint_as_float(__float_as_uint(ut) & 0xFFFFE000u);
+      Ut_hi[e] = hi;
+      Ut_lo[e] = ut - hi;
+    }
   }
 }
 
 // ------------------------------------------------------------------------- driver
 
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        double* lam, int* info, int* status, float** Ut, float** U, cudaStream_t s) {
+                        double* lam, int* info, int* status, float** Ut, float** U, bool split_ut, float** Ut_hi,
+                        float** Ut_lo, cudaStream_t s) {
   (void)status;
   if (K % kLeaf != 0) return HQ_ERR_UNSUPPORTED;
   HQ_CUDA_TRY(cudaFuncSetAttribute(chol_inv_leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -574,7 +584,12 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   *Ut = reinterpret_cast<float*>(A);
   *U = reinterpret_cast<float*>(A) + K * K;
   const int64_t grid = ceil_div(K * K, 4 * 256) < 148 * 32 ? ceil_div(K * K, 4 * 256) : 148 * 32;
-  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, *U, *Ut, info);
+  // the temporaries are dead too: the split U^T goes into their storage
+  float* hi = split_ut ? reinterpret_cast<float*>(T) : nullptr;
+  float* lo = split_ut ? reinterpret_cast<float*>(T) + K * K : nullptr;
+  if (Ut_hi != nullptr) *Ut_hi = hi;
+  if (Ut_lo != nullptr) *Ut_lo = lo;
+  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, *U, *Ut, hi, lo, info);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
 }

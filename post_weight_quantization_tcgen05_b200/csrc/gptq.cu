@@ -41,7 +41,8 @@ struct SweepArgs {
   int64_t N, K;
   const float* U;    // U row-major (upper triangular)
   int group;
-  float* Err;        // panel error buffer [N, P]
+  float* Err;        // panel error buffer [N, P] (the tf32 part when Err_lo is set)
+  float* Err_lo;     // NULL, or the fp32 remainder of each error (Err + Err_lo = error)
   int64_t err_ld;    // P
   int err_col;       // column of this block inside the panel buffer
   uint8_t* codes;
@@ -241,7 +242,18 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
   for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
     if (r0 + r >= a.N) break;
     const float* src = stage + r * LD + 4 * lane;
-    reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = make_float4(src[0], src[1], src[2], src[3]);
+    const float4 e4 = make_float4(src[0], src[1], src[2], src[3]);
+    if (a.Err_lo == nullptr) {
+      reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = e4;
+    } else {  // split for the 3xTF32 updates: tf32 part (low 13 mantissa bits cleared) + remainder
+      const float4 h4 = make_float4(__uint_as_float(__float_as_uint(e4.x) & 0xFFFFE000u),
+                                    __uint_as_float(__float_as_uint(e4.y) & 0xFFFFE000u),
+                                    __uint_as_float(__float_as_uint(e4.z) & 0xFFFFE000u),
+                                    __uint_as_float(__float_as_uint(e4.w) & 0xFFFFE000u));
+      reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = h4;
+      reinterpret_cast<float4*>(a.Err_lo + (r0 + r) * a.err_ld + a.err_col)[lane] =
+          make_float4(e4.x - h4.x, e4.y - h4.y, e4.z - h4.z, e4.w - h4.w);
+    }
     // lane writes bytes 2*lane, 2*lane+1 of the row's 64 code bytes
     const int8_t* cs = code_s + r * kBlk + 4 * lane;
     const uint32_t b0 = (cs[0] & 0xF) | ((cs[1] & 0xF) << 4);
@@ -365,6 +377,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   off = round_up(off + static_cast<size_t>(N) * K * sizeof(float), al);
   L.err = off;
   off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
+  L.err_lo = off;  // remainder part of the errors for the 3xTF32 updates
+  off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
   L.a = off;  // fp64 A, later U^T and U in fp32
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.x = off;
@@ -379,8 +393,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
 
 // W[:, c0 : c0+ncols] -= E[:, 0:kred] * U[k0 : k0+kred, c0 : c0+ncols]   (E row stride lde)
 static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
-                              int64_t lde, int64_t k0, int64_t kred, const float* Ut, const int* info, int* status,
-                              cudaStream_t s);
+                              const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut,
+                              const float* Ut_hi, const float* Ut_lo, const int* info, int* status, cudaStream_t s);
 
 hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
                       const float* imp, uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws,
@@ -390,6 +404,7 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   double* partials = reinterpret_cast<double*>(ws + L.partials);
   float* Wf = reinterpret_cast<float*>(ws + L.wf);
   float* Err = reinterpret_cast<float*>(ws + L.err);
+  float* Err_lo = reinterpret_cast<float*>(ws + L.err_lo);
   double* A = reinterpret_cast<double*>(ws + L.a);
   double* X = reinterpret_cast<double*>(ws + L.x);
   double* XT = reinterpret_cast<double*>(ws + L.xt);
@@ -398,7 +413,11 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
 
   float* Ut = nullptr;
   float* U = nullptr;
-  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, s);
+  float* Ut_hi = nullptr;
+  float* Ut_lo = nullptr;
+  const bool split = (update_impl == 0);  // 3xTF32 updates take pre-split operands
+  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, split, &Ut_hi,
+                               &Ut_lo, s);
   if (st != HQ_OK) return st;
 
   {
@@ -416,6 +435,7 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   a.U = U;
   a.group = static_cast<int>(group);
   a.Err = Err;
+  a.Err_lo = split ? Err_lo : nullptr;
   a.err_ld = P;
   a.codes = codes;
   a.scales = scales;
@@ -447,13 +467,14 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
                          N * (static_cast<double>(kBlk) / group) * 4.0, s);
       const int64_t j1 = j0 + kBlk;
       if (j1 < p1) {  // inner update of the rest of the panel
-        st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), P, j0, kBlk, Ut, &hdr->info,
-                          &hdr->status, s);
+        st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), Err_lo + (j0 - p0), P, j0, kBlk, Ut,
+                          Ut_hi, Ut_lo, &hdr->info, &hdr->status, s);
         if (st != HQ_OK) return st;
       }
     }
     if (p1 < K) {  // outer update of everything right of the panel
-      st = sweep_update(update_impl, Wf, N, K, p1, K - p1, Err, P, p0, p1 - p0, Ut, &hdr->info, &hdr->status, s);
+      st = sweep_update(update_impl, Wf, N, K, p1, K - p1, Err, Err_lo, P, p0, p1 - p0, Ut, Ut_hi, Ut_lo, &hdr->info,
+                        &hdr->status, s);
       if (st != HQ_OK) return st;
     }
   }
@@ -502,9 +523,26 @@ __global__ void __launch_bounds__(256) update_simt_kernel(float* __restrict__ C,
 }
 
 static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
-                              int64_t lde, int64_t k0, int64_t kred, const float* Ut, const int* info, int* status,
-                              cudaStream_t s) {
+                              const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut,
+                              const float* Ut_hi, const float* Ut_lo, const int* info, int* status, cudaStream_t s) {
   const float* B = Ut + c0 * K + k0;  // B(n, k) = U^T[c0 + n][k0 + k] = U[k0 + k][c0 + n]
+  if (impl == 0) {  // 3xTF32 from the pre-split operands (E, E_lo from the sweep; U^T split once)
+    UpdGemm g{};
+    g.C = Wf + c0;
+    g.ldc = K;
+    g.M = static_cast<int>(N);
+    g.N = static_cast<int>(ncols);
+    g.Kred = static_cast<int>(kred);
+    g.A_hi = E;
+    g.A_lo = E_lo;
+    g.lda = lde;
+    g.B_hi = Ut_hi + c0 * K + k0;
+    g.B_lo = Ut_lo + c0 * K + k0;
+    g.ldb = K;
+    g.skip = info;
+    g.status = status;
+    return upd_gemm(g, s);
+  }
   if (impl == 1) {
     const int64_t ctas = ceil_div(N, 64) * ceil_div(ncols, 64);
     update_simt_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(Wf + c0, K, N, ncols, E, lde, B, K, kred, info);

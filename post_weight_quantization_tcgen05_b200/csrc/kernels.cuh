@@ -34,6 +34,23 @@ struct Tf32Gemm {
 };
 hq_status tf32_gemm(const Tf32Gemm& g, cudaStream_t s);
 
+// gemm_upd.cu: C -= (A_hi + A_lo) (B_hi + B_lo)^T in 3xTF32 on tcgen05 (the GPTQ lazy updates),
+// operands pre-split into tf32 and remainder parts, K-major, 16-byte aligned rows.
+struct UpdGemm {
+  float* C;
+  int64_t ldc;
+  int M, N, Kred;
+  const float* A_hi;
+  const float* A_lo;
+  int64_t lda;
+  const float* B_hi;
+  const float* B_lo;
+  int64_t ldb;
+  const int* skip;
+  int* status;
+};
+hq_status upd_gemm(const UpdGemm& g, cudaStream_t s);
+
 // timing.cu: optional event timing of kernel classes (hq_debug_timing_*).  timer_start returns
 // -1 (and records nothing) unless the class is being timed; `work` is the launch's algorithmic
 // flops or bytes.
@@ -73,12 +90,16 @@ hq_status launch_rcp_nr(const double* d, double* out, int64_t n, cudaStream_t s)
 // factor.cu: U (row-major, upper) and U^T (row-major, lower) of the damped Hessian, in fp32,
 // from an fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; U and U^T are written into
 // the first and second halves of A's storage once A is no longer needed.
+// With split_ut, also the strict lower triangle of U^T split into a tf32 part and the fp32
+// remainder (U^T = Ut_hi + Ut_lo there), in T's storage; the upper parts of Ut_hi and Ut_lo are
+// not written.
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        double* lam, int* info, int* status, float** Ut, float** U, cudaStream_t s);
+                        double* lam, int* info, int* status, float** Ut, float** U, bool split_ut, float** Ut_hi,
+                        float** Ut_lo, cudaStream_t s);
 
 // gptq.cu
 struct GptqLayout {
-  size_t header, partials, wf, err, a, x, xt, t, total;
+  size_t header, partials, wf, err, err_lo, a, x, xt, t, total;
   int sweep_grid;
 };
 // Device-side header at the start of the GPTQ / RTN workspace.

@@ -20,11 +20,12 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D row-major tensor [outer, inner] with a 128-byte-swizzled box [box_outer, box_inner].
-// Out-of-range elements of a box read as zero.  Returns false if the driver refuses it
-// (base not 16-byte aligned, row stride not a multiple of 16 bytes, ...).
+// 2-D row-major tensor [outer, inner] with a swizzled box [box_outer, box_inner] (128-byte
+// swizzle unless stated).  Out-of-range elements of a box read as zero.  Returns false if the
+// driver refuses it (base not 16-byte aligned, row stride not a multiple of 16 bytes, ...).
 inline bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
-                         uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+                         uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                         CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -32,7 +33,7 @@ inline bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
