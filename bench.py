@@ -216,6 +216,7 @@ def run_ours(args, rank, world, local_rank):
     e2e = None if args.no_e2e else measure_e2e(args, layer, flush, world)
     # ---- per-kernel breakdown (outside the timed region: events around every launch)
     kernels = kernel_breakdown(hq, layer, flush)
+    codec = codec_throughput(hq, layer, flush)
     peaks = _peaks()
     syrk_flop = cfg.T * cfg.K * (cfg.K + 1)
     syrk_avg_s = statistics.mean(syrk_ms) / 1e3
@@ -226,6 +227,14 @@ def run_ours(args, rank, world, local_rank):
     return_line = build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops,
                              enc_bytes, dec_bytes, peaks, e2e, launches, clocks, dom, kernels,
                              fp64_mma_peak(hq))
+    hbm = peaks["hbm_gbs"]
+    return_line["codec_roofline"] = {
+        "kernels": "tril_encode_vec_kernel / tril_decode_vec_kernel", "bound": "hbm", "unit": "GB/s",
+        "encode": {"achieved": codec["encode_gbs"], "frac": codec["encode_gbs"] / hbm, "us": codec["encode_us"]},
+        "decode": {"achieved": codec["decode_gbs"], "frac": codec["decode_gbs"] / hbm, "us": codec["decode_us"]},
+        "peak": hbm, "peak_source": f"{peaks['source']} HBM copy",
+        "bytes": codec["bytes"],
+        "method": "each call alone after an L2 flush (write then read of 256 MiB), events around the call"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         return_line["cpu_baseline"] = cpu_baseline(cfg, layer)
     return return_line
@@ -267,6 +276,41 @@ def kernel_breakdown(hq, layer, flush, steps: int = 2):
         out[cls] = {"kernel": name, "ms_per_step": ms / steps, "launches_per_step": n / steps,
                     "achieved": work / (ms / 1e3) / scale, "unit": unit}
     return out
+
+
+def codec_throughput(hq, layer, flush, reps: int = 5):
+    """Encode and decode of the step's H, each launched right after an L2 flush and timed by
+    events around the call alone (in the step, the encode follows hq_gptq_quantize's host
+    synchronisation, so its stage time also holds the host's launch latency).  The flush ends
+    with a read so that no dirty lines are written back during the timed call."""
+    K = layer.cfg.K
+    enc_ms, dec_ms = [], []
+    # a write then a read of buffers larger than L2: the L2 holds clean lines of neither input
+    scratch = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=flush.device)
+
+    def clean_flush(r):
+        flush.fill_(r & 0xFF)
+        scratch.sum()
+
+    for r in range(reps + 1):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        clean_flush(r)
+        ev[0].record()
+        hq.hq_hessian_pack_bf16tril(layer.H, layer.tril)
+        ev[1].record()
+        clean_flush(r + 1)
+        ev[2].record()
+        hq.hq_hessian_unpack_bf16tril(layer.tril, K, layer.Hfull)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if r > 0:  # the first round warms up
+            enc_ms.append(ev[0].elapsed_time(ev[1]))
+            dec_ms.append(ev[2].elapsed_time(ev[3]))
+    enc_bytes = 2 * K * (K + 1) + hq.hq_bf16tril_bytes(K)  # H lower triangle read + payload written
+    dec_bytes = hq.hq_bf16tril_bytes(K) + 4 * K * K        # payload read + full H written
+    enc_s, dec_s = statistics.median(enc_ms) / 1e3, statistics.median(dec_ms) / 1e3
+    return {"encode_gbs": enc_bytes / enc_s / 1e9, "decode_gbs": dec_bytes / dec_s / 1e9,
+            "encode_us": enc_s * 1e6, "decode_us": dec_s * 1e6, "bytes": {"encode": enc_bytes, "decode": dec_bytes}}
 
 
 def fp64_mma_peak(hq):
