@@ -161,12 +161,20 @@ def _barrier(world):
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (a device time: the job ends with its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(units_per_rank: float, world: int, steps: int, total_ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own units each step (weak scaling), and
+    the job takes as long as its slowest rank."""
+    return units_per_rank * world * steps / (total_ms_max / 1e3)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -210,7 +218,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = _max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     weights = cfg.N * cfg.K
-    value = weights * world * args.steps / (total_ms / 1e3)
+    value = aggregate_rate(weights, world, args.steps, total_ms)
 
     # ---- e2e: same calls, inputs from pinned host memory, results copied back
     e2e = None if args.no_e2e else measure_e2e(args, layer, flush, world)
@@ -237,7 +245,86 @@ def run_ours(args, rank, world, local_rank):
         "method": "each call alone after an L2 flush (write then read of 256 MiB), events around the call"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         return_line["cpu_baseline"] = cpu_baseline(cfg, layer)
+    if world == 1 and not args.no_other_configs:
+        del layer
+        torch.cuda.empty_cache()
+        return_line["other_configs"] = other_configs(hq, dev, flush, peaks)
     return return_line
+
+
+def time_layer(hq, cfg, dev, flush, steps: int = 2, warmup: int = 1):
+    """Whole-path steps on one layer of `cfg` (the main measurement's protocol, fewer steps)."""
+    layer = Layer(hq, cfg, dev)
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for k in range(steps):
+        flush.fill_(k & 0xFF)
+        layer.step(stage_events=evs[k])
+    torch.cuda.synchronize()
+    step_ms = statistics.mean(e[0].elapsed_time(e[4]) for e in evs)
+    syrk_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    gptq_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    out = {"workload": f"{cfg.name}: W bf16 [{cfg.N}, {cfg.K}], X bf16 [{cfg.T}, {cfg.K}], group {cfg.group}"
+                       + (", imatrix" if cfg.use_imatrix else ""),
+           "steps": steps, "ms_per_step": step_ms, "weights_per_s": cfg.N * cfg.K / (step_ms / 1e3),
+           "gptq_quantize_ms": gptq_ms, "gptq_weights_per_s": cfg.N * cfg.K / (gptq_ms / 1e3),
+           "syrk_ms": syrk_ms, "xtx_tflops": cfg.T * cfg.K * (cfg.K + 1) / (syrk_ms / 1e3) / 1e12}
+    del layer
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_hessian_at_scale(hq, cfg, dev, flush, peaks, distinct: int = 8):
+    """SYRK over the configuration's 512 chunks of 8192 tokens into one fp32 H (the chunks cycle
+    through `distinct` pre-generated ones: the SYRK's cost does not depend on the values;
+    generation is outside the timed region), then the codec of that H, each call alone."""
+    import post_weight_quantization_tcgen05_b200 as hqm
+    K = cfg.K
+    scales = wl.channel_scales(cfg)
+    chunks = [wl.make_activation_chunk(cfg, c, dev, scales) for c in range(distinct)]
+    H = torch.zeros((K, K), dtype=torch.float32, device=dev)
+    for c in range(distinct):  # warm-up
+        hq.hq_hessian_accumulate(H, chunks[c])
+    H.zero_()
+    flush.fill_(1)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for c in range(cfg.n_chunks):
+        hq.hq_hessian_accumulate(H, chunks[c % distinct])
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+
+    class _L:  # what codec_throughput reads
+        pass
+    lay = _L()
+    lay.cfg, lay.H = cfg, H
+    lay.tril = torch.empty(hqm.hq_bf16tril_bytes(K), dtype=torch.uint8, device=dev)
+    lay.Hfull = torch.empty((K, K), dtype=torch.float32, device=dev)
+    codec = codec_throughput(hq, lay, flush)
+    hbm = peaks["hbm_gbs"]
+    out = {"workload": f"{cfg.name}: {cfg.n_chunks} chunks of X bf16 [{cfg.chunk}, {K}] into one H",
+           "syrk_ms": ms, "xtx_tflops": cfg.T * K * (K + 1) / (ms / 1e3) / 1e12,
+           "xtx_frac_of_bf16_peak": cfg.T * K * (K + 1) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "codec": {"encode_gbs": codec["encode_gbs"], "encode_frac": codec["encode_gbs"] / hbm,
+                     "decode_gbs": codec["decode_gbs"], "decode_frac": codec["decode_gbs"] / hbm}}
+    del chunks, H, lay
+    torch.cuda.empty_cache()
+    return out
+
+
+def other_configs(hq, dev, flush, peaks):
+    """The other single-GPU layer configurations (gate_up, down_proj at K = 17408, the Hessian at
+    scale), measured after the main line's timed region."""
+    out = {}
+    for idx in (2, 3):
+        cfg = wl.CONFIGS[idx]
+        out[cfg.name] = time_layer(hq, cfg, dev, flush)
+    out["hessian_at_scale"] = time_hessian_at_scale(hq, wl.CONFIGS[4], dev, flush, peaks)
+    return out
 
 
 # The kernel with the largest share of a step (ncu launch list of this benchmark) and the others
@@ -515,6 +602,8 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the gate_up / down_proj / Hessian-at-scale measurements after the main line")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -244,15 +244,46 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&acce[acc]);
       }
-      if (!ok) {
-        fail();
-      } else if (r < args.M) {
-        float* row = args.C + static_cast<int64_t>(r) * args.ldc;
-        const int cb = n0 + h * 128;
+      if (!ok) fail();
+      // H tile += sums, coalesced: once every MMA has completed the stage ring is free; the
+      // sums go there as a 128 x 256 tile (row r: 16-byte piece p at p ^ (r & 7)), then each
+      // warp adds rows of it to H with 16-byte accesses along the row.  Every epilogue warp
+      // meets the named barrier, also after a failed wait.
+      float4* tile = reinterpret_cast<float4*>(smem);
+      const int rl = q * 32 + lane;  // tile row
+      if (ok) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const int j = cb + i;
-          if (j <= r) row[j] += sum[i];
+        for (int k = 0; k < 32; ++k) {
+          const int p = h * 32 + k;
+          tile[rl * 64 + (p ^ (rl & 7))] = make_float4(sum[4 * k], sum[4 * k + 1], sum[4 * k + 2], sum[4 * k + 3]);
+        }
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (ok) {
+        const bool vec = (reinterpret_cast<uintptr_t>(args.C) & 15) == 0 && (args.ldc % 4) == 0;
+        for (int rr = warp - 2; rr < kGemmBM; rr += kEpiWarps) {
+          const int row = m0 + rr;
+          if (row >= args.M) break;
+          float* hrow = args.C + static_cast<int64_t>(row) * args.ldc;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int p = lane + 32 * half;  // 16-byte piece of the tile row
+            const int col = n0 + 4 * p;
+            const float4 v = tile[rr * 64 + (p ^ (rr & 7))];
+            if (vec && col + 3 <= row && col + 3 < args.Ncols) {  // entirely in the lower part
+              float4 o = *reinterpret_cast<float4*>(hrow + col);
+              o.x += v.x;
+              o.y += v.y;
+              o.z += v.z;
+              o.w += v.w;
+              *reinterpret_cast<float4*>(hrow + col) = o;
+            } else {
+              const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (col + e <= row && col + e < args.Ncols) hrow[col + e] += vv[e];
+            }
+          }
         }
       }
     } else {
