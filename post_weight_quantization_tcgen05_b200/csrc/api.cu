@@ -146,7 +146,7 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
   float* U = nullptr;
   hq_status st = launch_factor(H, K, damp, reinterpret_cast<double*>(ws + L.a), reinterpret_cast<double*>(ws + L.x),
                                reinterpret_cast<double*>(ws + L.xt), reinterpret_cast<double*>(ws + L.t), &hdr->lam,
-                               &hdr->info, &hdr->status, &Ut, &U, false, nullptr, nullptr, s);
+                               &hdr->info, &hdr->status, &Ut, &U, false, false, nullptr, nullptr, s);
   if (st != HQ_OK) return st;
   HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, Ut, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return finish_sync(s, hdr, nullptr);

@@ -530,18 +530,22 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
 
 // U[j][c] = X[K-1-j][K-1-c] and U^T[j][c] = X^T[K-1-j][K-1-c], rounded to fp32: 180-degree
 // rotations (U upper, U^T lower, zeros elsewhere because X and X^T hold zeros there).
-// With Ut_hi != NULL, also the strict lower part of U^T as a tf32 part (low 13 mantissa bits
-// cleared) plus the exact fp32 remainder, the operands of the 3xTF32 lazy updates.
+// With `scaled`, U^T[j][c] is divided by U[c][c] in fp64 first (U'^T, U' = diag(U)^-1 U, the
+// form the GPTQ sweep and its lazy updates use).  With Ut_hi != NULL, also the strict lower part
+// of the result as a tf32 part (low 13 mantissa bits cleared) plus the exact fp32 remainder, the
+// operands of the 3xTF32 lazy updates.
 __global__ void rotate_kernel(const double* __restrict__ X, const double* __restrict__ XT, int64_t K,
                               float* __restrict__ U, float* __restrict__ Ut, float* __restrict__ Ut_hi,
-                              float* __restrict__ Ut_lo, const int* __restrict__ info) {
+                              float* __restrict__ Ut_lo, bool scaled, const int* __restrict__ info) {
   if (*info != 0) return;
   const int64_t n = K * K;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t src = n - 1 - e;  // (K-1-j)*K + (K-1-c) for e = j*K + c
-    U[e] = static_cast<float>(X[src]);
-    const float ut = static_cast<float>(XT[src]);
+    if (U != nullptr) U[e] = static_cast<float>(X[src]);
+    double ut64 = XT[src];  // U^T[e / K][e % K] = U[e % K][e / K]
+    if (scaled) ut64 /= X[(K - 1 - e % K) * (K + 1)];  // divided by U[e % K][e % K]
+    const float ut = static_cast<float>(ut64);
     Ut[e] = ut;
     if (Ut_hi != nullptr && e % K < e / K) {
       const float hi = __uint_as_float(__float_as_uint(ut) & 0xFFFFE000u);
@@ -551,13 +555,35 @@ __global__ void rotate_kernel(const double* __restrict__ X, const double* __rest
   }
 }
 
+// The diagonal blocks of U' = diag(U)^-1 U in the GPTQ sweep's packed order
+// (sweep_upack_offset), U[j][c] = X[K-1-j][K-1-c].
+__global__ void sweep_pack_kernel(const double* __restrict__ X, int64_t K, float* __restrict__ Up,
+                                  const int* __restrict__ info) {
+  if (*info != 0) return;
+  constexpr int B = kSweepBlk;
+  const int64_t total = K * B;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = e / (B * B);
+    const int r = static_cast<int>(e % (B * B));
+    const int j = r / B, l = (r % B) / 8, m = r % 8;
+    const int c = 16 * (j / 16 + m) + l;
+    float v = 0.f;
+    if (c > j && c < B) {
+      const int64_t gj = b * B + j, gc = b * B + c;
+      v = static_cast<float>(X[(K - 1 - gj) * K + (K - 1 - gc)] / X[(K - 1 - gj) * (K + 1)]);
+    }
+    Up[b * B * B + sweep_upack_offset(j, l, m)] = v;
+  }
+}
+
 // ------------------------------------------------------------------------- driver
 
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        double* lam, int* info, int* status, float** Ut, float** U, bool split_ut, float** Ut_hi,
-                        float** Ut_lo, cudaStream_t s) {
+                        double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form, bool split_ut,
+                        float** Ut_hi, float** Ut_lo, cudaStream_t s) {
   (void)status;
-  if (K % kLeaf != 0) return HQ_ERR_UNSUPPORTED;
+  if (K % kLeaf != 0 || K % kSweepBlk != 0) return HQ_ERR_UNSUPPORTED;
   HQ_CUDA_TRY(cudaFuncSetAttribute(chol_inv_leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(kLeafSmem)));
   damp_stats_kernel<<<1, 1024, 0, s>>>(H, K, damp, lam, info);
@@ -580,7 +606,7 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   const hq_status st_join = stream_dep(side, side->s2, s);
   if (st != HQ_OK) return st;
   if (st_join != HQ_OK) return st_join;
-  // A is dead now: U^T and U (fp32) go into its storage
+  // A is dead now: the fp32 results go into its storage
   *Ut = reinterpret_cast<float*>(A);
   *U = reinterpret_cast<float*>(A) + K * K;
   const int64_t grid = ceil_div(K * K, 4 * 256) < 148 * 32 ? ceil_div(K * K, 4 * 256) : 148 * 32;
@@ -589,8 +615,14 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   float* lo = split_ut ? reinterpret_cast<float*>(T) + K * K : nullptr;
   if (Ut_hi != nullptr) *Ut_hi = hi;
   if (Ut_lo != nullptr) *Ut_lo = lo;
-  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, *U, *Ut, hi, lo, info);
+  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, sweep_form ? nullptr : *U, *Ut, hi, lo,
+                                                            sweep_form, info);
   HQ_LAUNCH_CHECK();
+  if (sweep_form) {
+    const int64_t pg = ceil_div(K * kSweepBlk, 256) < 148 * 16 ? ceil_div(K * kSweepBlk, 256) : 148 * 16;
+    sweep_pack_kernel<<<static_cast<unsigned>(pg), 256, 0, s>>>(X, K, *U, info);
+    HQ_LAUNCH_CHECK();
+  }
   return HQ_OK;
 }
 

@@ -4,25 +4,31 @@
 //
 // The sweep walks K in 128-column blocks grouped into panels of P columns (P = 512, or a
 // multiple of the group size when groups are wider than a block).  Per block:
-//   * sweep_block_kernel: the sequential part.  A group of eight lanes carries two rows;
-//     lane l holds columns l, l+8, l+16, ... of both rows as 16 "slots" each, in registers.
-//     The columns are visited in rounds of eight: at the end of a round every lane shifts its
-//     slots down by one, so the column being quantised is always slot 0 of lane (j mod 8), a
-//     compile-time lane inside the 8-way unrolled round, and the loop body stays small enough
-//     for the instruction cache.  Per column j and row: group scale at a group start (8-lane
-//     absmax), broadcast of w_j, code c = clamp(rint(w_j / s), -8, 7), error
-//     e = (w_j - c s) / U[j, j], and the feedback w_k -= e U[j, k] for k > j.  U's row j is
-//     pre-permuted (and XOR-swizzled against bank conflicts) in shared memory so that each
-//     lane reads its 16 values with four 16-byte loads, used for both of its rows.  It writes the block's
-//     errors into the panel's error buffer, the packed int4 codes, the scales and fp64 partial
-//     sums of the qerr numerator and denominator over the ORIGINAL weights.
-//   * inner lazy update of the rest of the panel, W[:, b+128 : panel end] -= Err_b U[b, ...]
+//   * sweep_block_kernel: the sequential part.  Sixteen lanes share two rows: lane l holds
+//     columns l, l+16, ..., l+112 of both rows as 8 "slots" each, in registers.  The columns
+//     are visited in rounds of sixteen; at the end of a round every lane shifts its slots down
+//     by one, so the column being quantised is always slot 0 of lane (j mod 16), a
+//     compile-time lane inside the 16-way unrolled round.  Per column j and row: group scale
+//     at a group start (16-lane absmax), broadcast of w_j, code c = clamp(rint(w_j / s), -8, 7),
+//     residual d = w_j - c s, and the feedback w_k -= d U'[j, k] for k > j, where
+//     U' = diag(U)^-1 U is U with each row divided by its diagonal entry, so that
+//     d U'[j, k] = e U[j, k] with the error e = d / U[j, j] of the method.  The factorisation
+//     hands over each 128 x 128 diagonal block of U' already permuted into the lanes' slot
+//     order (zero on and below the diagonal) so that a lane reads its 8 values for column j
+//     with two conflict-free 16-byte loads shared by its two rows.  At the end of a round each
+//     lane re-derives the code and residual of the column it holds in slot 0 (the same
+//     arithmetic on the same final weight) and stages them; the block then writes the
+//     residuals into the panel's buffer, the packed int4 codes, the scales and fp64 partial
+//     sums of the qerr numerator and denominator over the ORIGINAL weights.  A CTA holds
+//     ceil(N / 148) rows rounded up to a multiple of four, so one wave covers the layer.
+//   * inner lazy update of the rest of the panel, W[:, b+128 : panel end] -= D_b U'[b, ...]
 //     (contraction 128; the panel's N x P working weights stay in L2);
-// and after the panel the outer lazy update W[:, panel end:] -= Err_panel U[panel, ...] with
-// contraction P.  Both updates are dense contractions on the tensor cores (gemm_tf32.cuh, by
-// default 3xTF32) with B = U^T row-major.  Blocking only reorders exact sums: every column
-// still receives the feedback of every earlier column before it is quantised.
-// U^T comes from factor.cu.  The working copy of W is fp32 in the workspace.
+// and after the panel the outer lazy update W[:, panel end:] -= D_panel U'[panel, ...] with
+// contraction P.  Both updates are dense contractions on the tensor cores (gemm_upd.cu,
+// 3xTF32) with B = U'^T row-major.  Blocking only reorders exact sums: every column still
+// receives the feedback of every earlier column before it is quantised.
+// U'^T and the packed diagonal blocks of U' come from factor.cu.  The working copy of W is
+// fp32 in the workspace.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -30,19 +36,35 @@
 
 namespace hq {
 
-constexpr int kBlk = 128;        // sweep block width
-constexpr int kLanesPerRow = 8;
-constexpr int kSlots = kBlk / kLanesPerRow;  // 16 columns per lane
-constexpr int kRowsPerCta = 32;              // 4 warps x 4 lane groups x 2 rows
-constexpr int kSweepThreads = 128;
+constexpr int kBlk = 128;                    // sweep block width (== kSweepBlk)
+constexpr int kLanesPerRow = 16;             // lanes sharing one row's 128 columns
+constexpr int kSlots = kBlk / kLanesPerRow;  // 8 columns per lane and row
+constexpr int kRowsPerWarp = 4;              // two 16-lane groups x two rows
+constexpr int kMaxSweepThreads = 1024;
+constexpr int kMaxRowsPerCta = kMaxSweepThreads / 32 * kRowsPerWarp;  // 128
+static_assert(kBlk == kSweepBlk, "packed U' blocks are made for this block width");
+
+// Rows per CTA: the layer's rows spread over one wave of 148 CTAs, a multiple of 4, 4..128.
+static int sweep_rows_per_cta(int64_t N) {
+  int64_t r = ceil_div(N, int64_t(148));
+  r = ceil_div(r, int64_t(kRowsPerWarp)) * kRowsPerWarp;
+  if (r < kRowsPerWarp) r = kRowsPerWarp;
+  if (r > kMaxRowsPerCta) r = kMaxRowsPerCta;
+  return static_cast<int>(r);
+}
+
+static size_t sweep_smem_bytes(int rows) {
+  return (static_cast<size_t>(kBlk) * kBlk + static_cast<size_t>(rows) * (kBlk + 1) + rows * 4 + kBlk) * sizeof(float) +
+         static_cast<size_t>(rows) * kBlk;
+}
 
 struct SweepArgs {
   float* Wf;
   int64_t N, K;
-  const float* U;    // U row-major (upper triangular)
+  const float* Upack;  // packed diagonal blocks of U' (sweep_upack_offset order), kBlk^2 floats each
   int group;
-  float* Err;        // panel error buffer [N, P] (the tf32 part when Err_lo is set)
-  float* Err_lo;     // NULL, or the fp32 remainder of each error (Err + Err_lo = error)
+  float* Err;        // panel residual buffer [N, P] (the tf32 part when Err_lo is set)
+  float* Err_lo;     // NULL, or the fp32 remainder of each residual (Err + Err_lo = residual)
   int64_t err_ld;    // P
   int err_col;       // column of this block inside the panel buffer
   uint8_t* codes;
@@ -58,175 +80,178 @@ __device__ __forceinline__ float load_w(const void* W, int dt, int64_t idx) {
   return dt == HQ_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(W)[idx]) : static_cast<const float*>(W)[idx];
 }
 
-// c = clamp(rint(w / s), -8, 7) with w / s the IEEE fp32 quotient.  w * (1/s) is within a
-// couple of ulps of the quotient, so it rounds the same way unless it lies within 1e-5 of a
-// half-integer; only then is the exact division taken.  Rounding to nearest-even uses the
-// 1.5 * 2^23 shift (exact for |q| < 2^22; larger values are clamped anyway).
-__device__ __forceinline__ float quant_code(float w, float s, float rs) {
-  if (!(s > 0.f)) return 0.f;
+// c = clamp(rint(w / s), -8, 7) with w / s the IEEE fp32 quotient; rs = 1 / s, or 0 when
+// s == 0 (then c = 0 for every finite w).  w * rs is within a couple of ulps of the quotient,
+// so it rounds the same way unless it lies within 1e-5 of a half-integer; only then is the
+// exact division taken.  Rounding to nearest-even uses the 1.5 * 2^23 shift (exact for
+// |q| < 2^22; larger values are clamped anyway).  Two rows at a time, one branch for both.
+// The rare exact path, out of line so that the unrolled sweep loop stays compact.
+__device__ __noinline__ float exact_round_quotient(float w, float s) { return rintf(__fdiv_rn(w, s)); }
+
+__device__ __forceinline__ void quant_pair(float wa, float sa, float rsa, float wb, float sb, float rsb, float& ca,
+                                           float& cb) {
   constexpr float kShift = 12582912.f;
-  float q = w * rs;
-  float r = (q + kShift) - kShift;
-  if (fabsf(q - r) > 0.5f - 1e-5f) r = rintf(__fdiv_rn(w, s));
-  return fminf(fmaxf(r, -8.f), 7.f);
+  constexpr float kNear = 0.5f - 1e-5f;
+  const float qa = wa * rsa, qb = wb * rsb;
+  float ra = (qa + kShift) - kShift;
+  float rb = (qb + kShift) - kShift;
+  if (fmaxf(fabsf(qa - ra), fabsf(qb - rb)) > kNear) {
+    if (fabsf(qa - ra) > kNear) ra = exact_round_quotient(wa, sa);
+    if (fabsf(qb - rb) > kNear) rb = exact_round_quotient(wb, sb);
+  }
+  ca = fminf(fmaxf(ra, -8.f), 7.f);
+  cb = fminf(fmaxf(rb, -8.f), 7.f);
 }
+
+__device__ __forceinline__ float recip_or_zero(float s) { return s > 0.f ? __frcp_rn(s) : 0.f; }
 
 // GS: group size when it is 32, 64 or 128 (scales computed inside the block), or 0 when the
 // group spans several blocks (scale computed at the group's first block from Wf).
-// Offset (in floats) of chunk q (4 floats) of lane l's 16 U values for column j.  The XOR
-// keeps the eight lanes of a quarter-warp on eight different 16-byte bank groups.
-__device__ __forceinline__ int ur_off(int j, int l, int q) { return (j * kLanesPerRow + l) * kSlots + 4 * (q ^ (l >> 1)); }
-
 template <int GS>
-__global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a, int j0) {
+__global__ void __launch_bounds__(kMaxSweepThreads) sweep_block_kernel(SweepArgs a, int j0) {
   if (*a.info != 0) return;
-  constexpr int LD = kBlk + 1;  // padded row of the staging buffer
-  constexpr int kGS = (GS == 0 ? kLanesPerRow : GS) / kLanesPerRow;  // slots per group
-  extern __shared__ float sm[];
-  float* Ur = sm;                                  // [128 j][8 lanes][16 slots], swizzled
-  float* stage = Ur + kBlk * kBlk;                 // [32][129]: weights in, errors out
-  float* scl_s = stage + kRowsPerCta * LD;         // [32][4]
-  float* inv_diag = scl_s + kRowsPerCta * 4;       // [128]: 1 / U[j][j]
-  int8_t* code_s = reinterpret_cast<int8_t*>(inv_diag + kBlk);  // [32][128]
+  constexpr int LD = kBlk + 1;  // padded row of the residual stage
+  extern __shared__ float4 sm4[];
+  float* Ur = reinterpret_cast<float*>(sm4);      // packed U' block
+  const int rows = static_cast<int>(blockDim.x / 32) * kRowsPerWarp;
+  float* dst = Ur + kBlk * kBlk;                   // [rows][LD]: residuals
+  float* scl_s = dst + rows * LD;                  // [rows][4]
+  float* sup_s = scl_s + rows * 4;                 // [kBlk]: U'[j][j + 1], 0 for the last j
+  int8_t* code_s = reinterpret_cast<int8_t*>(sup_s + kBlk);  // [rows][kBlk]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, l = lane & (kLanesPerRow - 1);
-  const int rl0 = warp * (32 / kLanesPerRow) + lane / kLanesPerRow;  // rows rl0 and rl0 + 16
-  const int rl1 = rl0 + kRowsPerCta / 2;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  const int rlA = warp * kRowsPerWarp + (lane >> 4), rlB = rlA + 2;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows;
+  const int64_t rowA = r0 + rlA, rowB = r0 + rlB;
+  const bool vA = rowA < a.N, vB = rowB < a.N;
   const int64_t K = a.K;
 
-  // Ur: U[j0 + j][j0 + 8 * (j / 8 + m) + l] for slot m of lane l, zero past the block.
-  for (int e = tid; e < kBlk * kBlk; e += kSweepThreads) Ur[e] = 0.f;
-  __syncthreads();
-#pragma unroll 4
-  for (int e = tid; e < kBlk * (kBlk / 4); e += kSweepThreads) {
-    const int j = e >> 5, q4 = e & 31;  // row j, columns 4 q4 .. 4 q4 + 3
-    const float4 u = reinterpret_cast<const float4*>(a.U + (j0 + j) * K + j0)[q4];
-    const float uv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int col = 4 * q4 + i;
-      const int m = col / kLanesPerRow - j / kLanesPerRow;
-      if (m >= 0) Ur[ur_off(j, col % kLanesPerRow, m >> 2) + (m & 3)] = uv[i];
+  {  // packed U' block -> shared memory, all copies in flight at once
+    const float4* src = reinterpret_cast<const float4*>(a.Upack + static_cast<int64_t>(j0 / kBlk) * (kBlk * kBlk));
+    const uint32_t dst0 = static_cast<uint32_t>(__cvta_generic_to_shared(sm4));
+    for (int e = tid; e < kBlk * kBlk / 4; e += blockDim.x)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst0 + 16u * e), "l"(src + e) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int t = tid; t < kBlk; t += blockDim.x) {
+      const int c = t + 1;
+      sup_s[t] = c < kBlk ? a.Upack[static_cast<int64_t>(j0 / kBlk) * (kBlk * kBlk) +
+                                    sweep_upack_offset(t, c & (kLanesPerRow - 1), c / kLanesPerRow - t / kLanesPerRow)]
+                          : 0.f;
     }
   }
-  // weights: coalesced 512-byte rows into the staging buffer
-  for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
-    const float4 v = (r0 + r < a.N) ? reinterpret_cast<const float4*>(a.Wf + (r0 + r) * K + j0)[lane]
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    float* d = stage + r * LD + 4 * lane;
-    d[0] = v.x;
-    d[1] = v.y;
-    d[2] = v.z;
-    d[3] = v.w;
-  }
-  __syncthreads();
-  for (int j = tid; j < kBlk; j += kSweepThreads) inv_diag[j] = __frcp_rn(a.U[(j0 + j) * K + j0 + j]);
   float w0[kSlots], w1[kSlots];
 #pragma unroll
   for (int m = 0; m < kSlots; ++m) {
-    w0[m] = stage[rl0 * LD + kLanesPerRow * m + l];
-    w1[m] = stage[rl1 * LD + kLanesPerRow * m + l];
+    w0[m] = vA ? a.Wf[rowA * K + j0 + kLanesPerRow * m + l] : 0.f;
+    w1[m] = vB ? a.Wf[rowB * K + j0 + kLanesPerRow * m + l] : 0.f;
   }
 
-  float s0 = 0.f, rs0 = 0.f, s1 = 0.f, rs1 = 0.f;
+  float sA = 0.f, rsA = 0.f, sB = 0.f, rsB = 0.f;
   if (GS == 0) {
     // the group spans several blocks: its scale is taken at its first block from the current
     // weights of all its columns, and read back in the later blocks
     const int G = a.group;
     const int64_t g = j0 / G;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int rl = h ? rl1 : rl0;
-      const int64_t row = r0 + rl;
-      const bool valid = row < a.N;
-      float sc;
-      if (j0 % G == 0) {
-        float am = 0.f;
-        if (valid)
-          for (int i = l; i < G; i += kLanesPerRow) am = fmaxf(am, fabsf(a.Wf[row * K + j0 + i]));
-#pragma unroll
-        for (int x = 1; x < kLanesPerRow; x <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, x));
-        sc = __fdiv_rn(am, 7.f);
-        if (valid && l == 0) a.scales[row * (K / G) + g] = sc;
-      } else {
-        sc = valid ? a.scales[row * (K / G) + g] : 0.f;
+    if (j0 % G == 0) {
+      float amA = 0.f, amB = 0.f;
+      for (int i = l; i < G; i += kLanesPerRow) {
+        if (vA) amA = fmaxf(amA, fabsf(a.Wf[rowA * K + j0 + i]));
+        if (vB) amB = fmaxf(amB, fabsf(a.Wf[rowB * K + j0 + i]));
       }
-      if (l == 0) scl_s[rl * 4] = sc;
-      if (h) {
-        s1 = sc;
-        rs1 = __frcp_rn(sc);
-      } else {
-        s0 = sc;
-        rs0 = __frcp_rn(sc);
+#pragma unroll
+      for (int x = 1; x < kLanesPerRow; x <<= 1) {
+        amA = fmaxf(amA, __shfl_xor_sync(0xffffffffu, amA, x));
+        amB = fmaxf(amB, __shfl_xor_sync(0xffffffffu, amB, x));
       }
+      sA = __fdiv_rn(amA, 7.f);
+      sB = __fdiv_rn(amB, 7.f);
+      if (l == 0 && vA) a.scales[rowA * (K / G) + g] = sA;
+      if (l == 0 && vB) a.scales[rowB * (K / G) + g] = sB;
+    } else {
+      sA = vA ? a.scales[rowA * (K / G) + g] : 0.f;
+      sB = vB ? a.scales[rowB * (K / G) + g] : 0.f;
     }
+    rsA = recip_or_zero(sA);
+    rsB = recip_or_zero(sB);
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
-  float* err0 = stage + rl0 * LD;
-  float* err1 = stage + rl1 * LD;
-  int8_t* code0 = code_s + rl0 * kBlk;
-  int8_t* code1 = code_s + rl1 * kBlk;
-  const int src_base = lane & ~(kLanesPerRow - 1);
+
+  const int src_base = lane & kLanesPerRow;  // first lane of this 16-lane group
+  // Every lane carries the current value of the column being quantised (curA, curB): the
+  // value of column j + 1 is fetched from its owner lane BEFORE column j's feedback and then
+  // updated locally with the same fma the owner applies, so the broadcast is off the
+  // column-to-column dependency chain and the result is bit-identical to the owner's slot.
+  float curA = __shfl_sync(0xffffffffu, w0[0], src_base);
+  float curB = __shfl_sync(0xffffffffu, w1[0], src_base);
 #pragma unroll 1
   for (int R = 0; R < kSlots; ++R) {
 #pragma unroll
     for (int jr = 0; jr < kLanesPerRow; ++jr) {
       const int j = kLanesPerRow * R + jr;
-      if (GS != 0 && jr == 0 && (R % kGS) == 0) {
-        float am0 = 0.f, am1 = 0.f;
+      if (GS != 0 && jr == 0 && (R % (GS == 0 ? 1 : GS / kLanesPerRow)) == 0) {
+        constexpr int kGS = (GS == 0 ? kLanesPerRow : GS) / kLanesPerRow;  // slots per group
+        float amA = 0.f, amB = 0.f;
 #pragma unroll
         for (int m = 0; m < kGS; ++m) {
-          am0 = fmaxf(am0, fabsf(w0[m]));
-          am1 = fmaxf(am1, fabsf(w1[m]));
+          amA = fmaxf(amA, fabsf(w0[m]));
+          amB = fmaxf(amB, fabsf(w1[m]));
         }
 #pragma unroll
         for (int x = 1; x < kLanesPerRow; x <<= 1) {
-          am0 = fmaxf(am0, __shfl_xor_sync(0xffffffffu, am0, x));
-          am1 = fmaxf(am1, __shfl_xor_sync(0xffffffffu, am1, x));
+          amA = fmaxf(amA, __shfl_xor_sync(0xffffffffu, amA, x));
+          amB = fmaxf(amB, __shfl_xor_sync(0xffffffffu, amB, x));
         }
-        s0 = __fdiv_rn(am0, 7.f);
-        s1 = __fdiv_rn(am1, 7.f);
-        rs0 = __frcp_rn(s0);
-        rs1 = __frcp_rn(s1);
+        sA = __fdiv_rn(amA, 7.f);
+        sB = __fdiv_rn(amB, 7.f);
+        rsA = recip_or_zero(sA);
+        rsB = recip_or_zero(sB);
         if (l == 0) {
-          scl_s[rl0 * 4 + j / (GS == 0 ? 1 : GS)] = s0;
-          scl_s[rl1 * 4 + j / (GS == 0 ? 1 : GS)] = s1;
+          scl_s[rlA * 4 + j / (GS == 0 ? kBlk : GS)] = sA;
+          scl_s[rlB * 4 + j / (GS == 0 ? kBlk : GS)] = sB;
         }
       }
-      float u[kSlots];
-#pragma unroll
-      for (int q = 0; q < kSlots / 4; ++q) {
-        const float4 t = *reinterpret_cast<const float4*>(Ur + ur_off(j, l, q));
-        u[4 * q] = t.x;
-        u[4 * q + 1] = t.y;
-        u[4 * q + 2] = t.z;
-        u[4 * q + 3] = t.w;
-      }
-      const float idg = inv_diag[j];
-      const float wj0 = __shfl_sync(0xffffffffu, w0[0], src_base | jr);
-      const float wj1 = __shfl_sync(0xffffffffu, w1[0], src_base | jr);
-      const float c0 = quant_code(wj0, s0, rs0);
-      const float c1 = quant_code(wj1, s1, rs1);
-      const float e0 = fmaf(-c0, s0, wj0) * idg;
-      const float e1 = fmaf(-c1, s1, wj1) * idg;
-      if (l == jr) {
-        err0[j] = e0;
-        err1[j] = e1;
-        code0[j] = static_cast<int8_t>(c0);
-        code1[j] = static_cast<int8_t>(c1);
-      }
-      if (l > jr) {
-        w0[0] = fmaf(-e0, u[0], w0[0]);
-        w1[0] = fmaf(-e1, u[0], w1[0]);
-      }
-#pragma unroll
-      for (int m = 1; m < kSlots; ++m) {
-        w0[m] = fmaf(-e0, u[m], w0[m]);
-        w1[m] = fmaf(-e1, u[m], w1[m]);
-      }
+      const float4 u0 = *reinterpret_cast<const float4*>(Ur + sweep_upack_offset(j, l, 0));
+      const float4 u1 = *reinterpret_cast<const float4*>(Ur + sweep_upack_offset(j, l, 4));
+      const float usup = sup_s[j];
+      // column j + 1 before column j's feedback: slot 0 of lane jr + 1, or after the round's
+      // last column slot 1 of lane 0
+      const float preA = __shfl_sync(0xffffffffu, jr + 1 < kLanesPerRow ? w0[0] : w0[1], src_base | ((jr + 1) & 15));
+      const float preB = __shfl_sync(0xffffffffu, jr + 1 < kLanesPerRow ? w1[0] : w1[1], src_base | ((jr + 1) & 15));
+      float ca, cb;
+      quant_pair(curA, sA, rsA, curB, sB, rsB, ca, cb);
+      const float da = fmaf(-ca, sA, curA);
+      const float db = fmaf(-cb, sB, curB);
+      // U' is zero in the packed block on and left of column j: lanes l <= jr keep slot 0
+      w0[0] = fmaf(-da, u0.x, w0[0]);
+      w0[1] = fmaf(-da, u0.y, w0[1]);
+      w0[2] = fmaf(-da, u0.z, w0[2]);
+      w0[3] = fmaf(-da, u0.w, w0[3]);
+      w0[4] = fmaf(-da, u1.x, w0[4]);
+      w0[5] = fmaf(-da, u1.y, w0[5]);
+      w0[6] = fmaf(-da, u1.z, w0[6]);
+      w0[7] = fmaf(-da, u1.w, w0[7]);
+      w1[0] = fmaf(-db, u0.x, w1[0]);
+      w1[1] = fmaf(-db, u0.y, w1[1]);
+      w1[2] = fmaf(-db, u0.z, w1[2]);
+      w1[3] = fmaf(-db, u0.w, w1[3]);
+      w1[4] = fmaf(-db, u1.x, w1[4]);
+      w1[5] = fmaf(-db, u1.y, w1[5]);
+      w1[6] = fmaf(-db, u1.z, w1[6]);
+      w1[7] = fmaf(-db, u1.w, w1[7]);
+      curA = fmaf(-da, usup, preA);
+      curB = fmaf(-db, usup, preB);
+    }
+    {  // slot 0 of lane l now holds the final weight of column 16 R + l
+      const int col = kLanesPerRow * R + l;
+      float cA, cB;
+      quant_pair(w0[0], sA, rsA, w1[0], sB, rsB, cA, cB);
+      dst[rlA * LD + col] = fmaf(-cA, sA, w0[0]);
+      dst[rlB * LD + col] = fmaf(-cB, sB, w1[0]);
+      code_s[rlA * kBlk + col] = static_cast<int8_t>(cA);
+      code_s[rlB * kBlk + col] = static_cast<int8_t>(cB);
     }
 #pragma unroll
     for (int m = 0; m < kSlots - 1; ++m) {
@@ -236,13 +261,18 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
     w0[kSlots - 1] = 0.f;
     w1[kSlots - 1] = 0.f;
   }
+  if (GS == 0 && l == 0) {
+    scl_s[rlA * 4] = sA;
+    scl_s[rlB * 4] = sB;
+  }
   __syncthreads();
 
-  // errors -> panel buffer (coalesced rows), codes -> packed bytes, scales, qerr partials
-  for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
+  // residuals -> panel buffer (coalesced rows), codes -> packed bytes, scales, qerr partials
+  const int nwarps = static_cast<int>(blockDim.x / 32);
+  for (int r = warp; r < rows; r += nwarps) {
     if (r0 + r >= a.N) break;
-    const float* src = stage + r * LD + 4 * lane;
-    const float4 e4 = make_float4(src[0], src[1], src[2], src[3]);
+    const float* srcr = dst + r * LD + 4 * lane;
+    const float4 e4 = make_float4(srcr[0], srcr[1], srcr[2], srcr[3]);
     if (a.Err_lo == nullptr) {
       reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = e4;
     } else {  // split for the 3xTF32 updates: tf32 part (low 13 mantissa bits cleared) + remainder
@@ -262,30 +292,44 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
   }
   if (GS != 0) {
     constexpr int ng = (GS == 0) ? 1 : kBlk / GS;
-    for (int e = tid; e < kRowsPerCta * ng; e += kSweepThreads) {
+    for (int e = tid; e < rows * ng; e += blockDim.x) {
       const int r = e / ng, g = e % ng;
       if (r0 + r < a.N) a.scales[(r0 + r) * (K / (GS == 0 ? 1 : GS)) + j0 / (GS == 0 ? 1 : GS) + g] = scl_s[r * 4 + g];
     }
   }
+  // qerr partial sums over the ORIGINAL weights in fp64: warp w takes rows w + i * nwarps
+  // (i < 4, exactly the CTA's rows), lane columns 4 lane .. 4 lane + 3; all loads issued first
   double num = 0.0, den = 0.0;
-  for (int r = warp; r < kRowsPerCta; r += kSweepThreads / 32) {
-    if (r0 + r >= a.N) break;
+  {
+    float wo[kRowsPerWarp][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int k = 4 * lane + i;
-      const double wo = static_cast<double>(load_w(a.W, a.w_dtype, (r0 + r) * K + j0 + k));
-      const double sc = static_cast<double>(GS != 0 ? scl_s[r * 4 + k / (GS == 0 ? 1 : GS)] : scl_s[r * 4]);
-      const double q = static_cast<double>(code_s[r * kBlk + k]) * sc;
-      const double im = a.imp != nullptr ? static_cast<double>(a.imp[j0 + k]) : 1.0;
-      num += im * (wo - q) * (wo - q);
-      den += im * wo * wo;
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+      const int64_t row = r0 + warp + i * nwarps;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) wo[i][c] = row < a.N ? load_w(a.W, a.w_dtype, row * K + j0 + 4 * lane + c) : 0.f;
+    }
+    float im[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) im[c] = a.imp != nullptr ? a.imp[j0 + 4 * lane + c] : 1.f;
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+      const int r = warp + i * nwarps;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int k = 4 * lane + c;
+        const double w64 = static_cast<double>(wo[i][c]);
+        const double sc = static_cast<double>(GS != 0 ? scl_s[r * 4 + k / (GS == 0 ? 1 : GS)] : scl_s[r * 4]);
+        const double q = static_cast<double>(code_s[r * kBlk + k]) * sc;
+        num += static_cast<double>(im[c]) * (w64 - q) * (w64 - q);
+        den += static_cast<double>(im[c]) * w64 * w64;
+      }
     }
   }
   for (int off = 16; off > 0; off >>= 1) {
     num += __shfl_down_sync(0xffffffffu, num, off);
     den += __shfl_down_sync(0xffffffffu, den, off);
   }
-  __shared__ double red[kSweepThreads / 32][2];
+  __shared__ double red[kMaxSweepThreads / 32][2];
   if (lane == 0) {
     red[warp][0] = num;
     red[warp][1] = den;
@@ -293,7 +337,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
   __syncthreads();
   if (tid == 0) {
     double sn = 0.0, sd = 0.0;
-    for (int wq = 0; wq < kSweepThreads / 32; ++wq) {
+    for (int wq = 0; wq < nwarps; ++wq) {
       sn += red[wq][0];
       sd += red[wq][1];
     }
@@ -302,9 +346,6 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_kernel(SweepArgs a,
     p[1] = sd;
   }
 }
-
-constexpr size_t kSweepSmem =
-    (kBlk * kBlk + kRowsPerCta * (kBlk + 1) + kRowsPerCta * 4 + kBlk) * sizeof(float) + kRowsPerCta * kBlk;
 
 __global__ void w_prep_kernel(const void* __restrict__ W, int dt, int64_t n, float* __restrict__ Wf) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
@@ -351,7 +392,7 @@ hq_status launch_qerr_finalize(const double* partials, int64_t count, WsHeader* 
 bool gptq_shape_ok(int64_t N, int64_t K, int64_t group) {
   if (N < 1 || K < kBlk || K % kBlk != 0 || group < 32 || group % 32 != 0 || K % group != 0) return false;
   if (!(group == 32 || group == 64 || group == 128 || group % kBlk == 0)) return false;
-  if (K > 65536 || N > (int64_t(1) << 31) - kRowsPerCta) return false;
+  if (K > 65536 || N > (int64_t(1) << 31) - kMaxRowsPerCta) return false;
   return true;
 }
 
@@ -366,7 +407,8 @@ static int64_t panel_width(int64_t K, int64_t group) {
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   GptqLayout L{};
   const size_t al = 256;
-  L.sweep_grid = static_cast<int>(ceil_div(N, kRowsPerCta));
+  L.sweep_rows = sweep_rows_per_cta(N);
+  L.sweep_grid = static_cast<int>(ceil_div(N, int64_t(L.sweep_rows)));
   const int64_t P = panel_width(K, group);
   size_t off = 0;
   L.header = off;
@@ -379,7 +421,7 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
   L.err_lo = off;  // remainder part of the errors for the 3xTF32 updates
   off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
-  L.a = off;  // fp64 A, later U^T and U in fp32
+  L.a = off;  // fp64 A, later U'^T and the packed diagonal blocks of U' in fp32
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.x = off;
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
@@ -391,7 +433,7 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   return L;
 }
 
-// W[:, c0 : c0+ncols] -= E[:, 0:kred] * U[k0 : k0+kred, c0 : c0+ncols]   (E row stride lde)
+// W[:, c0 : c0+ncols] -= D[:, 0:kred] * U'[k0 : k0+kred, c0 : c0+ncols]   (residuals D, row stride lde)
 static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
                               const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut,
                               const float* Ut_hi, const float* Ut_lo, const int* info, int* status, cudaStream_t s);
@@ -416,8 +458,8 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   float* Ut_hi = nullptr;
   float* Ut_lo = nullptr;
   const bool split = (update_impl == 0);  // 3xTF32 updates take pre-split operands
-  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, split, &Ut_hi,
-                               &Ut_lo, s);
+  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, true, split,
+                               &Ut_hi, &Ut_lo, s);
   if (st != HQ_OK) return st;
 
   {
@@ -432,7 +474,7 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   a.Wf = Wf;
   a.N = N;
   a.K = K;
-  a.U = U;
+  a.Upack = U;
   a.group = static_cast<int>(group);
   a.Err = Err;
   a.Err_lo = split ? Err_lo : nullptr;
@@ -452,16 +494,18 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
     case 128: kern = sweep_block_kernel<128>; break;
     default: kern = sweep_block_kernel<0>; break;
   }
-  HQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSweepSmem)));
+  const size_t smem = sweep_smem_bytes(L.sweep_rows);
+  const int threads = L.sweep_rows / kRowsPerWarp * 32;
+  HQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
 
   for (int64_t p0 = 0; p0 < K; p0 += P) {
     const int64_t p1 = (p0 + P < K) ? p0 + P : K;
     for (int64_t j0 = p0; j0 < p1; j0 += kBlk) {
       a.err_col = static_cast<int>(j0 - p0);
       const int tm = timer_start(kTimeSweep, s);
-      kern<<<L.sweep_grid, kSweepThreads, kSweepSmem, s>>>(a, static_cast<int>(j0));
+      kern<<<L.sweep_grid, threads, smem, s>>>(a, static_cast<int>(j0));
       HQ_LAUNCH_CHECK();
-      // bytes: the block of working weights in, its errors out (fp32), the block of U^T, packed
+      // bytes: the block of working weights in, its residuals out (fp32), the block of U', packed
       // codes and the block's scales out
       timer_stop(tm, static_cast<double>(N) * kBlk * 8.0 + kBlk * kBlk * 4.0 + N * (kBlk / 2.0) +
                          N * (static_cast<double>(kBlk) / group) * 4.0, s);

@@ -87,20 +87,35 @@ hq_status f64_gemm(const F64Gemm& g, cudaStream_t s);
 // factor.cu: out[i] = 1 / d[i] by the leaf's Newton-Raphson reciprocal (for tests)
 hq_status launch_rcp_nr(const double* d, double* out, int64_t n, cudaStream_t s);
 
-// factor.cu: U (row-major, upper) and U^T (row-major, lower) of the damped Hessian, in fp32,
-// from an fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; U and U^T are written into
-// the first and second halves of A's storage once A is no longer needed.
-// With split_ut, also the strict lower triangle of U^T split into a tf32 part and the fp32
-// remainder (U^T = Ut_hi + Ut_lo there), in T's storage; the upper parts of Ut_hi and Ut_lo are
+// Packed diagonal blocks of U' = diag(U)^-1 U for the GPTQ sweep: block b (kSweepBlk^2 floats)
+// holds, for row j of the block, lane l (0..15) and slot m (0..7), the entry
+// U'[b kSweepBlk + j][b kSweepBlk + c] with c = 16 (j / 16 + m) + l when j < c < kSweepBlk,
+// and 0 otherwise (on and below the diagonal, and past the block).  A lane's 8 slots are two
+// 16-byte chunks, swapped for lanes 4-7 and 12-15 so that eight lanes reading chunk q of one
+// row j hit 32 different banks.
+constexpr int kSweepBlk = 128;
+__host__ __device__ __forceinline__ int sweep_upack_offset(int j, int l, int m) {
+  return ((j * 16 + l) * 2 + ((m >> 2) ^ ((l >> 2) & 1))) * 4 + (m & 3);
+}
+
+// factor.cu: the upper Cholesky factor U of the inverse of the damped Hessian, in fp32, from an
+// fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; the fp32 results are written into
+// A's storage once A is no longer needed: *Ut (first half) and *U (second half).
+//   sweep_form == false: *Ut = U^T (row-major, lower), *U = U (row-major, upper).
+//   sweep_form == true:  *Ut = U'^T with U' = diag(U)^-1 U (row-major, lower, unit diagonal),
+//                        *U = the packed diagonal blocks of U' (K / kSweepBlk blocks, see
+//                        sweep_upack_offset; K must be a multiple of kSweepBlk).
+// With split_ut, also the strict lower triangle of *Ut split into a tf32 part and the fp32
+// remainder (Ut = Ut_hi + Ut_lo there), in T's storage; the upper parts of Ut_hi and Ut_lo are
 // not written.
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        double* lam, int* info, int* status, float** Ut, float** U, bool split_ut, float** Ut_hi,
-                        float** Ut_lo, cudaStream_t s);
+                        double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form, bool split_ut,
+                        float** Ut_hi, float** Ut_lo, cudaStream_t s);
 
 // gptq.cu
 struct GptqLayout {
   size_t header, partials, wf, err, err_lo, a, x, xt, t, total;
-  int sweep_grid;
+  int sweep_rows, sweep_grid;  // rows per sweep CTA, sweep CTAs
 };
 // Device-side header at the start of the GPTQ / RTN workspace.
 struct WsHeader {
