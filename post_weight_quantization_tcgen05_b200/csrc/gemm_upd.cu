@@ -1,18 +1,20 @@
 // The GPTQ lazy trailing update on the tcgen05 tensor cores, fp32-accurate (3xTF32):
 //
 //   C[m, n] -= sum_k A(m, k) B(n, k)      m < M, n < N
-//   A(m, k) = A_hi[m * lda + k] + A_lo[m * lda + k]      (the sweep's errors E, split)
-//   B(n, k) = B_hi[n * ldb + k] + B_lo[n * ldb + k]      (U^T, split)
+//   A(m, k) = A_hi[m * lda + k] + A_lo[m * lda + k]      (the sweep's residuals D, split)
+//   B(n, k) = B_hi[n * ldb + k] + B_lo[n * ldb + k]      (U'^T, split)
 //
 // Both operands arrive split into a tf32 part (low 13 mantissa bits zero) and the fp32
 // remainder, so the kernel only streams them: the product is hi*hi + hi*lo + lo*hi, three
 // kind::tf32 MMAs per k-step into the same TMEM accumulator (about 2^-21 relative per product).
-// Persistent: one CTA per SM walks 128 x 256 output tiles; warp 0 issues TMA loads (a 4-stage
-// ring of 48 KB stages: A_hi, A_lo [128 x 16], B_hi, B_lo [256 x 16], 64-byte swizzle), warp 1
-// issues the MMAs into one of two 128 x 256 fp32 accumulators (all 512 TMEM columns), and warps
-// 2-5 drain the other accumulator into C while the next tile is being multiplied: C moves in
-// 128 x 32 chunks by TMA (load into a double-buffered shared-memory chunk, subtract there, TMA
-// store back), the next chunk's load in flight while one chunk is being worked on.
+// Persistent: one CTA per SM walks 128 x BN output tiles (BN = 256, or 128 / 64 when the
+// wide tiles would leave SMs without two tiles each, as in the small inner updates of a panel);
+// warp 0 issues TMA loads (a 4-stage ring of stages A_hi, A_lo [128 x 16], B_hi, B_lo
+// [BN x 16], 64-byte swizzle), warp 1 issues the MMAs into one of two 128 x BN fp32
+// accumulators (2 BN TMEM columns), and warps 2-5 drain the other accumulator into C while the
+// next tile is being multiplied: C moves in 128 x 32 chunks by TMA (load into a double-buffered
+// shared-memory chunk, subtract there, TMA store back), the next chunk's load in flight while
+// one chunk is being worked on.
 // Every wait is bounded; a CTA that times out records HQ_ERR_TIMEOUT and stops.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -22,17 +24,24 @@
 namespace hq {
 namespace {
 
-constexpr int kBM = 128, kBN = 256, kBK = 16;    // 16 fp32 = one 64-byte swizzled row per k-slice
+constexpr int kBM = 128, kBK = 16;                // 16 fp32 = one 64-byte swizzled row per k-slice
 constexpr int kStages = 4;
 constexpr int kATile = kBM * kBK * 4;              // 8 KB
-constexpr int kBTile = kBN * kBK * 4;              // 16 KB
-constexpr int kStage = 2 * kATile + 2 * kBTile;    // 48 KB
 constexpr int kChunk = 32;                         // epilogue: C columns per TMA round trip
 constexpr int kCBuf = kBM * kChunk * 4;            // 16 KB, 128-byte swizzled rows
 constexpr int kEpiBytes = 2 * kCBuf;               // double-buffered C chunks
-constexpr int kSmem = kStages * kStage + kEpiBytes + 1024 + 256;
 constexpr int kThreads = 192;
 constexpr int kSMs = 148;
+
+// Tile width BN (256, 128 or 64 output columns): the narrow tiles spread the small inner
+// updates of a panel over more SMs.
+template <int BN>
+struct UpdTile {
+  static constexpr int kBTile = BN * kBK * 4;             // 16 / 8 / 4 KB
+  static constexpr int kStage = 2 * kATile + 2 * kBTile;  // 48 / 32 / 24 KB
+  static constexpr int kSmem = kStages * kStage + kEpiBytes + 1024 + 256;
+  static constexpr int kTmemCols = 2 * BN;                // two accumulators
+};
 
 struct UpdArgs {
   float* C;
@@ -43,10 +52,14 @@ struct UpdArgs {
   int* status;
 };
 
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     upd_gemm_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
                     const __grid_constant__ CUtensorMap mBh, const __grid_constant__ CUtensorMap mBl,
                     const __grid_constant__ CUtensorMap mC, UpdArgs args) {
+  constexpr int kBN = BN;
+  constexpr int kBTile = UpdTile<BN>::kBTile;
+  constexpr int kStage = UpdTile<BN>::kStage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* cbuf = smem + kStages * kStage;  // two C chunks
@@ -79,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_barrier_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_alloc(tmem_slot, UpdTile<BN>::kTmemCols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -242,18 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 512);
+    ptx::tmem_dealloc(tmem, UpdTile<BN>::kTmemCols);
   }
 }
 
 }  // namespace
 
-hq_status upd_gemm(const UpdGemm& g, cudaStream_t s) {
-  if (g.M <= 0 || g.N <= 0 || g.Kred <= 0) return HQ_OK;
-  const void* ptrs[5] = {g.A_hi, g.A_lo, g.B_hi, g.B_lo, g.C};
-  for (const void* p : ptrs)
-    if (!aligned(p, 16)) return HQ_ERR_UNSUPPORTED;
-  if (g.lda % 4 != 0 || g.ldb % 4 != 0 || g.ldc % 4 != 0) return HQ_ERR_UNSUPPORTED;
+template <int BN>
+static hq_status upd_gemm_bn(const UpdGemm& g, cudaStream_t s) {
   const uint64_t kred = static_cast<uint64_t>(g.Kred);
   CUtensorMap mAh, mAl, mBh, mBl, mC;
   if (!make_tmap_2d(&mAh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.A_hi, kred, static_cast<uint64_t>(g.M),
@@ -261,9 +270,9 @@ hq_status upd_gemm(const UpdGemm& g, cudaStream_t s) {
       !make_tmap_2d(&mAl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.A_lo, kred, static_cast<uint64_t>(g.M),
                     static_cast<uint64_t>(g.lda) * 4, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_tmap_2d(&mBh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.B_hi, kred, static_cast<uint64_t>(g.N),
-                    static_cast<uint64_t>(g.ldb) * 4, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_64B) ||
+                    static_cast<uint64_t>(g.ldb) * 4, kBK, BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_tmap_2d(&mBl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.B_lo, kred, static_cast<uint64_t>(g.N),
-                    static_cast<uint64_t>(g.ldb) * 4, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_64B) ||
+                    static_cast<uint64_t>(g.ldb) * 4, kBK, BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_tmap_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.C, static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M),
                     static_cast<uint64_t>(g.ldc) * 4, kChunk, kBM))
     return HQ_ERR_CUDA;
@@ -274,18 +283,32 @@ hq_status upd_gemm(const UpdGemm& g, cudaStream_t s) {
   a.N = g.N;
   a.Kred = g.Kred;
   a.tiles_m = static_cast<int>(ceil_div(g.M, kBM));
-  a.tiles_n = static_cast<int>(ceil_div(g.N, kBN));
+  a.tiles_n = static_cast<int>(ceil_div(g.N, BN));
   a.skip = g.skip;
   a.status = g.status;
   const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
   if (ntiles > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(ntiles < kSMs ? ntiles : kSMs);
-  HQ_CUDA_TRY(cudaFuncSetAttribute(upd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+  constexpr int smem = UpdTile<BN>::kSmem;
+  HQ_CUDA_TRY(cudaFuncSetAttribute(upd_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int tm = timer_start(kTimeTf32Gemm, s);
-  upd_gemm_kernel<<<grid, kThreads, kSmem, s>>>(mAh, mAl, mBh, mBl, mC, a);
+  upd_gemm_kernel<BN><<<grid, kThreads, smem, s>>>(mAh, mAl, mBh, mBl, mC, a);
   HQ_LAUNCH_CHECK();
   timer_stop(tm, 2.0 * g.M * g.N * static_cast<double>(g.Kred), s);  // the product's flops
   return HQ_OK;
+}
+
+// The widest tile that still gives every SM two tiles, else the narrowest.
+hq_status upd_gemm(const UpdGemm& g, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0 || g.Kred <= 0) return HQ_OK;
+  const void* ptrs[5] = {g.A_hi, g.A_lo, g.B_hi, g.B_lo, g.C};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return HQ_ERR_UNSUPPORTED;
+  if (g.lda % 4 != 0 || g.ldb % 4 != 0 || g.ldc % 4 != 0) return HQ_ERR_UNSUPPORTED;
+  const int64_t tm = ceil_div(static_cast<int64_t>(g.M), int64_t(kBM));
+  if (tm * ceil_div(static_cast<int64_t>(g.N), int64_t(256)) >= 2 * kSMs) return upd_gemm_bn<256>(g, s);
+  if (tm * ceil_div(static_cast<int64_t>(g.N), int64_t(128)) >= 2 * kSMs) return upd_gemm_bn<128>(g, s);
+  return upd_gemm_bn<64>(g, s);
 }
 
 }  // namespace hq
