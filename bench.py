@@ -252,7 +252,7 @@ def run_ours(args, rank, world, local_rank):
     return return_line
 
 
-def time_layer(hq, cfg, dev, flush, steps: int = 2, warmup: int = 1):
+def time_layer(hq, cfg, dev, flush, steps: int = 2, warmup: int = 1, peaks=None):
     """Whole-path steps on one layer of `cfg` (the main measurement's protocol, fewer steps)."""
     layer = Layer(hq, cfg, dev)
     for _ in range(warmup):
@@ -271,6 +271,11 @@ def time_layer(hq, cfg, dev, flush, steps: int = 2, warmup: int = 1):
            "steps": steps, "ms_per_step": step_ms, "weights_per_s": cfg.N * cfg.K / (step_ms / 1e3),
            "gptq_quantize_ms": gptq_ms, "gptq_weights_per_s": cfg.N * cfg.K / (gptq_ms / 1e3),
            "syrk_ms": syrk_ms, "xtx_tflops": cfg.T * cfg.K * (cfg.K + 1) / (syrk_ms / 1e3) / 1e12}
+    if peaks is not None:  # kernel-level rooflines of the two tensor-core stages (one more step)
+        kernels = kernel_breakdown(hq, layer, flush, steps=1)
+        out["syrk_roofline"] = syrk_line(kernels, out["xtx_tflops"], peaks)
+        out["update_roofline"] = update_line(cfg, kernels, peaks)
+        out["kernels_ms"] = {k: v["ms_per_step"] for k, v in kernels.items()}
     del layer
     torch.cuda.empty_cache()
     return out
@@ -322,7 +327,7 @@ def other_configs(hq, dev, flush, peaks):
     out = {}
     for idx in (2, 3):
         cfg = wl.CONFIGS[idx]
-        out[cfg.name] = time_layer(hq, cfg, dev, flush)
+        out[cfg.name] = time_layer(hq, cfg, dev, flush, peaks=peaks)
     out["hessian_at_scale"] = time_hessian_at_scale(hq, wl.CONFIGS[4], dev, flush, peaks)
     return out
 
@@ -334,13 +339,38 @@ KERNEL_NAMES = {"f64_gemm_128": ("f64_gemm_kernel<128>", "TFLOP/s"),
                 "f64_gemm_64": ("f64_gemm_kernel<64> + split-K reduce", "TFLOP/s"),
                 "leaf": ("chol_inv_leaf_kernel", "TFLOP/s"),
                 "sweep": ("sweep_block_kernel", "GB/s"),
-                "tf32_gemm": ("tf32_gemm_kernel (3xTF32 lazy updates)", "TFLOP/s"),
+                "tf32_gemm": ("upd_gemm_kernel<BN> (3xTF32 lazy updates)", "TFLOP/s"),
                 "syrk": ("umma_gemm_kernel<kSyrkBF16>", "TFLOP/s")}
 # fp64 tensor-core peak: no measured figure exists for fp64, so the measured bf16 burst is scaled
 # by NVIDIA's nominal dense ratio for B200 (fp64 tensor 37 TFLOP/s : bf16 2250 TFLOP/s)
 FP64_OVER_BF16 = 37.0 / 2250.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "f64_gemm_kernel_128_q_proj.md")
 KERNEL_SOURCE = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "csrc", "gemm_f64.cu")
+
+
+def update_roofline_ms(cfg, peaks) -> float:
+    """Sum over the sweep's lazy-update launches of each launch's roofline time: the larger of
+    its tensor time (three tf32 MMAs per product at the tf32 peak, taken as half the measured
+    bf16 burst, NVIDIA's nominal dense ratio) and its DRAM time at the measured HBM rate (C read
+    and written, the split residuals and the split U' block read once, 4 bytes each)."""
+    N, K = cfg.N, cfg.K
+    P = min(512 if cfg.group <= 128 else cfg.group * max(512 // cfg.group, 1), K)
+    tf32 = peaks["bf16_tflops"] * 1e12 / 2.0
+    hbm = peaks["hbm_gbs"] * 1e9
+    launches = []
+    for p0 in range(0, K, P):
+        p1 = min(p0 + P, K)
+        for j0 in range(p0, p1, 128):
+            if j0 + 128 < p1:
+                launches.append((p1 - j0 - 128, 128))
+        if p1 < K:
+            launches.append((K - p1, p1 - p0))
+    total = 0.0
+    for ncols, kred in launches:
+        flops = 3 * 2.0 * N * ncols * kred
+        nbytes = 8.0 * N * ncols + 8.0 * N * kred + 8.0 * ncols * kred
+        total += max(flops / tf32, nbytes / hbm)
+    return total * 1e3
 
 
 def kernel_breakdown(hq, layer, flush, steps: int = 2):
@@ -468,6 +498,29 @@ def measure_e2e(args, layer, flush, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def syrk_line(kernels, stage_tflops, peaks):
+    """The SYRK kernel against the bf16 peak: `achieved` from the kernel's own launch events,
+    `stage_achieved` from the stage events (which also hold the zeroing of H and launch gaps)."""
+    k = kernels.get("syrk") if kernels else None
+    achieved = k["achieved"] if k else stage_tflops
+    return {"kernel": "umma_gemm_kernel<kSyrkBF16> (X^T X)", "bound": "tensor", "achieved": achieved,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "stage_achieved": stage_tflops, "peak_source": peaks["source"] + " bf16 dense burst"}
+
+
+def update_line(cfg, kernels, peaks):
+    """The lazy updates against their per-launch roofline (update_roofline_ms)."""
+    k = kernels.get("tf32_gemm") if kernels else None
+    if not k:
+        return None
+    roof = update_roofline_ms(cfg, peaks)
+    return {"kernel": "upd_gemm_kernel<BN> (3xTF32 lazy updates)", "bound": "tensor / hbm per launch",
+            "ms_per_step": k["ms_per_step"], "roofline_ms_per_step": roof, "frac": roof / k["ms_per_step"],
+            "achieved_useful_tflops": k["achieved"], "launches_per_step": k["launches_per_step"],
+            "peak_source": (peaks["source"] + " bf16 dense burst / 2 (nominal tf32 ratio), 3 MMAs per product; "
+                            + peaks["source"] + " HBM copy")}
+
+
 def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops, enc_bytes,
                dec_bytes, peaks, e2e, launches, clocks, dom, kernels, fp64_peak_measured):
     dom_ms, dom_flop, dom_n = dom
@@ -505,10 +558,8 @@ def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, d
                       "decode": dec_bytes / (statistics.mean(dec_ms) / 1e3) / 1e9},
         "roofline": roofline,
         "kernels": kernels,
-        "syrk_roofline": {"kernel": "umma_gemm_kernel<kSyrkBF16> (X^T X)", "bound": "tensor",
-                          "achieved": syrk_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                          "frac": syrk_tflops / peaks["bf16_tflops"],
-                          "peak_source": peaks["source"] + " bf16 dense burst"},
+        "syrk_roofline": syrk_line(kernels, syrk_tflops, peaks),
+        "update_roofline": update_line(cfg, kernels, peaks),
         "e2e": e2e,
         "gpu_launches": int(launches) * args.steps,
         "gpu_launches_per_step": int(launches),
