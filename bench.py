@@ -340,7 +340,7 @@ KERNEL_NAMES = {"f64_gemm_128": ("f64_gemm_kernel<128>", "TFLOP/s"),
                 "leaf": ("chol_inv_leaf_kernel", "TFLOP/s"),
                 "sweep": ("sweep_block_kernel", "GB/s"),
                 "tf32_gemm": ("upd_gemm_kernel<BN> (3xTF32 lazy updates)", "TFLOP/s"),
-                "syrk": ("umma_gemm_kernel<kSyrkBF16>", "TFLOP/s")}
+                "syrk": ("syrk_tc_kernel (persistent tcgen05 SYRK)", "TFLOP/s")}
 # fp64 tensor-core peak: no measured figure exists for fp64, so the measured bf16 burst is scaled
 # by NVIDIA's nominal dense ratio for B200 (fp64 tensor 37 TFLOP/s : bf16 2250 TFLOP/s)
 FP64_OVER_BF16 = 37.0 / 2250.0
@@ -503,7 +503,7 @@ def syrk_line(kernels, stage_tflops, peaks):
     `stage_achieved` from the stage events (which also hold the zeroing of H and launch gaps)."""
     k = kernels.get("syrk") if kernels else None
     achieved = k["achieved"] if k else stage_tflops
-    return {"kernel": "umma_gemm_kernel<kSyrkBF16> (X^T X)", "bound": "tensor", "achieved": achieved,
+    return {"kernel": "syrk_tc_kernel (X^T X)", "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
             "stage_achieved": stage_tflops, "peak_source": peaks["source"] + " bf16 dense burst"}
 

@@ -1,16 +1,30 @@
 // Calibration Hessian accumulation H += X^T X over the lower triangle of H.
 //
-// bf16 X with K a multiple of 8 and a 16-byte aligned base goes through the tcgen05 GEMM
-// (gemm_tc.cuh, kSyrkBF16): TMA brings 64-token x 64-channel bf16 boxes, the tensor core
-// multiplies them as MN-major operands and accumulates 1024-token segments in TMEM in fp32,
-// and the segments are summed in fp32 registers.  Every other input
-// (fp32 X, odd K, unaligned X) takes the fp32 CUDA-core kernel below, which computes the same
-// sum with exact products and fp32 accumulation.
+// bf16 X with K a multiple of 8 and a 16-byte aligned base goes through the persistent tcgen05
+// kernel below; every other input (fp32 X, odd K, unaligned X) takes the fp32 CUDA-core kernel,
+// which computes the same sum with exact products and fp32 accumulation.
+//
+// Tensor-core path: one CTA per SM walks 128 x 256 lower-triangle tiles of H (static round
+// robin; all tiles cost the same).  Warp 0 issues TMA loads of 64-token x 64-channel bf16 boxes
+// into a 4-stage ring of 48 KB stages (A: channels m0..m0+127, B: n0..n0+255, both MN-major);
+// warp 1 allocates all 512 TMEM columns and issues kind::f16 MMAs from one thread; warps 2-9
+// drain the accumulators.  The tensor core's fp32 accumulation loses precision in proportion to
+// the number of MMAs chained into one accumulator (measured: 1.2e-5 relative Frobenius error
+// after 256 chained K=16 steps; 4096-token segments failed the 1e-5 budget), so at most
+// kSyrkSegK tokens (64 MMAs) are chained per accumulator: two 256-column accumulators alternate
+// segment by segment, across tile boundaries too, and the epilogue warps (two per TMEM lane
+// quadrant, 128 columns each) add every finished segment into fp32 registers while the tensor
+// core fills the other accumulator.  After a tile's last segment each thread adds its row's 128
+// sums to H with 16-byte read-modify-writes (lower part only), which overlaps the next tile's
+// first segments.
+//
+// Every wait is bounded: on expiry the CTA records HQ_ERR_TIMEOUT, waits (bounded) for its
+// in-flight TMA and MMA work, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
-#include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 #include "tmap.cuh"
 
 namespace hq {
@@ -95,6 +109,226 @@ hq_status launch_syrk_simt(float* H, const void* X, int x_dtype, int64_t T, int6
 
 // ---------------------------------------------------------------- tensor-core path
 
+constexpr int kSyBM = 128;
+constexpr int kSyBN = 256;
+constexpr int kSyBK = 64;               // tokens per stage
+constexpr int kSyStages = 4;
+constexpr int kSyStageBytes = 49152;    // A 16 KB + B 32 KB
+constexpr int kSySmem = kSyStages * kSyStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kSyrkSegK = 1024;         // tokens chained in one TMEM accumulator
+constexpr int kSySegIters = kSyrkSegK / kSyBK;
+constexpr int kSyEpiWarps = 8;
+constexpr int kSyThreads = 64 + 32 * kSyEpiWarps;
+constexpr int kSySMs = 148;
+
+// Lower-triangle tile enumeration of a K x K output with 128 x 256 tiles: tile row bi holds
+// column tiles bj with bj * 256 <= bi * 128 + 127.
+__host__ __device__ inline int syrk_tiles_in_row(int bi, int tiles_n) {
+  int c = (bi * kSyBM + kSyBM - 1) / kSyBN + 1;
+  return c < tiles_n ? c : tiles_n;
+}
+
+__device__ inline void syrk_tile_coords(int t, int tiles_n, int& m0, int& n0) {
+  int bi = 0;
+  while (true) {
+    const int c = syrk_tiles_in_row(bi, tiles_n);
+    if (t < c) break;
+    t -= c;
+    ++bi;
+  }
+  m0 = bi * kSyBM;
+  n0 = t * kSyBN;
+}
+
+struct SyrkArgs {
+  float* H;
+  int K;         // H is K x K, row-major
+  int T;         // tokens
+  int tiles;     // lower-triangle tiles
+  int* status;
+};
+
+__global__ void __launch_bounds__(kSyThreads, 1)
+    syrk_tc_kernel(const __grid_constant__ CUtensorMap mapX, SyrkArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSyStages * kSyStageBytes);
+  uint64_t* empty = full + kSyStages;
+  uint64_t* accf = empty + kSyStages;  // [2] accumulator filled
+  uint64_t* acce = accf + 2;           // [2] accumulator drained
+  uint64_t* drain = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tiles_n = (args.K + kSyBN - 1) / kSyBN;
+  const int kiters = (args.T + kSyBK - 1) / kSyBK;
+  const int nseg = (kiters + kSySegIters - 1) / kSySegIters;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSyStages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&accf[a], 1);
+      ptx::mbar_init(&acce[a], kSyEpiWarps);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    record_status(args.status, HQ_ERR_TIMEOUT);
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    ptx::prefetch_tensormap(&mapX);
+    int g = 0;  // stages issued by this CTA
+    bool ok = true;
+    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
+      int m0, n0;
+      syrk_tile_coords(t, tiles_n, m0, n0);
+      for (int k = 0; k < kiters; ++k, ++g) {
+        const int s = g % kSyStages;
+        if (g >= kSyStages && !ptx::mbar_wait(&empty[s], ((g / kSyStages) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * kSyStageBytes;
+        uint8_t* sb = sa + 16384;
+        const int t0 = k * kSyBK;
+        ptx::mbar_arrive_expect_tx(&full[s], kSyStageBytes);
+        ptx::tma_load_2d(sa, &mapX, m0, t0, &full[s]);
+        ptx::tma_load_2d(sa + 8192, &mapX, m0 + 64, t0, &full[s]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tma_load_2d(sb + c * 8192, &mapX, n0 + 64 * c, t0, &full[s]);
+      }
+    }
+    if (!ok) {
+      fail();
+      // let the copies already issued land before the CTA's shared memory goes away
+      const int first = g > kSyStages ? g - kSyStages : 0;
+      for (int k = first; k < g; ++k) ptx::mbar_wait(&full[k % kSyStages], (k / kSyStages) & 1, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdesc = ptx::idesc(ptx::kFmtBF16, kSyBM, kSyBN, true, true);
+    bool ok = true;
+    int g = 0;   // stages consumed
+    int sg = 0;  // segments issued (accumulator = sg & 1)
+    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
+      int k = 0;
+      for (int seg = 0; seg < nseg && ok; ++seg, ++sg) {
+        const int acc = sg & 1;
+        if (sg >= 2 && !ptx::mbar_wait(&acce[acc], ((sg >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t dacc = tmem + static_cast<uint32_t>(acc * kSyBN);
+        const int kbeg = seg * kSySegIters;
+        const int kend = (kiters < kbeg + kSySegIters) ? kiters : kbeg + kSySegIters;
+        for (; k < kend; ++k, ++g) {
+          const int s = g % kSyStages;
+          if (!ptx::mbar_wait(&full[s], (g / kSyStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = ptx::smem_u32(smem + s * kSyStageBytes);
+          const uint32_t sb = sa + 16384;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // MN-major: 64-element chunks 8 KB apart (LBO), 8-row groups 1 KB apart (SBO);
+            // each MMA consumes 16 tokens = 2 KB.
+            const uint64_t ad = ptx::sdesc_sw128(sa + kk * 2048, 8192, 1024);
+            const uint64_t bd = ptx::sdesc_sw128(sb + kk * 2048, 8192, 1024);
+            ptx::mma_bf16(dacc, ad, bd, kIdesc, (k > kbeg || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(&empty[s]);
+        }
+        if (ok) ptx::mma_commit(&accf[acc]);
+      }
+    }
+    if (!ok) {
+      fail();
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, nullptr);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;             // TMEM lane quadrant this warp may access
+    const int h = (warp - 2) >> 2;      // which 128-column half of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const bool vec = (reinterpret_cast<uintptr_t>(args.H) & 15) == 0 && (args.K % 4) == 0;
+    bool ok = true;
+    int sg = 0;
+    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
+      int m0, n0;
+      syrk_tile_coords(t, tiles_n, m0, n0);
+      float sum[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) sum[i] = 0.f;
+      for (int seg = 0; seg < nseg; ++seg, ++sg) {
+        const int acc = sg & 1;
+        if (!ptx::mbar_wait(&accf[acc], (sg >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        ptx::tmem_add128(tmem + lane_off + static_cast<uint32_t>(acc * kSyBN + h * 128), sum);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&acce[acc]);
+      }
+      if (!ok) break;
+      // row `row`, columns c0 .. c0 + 127 of H += sum (lower part only)
+      const int row = m0 + q * 32 + lane;
+      if (row < args.K) {
+        float* hrow = args.H + static_cast<int64_t>(row) * args.K;
+        const int c0 = n0 + h * 128;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int col = c0 + 4 * k;
+          if (vec && col + 3 <= row && col + 3 < args.K) {
+            float4 o = *reinterpret_cast<float4*>(hrow + col);
+            o.x += sum[4 * k];
+            o.y += sum[4 * k + 1];
+            o.z += sum[4 * k + 2];
+            o.w += sum[4 * k + 3];
+            *reinterpret_cast<float4*>(hrow + col) = o;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (col + e <= row && col + e < args.K) hrow[col + e] += sum[4 * k + e];
+          }
+        }
+      }
+    }
+    if (!ok) fail();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
 bool syrk_tc_eligible(const void* X, int x_dtype, int64_t T, int64_t K) {
   return x_dtype == HQ_BF16 && (K % 8) == 0 && aligned(X, 16) && K <= (1 << 24) && T <= 0x7FFFFFFF;
 }
@@ -104,21 +338,21 @@ hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev
   if (!make_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K), static_cast<uint64_t>(T),
                     static_cast<uint64_t>(K) * 2, 64, 64))
     return HQ_ERR_CUDA;
-  HQ_CUDA_TRY(cudaFuncSetAttribute(umma_gemm_kernel<GemmMode::kSyrkBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   kGemmSmemBytes));
-  const int tiles_m = static_cast<int>(ceil_div(K, kGemmBM));
-  const int tiles_n = static_cast<int>(ceil_div(K, kGemmBN));
+  HQ_CUDA_TRY(cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSySmem));
+  const int tiles_m = static_cast<int>(ceil_div(K, kSyBM));
+  const int tiles_n = static_cast<int>(ceil_div(K, kSyBN));
   int64_t tiles = 0;
   for (int bi = 0; bi < tiles_m; ++bi) tiles += syrk_tiles_in_row(bi, tiles_n);
-  GemmArgs a{};
-  a.C = H;
-  a.ldc = K;
-  a.M = static_cast<int>(K);
-  a.Ncols = static_cast<int>(K);
-  a.Kred = static_cast<int>(T);
+  if (tiles > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
+  SyrkArgs a{};
+  a.H = H;
+  a.K = static_cast<int>(K);
+  a.T = static_cast<int>(T);
+  a.tiles = static_cast<int>(tiles);
   a.status = dev_status;
+  const int grid = static_cast<int>(tiles < kSySMs ? tiles : kSySMs);
   const int tm = timer_start(kTimeSyrk, s);
-  umma_gemm_kernel<GemmMode::kSyrkBF16><<<static_cast<unsigned>(tiles), gemm_threads(GemmMode::kSyrkBF16), kGemmSmemBytes, s>>>(map, map, a);
+  syrk_tc_kernel<<<grid, kSyThreads, kSySmem, s>>>(map, a);
   HQ_LAUNCH_CHECK();
   timer_stop(tm, static_cast<double>(T) * K * (K + 1), s);  // 2 flops x T x K (K + 1) / 2 lower entries
   return HQ_OK;
