@@ -128,16 +128,38 @@ __host__ __device__ inline int syrk_tiles_in_row(int bi, int tiles_n) {
   return c < tiles_n ? c : tiles_n;
 }
 
-__device__ inline void syrk_tile_coords(int t, int tiles_n, int& m0, int& n0) {
-  int bi = 0;
-  while (true) {
-    const int c = syrk_tiles_in_row(bi, tiles_n);
-    if (t < c) break;
-    t -= c;
-    ++bi;
+// Tile order: bands of kSyBand tile rows; inside a band column-tile by column-tile, and inside a
+// column down the band's rows that hold it.  The 148 tiles in flight at a time then cover a
+// compact block of H, so the X columns they read are few and shared through L2.
+constexpr int kSyBand = 16;
+
+__device__ inline void syrk_tile_coords(int t, int tiles_m, int tiles_n, int& m0, int& n0) {
+  for (int r0 = 0; r0 < tiles_m; r0 += kSyBand) {
+    const int r1 = r0 + kSyBand < tiles_m ? r0 + kSyBand : tiles_m;
+    int band = 0;
+    for (int bi = r0; bi < r1; ++bi) band += syrk_tiles_in_row(bi, tiles_n);
+    if (t >= band) {
+      t -= band;
+      continue;
+    }
+    for (int bj = 0;; ++bj) {
+      // rows of the band holding column tile bj: bi with syrk_tiles_in_row(bi) > bj
+      int first = r1;
+      for (int bi = r0; bi < r1; ++bi)
+        if (syrk_tiles_in_row(bi, tiles_n) > bj) {
+          first = bi;
+          break;
+        }
+      const int n = r1 - first;
+      if (t < n) {
+        m0 = (first + t) * kSyBM;
+        n0 = bj * kSyBN;
+        return;
+      }
+      t -= n;
+    }
   }
-  m0 = bi * kSyBM;
-  n0 = t * kSyBN;
+  m0 = n0 = 0;  // not reached for t < tiles
 }
 
 struct SyrkArgs {
@@ -162,6 +184,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int tiles_m = (args.K + kSyBM - 1) / kSyBM;
   const int tiles_n = (args.K + kSyBN - 1) / kSyBN;
   const int kiters = (args.T + kSyBK - 1) / kSyBK;
   const int nseg = (kiters + kSySegIters - 1) / kSySegIters;
@@ -200,7 +223,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
       int m0, n0;
-      syrk_tile_coords(t, tiles_n, m0, n0);
+      syrk_tile_coords(t, tiles_m, tiles_n, m0, n0);
       for (int k = 0; k < kiters; ++k, ++g) {
         const int s = g % kSyStages;
         if (g >= kSyStages && !ptx::mbar_wait(&empty[s], ((g / kSyStages) - 1) & 1, abort_flag)) {
@@ -278,7 +301,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
     int sg = 0;
     for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
       int m0, n0;
-      syrk_tile_coords(t, tiles_n, m0, n0);
+      syrk_tile_coords(t, tiles_m, tiles_n, m0, n0);
       float sum[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) sum[i] = 0.f;
