@@ -655,7 +655,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the gate_up / down_proj / Hessian-at-scale measurements after the main line")
+    ap.add_argument("--profile-case", choices=["step"], default=None,
+                    help="run one untimed step of the configuration on cuda:0 and exit (for ncu captures)")
     args = ap.parse_args()
+
+    if args.profile_case == "step":
+        import post_weight_quantization_tcgen05_b200 as hq
+        layer = Layer(hq, wl.CONFIGS[args.config], torch.device("cuda:0"))
+        layer.step()
+        torch.cuda.synchronize()
+        print(f"one step of {wl.CONFIGS[args.config].name} done", flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
