@@ -116,6 +116,20 @@ hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, con
                            float* scales, double* qerr_out, double* qerr_dev, void* workspace,
                            size_t workspace_bytes, hq_stream_t stream);
 
+/*
+ * The two fp64 sums behind the qerr of the last hq_gptq_quantize or hq_rtn_quantize that ran
+ * with this workspace ([gptq] qerr definition): terms_dev[0] = sum imp[k] (W[n,k] - q[n,k])^2,
+ * terms_dev[1] = sum imp[k] W[n,k]^2, so that qerr = sqrt(terms[0] / terms[1]).  For callers that
+ * split a layer's rows over several calls or devices: the sums of the parts add up (in any
+ * order, up to fp64 rounding) to the whole layer's.
+ *   workspace : the workspace of that call (device, 256-byte aligned), read only.
+ *   terms_dev : DEVICE double[2] out, written asynchronously on `stream` after the call's work
+ *               when enqueued on the same stream.
+ * Returns HQ_ERR_INVALID for NULL pointers; nothing else is checked (the workspace must hold a
+ * finished call's results).
+ */
+hq_status hq_qerr_terms(const void* workspace, double* terms_dev, hq_stream_t stream);
+
 /* Bytes of workspace hq_rtn_quantize needs (0 if the shape is invalid). */
 size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group);
 

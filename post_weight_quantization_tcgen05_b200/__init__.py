@@ -55,6 +55,7 @@ _SIGS = {
     "hq_rtn_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "hq_rtn_quantize": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hq_rtn_quantize_noalloc": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "hq_qerr_terms": (_int, [_vp, _vp, _vp]),
     "hq_bf16tril_bytes": (_sz, [_i64]),
     "hq_hessian_pack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
     "hq_hessian_unpack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
@@ -193,6 +194,12 @@ def hq_rtn_quantize_noalloc(W, group: int, codes, scales, imp=None, want_qerr: b
                                      ctypes.byref(q) if want_qerr else None, _ptr(qerr_dev), _stream(stream))
     _check(st, "hq_rtn_quantize_noalloc")
     return q.value if want_qerr else None
+
+
+def hq_qerr_terms(workspace, terms_dev, stream=None) -> None:
+    """terms_dev (fp64 [2], device) <- the qerr numerator and denominator sums of the last
+    quantisation that used `workspace`."""
+    _check(lib.hq_qerr_terms(_ptr(workspace), _ptr(terms_dev), _stream(stream)), "hq_qerr_terms")
 
 
 def hq_debug_factor(H, damp: float, Ut_out, workspace, stream=None) -> None:

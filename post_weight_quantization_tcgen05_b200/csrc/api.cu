@@ -59,6 +59,12 @@ hq_status gptq_common(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   return finish_sync(s, reinterpret_cast<const WsHeader*>(ws + L.header), qerr_out);
 }
 
+// Both the GPTQ and the RTN workspace start with the status header (layout offset 0).
+__global__ void qerr_terms_kernel(const WsHeader* __restrict__ hdr, double* __restrict__ out) {
+  out[0] = hdr->num;
+  out[1] = hdr->den;
+}
+
 }  // namespace
 
 extern "C" {
@@ -226,6 +232,14 @@ hq_status hq_rtn_quantize(const void* W, int w_dtype, int64_t N, int64_t K, int6
   if (st != HQ_OK) return st;
   if (qerr_out == nullptr) return HQ_OK;
   return finish_sync(s, reinterpret_cast<const WsHeader*>(ws), qerr_out);
+}
+
+hq_status hq_qerr_terms(const void* workspace, double* terms_dev, hq_stream_t stream) {
+  if (workspace == nullptr || terms_dev == nullptr) return HQ_ERR_INVALID;
+  qerr_terms_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<const WsHeader*>(workspace),
+                                                                     terms_dev);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
 }
 
 size_t hq_bf16tril_bytes(int64_t K) {

@@ -97,3 +97,5 @@ def test_invalid_arguments_refused_before_launch(hq):
     assert L.hq_hessian_pack_bf16tril(fake, 8, ctypes.c_void_p(258), None) == hq.HQ_ERR_INVALID  # out not 16-B aligned
     assert L.hq_hessian_unpack_bf16tril(None, 8, fake, None) == hq.HQ_ERR_INVALID
     assert L.hq_imatrix(fake, 8, 0, fake, None) == hq.HQ_ERR_INVALID
+    assert L.hq_qerr_terms(None, fake, None) == hq.HQ_ERR_INVALID
+    assert L.hq_qerr_terms(fake, None, None) == hq.HQ_ERR_INVALID
