@@ -311,14 +311,43 @@ def time_hessian_at_scale(hq, cfg, dev, flush, peaks, distinct: int = 8):
     lay.Hfull = torch.empty((K, K), dtype=torch.float32, device=dev)
     codec = codec_throughput(hq, lay, flush)
     hbm = peaks["hbm_gbs"]
+    psd = time_psd_projection(hq, lay.Hfull, peaks)  # the decoded (stored) H, as a reader gets it
     out = {"workload": f"{cfg.name}: {cfg.n_chunks} chunks of X bf16 [{cfg.chunk}, {K}] into one H",
            "syrk_ms": ms, "xtx_tflops": cfg.T * K * (K + 1) / (ms / 1e3) / 1e12,
            "xtx_frac_of_bf16_peak": cfg.T * K * (K + 1) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
            "codec": {"encode_gbs": codec["encode_gbs"], "encode_frac": codec["encode_gbs"] / hbm,
-                     "decode_gbs": codec["decode_gbs"], "decode_frac": codec["decode_gbs"] / hbm}}
+                     "decode_gbs": codec["decode_gbs"], "decode_frac": codec["decode_gbs"] / hbm},
+           "psd_projection": psd}
     del chunks, H, lay
     torch.cuda.empty_cache()
     return out
+
+
+def time_psd_projection(hq, Hstored, peaks, steps: int = 40):
+    """hq_hessian_project_psd on a copy of a decoded Hessian (one untimed call first): its time
+    and its rate against the tensor roofline of its products (three tf32 MMAs per product, tf32
+    peak taken as half the measured bf16 burst, NVIDIA's nominal dense ratio)."""
+    K = Hstored.shape[0]
+    ws = hq.alloc_workspace(hq.hq_psd_workspace_bytes(K), Hstored.device)
+    P = Hstored.clone()
+    hq.hq_hessian_project_psd(P, ws, steps=steps)
+    P.copy_(Hstored)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    hq.hq_hessian_project_psd(P, ws, steps=steps)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    flops = 4.0 * (steps + 0.5) * float(K) ** 3
+    useful = flops / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"] / 2.0 / 3.0
+    moved = float(torch.linalg.norm(P - Hstored) / torch.linalg.norm(Hstored))
+    del ws, P
+    return {"kernels": "upd_gemm_kernel<BN> (3xTF32 Newton-Schulz products) + elementwise", "K": K,
+            "steps": steps, "ms": ms, "achieved_useful_tflops": useful, "peak_useful_tflops": peak,
+            "frac": useful / peak, "relative_change": moved,
+            "peak_source": peaks["source"] + " bf16 dense burst / 2 (nominal tf32 ratio) / 3 MMAs per product"}
 
 
 def other_configs(hq, dev, flush, peaks):

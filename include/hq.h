@@ -167,6 +167,27 @@ hq_status hq_rtn_quantize_noalloc(const void* W, int w_dtype, int64_t N, int64_t
                                   const float* imp, uint8_t* codes, float* scales, double* qerr_out,
                                   double* qerr_dev, hq_stream_t stream);
 
+/* Bytes of workspace hq_hessian_project_psd needs (0 if K is unsupported). */
+size_t hq_psd_workspace_bytes(int64_t K);
+
+/*
+ * H <- its projection onto the positive semidefinite cone ([calib] "REQUIRED: project to PSD
+ * before Cholesky", "The fix"): the matrix that eigendecomposing H = V diag(l) V^T, clipping the
+ * negative eigenvalues to zero, rebuilding and symmetrising gives.  Computed without an
+ * eigendecomposition as (H + H sign(H)) / 2, sign(H) from `steps` Newton-Schulz steps
+ * X <- X (3I - X^2) / 2 on the tensor cores started at H / ||H||_F, then (P + P^T) / 2.  fp32
+ * iterates, 3xTF32 products.  An eigenvalue below about 1.5^-steps ||H||_F in magnitude is not
+ * resolved and moves the result by at most its size; 40 steps resolve 1e-7 ||H||_F.  Cost:
+ * 4 (steps + 1/2) K^3 flops.
+ *   H         : fp32 [K, K] device, both triangles (e.g. from hq_hessian_unpack_bf16tril),
+ *               symmetric; overwritten.  16-byte aligned, K a multiple of 4, K <= 65536.
+ *   steps     : 0 .. 1000 (0 gives (H + H H / ||H||_F) / 2 symmetrised: no projection).
+ *   workspace : device, 256-byte aligned, at least hq_psd_workspace_bytes(K) bytes.
+ * Synchronises `stream` at the end (HQ_ERR_TIMEOUT if a bounded wait in a product expired).
+ */
+hq_status hq_hessian_project_psd(float* H, int64_t K, int steps, void* workspace, size_t workspace_bytes,
+                                 hq_stream_t stream);
+
 /* Bf16TrilDiagF32 payload size: K*4 + K*(K-1)/2*2 bytes ([calib] "Hessian storage"). */
 size_t hq_bf16tril_bytes(int64_t K);
 

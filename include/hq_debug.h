@@ -52,6 +52,15 @@ hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, cons
                              hq_stream_t stream);
 
 /*
+ * The GPTQ lazy-update product (persistent tcgen05 kernel, 3xTF32 from pre-split operands):
+ *   C[m, n] -= sum_k (A_hi + A_lo)[m * lda + k] (B_hi + B_lo)[n * ldb + k]   (hi*lo + lo*hi +
+ *   hi*hi; lo*lo dropped), m < M, n < N.  All pointers 16-byte aligned, lda, ldb, ldc multiples
+ * of 4.  No counterpart on the pages: a building block of the path.
+ */
+hq_status hq_debug_upd_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A_hi, const float* A_lo,
+                            int64_t lda, const float* B_hi, const float* B_lo, int64_t ldb, hq_stream_t stream);
+
+/*
  * The fp64 GEMM of the factorisation (fp64 tensor cores, mma.sync m8n8k4):
  *   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]
  * for m < M, n < N (if `lower`, M == N and only elements with m >= n are written).

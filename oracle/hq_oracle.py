@@ -13,7 +13,9 @@ Pages cited (by title and section):
       mirrored on read, bf16 conversion by truncation (f32_bits >> 16).  Full Hessians XX^T.
     - "REQUIRED: project to PSD before Cholesky" / "The fix": damping is expressed as a
       multiple of mean(diag(H)); damping that dominates the diagonal turns GPTQ into
-      round-to-nearest.
+      round-to-nearest.  A stored (bf16) Hessian is made positive semidefinite by an
+      eigendecomposition whose negative eigenvalues are clipped to zero, the matrix rebuilt
+      from the clipped spectrum and then symmetrised.
 * [gptq]   ork-driver wiki, "Exp 2026-08-18 GPTQ Int4":
     - experiment summary: error-compensated column-sequential int4 rounding (GPTQ), a
       Cholesky-based Hessian inverse plus an error-feedback sweep, uniform symmetric int4
@@ -54,6 +56,7 @@ __all__ = [
     "hessian_accumulate",
     "imatrix",
     "damp_hessian",
+    "project_psd",
     "cholesky_lower",
     "upper_factor_of_inverse",
     "upper_factor_by_reversal",
@@ -117,6 +120,15 @@ def damp_hessian(H, damp: float):
         raise ValueError("mean(diag H) must be positive")
     lam = float(damp) * mean_diag
     return H64 + lam * np.eye(K), lam
+
+
+def project_psd(H) -> np.ndarray:
+    """[calib] "The fix": with H = V diag(l) V^T (symmetric eigendecomposition, LAPACK as one
+    step), rebuild V diag(max(l, 0)) V^T, then return its symmetric part (P + P^T) / 2."""
+    H64 = np.asarray(H, dtype=np.float64)
+    l, V = np.linalg.eigh(H64)
+    P = (V * np.maximum(l, 0.0)) @ V.T
+    return (P + P.T) / 2.0
 
 
 def cholesky_lower(A) -> np.ndarray:

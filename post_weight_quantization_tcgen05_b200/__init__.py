@@ -56,6 +56,8 @@ _SIGS = {
     "hq_rtn_quantize": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hq_rtn_quantize_noalloc": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "hq_qerr_terms": (_int, [_vp, _vp, _vp]),
+    "hq_psd_workspace_bytes": (_sz, [_i64]),
+    "hq_hessian_project_psd": (_int, [_vp, _i64, _int, _vp, _sz, _vp]),
     "hq_bf16tril_bytes": (_sz, [_i64]),
     "hq_hessian_pack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
     "hq_hessian_unpack_bf16tril": (_int, [_vp, _i64, _vp, _vp]),
@@ -66,6 +68,7 @@ _SIGS = {
     "hq_debug_launch_count": (ctypes.c_uint64, []),
     "hq_debug_tf32_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _f, _f, _int, _int, _vp]),
     "hq_debug_rcp_f64": (_int, [_vp, _vp, _i64, _vp]),
+    "hq_debug_upd_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _i64, _vp, _vp, _i64, _vp]),
     "hq_debug_fp64_mma_rate": (ctypes.c_double, [_vp, _i64, _vp]),
     "hq_debug_timing_start": (_int, [_int]),
     "hq_debug_timing_stop": (_int, []),
@@ -196,6 +199,20 @@ def hq_rtn_quantize_noalloc(W, group: int, codes, scales, imp=None, want_qerr: b
     return q.value if want_qerr else None
 
 
+def hq_psd_workspace_bytes(K: int) -> int:
+    return int(lib.hq_psd_workspace_bytes(int(K)))
+
+
+def hq_hessian_project_psd(H, workspace=None, steps: int = 40, stream=None) -> None:
+    """H (fp32 [K, K], symmetric, device) <- its projection onto the PSD cone, in place."""
+    K = H.shape[0]
+    if workspace is None:
+        workspace = alloc_workspace(hq_psd_workspace_bytes(K), H.device)
+    _check(lib.hq_hessian_project_psd(_ptr(H), K, int(steps), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "hq_hessian_project_psd")
+
+
 def hq_qerr_terms(workspace, terms_dev, stream=None) -> None:
     """terms_dev (fp64 [2], device) <- the qerr numerator and denominator sums of the last
     quantisation that used `workspace`."""
@@ -247,6 +264,14 @@ def hq_debug_timing_read(cls: str):
     _check(lib.hq_debug_timing_read(TIMING_CLASSES[cls], ctypes.byref(ms), ctypes.byref(work), ctypes.byref(n)),
            "hq_debug_timing_read")
     return ms.value, work.value, n.value
+
+
+def hq_debug_upd_gemm(C, A_hi, A_lo, B_hi, B_lo, stream=None) -> None:
+    """C -= (A_hi + A_lo) (B_hi + B_lo)^T by the lazy-update kernel (3xTF32)."""
+    M, Kred = A_hi.shape
+    N = B_hi.shape[0]
+    _check(lib.hq_debug_upd_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A_hi), _ptr(A_lo), A_hi.stride(0),
+                                 _ptr(B_hi), _ptr(B_lo), B_hi.stride(0), _stream(stream)), "hq_debug_upd_gemm")
 
 
 def hq_debug_rcp_f64(d, out, stream=None) -> None:

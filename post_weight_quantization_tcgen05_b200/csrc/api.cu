@@ -213,6 +213,27 @@ hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, cons
   return tf32_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
+hq_status hq_debug_upd_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A_hi, const float* A_lo,
+                            int64_t lda, const float* B_hi, const float* B_lo, int64_t ldb, hq_stream_t stream) {
+  if (C == nullptr || A_hi == nullptr || A_lo == nullptr || B_hi == nullptr || B_lo == nullptr || M < 0 || N < 0 ||
+      Kred < 1)
+    return HQ_ERR_INVALID;
+  if (ldc < N || lda < Kred || ldb < Kred) return HQ_ERR_INVALID;
+  UpdGemm g{};
+  g.C = C;
+  g.ldc = ldc;
+  g.M = M;
+  g.N = N;
+  g.Kred = Kred;
+  g.A_hi = A_hi;
+  g.A_lo = A_lo;
+  g.lda = lda;
+  g.B_hi = B_hi;
+  g.B_lo = B_lo;
+  g.ldb = ldb;
+  return upd_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
 size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group) {
   if (N < 1 || K < 2 || group < 2 || group % 2 != 0 || K % group != 0) return 0;
   return rtn_workspace(N, K, group);
@@ -240,6 +261,27 @@ hq_status hq_qerr_terms(const void* workspace, double* terms_dev, hq_stream_t st
                                                                      terms_dev);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
+}
+
+size_t hq_psd_workspace_bytes(int64_t K) {
+  return (K >= 4 && K % 4 == 0 && K <= 65536) ? psd_workspace(K) : 0;
+}
+
+hq_status hq_hessian_project_psd(float* H, int64_t K, int steps, void* workspace, size_t workspace_bytes,
+                                 hq_stream_t stream) {
+  if (H == nullptr || K < 1 || steps < 0 || steps > 1000) return HQ_ERR_INVALID;
+  if (K % 4 != 0 || K > 65536 || !aligned(H, 16)) return HQ_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < psd_workspace(K)) return HQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + 128);
+  HQ_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  hq_status st = launch_psd(H, K, steps, ws, status, s);
+  if (st != HQ_OK) return st;
+  int h_status = 0;
+  HQ_CUDA_TRY(cudaMemcpyAsync(&h_status, status, sizeof(int), cudaMemcpyDeviceToHost, s));
+  HQ_CUDA_TRY(cudaStreamSynchronize(s));
+  return h_status == HQ_ERR_TIMEOUT ? HQ_ERR_TIMEOUT : HQ_OK;
 }
 
 size_t hq_bf16tril_bytes(int64_t K) {

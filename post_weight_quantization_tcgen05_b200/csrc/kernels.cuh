@@ -51,6 +51,11 @@ struct UpdGemm {
 };
 hq_status upd_gemm(const UpdGemm& g, cudaStream_t s);
 
+// psd.cu: H <- its projection onto the PSD cone (steps Newton-Schulz steps for sign(H));
+// workspace of psd_workspace(K) bytes, 256-byte aligned; `status` a device int (timeouts).
+size_t psd_workspace(int64_t K);
+hq_status launch_psd(float* H, int64_t K, int steps, uint8_t* ws, int* status, cudaStream_t s);
+
 // timing.cu: optional event timing of kernel classes (hq_debug_timing_*).  timer_start returns
 // -1 (and records nothing) unless the class is being timed; `work` is the launch's algorithmic
 // flops or bytes.

@@ -78,3 +78,10 @@ def check_gptq_parity(W64, U64, group, codes_gpu, scales_gpu, what=""):
     assert srel <= SCALE_REL, f"{what}: teacher-forced scale rel err {srel:.3e}"
     assert tie <= TIE_TOL, f"{what}: a differing code is {tie:.3e} steps from its rounding boundary"
     return ref_codes, ref_scales
+
+
+def split_tf32(x: torch.Tensor):
+    """(hi, lo): hi = x with the low 13 mantissa bits cleared (a tf32 value), lo = x - hi
+    (exact in fp32): the operand split the lazy-update kernel consumes."""
+    hi = (x.view(torch.int32) & -8192).view(torch.float32)
+    return hi, x - hi

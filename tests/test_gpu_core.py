@@ -368,6 +368,28 @@ def test_f64_gemm_against_fp64(hq, cuda_device, M, N, Kred, lower, tri, split):
     assert err < 1e-13, err
 
 
+@pytest.mark.parametrize("M,N,Kred", [(5120, 384, 128), (5120, 4608, 512), (512, 512, 512), (512, 512, 1024),
+                                       (1000, 600, 300), (132, 72, 36)])
+def test_upd_gemm_against_fp64(hq, cuda_device, M, N, Kred):
+    """The persistent 3xTF32 lazy-update kernel (every tile width it picks) against fp64:
+    C -= A B^T with A, B given as tf32 part + remainder.  The tensor core's fp32 accumulation
+    drifts with the number of chained MMAs (about 4e-6 relative at a contraction of 512), so
+    the bound scales with the contraction."""
+    from gpu_helpers import split_tf32
+    g = _gen(M + 7 * N + Kred)
+    A = torch.randn((M, Kred), generator=g, device="cuda")
+    B = torch.randn((N, Kred), generator=g, device="cuda")
+    C0 = torch.randn((M, N), generator=g, device="cuda")
+    Ah, Al = split_tf32(A)
+    Bh, Bl = split_tf32(B)
+    C = C0.clone()
+    hq.hq_debug_upd_gemm(C, Ah, Al, Bh, Bl)
+    torch.cuda.synchronize()
+    ref = C0.double() - A.double() @ B.double().T
+    err = ((C.double() - ref).norm() / (A.double() @ B.double().T).norm()).item()
+    assert err < 1e-6 + 1e-8 * Kred, err
+
+
 @pytest.mark.parametrize("split3", [True, False])
 @pytest.mark.parametrize("M,N,Kred,lower", [(128, 128, 32, False), (300, 200, 100, False), (5120, 384, 128, False),
                                              (640, 640, 512, True), (1, 7, 4, False)])

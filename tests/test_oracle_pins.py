@@ -473,3 +473,67 @@ def test_factor_pins_catch_transposed_factor():
     wrong = np.linalg.cholesky(np.linalg.inv(Hd))  # lower factor instead of upper
     assert np.abs(U @ Hd @ U.T - np.eye(K)).max() < 1e-9
     assert np.abs(np.triu(wrong) @ Hd @ np.triu(wrong).T - np.eye(K)).max() > 1e-3
+
+
+# ----------------------------------------------------------------------------- PSD projection
+
+def test_psd_projection_2x2_closed_form():
+    """[calib] "The fix" on a 2 x 2 symmetric matrix with one negative eigenvalue: the result
+    is l+ v v^T with l+ = (a + c)/2 + sqrt(((a - c)/2)^2 + b^2) and v the unit vector along
+    (b, l+ - a), written out by hand."""
+    for a, b, c in ((1.0, 2.0, 0.5), (-1.0, 0.3, 2.0), (0.2, -1.5, 0.1)):
+        lp = (a + c) / 2 + math.sqrt(((a - c) / 2) ** 2 + b * b)
+        lm = (a + c) / 2 - math.sqrt(((a - c) / 2) ** 2 + b * b)
+        assert lm < 0 < lp
+        v = np.array([b, lp - a])
+        v /= np.linalg.norm(v)
+        want = lp * np.outer(v, v)
+        got = O.project_psd(np.array([[a, b], [b, c]]))
+        assert np.allclose(got, want, rtol=0, atol=1e-14)
+
+
+def test_psd_projection_diagonal_clips_and_psd_input_unchanged():
+    d = np.array([3.0, -1.0, 0.0, 2.5, -4.0])
+    assert np.array_equal(O.project_psd(np.diag(d)), np.diag(np.maximum(d, 0.0)))
+    rng = np.random.default_rng(2)
+    A = rng.standard_normal((40, 60))
+    H = A @ A.T
+    assert np.abs(O.project_psd(H) - H).max() <= 1e-12 * np.abs(H).max()
+
+
+def test_psd_projection_nearest_psd_properties():
+    """The projection onto the PSD cone (nearest in Frobenius norm): P is PSD, idempotent,
+    orthogonal to H - P (<P, H - P> = 0), and ||H - P||^2 is the sum of the squared negative
+    eigenvalues of H."""
+    rng = np.random.default_rng(9)
+    B = rng.standard_normal((50, 50))
+    H = (B + B.T) / 2
+    P = O.project_psd(H)
+    l = np.linalg.eigvalsh(H)
+    assert np.linalg.eigvalsh(P).min() >= -1e-12 * np.abs(l).max()
+    assert np.abs(O.project_psd(P) - P).max() <= 1e-12 * np.abs(P).max()
+    assert abs(np.sum(P * (H - P))) <= 1e-12 * np.sum(H * H)
+    assert np.sum((H - P) ** 2) == pytest.approx(np.sum(l[l < 0] ** 2), rel=1e-10)
+
+
+def test_psd_projection_of_a_bf16_stored_hessian_is_small():
+    """[calib] "The fix": on a Hessian stored with bf16 off-diagonals, the projection removes
+    less than bf16's own quantisation step (2^-8 relative); the stored matrix is indefinite."""
+    import workloads as wl
+    cfg = wl.correlated_config(16, 512, T=2048, group=128, seed=3)
+    X = wl.make_activations(cfg, "cpu").double().numpy()
+    H = (X.T @ X).astype(np.float32)
+    Hs = O.bf16tril_decode(O.bf16tril_encode(H), 512)
+    assert np.linalg.eigvalsh(Hs).min() < 0
+    P = O.project_psd(Hs)
+    rel = np.linalg.norm(P - Hs) / np.linalg.norm(Hs)
+    assert 0 < rel < 2.0 ** -8
+
+
+def test_psd_pins_catch_clipping_the_wrong_side():
+    def wrong(H):
+        l, V = np.linalg.eigh(np.asarray(H, dtype=np.float64))
+        P = (V * np.minimum(l, 0.0)) @ V.T
+        return (P + P.T) / 2
+    d = np.array([3.0, -1.0])
+    assert not np.array_equal(wrong(np.diag(d)), np.diag(np.maximum(d, 0.0)))
