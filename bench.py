@@ -243,6 +243,8 @@ def run_ours(args, rank, world, local_rank):
         "peak": hbm, "peak_source": f"{peaks['source']} HBM copy",
         "bytes": codec["bytes"],
         "method": "each call alone after an L2 flush (write then read of 256 MiB), events around the call"}
+    if world == 1 and not args.no_other_configs:
+        return_line["hadamard_rotation"] = time_hadamard(hq, layer, flush, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         return_line["cpu_baseline"] = cpu_baseline(cfg, layer)
     if world == 1 and not args.no_other_configs:
@@ -250,6 +252,38 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         return_line["other_configs"] = other_configs(hq, dev, flush, peaks)
     return return_line
+
+
+def time_hadamard(hq, layer, flush, peaks, block: int = 256):
+    """The rotate-then-GPTQ rotation on the layer: W' = W R (bf16 in, fp32 out) and H' = R^T H R
+    (mirror the lower triangle, rows pass, columns pass), each timed alone after an L2 flush;
+    rates are the algorithmic bytes (W: 2 + 4 bytes per weight; H: 4 read + 4 written per element
+    by each of its three passes) over the time, against the measured HBM copy rate."""
+    from post_weight_quantization_tcgen05_b200 import quarot
+    N, K = layer.W.shape
+    g = torch.Generator(device=layer.W.device)
+    g.manual_seed(42)
+    s = quarot.random_signs(K, g, device=layer.W.device)
+    Wr = torch.empty((N, K), dtype=torch.float32, device=layer.W.device)
+    Hr = torch.empty((K, K), dtype=torch.float32, device=layer.W.device)
+    out = {}
+    for name, fn, nbytes in (("weights", lambda: hq.hq_hadamard_rotate_weights(layer.W, s, block, Wr), 6.0 * N * K),
+                             ("hessian", lambda: hq.hq_hadamard_rotate_hessian(layer.H, s, block, Hr), 24.0 * K * K)):
+        fn()
+        flush.fill_(3)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"ms": ms, "achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    del Wr, Hr
+    out.update({"kernels": "hadamard_rows_kernel, hadamard_cols_kernel, mirror_lower_kernel", "block": block,
+                "bound": "hbm", "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"] + " HBM copy"})
+    return out
 
 
 def time_layer(hq, cfg, dev, flush, steps: int = 2, warmup: int = 1, peaks=None):

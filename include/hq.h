@@ -188,6 +188,25 @@ size_t hq_psd_workspace_bytes(int64_t K);
 hq_status hq_hessian_project_psd(float* H, int64_t K, int steps, void* workspace, size_t workspace_bytes,
                                  hq_stream_t stream);
 
+/*
+ * Hadamard rotation ahead of GPTQ ([gptq] experiment summary: GPTQ composes with Hadamard,
+ * "rotate then GPTQ").  R = diag(signs) blockdiag(M, ..., M), M = Hadamard_block / sqrt(block)
+ * the orthonormal Walsh-Hadamard matrix (Sylvester: M[i][j] = (-1)^popcount(i & j) / sqrt(block)).
+ * R is orthogonal: quantising W' = W R against H' = R^T H R (the Hessian of the rotated
+ * activations X R) and feeding the layer R^T x leaves its output unchanged.
+ *   block : a power of two, 2 .. 1024, dividing K.
+ *   signs : device fp32 [K] of +1 / -1, drawn by the caller (the method's random signs).
+ * hq_hadamard_rotate_weights: W_out (fp32 [N, K], may equal W when W is fp32) = W R; W bf16 or
+ *   fp32 [N, K].
+ * hq_hadamard_rotate_hessian: H_out (fp32 [K, K], both triangles, distinct from H) = R^T H R,
+ *   H read as the symmetric matrix of its lower triangle (diagonal included); H unchanged.
+ * Asynchronous.  HQ_ERR_UNSUPPORTED for a block that is not a power of two dividing K.
+ */
+hq_status hq_hadamard_rotate_weights(const void* W, int w_dtype, int64_t N, int64_t K, int64_t block,
+                                     const float* signs, float* W_out, hq_stream_t stream);
+hq_status hq_hadamard_rotate_hessian(const float* H, int64_t K, int64_t block, const float* signs, float* H_out,
+                                     hq_stream_t stream);
+
 /* Bf16TrilDiagF32 payload size: K*4 + K*(K-1)/2*2 bytes ([calib] "Hessian storage"). */
 size_t hq_bf16tril_bytes(int64_t K);
 

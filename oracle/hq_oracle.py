@@ -57,6 +57,10 @@ __all__ = [
     "imatrix",
     "damp_hessian",
     "project_psd",
+    "hadamard_matrix",
+    "hadamard_rotation",
+    "rotate_weights",
+    "rotate_hessian",
     "cholesky_lower",
     "upper_factor_of_inverse",
     "upper_factor_by_reversal",
@@ -129,6 +133,43 @@ def project_psd(H) -> np.ndarray:
     l, V = np.linalg.eigh(H64)
     P = (V * np.maximum(l, 0.0)) @ V.T
     return (P + P.T) / 2.0
+
+
+def hadamard_matrix(B: int) -> np.ndarray:
+    """The orthonormal Walsh-Hadamard matrix of order B (a power of two), Sylvester ordering:
+    M[i][j] = (-1)^popcount(i & j) / sqrt(B)."""
+    if B < 1 or B & (B - 1):
+        raise ValueError("B must be a power of two")
+    i = np.arange(B)
+    bits = np.bitwise_and.outer(i, i)
+    parity = np.zeros((B, B), dtype=np.int64)
+    while bits.any():
+        parity ^= bits & 1
+        bits >>= 1
+    return (1.0 - 2.0 * parity) / np.sqrt(B)
+
+
+def hadamard_rotation(signs, B: int) -> np.ndarray:
+    """[gptq] experiment summary ("rotate then GPTQ"): R = diag(signs) blockdiag(M_B, ..., M_B),
+    K = len(signs) a multiple of B."""
+    s = np.asarray(signs, dtype=np.float64)
+    K = s.size
+    if K % B:
+        raise ValueError("B must divide K")
+    return s[:, None] * np.kron(np.eye(K // B), hadamard_matrix(B))
+
+
+def rotate_weights(W, signs, B: int) -> np.ndarray:
+    """W' = W R."""
+    return np.asarray(W, dtype=np.float64) @ hadamard_rotation(signs, B)
+
+
+def rotate_hessian(H, signs, B: int) -> np.ndarray:
+    """H' = R^T H R, H taken as the symmetric matrix of its lower triangle."""
+    L = np.tril(np.asarray(H, dtype=np.float64))
+    Hs = L + np.tril(L, -1).T
+    R = hadamard_rotation(signs, B)
+    return R.T @ Hs @ R
 
 
 def cholesky_lower(A) -> np.ndarray:

@@ -56,6 +56,8 @@ _SIGS = {
     "hq_rtn_quantize": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hq_rtn_quantize_noalloc": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "hq_qerr_terms": (_int, [_vp, _vp, _vp]),
+    "hq_hadamard_rotate_weights": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "hq_hadamard_rotate_hessian": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "hq_psd_workspace_bytes": (_sz, [_i64]),
     "hq_hessian_project_psd": (_int, [_vp, _i64, _int, _vp, _sz, _vp]),
     "hq_bf16tril_bytes": (_sz, [_i64]),
@@ -211,6 +213,20 @@ def hq_hessian_project_psd(H, workspace=None, steps: int = 40, stream=None) -> N
     _check(lib.hq_hessian_project_psd(_ptr(H), K, int(steps), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)),
            "hq_hessian_project_psd")
+
+
+def hq_hadamard_rotate_weights(W, signs, block: int, W_out, stream=None) -> None:
+    """W_out (fp32 [N, K]) = W R, R = diag(signs) blockdiag(Hadamard_block / sqrt(block))."""
+    N, K = W.shape
+    _check(lib.hq_hadamard_rotate_weights(_ptr(W), _dtype(W), N, K, int(block), _ptr(signs), _ptr(W_out),
+                                          _stream(stream)), "hq_hadamard_rotate_weights")
+
+
+def hq_hadamard_rotate_hessian(H, signs, block: int, H_out, stream=None) -> None:
+    """H_out (fp32 [K, K]) = R^T H R, H read from its lower triangle."""
+    K = H.shape[0]
+    _check(lib.hq_hadamard_rotate_hessian(_ptr(H), K, int(block), _ptr(signs), _ptr(H_out), _stream(stream)),
+           "hq_hadamard_rotate_hessian")
 
 
 def hq_qerr_terms(workspace, terms_dev, stream=None) -> None:

@@ -284,6 +284,28 @@ hq_status hq_hessian_project_psd(float* H, int64_t K, int steps, void* workspace
   return h_status == HQ_ERR_TIMEOUT ? HQ_ERR_TIMEOUT : HQ_OK;
 }
 
+hq_status hq_hadamard_rotate_weights(const void* W, int w_dtype, int64_t N, int64_t K, int64_t block,
+                                     const float* signs, float* W_out, hq_stream_t stream) {
+  if (W == nullptr || signs == nullptr || W_out == nullptr || N < 0 || !valid_dtype(w_dtype)) return HQ_ERR_INVALID;
+  if (!hadamard_shape_ok(K, block)) return HQ_ERR_UNSUPPORTED;
+  if (w_dtype == HQ_BF16 && static_cast<const void*>(W_out) == W) return HQ_ERR_INVALID;
+  return launch_hadamard_rows(W, w_dtype, N, K, static_cast<int>(block), signs, W_out,
+                              static_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_hadamard_rotate_hessian(const float* H, int64_t K, int64_t block, const float* signs, float* H_out,
+                                     hq_stream_t stream) {
+  if (H == nullptr || signs == nullptr || H_out == nullptr) return HQ_ERR_INVALID;
+  if (H == H_out) return HQ_ERR_INVALID;
+  if (!hadamard_shape_ok(K, block)) return HQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  hq_status st = launch_mirror_lower(H, K, H_out, s);
+  if (st != HQ_OK) return st;
+  st = launch_hadamard_rows(H_out, HQ_F32, K, K, static_cast<int>(block), signs, H_out, s);
+  if (st != HQ_OK) return st;
+  return launch_hadamard_cols(H_out, K, static_cast<int>(block), signs, s);
+}
+
 size_t hq_bf16tril_bytes(int64_t K) {
   if (K < 1) return 0;
   return static_cast<size_t>(K) * 4 + static_cast<size_t>(K) * (K - 1) / 2 * 2;

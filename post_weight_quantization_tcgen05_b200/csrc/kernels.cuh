@@ -56,6 +56,13 @@ hq_status upd_gemm(const UpdGemm& g, cudaStream_t s);
 size_t psd_workspace(int64_t K);
 hq_status launch_psd(float* H, int64_t K, int steps, uint8_t* ws, int* status, cudaStream_t s);
 
+// hadamard.cu: rotation by R = diag(s) blockdiag(Hadamard_B / sqrt B)
+bool hadamard_shape_ok(int64_t K, int64_t B);
+hq_status launch_hadamard_rows(const void* A, int a_dtype, int64_t rows, int64_t K, int B, const float* s,
+                               float* out, cudaStream_t st);  // out = A R (out may be A when fp32)
+hq_status launch_hadamard_cols(float* A, int64_t K, int B, const float* s, cudaStream_t st);  // A <- R^T A
+hq_status launch_mirror_lower(const float* H, int64_t K, float* out, cudaStream_t st);
+
 // timing.cu: optional event timing of kernel classes (hq_debug_timing_*).  timer_start returns
 // -1 (and records nothing) unless the class is being timed; `work` is the launch's algorithmic
 // flops or bytes.

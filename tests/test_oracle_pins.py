@@ -537,3 +537,42 @@ def test_psd_pins_catch_clipping_the_wrong_side():
         return (P + P.T) / 2
     d = np.array([3.0, -1.0])
     assert not np.array_equal(wrong(np.diag(d)), np.diag(np.maximum(d, 0.0)))
+
+
+# ----------------------------------------------------------------------------- Hadamard rotation
+
+def test_hadamard_matrix_sylvester_recursion_and_order_2():
+    """The popcount definition against the Sylvester doubling M_2n = [[M, M], [M, -M]] / sqrt 2
+    and the hand-written order 2."""
+    assert np.allclose(O.hadamard_matrix(2), np.array([[1.0, 1.0], [1.0, -1.0]]) / math.sqrt(2), atol=1e-15)
+    M = np.array([[1.0]])
+    for n in (2, 4, 8, 16, 32, 64):
+        M = np.block([[M, M], [M, -M]]) / math.sqrt(2)
+        assert np.allclose(O.hadamard_matrix(n), M, atol=1e-14)
+        assert np.allclose(O.hadamard_matrix(n) @ O.hadamard_matrix(n).T, np.eye(n), atol=1e-13)
+
+
+def test_rotation_is_orthogonal_and_preserves_the_quadratic_form():
+    """R orthogonal; W' R^T = W; H' = R^T H R has H's spectrum; the layer's output pairing
+    W H W^T is unchanged (trace identity of the loss)."""
+    rng = np.random.default_rng(6)
+    K, B = 64, 16
+    s = rng.choice([-1.0, 1.0], K)
+    R = O.hadamard_rotation(s, B)
+    assert np.allclose(R.T @ R, np.eye(K), atol=1e-13)
+    W = rng.standard_normal((5, K))
+    Wr = O.rotate_weights(W, s, B)
+    assert np.allclose(Wr @ R.T, W, atol=1e-12)
+    A = rng.standard_normal((K, 2 * K))
+    H = A @ A.T
+    Hr = O.rotate_hessian(np.tril(H), s, B)
+    assert np.allclose(np.linalg.eigvalsh(Hr), np.linalg.eigvalsh(H), rtol=1e-10, atol=1e-9)
+    assert np.trace(Wr @ Hr @ Wr.T) == pytest.approx(np.trace(W @ H @ W.T), rel=1e-12)
+
+
+def test_rotation_pins_catch_a_missing_sign_vector():
+    rng = np.random.default_rng(7)
+    s = rng.choice([-1.0, 1.0], 32)
+    W = rng.standard_normal((3, 32))
+    wrong = W @ np.kron(np.eye(2), O.hadamard_matrix(16))  # signs dropped
+    assert not np.allclose(wrong, O.rotate_weights(W, s, 16))
