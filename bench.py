@@ -256,9 +256,11 @@ def run_ours(args, rank, world, local_rank):
 
 def time_hadamard(hq, layer, flush, peaks, block: int = 256):
     """The rotate-then-GPTQ rotation on the layer: W' = W R (bf16 in, fp32 out) and H' = R^T H R
-    (mirror the lower triangle, rows pass, columns pass), each timed alone after an L2 flush;
-    rates are the algorithmic bytes (W: 2 + 4 bytes per weight; H: 4 read + 4 written per element
-    by each of its three passes) over the time, against the measured HBM copy rate."""
+    (columns pass on the lower blocks, then rows pass with the transposed writes), each timed alone
+    after an L2 flush; rates are the algorithmic bytes (W: 2 read + 4 written per weight; H: its
+    lower triangle read once, K(K+1)/2 x 4, and H' written once, K^2 x 4) over the time, against
+    the measured HBM copy rate.  The two-pass Hessian design moves about twice those bytes
+    (`design_bytes`)."""
     from post_weight_quantization_tcgen05_b200 import quarot
     N, K = layer.W.shape
     g = torch.Generator(device=layer.W.device)
@@ -268,7 +270,8 @@ def time_hadamard(hq, layer, flush, peaks, block: int = 256):
     Hr = torch.empty((K, K), dtype=torch.float32, device=layer.W.device)
     out = {}
     for name, fn, nbytes in (("weights", lambda: hq.hq_hadamard_rotate_weights(layer.W, s, block, Wr), 6.0 * N * K),
-                             ("hessian", lambda: hq.hq_hadamard_rotate_hessian(layer.H, s, block, Hr), 24.0 * K * K)):
+                             ("hessian", lambda: hq.hq_hadamard_rotate_hessian(layer.H, s, block, Hr),
+                              4.0 * K * (K + 1) / 2 + 4.0 * K * K)):
         fn()
         flush.fill_(3)
         a = torch.cuda.Event(enable_timing=True)
@@ -281,7 +284,11 @@ def time_hadamard(hq, layer, flush, peaks, block: int = 256):
         gbs = nbytes / (ms / 1e3) / 1e9
         out[name] = {"ms": ms, "achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
     del Wr, Hr
-    out.update({"kernels": "hadamard_rows_kernel, hadamard_cols_kernel, mirror_lower_kernel", "block": block,
+    nb = K // block
+    lower = nb * (nb + 1) / 2 * block * block * 4.0
+    out["hessian"]["design_bytes"] = 3 * lower + 4.0 * K * K  # pass 1 r+w lower blocks, pass 2 r lower, w all
+    out.update({"kernels": "hadamard_rows_warp_kernel (W); hadamard_cols_lower_kernel + hadamard_rows_mirror_kernel (H)",
+                "block": block,
                 "bound": "hbm", "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"] + " HBM copy"})
     return out
 

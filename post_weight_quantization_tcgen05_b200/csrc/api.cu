@@ -298,12 +298,7 @@ hq_status hq_hadamard_rotate_hessian(const float* H, int64_t K, int64_t block, c
   if (H == nullptr || signs == nullptr || H_out == nullptr) return HQ_ERR_INVALID;
   if (H == H_out) return HQ_ERR_INVALID;
   if (!hadamard_shape_ok(K, block)) return HQ_ERR_UNSUPPORTED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  hq_status st = launch_mirror_lower(H, K, H_out, s);
-  if (st != HQ_OK) return st;
-  st = launch_hadamard_rows(H_out, HQ_F32, K, K, static_cast<int>(block), signs, H_out, s);
-  if (st != HQ_OK) return st;
-  return launch_hadamard_cols(H_out, K, static_cast<int>(block), signs, s);
+  return launch_hadamard_hessian(H, K, static_cast<int>(block), signs, H_out, static_cast<cudaStream_t>(stream));
 }
 
 size_t hq_bf16tril_bytes(int64_t K) {

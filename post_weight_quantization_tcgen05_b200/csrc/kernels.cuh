@@ -62,6 +62,8 @@ hq_status launch_hadamard_rows(const void* A, int a_dtype, int64_t rows, int64_t
                                float* out, cudaStream_t st);  // out = A R (out may be A when fp32)
 hq_status launch_hadamard_cols(float* A, int64_t K, int B, const float* s, cudaStream_t st);  // A <- R^T A
 hq_status launch_mirror_lower(const float* H, int64_t K, float* out, cudaStream_t st);
+// out = R^T H R (both triangles), H read as the symmetric matrix of its lower triangle; out != H.
+hq_status launch_hadamard_hessian(const float* H, int64_t K, int B, const float* s, float* out, cudaStream_t st);
 
 // timing.cu: optional event timing of kernel classes (hq_debug_timing_*).  timer_start returns
 // -1 (and records nothing) unless the class is being timed; `work` is the launch's algorithmic

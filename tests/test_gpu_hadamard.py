@@ -19,7 +19,8 @@ def hq():
 
 
 @pytest.mark.parametrize("K,B,wdt", [(512, 256, "bf16"), (512, 128, "f32"), (384, 128, "bf16"), (256, 2, "f32"),
-                                     (1024, 1024, "f32")])
+                                     (1024, 1024, "f32"), (96, 32, "bf16"), (64, 64, "f32"), (96, 16, "bf16"),
+                                     (2048, 512, "bf16"), (1280, 256, "f32")])
 def test_rotation_matches_oracle(hq, cuda_device, K, B, wdt):
     from post_weight_quantization_tcgen05_b200 import quarot
     g = torch.Generator(device="cuda")
@@ -41,6 +42,13 @@ def test_rotation_matches_oracle(hq, cuda_device, K, B, wdt):
     ew = np.linalg.norm(to_np64(Wr) - rw) / np.linalg.norm(rw)
     eh = np.linalg.norm(to_np64(Hr) - rh) / np.linalg.norm(rh)
     assert ew < 1e-6 and eh < 1e-6, (ew, eh)
+    # H' is symmetric: with blocks of 32 and more the off-diagonal blocks are written as exact
+    # transposes of each other
+    nb = K // B if B >= 32 else 0
+    for bi in range(nb):
+        for bj in range(bi):
+            assert torch.equal(Hr[bi * B:(bi + 1) * B, bj * B:(bj + 1) * B],
+                               Hr[bj * B:(bj + 1) * B, bi * B:(bi + 1) * B].T)
     # in place on fp32 weights gives the same bytes
     if wdt == "f32":
         W2 = W.clone()
@@ -74,3 +82,29 @@ def test_rotate_then_gptq(hq, cuda_device):
     Qr = oracle.dequantize(c, scales.cpu().numpy(), G)
     Wn = to_np64(W)
     assert q == pytest.approx(np.linalg.norm(Wn - Qr @ R.T) / np.linalg.norm(Wn), rel=1e-4)
+
+
+@pytest.mark.parametrize("B", [32, 256])
+def test_rotation_unaligned_buffers(hq, cuda_device, B):
+    """Buffers that are not 16-byte aligned take the shared-memory kernels: same values."""
+    from post_weight_quantization_tcgen05_b200 import quarot
+    N, K = 40, 512
+    g = torch.Generator(device="cuda")
+    g.manual_seed(B)
+    s = quarot.random_signs(K, g)
+    W = torch.randn((N, K), device="cuda", generator=g)
+    Wr = torch.empty((N, K), device="cuda")
+    hq.hq_hadamard_rotate_weights(W, s, B, Wr)
+    buf = torch.empty(N * K + 1, device="cuda")
+    Wu = buf[1:].view(N, K)
+    hq.hq_hadamard_rotate_weights(W, s, B, Wu)
+    hbuf = torch.empty(K * K + 1, device="cuda")
+    Hu = hbuf[1:].view(K, K)
+    A = torch.randn((K, K), device="cuda", generator=g, dtype=torch.float64)
+    H = (A @ A.T).float()
+    Hr = torch.empty((K, K), device="cuda")
+    hq.hq_hadamard_rotate_hessian(H, s, B, Hr)
+    hq.hq_hadamard_rotate_hessian(H, s, B, Hu)
+    torch.cuda.synchronize()
+    assert torch.allclose(Wu, Wr, rtol=1e-5, atol=1e-5 * float(Wr.abs().max()))
+    assert torch.allclose(Hu, Hr, rtol=1e-5, atol=1e-5 * float(Hr.abs().max()))
