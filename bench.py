@@ -573,9 +573,11 @@ def syrk_line(kernels, stage_tflops, peaks):
     `stage_achieved` from the stage events (which also hold the zeroing of H and launch gaps)."""
     k = kernels.get("syrk") if kernels else None
     achieved = k["achieved"] if k else stage_tflops
+    sus = peaks.get("bf16_tflops_sustained")
     return {"kernel": "syrk_tc_kernel (X^T X)", "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-            "stage_achieved": stage_tflops, "peak_source": peaks["source"] + " bf16 dense burst"}
+            "peak_sustained": sus, "frac_sustained": achieved / sus if sus else None,
+            "stage_achieved": stage_tflops, "peak_source": peaks["source"] + " bf16 dense burst (and sustained)"}
 
 
 def update_line(cfg, kernels, peaks):
@@ -584,8 +586,12 @@ def update_line(cfg, kernels, peaks):
     if not k:
         return None
     roof = update_roofline_ms(cfg, peaks)
+    sus = peaks.get("bf16_tflops_sustained")
+    roof_sus = update_roofline_ms(cfg, dict(peaks, bf16_tflops=sus)) if sus else None
     return {"kernel": "upd_gemm_kernel<BN> (3xTF32 lazy updates)", "bound": "tensor / hbm per launch",
             "ms_per_step": k["ms_per_step"], "roofline_ms_per_step": roof, "frac": roof / k["ms_per_step"],
+            "roofline_ms_per_step_sustained": roof_sus,
+            "frac_sustained": roof_sus / k["ms_per_step"] if roof_sus else None,
             "achieved_useful_tflops": k["achieved"], "launches_per_step": k["launches_per_step"],
             "peak_source": (peaks["source"] + " bf16 dense burst / 2 (nominal tf32 ratio), 3 MMAs per product; "
                             + peaks["source"] + " HBM copy")}
