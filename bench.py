@@ -256,8 +256,8 @@ def run_ours(args, rank, world, local_rank):
 
 def time_hadamard(hq, layer, flush, peaks, block: int = 256):
     """The rotate-then-GPTQ rotation on the layer: W' = W R (bf16 in, fp32 out) and H' = R^T H R
-    (columns pass on the lower blocks, then rows pass with the transposed writes), each timed alone
-    after an L2 flush; rates are the algorithmic bytes (W: 2 read + 4 written per weight; H: its
+    (columns pass on the lower blocks, then rows pass with the transposed writes), each call timed
+    alone after an L2 flush (median of 5); rates are the algorithmic bytes (W: 2 read + 4 written per weight; H: its
     lower triangle read once, K(K+1)/2 x 4, and H' written once, K^2 x 4) over the time, against
     the measured HBM copy rate.  The two-pass Hessian design moves about twice those bytes
     (`design_bytes`)."""
@@ -273,14 +273,17 @@ def time_hadamard(hq, layer, flush, peaks, block: int = 256):
                              ("hessian", lambda: hq.hq_hadamard_rotate_hessian(layer.H, s, block, Hr),
                               4.0 * K * (K + 1) / 2 + 4.0 * K * K)):
         fn()
-        flush.fill_(3)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        fn()
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
+        times = []
+        for rep in range(5):  # each call after an L2 flush; the median
+            flush.fill_(3 + rep)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
         gbs = nbytes / (ms / 1e3) / 1e9
         out[name] = {"ms": ms, "achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
     del Wr, Hr
@@ -731,8 +734,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the gate_up / down_proj / Hessian-at-scale measurements after the main line")
-    ap.add_argument("--profile-case", choices=["step"], default=None,
-                    help="run one untimed step of the configuration on cuda:0 and exit (for ncu captures)")
+    ap.add_argument("--profile-case", choices=["step", "rotation"], default=None,
+                    help="run one untimed step (or one Hadamard rotation of W and H) of the configuration on "
+                         "cuda:0 and exit (for ncu captures)")
     args = ap.parse_args()
 
     if args.profile_case == "step":
@@ -741,6 +745,22 @@ def main():
         layer.step()
         torch.cuda.synchronize()
         print(f"one step of {wl.CONFIGS[args.config].name} done", flush=True)
+        return
+    if args.profile_case == "rotation":
+        import post_weight_quantization_tcgen05_b200 as hq
+        from post_weight_quantization_tcgen05_b200 import quarot
+        cfg = wl.CONFIGS[args.config]
+        layer = Layer(hq, cfg, torch.device("cuda:0"))
+        layer.step()  # the layer's Hessian
+        g = torch.Generator(device="cuda:0")
+        g.manual_seed(42)
+        s = quarot.random_signs(cfg.K, g, device=torch.device("cuda:0"))
+        Wr = torch.empty((cfg.N, cfg.K), dtype=torch.float32, device="cuda:0")
+        Hr = torch.empty((cfg.K, cfg.K), dtype=torch.float32, device="cuda:0")
+        hq.hq_hadamard_rotate_weights(layer.W, s, 256, Wr)
+        hq.hq_hadamard_rotate_hessian(layer.H, s, 256, Hr)
+        torch.cuda.synchronize()
+        print(f"one rotation of {cfg.name} done", flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
