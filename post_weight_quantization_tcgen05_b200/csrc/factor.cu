@@ -380,6 +380,18 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
   }
 }
 
+// X and X^T := 0 on the diagonal kLeaf x kLeaf blocks (one CTA per block).
+__global__ void __launch_bounds__(256) zero_diag_blocks_kernel(double* __restrict__ X, double* __restrict__ XT,
+                                                               int64_t K) {
+  const int64_t d0 = static_cast<int64_t>(blockIdx.x) * kLeaf;
+  for (int e = threadIdx.x; e < kLeaf * kLeaf / 2; e += blockDim.x) {
+    const int r = e / (kLeaf / 2), c = 2 * (e % (kLeaf / 2));
+    const int64_t off = (d0 + r) * K + d0 + c;
+    *reinterpret_cast<double2*>(X + off) = make_double2(0.0, 0.0);
+    *reinterpret_cast<double2*>(XT + off) = make_double2(0.0, 0.0);
+  }
+}
+
 // ------------------------------------------------------------------------- 3b. recursion
 
 // A second stream per (host thread, device) for the work off the recursion's critical path,
@@ -533,7 +545,7 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
 // With `scaled`, U^T[j][c] is divided by U[c][c] in fp64 first (U'^T, U' = diag(U)^-1 U, the
 // form the GPTQ sweep and its lazy updates use).  With Ut_hi != NULL, also the strict lower part
 // of the result as a tf32 part (low 13 mantissa bits cleared) plus the exact fp32 remainder, the
-// operands of the 3xTF32 lazy updates.
+// operands of the 3xTF32 lazy updates; with Ut == NULL as well, only that split part is produced.
 __global__ void rotate_kernel(const double* __restrict__ X, const double* __restrict__ XT, int64_t K,
                               float* __restrict__ U, float* __restrict__ Ut, float* __restrict__ Ut_hi,
                               float* __restrict__ Ut_lo, bool scaled, const int* __restrict__ info) {
@@ -542,11 +554,13 @@ __global__ void rotate_kernel(const double* __restrict__ X, const double* __rest
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t src = n - 1 - e;  // (K-1-j)*K + (K-1-c) for e = j*K + c
+    // with Ut == NULL only the strict lower split is wanted: the rest is neither read nor written
+    if (Ut == nullptr && e % K >= e / K) continue;
     if (U != nullptr) U[e] = static_cast<float>(X[src]);
     double ut64 = XT[src];  // U^T[e / K][e % K] = U[e % K][e / K]
     if (scaled) ut64 /= X[(K - 1 - e % K) * (K + 1)];  // divided by U[e % K][e % K]
     const float ut = static_cast<float>(ut64);
-    Ut[e] = ut;
+    if (Ut != nullptr) Ut[e] = ut;
     if (Ut_hi != nullptr && e % K < e / K) {
       const float hi = __uint_as_float(__float_as_uint(ut) & 0xFFFFE000u);
       Ut_hi[e] = hi;
@@ -593,8 +607,15 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
     reverse_damp_kernel<<<static_cast<unsigned>(nb * (nb + 1) / 2), 256, 0, s>>>(H, K, lam, A, info);
     HQ_LAUNCH_CHECK();
   }
-  HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(double), s));
-  HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(double), s));
+  if (sweep_form && split_ut) {
+    // the products' triangular tiles and the leaves read zeros only inside the diagonal leaf
+    // blocks, and nothing downstream reads X or X^T outside their triangles
+    zero_diag_blocks_kernel<<<static_cast<unsigned>(K / kLeaf), 256, 0, s>>>(X, XT, K);
+    HQ_LAUNCH_CHECK();
+  } else {
+    HQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(K) * K * sizeof(double), s));
+    HQ_CUDA_TRY(cudaMemsetAsync(XT, 0, static_cast<size_t>(K) * K * sizeof(double), s));
+  }
   SideStream* side = nullptr;
   hq_status st = side_stream(&side);
   if (st != HQ_OK) return st;
@@ -615,7 +636,9 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   float* lo = split_ut ? reinterpret_cast<float*>(T) + K * K : nullptr;
   if (Ut_hi != nullptr) *Ut_hi = hi;
   if (Ut_lo != nullptr) *Ut_lo = lo;
-  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, sweep_form ? nullptr : *U, *Ut, hi, lo,
+  // the 3xTF32 updates of the sweep read only the split strict lower part of U'^T
+  float* ut_plain = (sweep_form && split_ut) ? nullptr : *Ut;
+  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, sweep_form ? nullptr : *U, ut_plain, hi, lo,
                                                             sweep_form, info);
   HQ_LAUNCH_CHECK();
   if (sweep_form) {
