@@ -2,13 +2,13 @@
 // Bf16TrilDiagF32 (quant_type 130)"): K fp32 diagonal values, then the strict lower
 // triangle as bf16 obtained by truncation (fp32 bits >> 16) at index i(i-1)/2 + j.
 //
-// Encode: for K % 4 == 0 one grid-stride pass of 16-byte payload stores (see
-// tril_encode_vec_kernel); otherwise one CTA per row i, whose triangle segment starts at an arbitrary 2-byte offset: a
-// scalar head up to the next 16-byte boundary, then 8 values per 16-byte store, then a scalar
-// tail.  Loads of H are coalesced fp32 either way.
+// Encode: for K % 4 == 0 one pass over row pairs with float4 loads and 16-byte payload stores
+// (tril_encode_pair_kernel); otherwise one CTA per row i, whose triangle segment starts at an
+// arbitrary 2-byte offset: a scalar head up to the next 16-byte boundary, then 8 values per
+// 16-byte store, then a scalar tail.
 // Decode ("mirrored on read"): 64 x 64 tiles of the lower triangle; each tile reads its rows'
-// triangle segments (coalesced u16), writes H[i, j] row-wise and the mirror H[j, i] through a
-// shared-memory transpose so both stores are coalesced.
+// triangle segments (aligned 8-byte words for K % 4 == 0, else u16), writes H[i, j] row-wise and
+// the mirror H[j, i] through a shared-memory transpose so both stores are coalesced.
 #include <algorithm>
 
 #include "common.cuh"
@@ -52,71 +52,78 @@ __global__ void __launch_bounds__(256) tril_encode_rows_kernel(const float* __re
   }
 }
 
-// One pass for K % 4 == 0 (the payload then starts 16-byte aligned) and K <= 46340 (every
-// index fits 32 bits).  A warp takes 256 consecutive payload values p = w0 .. w0 + 255: lane l
-// loads p = w0 + l + 32 k (k = 0..7), so each load instruction reads 32 consecutive values of
-// H (mostly one row: 128 contiguous bytes), truncates them into a shared-memory strip in
-// payload order, and then stores 16-byte pieces p = w0 + 256 h + 8 l .. + 7.  The row of w0 is found
-// once per warp range; every lane steps from there along the rows.  The diagonal goes in
-// 16-byte stores of four values.
-constexpr int kEncThreads = 256;
-constexpr int kEncRange = 256;  // payload values per warp range (8 loads in flight per lane)
+constexpr int kEncThreads = 256;  // the per-row encoder (any K)
 
-__global__ void __launch_bounds__(kEncThreads) tril_encode_vec_kernel(const float* __restrict__ H, int K,
-                                                                      uint8_t* __restrict__ out) {
-  __shared__ __align__(16) uint16_t strip[kEncThreads / 32][kEncRange];
+// One pass for K % 4 == 0 (16-byte aligned rows of H and payload start) and K <= 46340 (payload
+// indices fit 32 bits), balanced by rows: CTA p takes rows 1 + p and K - 1 - p (K values between
+// them).  A warp takes 512-value chunks of a row: each lane loads four float4 of H (512
+// contiguous bytes per load instruction), truncates them into the warp's shared-memory strip at
+// their payload positions (the strip starts at the 16-byte boundary at or below the chunk's
+// first payload value), and the chunk's payload piece is then stored as aligned 16-byte words,
+// its unaligned head and tail (shared with the neighbouring pieces) as 2-byte stores.  CTA p
+// also writes diagonal entries 4p .. 4p + 3.
+constexpr int kEncChunk = 512;                   // values per warp chunk (4 float4 per lane)
+constexpr int kEncStrip = kEncChunk + 16;        // strip length in u16 (alignment slack)
+constexpr int kEncPairThreads = 128;             // 4 warps: about 3 chunks each per row pair
+
+__global__ void __launch_bounds__(kEncPairThreads) tril_encode_pair_kernel(const float* __restrict__ H, int K,
+                                                                           uint8_t* __restrict__ out) {
+  __shared__ __align__(16) uint16_t strip[kEncPairThreads / 32][kEncStrip];
   const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
-  const int npay = K * (K - 1) / 2;  // payload values
-  const int nw = (npay + kEncRange - 1) / kEncRange;  // warp ranges
   uint16_t* my = strip[w];
-  uint4* pay4 = reinterpret_cast<uint4*>(out + 4 * static_cast<int64_t>(K));
   uint16_t* pay = reinterpret_cast<uint16_t*>(out + 4 * static_cast<int64_t>(K));
-  const int wstride = gridDim.x * (kEncThreads / 32);
-  for (int r = blockIdx.x * (kEncThreads / 32) + w; r < nw; r += wstride) {
-    const int w0 = kEncRange * r;
-    // row of w0: i (i - 1) / 2 <= w0 < i (i + 1) / 2
-    int i = static_cast<int>((1.0f + sqrtf(1.0f + 8.0f * static_cast<float>(w0))) * 0.5f);
-    while (static_cast<int64_t>(i) * (i - 1) / 2 > w0) --i;
-    while (static_cast<int64_t>(i) * (i + 1) / 2 <= w0) ++i;
-    int j = w0 - static_cast<int>(static_cast<int64_t>(i) * (i - 1) / 2) + lane;
-    while (j >= i && i < K) {
-      j -= i;
-      ++i;
+  uint4* pay4 = reinterpret_cast<uint4*>(pay);
+  const int p = blockIdx.x;
+  const int ra = 1 + p, rb = K - 1 - p;
+  const int na = (ra + kEncChunk - 1) / kEncChunk;
+  const int nb = rb > ra ? (rb + kEncChunk - 1) / kEncChunk : 0;
+  for (int t = w; t < na + nb; t += kEncPairThreads / 32) {
+    const int i = t < na ? ra : rb;
+    const int c0 = (t < na ? t : t - na) * kEncChunk;
+    const int len = min(kEncChunk, i - c0);  // values of row i in this chunk
+    const int P0 = i * (i - 1) / 2 + c0;     // payload index of (i, c0)
+    const int base = P0 & ~7;
+    const float* src = H + static_cast<int64_t>(i) * K + c0;
+    float4 v[kEncChunk / 128];
+#pragma unroll
+    for (int u = 0; u < kEncChunk / 128; ++u) {
+      const int c = 4 * lane + 128 * u;
+      v[u] = c < len ? reinterpret_cast<const float4*>(src)[c / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int k = 0; k < kEncRange / 32; ++k) {
-      const bool in = w0 + lane + 32 * k < npay;
-      my[lane + 32 * k] = in ? static_cast<uint16_t>(__float_as_uint(H[i * K + j]) >> 16) : uint16_t(0);
-      j += 32;
-      while (j >= i && i < K) {
-        j -= i;
-        ++i;
-      }
+    for (int u = 0; u < kEncChunk / 128; ++u) {
+      const int c = 4 * lane + 128 * u;
+      const int d = P0 - base + c;
+      const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (c + q < len) my[d + q] = static_cast<uint16_t>(__float_as_uint(f[q]) >> 16);
     }
     __syncwarp();
-#pragma unroll
-    for (int h = 0; h < kEncRange / 256; ++h) {
-      const int q0 = w0 + 256 * h + 8 * lane;
-      if (q0 + 8 <= npay) {
-        pay4[q0 / 8] = reinterpret_cast<const uint4*>(my)[32 * h + lane];
-      } else {
-        for (int e = 0; q0 + e < npay; ++e) pay[q0 + e] = my[256 * h + 8 * lane + e];
-      }
-    }
+    const int P1 = P0 + len;
+    const int A0 = (P0 + 7) & ~7, A1 = P1 & ~7;
+    for (int a = A0 + 8 * lane; a + 8 <= A1; a += 256) pay4[a / 8] = *reinterpret_cast<const uint4*>(my + (a - base));
+    const int h1 = min(A0, P1);
+    if (P0 + lane < h1) pay[P0 + lane] = my[P0 + lane - base];
+    const int t0 = max(A1, A0);
+    if (t0 + lane < P1) pay[t0 + lane] = my[t0 + lane - base];
     __syncwarp();
   }
-  float4* diag4 = reinterpret_cast<float4*>(out);
-  for (int u = blockIdx.x * kEncThreads + threadIdx.x; u < K / 4; u += gridDim.x * kEncThreads) {
-    const int i = 4 * u;
-    diag4[u] = make_float4(H[i * (K + 1)], H[(i + 1) * (K + 1)], H[(i + 2) * (K + 1)], H[(i + 3) * (K + 1)]);
+  if (4 * p < K) {  // diagonal entries 4p .. 4p + 3 (K % 4 == 0)
+    float4* diag4 = reinterpret_cast<float4*>(out);
+    if (threadIdx.x == 0) {
+      const int i = 4 * p;
+      diag4[p] = make_float4(H[static_cast<int64_t>(i) * (K + 1)], H[static_cast<int64_t>(i + 1) * (K + 1)],
+                             H[static_cast<int64_t>(i + 2) * (K + 1)], H[static_cast<int64_t>(i + 3) * (K + 1)]);
+    }
   }
 }
 
 hq_status launch_tril_encode(const float* H, int64_t K, uint8_t* out, cudaStream_t s) {
-  if (K % 4 == 0 && K <= 46340 && aligned(out, 16)) {
-    const int64_t nw = ceil_div(K * (K - 1) / 2, kEncRange);  // warp ranges
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(nw, kEncThreads / 32), 148 * 8));
-    tril_encode_vec_kernel<<<static_cast<unsigned>(grid), kEncThreads, 0, s>>>(H, static_cast<int>(K), out);
+  if (K % 4 == 0 && K <= 46340 && aligned(out, 16) && aligned(H, 16)) {
+    // row pairs, and at least K / 4 CTAs for the diagonal
+    const int64_t grid = std::max<int64_t>(K / 2, K / 4);
+    tril_encode_pair_kernel<<<static_cast<unsigned>(grid), kEncPairThreads, 0, s>>>(H, static_cast<int>(K), out);
     HQ_LAUNCH_CHECK();
     return HQ_OK;
   }
@@ -194,19 +201,49 @@ __global__ void __launch_bounds__(256) tril_decode_vec_kernel(const uint8_t* __r
   const int i0 = bi * kDecTile, j0 = bj * kDecTile;
   const float* diag = reinterpret_cast<const float*>(in);
   const uint16_t* tri = reinterpret_cast<const uint16_t*>(in + 4 * static_cast<int64_t>(K));
+  const uint2* tri8 = reinterpret_cast<const uint2*>(tri);  // 8-byte words (the payload starts 16-byte aligned)
+  const int npay = K * (K - 1) / 2;
   const int c4 = 4 * (threadIdx.x % 16);
+  const int hl = threadIdx.x % 16;  // lane within the half-warp that owns a row
+  // A row's 64 values start at payload index s = i(i-1)/2 + j0, 2-byte aligned: lane hl loads the
+  // aligned word holding values s - m + 4 hl .. + 3 (m = s mod 4) and takes its four values from
+  // that word and the next lane's (lane 15 loads the 17th word itself).  Words that would reach
+  // past the payload are read value by value.
+  auto word = [&](int x) -> uint64_t {
+    if (4 * x + 4 <= npay) {
+      const uint2 v = tri8[x];
+      return static_cast<uint64_t>(v.x) | (static_cast<uint64_t>(v.y) << 32);
+    }
+    uint64_t v = 0;
+    for (int q = 0; q < 4; ++q)
+      if (4 * x + q < npay) v |= static_cast<uint64_t>(tri[4 * x + q]) << (16 * q);
+    return v;
+  };
 #pragma unroll
   for (int k = 0; k < kDecTile / 16; ++k) {
     const int r = threadIdx.x / 16 + 16 * k;
     const int i = i0 + r;
-    const int rowbase = static_cast<int>(static_cast<int64_t>(i) * (i - 1) / 2);
+    const int ncol = i < K ? min(i, j0 + kDecTile) - j0 : 0;  // payload values of this row in the tile
+    uint64_t own = 0, nxt = 0;
+    int m = 0;
+    if (ncol > 0) {
+      const int sidx = i * (i - 1) / 2 + j0;
+      m = sidx & 3;
+      const int wb = (sidx - m) / 4;
+      if (4 * hl < m + ncol) own = word(wb + hl);
+      if (hl == 15 && m + ncol > 64) nxt = word(wb + 16);
+    }
+    const uint64_t from_next = __shfl_down_sync(0xffffffffu, own, 1, 16);
+    if (hl != 15) nxt = from_next;
+    // values m + 4 hl .. m + 4 hl + 3 of the window = bits 16 m .. of (nxt : own)
+    const uint64_t vals = m == 0 ? own : ((own >> (16 * m)) | (nxt << (64 - 16 * m)));
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int j = j0 + c4 + q;
       float v = 0.f;
       if (i < K && j < K) {
         if (j < i)
-          v = __uint_as_float(static_cast<uint32_t>(tri[rowbase + j]) << 16);
+          v = __uint_as_float(static_cast<uint32_t>((vals >> (16 * q)) & 0xFFFFu) << 16);
         else if (j == i)
           v = diag[i];
       }
@@ -242,11 +279,12 @@ __global__ void __launch_bounds__(256) tril_decode_vec_kernel(const uint8_t* __r
   }
 }
 
+
 hq_status launch_tril_decode(const uint8_t* in, int64_t K, float* H, cudaStream_t s) {
   const int64_t nb = ceil_div(K, kDecTile);
   const int64_t tiles = nb * (nb + 1) / 2;
   if (tiles > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
-  if (K % 4 == 0 && K <= 46340 && aligned(H, 16))
+  if (K % 4 == 0 && K <= 46340 && aligned(H, 16) && aligned(in, 8))
     tril_decode_vec_kernel<<<static_cast<unsigned>(tiles), 256, 0, s>>>(in, static_cast<int>(K), H);
   else
     tril_decode_kernel<<<static_cast<unsigned>(tiles), 256, 0, s>>>(in, K, H);

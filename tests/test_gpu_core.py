@@ -41,7 +41,7 @@ def _random_h(K, seed):
     return H
 
 
-@pytest.mark.parametrize("K", [1, 2, 3, 4, 5, 12, 64, 127, 128, 129, 1000, 2049])
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 5, 12, 64, 127, 128, 129, 516, 1000, 2049, 2052])
 def test_codec_encode_bit_exact(hq, cuda_device, K):
     H = _random_h(K, 100 + K)
     out = torch.full((hq.hq_bf16tril_bytes(K),), 0xAB, dtype=torch.uint8, device="cuda")
@@ -51,7 +51,7 @@ def test_codec_encode_bit_exact(hq, cuda_device, K):
     assert out.cpu().numpy().tobytes() == ref
 
 
-@pytest.mark.parametrize("K", [1, 2, 3, 4, 12, 64, 129, 1000, 2049])
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 12, 64, 68, 129, 516, 1000, 2049, 2052])
 def test_codec_decode_bit_exact(hq, cuda_device, K):
     nb = hq.hq_bf16tril_bytes(K)
     g = _gen(200 + K)
