@@ -542,10 +542,42 @@ def measure_e2e(args, layer, flush, world):
     tril_h = torch.empty(layer.tril.shape, dtype=layer.tril.dtype).pin_memory()
     qerr_h = torch.empty(1, dtype=torch.float64).pin_memory()
     e2e_steps = max(1, min(args.steps, 5))
+    hq, main = layer.hq, torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def pipelined_step():
+        """The step's calls with its copies overlapped as a host pipeline would: X then W go up on
+        one copy stream; the SYRK starts once X is in; the packed Hessian (which depends on H
+        alone) is encoded right after it and copied back on a second copy stream while the
+        factorisation runs; the quantisation waits for W."""
+        x_in, w_in, tril_out, tril_back = (torch.cuda.Event() for _ in range(4))
+        h2d_s.wait_stream(main)
+        with torch.cuda.stream(h2d_s):
+            Xd.copy_(Xh, non_blocking=True)
+            x_in.record()
+            Wd.copy_(Wh, non_blocking=True)
+            w_in.record()
+        main.wait_event(x_in)
+        layer.H.zero_()
+        hq.hq_hessian_accumulate(layer.H, Xd, dev_status=layer.status)
+        hq.hq_imatrix(layer.H, cfg.T, layer.imp)
+        hq.hq_hessian_pack_bf16tril(layer.H, layer.tril)
+        tril_out.record()
+        d2h_s.wait_event(tril_out)
+        with torch.cuda.stream(d2h_s):
+            tril_h.copy_(layer.tril, non_blocking=True)
+            tril_back.record()
+        main.wait_event(w_in)
+        hq.hq_gptq_quantize(Wd, layer.H, cfg.group, cfg.damp, layer.codes, layer.scales, layer.ws,
+                            imp=layer.imp if cfg.use_imatrix else None, want_qerr=False, qerr_dev=layer.qerr)
+        hq.hq_hessian_unpack_bf16tril(layer.tril, cfg.K, layer.Hfull)
+        codes_h.copy_(layer.codes, non_blocking=True)
+        scales_h.copy_(layer.scales, non_blocking=True)
+        qerr_h.copy_(layer.qerr, non_blocking=True)
+        main.wait_event(tril_back)  # the step ends when every copy has landed
+
     for _ in range(2):
-        Xd.copy_(Xh, non_blocking=True)
-        Wd.copy_(Wh, non_blocking=True)
-        layer.step(Xd, Wd)
+        pipelined_step()
     torch.cuda.synchronize()
     e_start = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     e_end = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
@@ -553,13 +585,7 @@ def measure_e2e(args, layer, flush, world):
     for k in range(e2e_steps):
         flush.fill_(k & 0xFF)
         e_start[k].record()
-        Xd.copy_(Xh, non_blocking=True)
-        Wd.copy_(Wh, non_blocking=True)
-        layer.step(Xd, Wd)
-        codes_h.copy_(layer.codes, non_blocking=True)
-        scales_h.copy_(layer.scales, non_blocking=True)
-        tril_h.copy_(layer.tril, non_blocking=True)
-        qerr_h.copy_(layer.qerr, non_blocking=True)
+        pipelined_step()
         e_end[k].record()
     torch.cuda.synchronize()
     _barrier(world)
