@@ -10,7 +10,8 @@ One step = the whole hot path over one seeded synthetic layer, q_proj-like by de
 Metric: GPTQ-int4 weights/s = N*K / step time (whole job, all ranks).  Inputs are resident in
 HBM; L2 is flushed (a 256 MiB write) between timed steps.  `e2e` repeats the measurement through
 the same C ABI calls with the inputs in pinned host memory: their H2D copies and the D2H copy of
-the results (codes, scales, encoded H, qerr) are inside its timed region.
+the results (codes, scales, encoded H, qerr) are inside its timed region, overlapped with the
+compute on two copy streams (the encoded H goes back while the factorisation runs).
 
 Under torchrun every rank quantises its own independent layer (weak scaling, no collective in
 the data path); times are the max over ranks.  `--impl reference` times the fp64 CPU oracle
