@@ -717,7 +717,50 @@ def cpu_baseline(cfg, layer=None, rows: int = 32):
     return {"value": cfg.N * cfg.K / est, "unit": "weights/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": (f"full fp64 Hessian of X [{cfg.T}, {cfg.K}], full factorisation and codec, sweep of "
                        f"{rows} of {cfg.N} rows scaled to all rows (rows are independent)"),
-            "stages_s": det}
+            "stages_s": det, "host": _host_cpu(), "tiny_single_thread": _oracle_tiny_single_thread()}
+
+
+def _host_cpu():
+    """The host's CPU model and logical core count (recorded beside the oracle's timing)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
+def _oracle_tiny_single_thread(reps: int = 5):
+    """The oracle's whole path on the tiny layer (W [64, 128], X [512, 128], group 32) with the
+    BLAS limited to one thread: the median of `reps` runs."""
+    import oracle
+    cfg = wl.CONFIGS[0]
+    X = wl.make_activations(cfg, "cpu").double().numpy()
+    W = wl.make_weights(cfg, "cpu").double().numpy()
+    try:
+        import threadpoolctl
+        limit = threadpoolctl.threadpool_limits(1)
+    except Exception:
+        limit = None
+    try:
+        times = []
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            H = oracle.hessian(X)
+            r = oracle.gptq_quantize(W, H, cfg.group, cfg.damp)
+            oracle.qerr(W, r["codes"], r["scales"], cfg.group)
+            oracle.bf16tril_decode(oracle.bf16tril_encode(H.astype(np.float32)), cfg.K)
+            times.append(time.perf_counter() - t0)
+    finally:
+        if limit is not None:
+            limit.restore_original_limits()
+    t = statistics.median(times)
+    return {"workload": f"{cfg.name}: W [{cfg.N}, {cfg.K}], X [{cfg.T}, {cfg.K}], group {cfg.group}",
+            "threads": 1, "s_per_step": t, "weights_per_s": cfg.N * cfg.K / t}
 
 
 def run_reference(args):
@@ -744,7 +787,8 @@ def run_reference(args):
         "ms_per_step": statistics.mean(ests) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": f"{cfg.name}: W [{cfg.N}, {cfg.K}], X [{cfg.T}, {cfg.K}], group {cfg.group}"},
-        "cpu_baseline": {"value": value, "unit": "weights/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "weights/s", "cores": cores, "kind": "oracle", "sample": sample,
+                         "host": _host_cpu()},
         "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }

@@ -54,3 +54,14 @@ def test_single_rank_rate_is_plain_throughput():
     import bench
     assert bench._max_over_ranks(12.5, 1) == 12.5
     assert bench.aggregate_rate(5120 * 5120, 1, 10, 100.0) == pytest.approx(5120 * 5120 * 10 / 0.1)
+
+
+def test_cpu_baseline_host_fields():
+    """The oracle baseline records the host's CPU model and core count, and times the tiny
+    layer's whole path single-threaded."""
+    import bench
+    host = bench._host_cpu()
+    assert host["nproc"] >= 1
+    tiny = bench._oracle_tiny_single_thread(reps=1)
+    assert tiny["threads"] == 1 and tiny["s_per_step"] > 0 and tiny["weights_per_s"] > 0
+    assert "W [64, 128]" in tiny["workload"]
