@@ -246,6 +246,7 @@ def run_ours(args, rank, world, local_rank):
         "method": "each call alone after an L2 flush (write then read of 256 MiB), events around the call"}
     if world == 1 and not args.no_other_configs:
         return_line["hadamard_rotation"] = time_hadamard(hq, layer, flush, peaks)
+        return_line["syrk_per_call"] = time_syrk_per_call(hq, layer, flush, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         return_line["cpu_baseline"] = cpu_baseline(cfg, layer)
     if world == 1 and not args.no_other_configs:
@@ -467,6 +468,49 @@ def kernel_breakdown(hq, layer, flush, steps: int = 2):
         out[cls] = {"kernel": name, "ms_per_step": ms / steps, "launches_per_step": n / steps,
                     "achieved": work / (ms / 1e3) / scale, "unit": unit}
     return out
+
+
+def time_syrk_per_call(hq, layer, flush, peaks, tokens: int = 512, reps: int = 3):
+    """The layer's Hessian accumulated call by call as its chunks arrive (16 calls of 512 tokens
+    for q_proj) instead of in one call; each pass timed by events after an L2 flush (median of
+    `reps`).  Per call the roofline is the larger of its flops at the bf16 burst and the
+    read-modify-write of H's lower triangle at the measured HBM rate."""
+    try:
+        cfg = layer.cfg
+        K, T = cfg.K, cfg.T
+        calls = T // tokens
+        H = torch.zeros((K, K), dtype=torch.float32, device=layer.X.device)
+        chunks = [layer.X[c * tokens:(c + 1) * tokens] for c in range(calls)]
+
+        def one_pass():
+            for x in chunks:
+                hq.hq_hessian_accumulate(H, x)
+
+        one_pass()
+        times = []
+        for rep in range(reps):
+            flush.fill_(7 + rep)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            one_pass()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        del H
+        flop_call = tokens * K * (K + 1)
+        rmw_call = 2.0 * 4.0 * K * (K + 1) / 2  # H's lower triangle read and written
+        roof_us = max(flop_call / (peaks["bf16_tflops"] * 1e12), rmw_call / (peaks["hbm_gbs"] * 1e9)) * 1e6
+        per_call_us = ms * 1e3 / calls
+        return {"workload": f"{cfg.name}: {calls} calls of X bf16 [{tokens}, {K}] into one H",
+                "ms": ms, "us_per_call": per_call_us, "tflops": calls * flop_call / (ms / 1e3) / 1e12,
+                "roofline_us_per_call": roof_us, "frac": roof_us / per_call_us,
+                "bound": "hbm (H read-modify-write)" if rmw_call / (peaks["hbm_gbs"] * 1e9) >
+                flop_call / (peaks["bf16_tflops"] * 1e12) else "tensor",
+                "peak_source": peaks["source"] + " bf16 dense burst and HBM copy"}
+    except Exception as e:  # a measurement beside the line: never lose the line for it
+        return {"error": str(e)}
 
 
 def codec_throughput(hq, layer, flush, reps: int = 5):
