@@ -21,7 +21,8 @@ def random_signs(K: int, generator: torch.Generator, device="cuda") -> torch.Ten
 
 def rotate_then_gptq(hq, W, H, signs, block: int, group: int, damp: float, codes, scales, workspace, imp=None):
     """GPTQ of W' = W R against H' = R^T H R (H read from its lower triangle).  Returns
-    (qerr, W', H')."""
+    (qerr, W', H').  `imp`, when given, weights the columns of W', i.e. the ROTATED channels
+    (the imatrix of the rotated layer is diag(H') / T, not diag(H) / T)."""
     N, K = W.shape
     Wr = torch.empty((N, K), dtype=torch.float32, device=W.device)
     Hr = torch.empty((K, K), dtype=torch.float32, device=W.device)
