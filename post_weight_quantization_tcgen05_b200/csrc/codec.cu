@@ -52,8 +52,6 @@ __global__ void __launch_bounds__(256) tril_encode_rows_kernel(const float* __re
   }
 }
 
-constexpr int kEncThreads = 256;  // the per-row encoder (any K)
-
 // One pass for K % 4 == 0 (16-byte aligned rows of H and payload start) and K <= 46340 (payload
 // indices fit 32 bits), balanced by rows: CTA p takes rows 1 + p and K - 1 - p (K values between
 // them).  A warp takes 512-value chunks of a row: each lane loads four float4 of H (512
