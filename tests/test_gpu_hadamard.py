@@ -108,3 +108,20 @@ def test_rotation_unaligned_buffers(hq, cuda_device, B):
     torch.cuda.synchronize()
     assert torch.allclose(Wu, Wr, rtol=1e-5, atol=1e-5 * float(Wr.abs().max()))
     assert torch.allclose(Hu, Hr, rtol=1e-5, atol=1e-5 * float(Hr.abs().max()))
+
+
+@pytest.mark.parametrize("N,K,B", [(1500, 1024, 32), (9600, 1024, 256)])
+def test_weight_rotation_beyond_one_wave(hq, cuda_device, N, K, B):
+    """More blocks than one wave of warps holds (148 x 8 CTAs of 8 warps, 4 blocks each): the
+    grid-stride loop of the weight rotation, against the oracle."""
+    from post_weight_quantization_tcgen05_b200 import quarot
+    assert N * (K // B) > 148 * 8 * 8 * 4
+    g = torch.Generator(device="cuda")
+    g.manual_seed(N + B)
+    s = quarot.random_signs(K, g)
+    W = (torch.randn((N, K), device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    Wr = torch.empty((N, K), device="cuda")
+    hq.hq_hadamard_rotate_weights(W, s, B, Wr)
+    torch.cuda.synchronize()
+    rw = oracle.rotate_weights(to_np64(W), s.cpu().numpy(), B)
+    assert np.linalg.norm(to_np64(Wr) - rw) / np.linalg.norm(rw) < 1e-6
