@@ -22,7 +22,8 @@
 // (chol_inv_leaf_kernel).  Steps:
 //   1. lambda = damp * mean(diag H)            (fp64 reduction, one CTA)
 //   2. A = J (H + lambda I) J in fp64, lower triangle (tiled transpose of H's lower triangle)
-//   3. X = L^-1 and X^T by the recursion above
+//   3. X = L^-1 and X^T by the recursion above (zeros are read only inside the diagonal leaf
+//      blocks, so for the sweep's split output only those blocks are cleared first)
 //   4. U = J X J and U^T = J X^T J, both row-major (180-degree rotated copies)
 // A device flag `info` receives the first failing pivot (1-based, in M's order) and stops
 // every later kernel.
