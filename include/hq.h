@@ -201,6 +201,9 @@ hq_status hq_hessian_project_psd(float* H, int64_t K, int steps, void* workspace
  * hq_hadamard_rotate_hessian: H_out (fp32 [K, K], both triangles, distinct from H) = R^T H R,
  *   H read as the symmetric matrix of its lower triangle (diagonal included); H unchanged.
  * Asynchronous.  HQ_ERR_UNSUPPORTED for a block that is not a power of two dividing K.
+ * Any alignment is accepted; blocks of 32 and more with 16-byte aligned W, W_out / H_out and
+ * signs take the warp-level kernels (one read and one write of W; two passes over H's lower
+ * blocks), other cases simpler shared-memory kernels with the same results up to rounding order.
  */
 hq_status hq_hadamard_rotate_weights(const void* W, int w_dtype, int64_t N, int64_t K, int64_t block,
                                      const float* signs, float* W_out, hq_stream_t stream);
@@ -216,14 +219,17 @@ size_t hq_bf16tril_bytes(int64_t K);
  *   out[4K + 2*(i(i-1)/2 + j)] = (fp32 bits of H[i,j]) >> 16 as little-endian u16, i > j
  *                            (bf16 by truncation, not rounding).
  *   H fp32 [K, K] (diagonal and strict lower triangle read), out hq_bf16tril_bytes(K) bytes.
- *   K >= 1.  Asynchronous.  Bit-exact by definition.
+ *   K >= 1.  Asynchronous.  Bit-exact by definition.  K % 4 == 0, K <= 46340 and 16-byte
+ *   aligned H and out take the one-pass vector kernel; other cases a per-row kernel (same bytes).
  */
 hq_status hq_hessian_pack_bf16tril(const float* H, int64_t K, uint8_t* out, hq_stream_t stream);
 
 /*
  * Bf16TrilDiagF32 decode, "mirrored on read": H[i,i] = diagonal; H[i,j] = H[j,i] =
  * fp32(bits << 16) for i > j.  in: hq_bf16tril_bytes(K) bytes; H_full fp32 [K, K] out (both
- * triangles written).  K >= 1.  Asynchronous.
+ * triangles written).  K >= 1.  Asynchronous.  K % 4 == 0, K <= 46340, 16-byte aligned H_full
+ * and 8-byte aligned in take the word-gather kernel; other cases a scalar-gather kernel (same
+ * values).
  */
 hq_status hq_hessian_unpack_bf16tril(const uint8_t* in, int64_t K, float* H_full,
                                      hq_stream_t stream);
