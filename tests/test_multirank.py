@@ -65,3 +65,34 @@ def test_cpu_baseline_host_fields():
     tiny = bench._oracle_tiny_single_thread(reps=1)
     assert tiny["threads"] == 1 and tiny["s_per_step"] > 0 and tiny["weights_per_s"] > 0
     assert "W [64, 128]" in tiny["workload"]
+
+
+def test_bench_line_carries_the_contract_keys():
+    """The JSON line's keys and types (built from stand-in measurements); the dominant kernel's
+    DRAM traffic comes from its committed profile, or is null once the kernel source changed."""
+    import json
+    import types
+
+    import bench
+    import workloads as wl
+    cfg = wl.CONFIGS[1]
+    args = types.SimpleNamespace(steps=10, warmup=3)
+    peaks = bench._peaks()
+    kernels = {"syrk": {"achieved": 1000.0, "ms_per_step": 0.2, "launches_per_step": 1.0},
+               "tf32_gemm": {"achieved": 120.0, "ms_per_step": 1.1, "launches_per_step": 39.0}}
+    e2e = {"value": 2.0e9, "unit": "weights/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    line = bench.build_line(args, cfg, 1, 2.8e9, 9.3, [0.2], [9.0], [0.03], [0.03], 900.0, 7.9e7, 1.3e8,
+                            peaks, e2e, 394, clocks, (33.0, 6.7e11, 40), kernels, 37.0)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["unit"] == "weights/s" and line["higher_is_better"] is True and line["scaling"] == "weak"
+    assert "workload" in line["config"] and "model" not in line["config"]
+    roof = line["roofline"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in roof, key
+    assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    assert roof["traffic"] is None or roof["traffic"] > 0
+    assert line["gpu_launches"] == 3940
+    json.dumps(line)
