@@ -227,6 +227,10 @@ def run_ours(args, rank, world, local_rank):
     kernels = kernel_breakdown(hq, layer, flush)
     codec = codec_throughput(hq, layer, flush)
     peaks = _peaks()
+    dense = measure_dense_peaks(hq, dev)
+    peaks["tf32_tflops"] = dense.get("tf32_tflops") or peaks["bf16_tflops"] / 2.0
+    peaks["fp64_tflops"] = dense.get("fp64_tflops")
+    peaks["int8_tops"] = dense.get("int8_tops")
     syrk_flop = cfg.T * cfg.K * (cfg.K + 1)
     syrk_avg_s = statistics.mean(syrk_ms) / 1e3
     syrk_tflops = syrk_flop / syrk_avg_s / 1e12
@@ -234,8 +238,7 @@ def run_ours(args, rank, world, local_rank):
     dec_bytes = hq.hq_bf16tril_bytes(cfg.K) + 4 * cfg.K * cfg.K
     clocks = clk.summary()
     return_line = build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops,
-                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks, dom, kernels,
-                             fp64_mma_peak(hq))
+                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense)
     hbm = peaks["hbm_gbs"]
     return_line["codec_roofline"] = {
         "kernels": "tril_encode_pair_kernel / tril_decode_vec_kernel", "bound": "hbm", "unit": "GB/s",
@@ -423,14 +426,14 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "f64_gemm_kernel_128_q_proj.md"
 KERNEL_SOURCE = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "csrc", "gemm_f64.cu")
 
 
-def update_roofline_ms(cfg, peaks) -> float:
+def update_roofline_ms(cfg, peaks, tf32_tflops=None) -> float:
     """Sum over the sweep's lazy-update launches of each launch's roofline time: the larger of
-    its tensor time (three tf32 MMAs per product at the tf32 peak, taken as half the measured
-    bf16 burst, NVIDIA's nominal dense ratio) and its DRAM time at the measured HBM rate (C read
-    and written, the split residuals and the split U' block read once, 4 bytes each)."""
+    its tensor time (three tf32 MMAs per product at the measured tf32 rate) and its DRAM time at
+    the measured HBM rate (C read and written, the split residuals and the split U' block read
+    once, 4 bytes each)."""
     N, K = cfg.N, cfg.K
     P = min(512 if cfg.group <= 128 else cfg.group * max(512 // cfg.group, 1), K)
-    tf32 = peaks["bf16_tflops"] * 1e12 / 2.0
+    tf32 = (tf32_tflops or peaks["tf32_tflops"]) * 1e12
     hbm = peaks["hbm_gbs"] * 1e9
     launches = []
     for p0 in range(0, K, P):
@@ -556,6 +559,57 @@ def fp64_mma_peak(hq):
         return None
 
 
+def _best_matmul_rate(fn, flops: float, reps: int) -> float:
+    """flops / the shortest of `reps` timed calls of fn (CUDA events, after one warm-up call)."""
+    fn()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        best = min(best, a.elapsed_time(b) / 1e3)
+    return flops / best / 1e12
+
+
+def measure_dense_peaks(hq, dev, n: int = 8192):
+    """Dense matrix-product rates of this GPU for the operand types the path uses besides bf16,
+    measured the way the bf16 figure of MEASURED_PEAKS.json is (a library GEMM of n^3, the best
+    of several calls): tf32 (fp32 torch.matmul with tensor-float-32 allowed), fp64 (fp64
+    torch.matmul; the fp64 peak is the larger of that and the library's fp64 MMA rate) and int8
+    (torch._int_mm, int32 accumulation)."""
+    out = {"method": f"torch.matmul {n}^3 (2 n^3 flops), best of several calls, CUDA events"}
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    flops = 2.0 * n ** 3
+    try:
+        a = torch.randn((n, n), generator=g, device=dev)
+        b = torch.randn((n, n), generator=g, device=dev)
+        prev = torch.backends.cuda.matmul.allow_tf32
+        torch.backends.cuda.matmul.allow_tf32 = True
+        try:
+            out["tf32_tflops"] = _best_matmul_rate(lambda: a @ b, flops, 10)
+        finally:
+            torch.backends.cuda.matmul.allow_tf32 = prev
+        a64, b64 = a.double(), b.double()
+        del a, b
+        out["fp64_gemm_tflops"] = _best_matmul_rate(lambda: a64 @ b64, flops, 5)
+        del a64, b64
+        ai = torch.randint(-128, 128, (n, n), generator=g, device=dev, dtype=torch.int32).to(torch.int8)
+        bi = torch.randint(-128, 128, (n, n), generator=g, device=dev, dtype=torch.int32).to(torch.int8)
+        out["int8_tops"] = _best_matmul_rate(lambda: torch._int_mm(ai, bi), flops, 10)
+        del ai, bi
+    except Exception as e:  # a measurement beside the line: never lose the line for it
+        out["error"] = str(e)
+    torch.cuda.empty_cache()
+    out["fp64_mma_rate_tflops"] = fp64_mma_peak(hq)
+    rates = [r for r in (out.get("fp64_gemm_tflops"), out["fp64_mma_rate_tflops"]) if r]
+    out["fp64_tflops"] = max(rates) if rates else None
+    return out
+
+
 def profiled_traffic():
     """dram bytes per launch of the dominant kernel from the committed ncu summary, or None when
     the kernel's source has changed since that capture."""
@@ -661,30 +715,32 @@ def update_line(cfg, kernels, peaks):
         return None
     roof = update_roofline_ms(cfg, peaks)
     sus = peaks.get("bf16_tflops_sustained")
-    roof_sus = update_roofline_ms(cfg, dict(peaks, bf16_tflops=sus)) if sus else None
+    # sustained tf32: the measured tf32 burst scaled by the bf16 sustained / burst ratio
+    tf32_sus = peaks["tf32_tflops"] * sus / peaks["bf16_tflops"] if sus else None
+    roof_sus = update_roofline_ms(cfg, peaks, tf32_sus) if sus else None
     return {"kernel": "upd_gemm_kernel<BN> (3xTF32 lazy updates)", "bound": "tensor / hbm per launch",
             "ms_per_step": k["ms_per_step"], "roofline_ms_per_step": roof, "frac": roof / k["ms_per_step"],
             "roofline_ms_per_step_sustained": roof_sus,
             "frac_sustained": roof_sus / k["ms_per_step"] if roof_sus else None,
             "achieved_useful_tflops": k["achieved"], "launches_per_step": k["launches_per_step"],
-            "peak_source": (peaks["source"] + " bf16 dense burst / 2 (nominal tf32 ratio), 3 MMAs per product; "
-                            + peaks["source"] + " HBM copy")}
+            "tf32_tflops": peaks["tf32_tflops"],
+            "peak_source": ("tf32 dense rate measured in this run (torch.matmul fp32 with TF32, 3 MMAs per "
+                            "product); " + peaks["source"] + " HBM copy")}
 
 
 def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops, enc_bytes,
-               dec_bytes, peaks, e2e, launches, clocks, dom, kernels, fp64_peak_measured):
+               dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense):
     dom_ms, dom_flop, dom_n = dom
     achieved = dom_flop / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
-    peak = peaks["bf16_tflops"] * FP64_OVER_BF16
+    peak = peaks.get("fp64_tflops") or peaks["bf16_tflops"] * FP64_OVER_BF16
     roofline = {"kernel": KERNEL_NAMES[DOMINANT][0] + " (fp64 MMA, factorisation products)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak if achieved is not None else None, "traffic": profiled_traffic(),
                 "launches_per_step": dom_n / max(args.steps, 1), "ms_per_step": dom_ms / max(args.steps, 1),
-                "peak_source": (f"{peaks['source']} bf16 dense burst {peaks['bf16_tflops']} TFLOP/s x nominal "
-                                f"fp64-tensor/bf16 ratio 37/2250"),
-                "fp64_mma_rate_measured": fp64_peak_measured,
-                "frac_of_measured_fp64_mma": (achieved / fp64_peak_measured
-                                              if achieved is not None and fp64_peak_measured else None)}
+                "peak_source": ("fp64 dense rate measured in this run: the larger of the fp64 torch.matmul "
+                                "(cuBLAS) rate and the library's fp64 MMA rate" if peaks.get("fp64_tflops") else
+                                f"{peaks['source']} bf16 dense burst x nominal fp64-tensor/bf16 ratio 37/2250"),
+                "dense_peaks_measured": dense}
     line = {
         "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
         "value": value,
@@ -698,9 +754,8 @@ def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, d
         "vs_baseline": None,
         "dtype": "bf16 in; bf16 tcgen05 SYRK (fp32 accumulate), fp64 factorisation, fp32 sweep, 3xTF32 updates",
         "data": "synthetic (seeded; shapes and distributions of the q_proj-like layer)",
-        "config": {"workload": f"{cfg.name}: W bf16 [{cfg.N}, {cfg.K}], X bf16 [{cfg.T}, {cfg.K}] "
-                               f"({cfg.n_chunks} chunks of {cfg.chunk}), group {cfg.group}, damp {cfg.damp}",
-                   "layers_per_gpu": 1, "l2": "flushed between timed steps (256 MiB write)"},
+        "config": {"workload": workload_string(cfg), "layers_per_gpu": 1,
+                   "l2": "flushed between timed steps (256 MiB write)"},
         "stages_ms": {"syrk": statistics.mean(syrk_ms), "imatrix+factor+sweep": statistics.mean(gptq_ms),
                       "tril_encode": statistics.mean(enc_ms), "tril_decode": statistics.mean(dec_ms)},
         "xtx_tflops": syrk_tflops,
@@ -729,9 +784,15 @@ def _blas_threads():
         return os.cpu_count()
 
 
-def oracle_sample(cfg, X, W, rows: int):
-    """Times the oracle on one layer: full Hessian, factorisation and codec, sweep on `rows`
-    rows; returns (estimated seconds for the whole layer, details)."""
+def workload_string(cfg) -> str:
+    """The workload's description, the same in both arms' lines."""
+    return (f"{cfg.name}: W bf16 [{cfg.N}, {cfg.K}], X bf16 [{cfg.T}, {cfg.K}] ({cfg.n_chunks} chunks of "
+            f"{cfg.chunk}), group {cfg.group}, damp {cfg.damp}")
+
+
+def oracle_fixed(cfg, X):
+    """The oracle's per-layer stages, timed: the fp64 Hessian of all the layer's tokens, damping
+    and the factorisation, the codec of H.  Returns (U, seconds per stage)."""
     import oracle
     t0 = time.perf_counter()
     H = oracle.hessian(X)
@@ -739,29 +800,45 @@ def oracle_sample(cfg, X, W, rows: int):
     Hd, _ = oracle.damp_hessian(H, cfg.damp)
     U = oracle.upper_factor_of_inverse(Hd)
     t2 = time.perf_counter()
-    codes, scales, _ = oracle.gptq_sweep(W[:rows], U, cfg.group)
-    oracle.qerr(W[:rows], codes, scales, cfg.group)
-    t3 = time.perf_counter()
     buf = oracle.bf16tril_encode(H.astype(np.float32))
     oracle.bf16tril_decode(buf, cfg.K)
-    t4 = time.perf_counter()
-    sweep_full = (t3 - t2) * cfg.N / rows
-    est = (t1 - t0) + (t2 - t1) + sweep_full + (t4 - t3)
-    return est, {"syrk_s": t1 - t0, "factor_s": t2 - t1, "sweep_s_sample": t3 - t2, "codec_s": t4 - t3}
+    t3 = time.perf_counter()
+    return U, {"syrk_s": t1 - t0, "factor_s": t2 - t1, "codec_s": t3 - t2}
 
 
-def cpu_baseline(cfg, layer=None, rows: int = 32):
+def oracle_sweep_rows(cfg, W, U, r0: int, rows: int) -> float:
+    """Seconds the oracle's sweep and qerr take on rows r0 .. r0 + rows of W (rows are
+    independent given U, so a layer's sweep time is proportional to its rows)."""
+    import oracle
+    Ws = W[r0:r0 + rows]
+    t0 = time.perf_counter()
+    codes, scales, _ = oracle.gptq_sweep(Ws, U, cfg.group)
+    oracle.qerr(Ws, codes, scales, cfg.group)
+    return time.perf_counter() - t0
+
+
+ORACLE_SAMPLE_ROWS = 512  # rows per timed sweep: enough that the per-column overhead is a few %
+
+
+def cpu_baseline(cfg, layer=None, rows: int = ORACLE_SAMPLE_ROWS):
+    """The oracle on a bounded sample of the layer: its per-layer stages in full, then the sweep
+    of `rows` rows, scaled to the layer's rows."""
     if layer is not None:
         X = layer.X.double().cpu().numpy()
         W = layer.W.double().cpu().numpy()
     else:
         X = wl.make_activations(cfg, "cpu").double().numpy()
         W = wl.make_weights(cfg, "cpu").double().numpy()
-    est, det = oracle_sample(cfg, X, W, rows)
+    U, fixed = oracle_fixed(cfg, X)
+    rows = min(rows, cfg.N)
+    t_sweep = oracle_sweep_rows(cfg, W, U, 0, rows)
+    est = sum(fixed.values()) + t_sweep * cfg.N / rows
     return {"value": cfg.N * cfg.K / est, "unit": "weights/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": (f"full fp64 Hessian of X [{cfg.T}, {cfg.K}], full factorisation and codec, sweep of "
-                       f"{rows} of {cfg.N} rows scaled to all rows (rows are independent)"),
-            "stages_s": det, "host": _host_cpu(), "tiny_single_thread": _oracle_tiny_single_thread()}
+            "sample": (f"{workload_string(cfg)}: the oracle's fp64 Hessian of all {cfg.T} tokens, factorisation "
+                       f"and codec in full, and its sweep of {rows} of the {cfg.N} rows, scaled to all rows "
+                       f"(rows are independent given U)"),
+            "stages_s": dict(fixed, sweep_s=t_sweep, sweep_rows=rows), "host": _host_cpu(),
+            "tiny_single_thread": _oracle_tiny_single_thread()}
 
 
 def _host_cpu():
@@ -807,34 +884,47 @@ def _oracle_tiny_single_thread(reps: int = 5):
             "threads": 1, "s_per_step": t, "weights_per_s": cfg.N * cfg.K / t}
 
 
-def run_reference(args):
+def run_reference(args, budget_s: float = 150.0):
+    """The base contract's reference arm: the fp64 oracle, as it stands, on the host cores.  The
+    oracle's per-layer stages (Hessian, factorisation, codec) run once before the timed loop;
+    each step then sweeps the next block of rows (up to ORACLE_SAMPLE_ROWS, fewer when
+    warm-up + steps would otherwise exceed `budget_s`).  `ms_per_step` is the measured time of a
+    step; `value` scales the mean per-row sweep time to the layer and adds the per-layer
+    stages."""
     cfg = wl.CONFIGS[args.config]
     X = wl.make_activations(cfg, "cpu").double().numpy()
     W = wl.make_weights(cfg, "cpu").double().numpy()
-    rows = 8
+    U, fixed = oracle_fixed(cfg, X)
+    del X
+    t_row = oracle_sweep_rows(cfg, W, U, 0, 32) / 32
+    n_steps = max(args.warmup + args.steps, 1)
+    rows = int(budget_s / n_steps / max(t_row, 1e-9)) // 64 * 64
+    rows = max(64, min(ORACLE_SAMPLE_ROWS, rows, cfg.N))
+    r0 = 0
     for _ in range(args.warmup):
-        oracle_sample(cfg, X, W, rows)
-    ests = []
-    t0 = time.perf_counter()
+        oracle_sweep_rows(cfg, W, U, r0, rows)
+        r0 = (r0 + rows) % (cfg.N - rows + 1)
+    step_s = []
     for _ in range(args.steps):
-        est, _ = oracle_sample(cfg, X, W, rows)
-        ests.append(est)
-    wall = time.perf_counter() - t0
-    value = cfg.N * cfg.K / statistics.mean(ests)
+        step_s.append(oracle_sweep_rows(cfg, W, U, r0, rows))
+        r0 = (r0 + rows) % (cfg.N - rows + 1)
+    per_row = statistics.mean(step_s) / rows
+    est = sum(fixed.values()) + per_row * cfg.N
+    value = cfg.N * cfg.K / est
     cores = _blas_threads()
-    sample = (f"per step: full fp64 Hessian of X [{cfg.T}, {cfg.K}], full factorisation and codec, sweep of "
-              f"{rows} of {cfg.N} rows scaled to all rows")
+    sample = (f"{workload_string(cfg)}: per step the oracle's sweep (and qerr) of {rows} of the {cfg.N} rows; "
+              f"its Hessian of all {cfg.T} tokens, factorisation and codec ({sum(fixed.values()):.1f} s) once "
+              f"before the timed steps; value = weights / (those stages + mean per-row sweep time x {cfg.N} rows)")
     return {
         "impl": "reference",
         "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
         "value": value, "unit": "weights/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": statistics.mean(ests) * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": f"{cfg.name}: W [{cfg.N}, {cfg.K}], X [{cfg.T}, {cfg.K}], group {cfg.group}"},
+        "ms_per_step": statistics.mean(step_s) * 1e3 if step_s else None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": workload_string(cfg), "layers_per_gpu": 1},
         "cpu_baseline": {"value": value, "unit": "weights/s", "cores": cores, "kind": "oracle", "sample": sample,
-                         "host": _host_cpu()},
+                         "host": _host_cpu(), "stages_s": fixed, "rows_per_step": rows},
         "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "wall_s": wall,
     }
 
 

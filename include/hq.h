@@ -110,6 +110,10 @@ size_t hq_gptq_workspace_bytes(int64_t N, int64_t K, int64_t group);
  * events, kept for the thread's lifetime); it is joined back into `stream` before the call's
  * later work, so ordering on `stream` is as if everything ran there.  codes and scales do not
  * depend on whether qerr is requested, and are identical run to run.
+ * Non-finite inputs: a NaN or infinite weight affects only its own row's codes and scales
+ * (rows are independent) and makes qerr non-finite; a non-finite mean(diag H) is refused as
+ * HQ_ERR_INVALID after the damping stage; any other NaN or infinity in H's lower triangle
+ * reaches a Cholesky pivot and is reported as HQ_ERR_NOT_PD.
  */
 hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
                            int64_t group, float damp, const float* imp, uint8_t* codes,
@@ -134,8 +138,8 @@ hq_status hq_qerr_terms(const void* workspace, double* terms_dev, hq_stream_t st
 size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group);
 
 /*
- * Round-to-nearest int4 with the same quantiser and no error feedback (ork's "crude
- * symmetric absmax/7 rounding", [gptq] experiment summary): s = fp32(max|W[n,group]|/7),
+ * Round-to-nearest int4 with the same quantiser and no error feedback, the RTN baseline of
+ * symmetric absmax/7 rounding ([gptq] experiment summary): s = fp32(max|W[n,group]|/7),
  * c = clamp(rint(W/s), -8, 7).  Same argument meanings and output layouts as
  * hq_gptq_quantize.  Synchronises `stream` only when qerr_out != NULL.
  */
@@ -153,11 +157,18 @@ hq_status hq_rtn_quantize(const void* W, int w_dtype, int64_t N, int64_t K, int6
  * `workspace` / `workspace_bytes`.
  *   - Scratch (qerr partial sums, status) lives in one fixed array in the library's device
  *     memory: HQ_RTN_NOALLOC_MAX_GROUPS * 16 + 256 bytes (16 MiB + 256 B), held on every GPU
- *     that loads the library until the process exits.  N * (K / group) above
- *     HQ_RTN_NOALLOC_MAX_GROUPS is refused with HQ_ERR_UNSUPPORTED before any launch.
- *   - The call allocates nothing (no cudaMalloc, no allocating library routine).  The first
- *     call on a device looks up the array's device address (cudaGetSymbolAddress) with that
- *     device current; make that first call before any stream capture.
+ *     where the library's module holding it has been loaded, until the process exits.
+ *     N * (K / group) above HQ_RTN_NOALLOC_MAX_GROUPS is refused with HQ_ERR_UNSUPPORTED
+ *     before any launch; exactly HQ_RTN_NOALLOC_MAX_GROUPS groups are accepted.
+ *   - The call allocates nothing itself (no cudaMalloc, no allocating library routine).  The
+ *     array is committed when that module is loaded on a device; under CUDA's lazy module
+ *     loading (the default, CUDA_MODULE_LOADING=LAZY) that is the first call on the device,
+ *     which can therefore fail with HQ_ERR_CUDA if the device has no free memory left.  A caller
+ *     that must not allocate later makes one warm-up call on each device before it reserves its
+ *     memory pool or starts a stream capture; later calls commit nothing new.
+ *   - The first call on a device (and the first after the current context changes, e.g. after
+ *     a device reset) looks up the array's device address (cudaGetSymbolAddress) with that
+ *     device current, and caches it per device and context.
  *   - Every call on a device shares the one array and it keeps the last call's contents; each
  *     call re-initialises what it needs.  Calls whose GPU work overlaps (different streams,
  *     different host threads) race on it: serialise them.

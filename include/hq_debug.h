@@ -41,6 +41,24 @@ hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype,
                                            int* dev_status, int impl, hq_stream_t stream);
 
 /*
+ * The failure path of the tensor-core SYRK's bounded waits, made to run on purpose (no
+ * counterpart on the pages; the library's rule that a device-side wait never hangs).  The
+ * tcgen05 SYRK of hq_hessian_accumulate on bf16 X with
+ *   wait_limit_cycles : 1000 .. 4e9, the SM cycles any pipeline wait may take before the CTA
+ *                       records HQ_ERR_TIMEOUT in *dev_status, stops issuing, waits for the copies
+ *                       and tensor-core work it already issued, frees its tensor memory and returns;
+ *   withhold_stage    : -1 (an ordinary call), or 0 .. 3: the MMA issuer never releases that
+ *                       stage of the 4-stage operand ring after its first use, so the producer's
+ *                       wait to refill it expires (when X has more than 4 x 64 tokens) before it
+ *                       issues another load.  The stream and context stay usable; H is then
+ *                       partly or not updated.
+ *   dev_status : device int, required (zeroed by the caller).  X bf16 [T, K], K % 8 == 0, 16-byte
+ *                aligned (the tensor-core path), else HQ_ERR_UNSUPPORTED.  Asynchronous.
+ */
+hq_status hq_debug_hessian_accumulate_timeout(float* H, const void* X, int64_t T, int64_t K, int* dev_status,
+                                              int64_t wait_limit_cycles, int withhold_stage, hq_stream_t stream);
+
+/*
  * The tensor-core fp32 GEMM used by the GPTQ lazy updates:
  *   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]
  * for m < M, n < N (if `lower`, only elements with m >= n are written).  split3 = 1 selects

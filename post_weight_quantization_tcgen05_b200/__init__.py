@@ -26,6 +26,8 @@ HQ_ERR_CUDA = 5
 HQ_ERR_WORKSPACE = 6
 HQ_F32 = 0
 HQ_BF16 = 1
+# groups N * (K / group) that hq_rtn_quantize_noalloc's fixed scratch holds (hq.h)
+HQ_RTN_NOALLOC_MAX_GROUPS = 1048576
 
 _DTYPE = {torch.float32: HQ_F32, torch.bfloat16: HQ_BF16}
 
@@ -67,6 +69,7 @@ _SIGS = {
     "hq_debug_gptq_quantize_impl": (_int, [_vp, _int, _i64, _i64, _vp, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                            _int, _vp]),
     "hq_debug_hessian_accumulate_impl": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _int, _vp]),
+    "hq_debug_hessian_accumulate_timeout": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _int, _vp]),
     "hq_debug_launch_count": (ctypes.c_uint64, []),
     "hq_debug_tf32_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _f, _f, _int, _int, _vp]),
     "hq_debug_rcp_f64": (_int, [_vp, _vp, _i64, _vp]),
@@ -140,6 +143,18 @@ def hq_debug_hessian_accumulate_impl(H, X, impl: int, dev_status=None, stream=No
     T, K = X.shape
     _check(lib.hq_debug_hessian_accumulate_impl(_ptr(H), _ptr(X), _dtype(X), T, K, _ptr(dev_status), int(impl),
                                                 _stream(stream)), "hq_debug_hessian_accumulate_impl")
+
+
+def hq_debug_hessian_accumulate_timeout(H, X, dev_status, wait_limit_cycles: int, withhold_stage: int = -1,
+                                        stream=None) -> None:
+    """The tensor-core SYRK with a runtime wait limit and, for the test of its timeout path, one
+    operand stage the MMA issuer never releases (hq_debug.h)."""
+    if X.dtype != torch.bfloat16:
+        raise ValueError("the tensor-core SYRK takes bf16 X")
+    T, K = X.shape
+    st = lib.hq_debug_hessian_accumulate_timeout(_ptr(H), _ptr(X), T, K, _ptr(dev_status), int(wait_limit_cycles),
+                                                 int(withhold_stage), _stream(stream))
+    _check(st, "hq_debug_hessian_accumulate_timeout")
 
 
 def hq_imatrix(H, tokens: int, imp, stream=None) -> None:

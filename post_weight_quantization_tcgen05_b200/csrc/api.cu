@@ -97,6 +97,16 @@ hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype,
   return launch_syrk_simt(H, X, x_dtype, T, K, s);
 }
 
+hq_status hq_debug_hessian_accumulate_timeout(float* H, const void* X, int64_t T, int64_t K, int* dev_status,
+                                              int64_t wait_limit_cycles, int withhold_stage, hq_stream_t stream) {
+  if (H == nullptr || X == nullptr || dev_status == nullptr || K < 1 || T < 1) return HQ_ERR_INVALID;
+  if (wait_limit_cycles < 1000 || wait_limit_cycles > kWaitLimitCycles || withhold_stage < -1 || withhold_stage > 3)
+    return HQ_ERR_INVALID;
+  if (!syrk_tc_eligible(X, HQ_BF16, T, K) || K > (int64_t(1) << 20) || T > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
+  return launch_syrk_tc(H, X, T, K, dev_status, static_cast<cudaStream_t>(stream), wait_limit_cycles,
+                        withhold_stage);
+}
+
 hq_status hq_hessian_accumulate(float* H, const void* X, int x_dtype, int64_t T, int64_t K, int* dev_status,
                                 hq_stream_t stream) {
   return hq_debug_hessian_accumulate_impl(H, X, x_dtype, T, K, dev_status, 0, stream);

@@ -5,12 +5,16 @@
 #include <stdint.h>
 
 #include "../../include/hq.h"
+#include "common.cuh"
 
 namespace hq {
 
 // syrk.cu
 bool syrk_tc_eligible(const void* X, int x_dtype, int64_t T, int64_t K);
-hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev_status, cudaStream_t s);
+// wait_limit: cycles a pipeline wait may take before the kernel records HQ_ERR_TIMEOUT and stops;
+// withhold_stage >= 0 (tests of that path only): the MMA issuer never releases that ring stage.
+hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev_status, cudaStream_t s,
+                         long long wait_limit = kWaitLimitCycles, int withhold_stage = -1);
 hq_status launch_syrk_simt(float* H, const void* X, int x_dtype, int64_t T, int64_t K, cudaStream_t s);
 
 // codec.cu

@@ -1,5 +1,5 @@
-// Round-to-nearest int4 ("ork's crude symmetric absmax/7 rounding", ork-driver wiki
-// "Exp 2026-08-18 GPTQ Int4", experiment summary): the GPTQ quantiser without error feedback.
+// Round-to-nearest int4, the RTN baseline: symmetric absmax/7 rounding (ork-driver wiki
+// "Exp 2026-08-18 GPTQ Int4", experiment summary), i.e. the GPTQ quantiser without error feedback.
 // One warp per (row, group): absmax by shuffles, scale s = fp32(absmax / 7), codes
 // c = clamp(rint(w / s), -8, 7) packed two per byte, fp64 qerr partials per warp.
 #include <cuda_bf16.h>

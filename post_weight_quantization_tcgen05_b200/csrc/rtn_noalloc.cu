@@ -7,10 +7,15 @@
 // allocation after start-up, or a plugin that runs under another framework's allocator and has
 // no handle to it.  For them this entry point keeps its scratch -- the qerr partial sums and
 // the small status header -- in one fixed array that lives in the library's own device memory
-// for as long as the library is loaded, on every GPU that loads it.  The caller still provides
+// for as long as the library is loaded, on every GPU that loads it.  The array is committed on a
+// device when the library's module that holds it is loaded there; under CUDA's lazy module
+// loading (the default) that is the first call on that device.  The caller still provides
 // W, codes and scales.  The kernels are the same ones hq_rtn_quantize launches, so the results
 // are identical.
+#include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "../../include/hq.h"
 #include "common.cuh"
@@ -25,25 +30,63 @@ constexpr size_t kNoallocBytes = kNoallocHeader + static_cast<size_t>(HQ_RTN_NOA
 
 static __device__ __align__(256) unsigned char g_rtn_scratch[kNoallocBytes];
 
-// The array's device address on each device.  In host code `g_rtn_scratch` names a host-side
-// stand-in, not device memory, so the address is looked up once per device (with that device
-// current) and passed to the kernels.
+// The array's device address, per device and context.  In host code `g_rtn_scratch` names a
+// host-side stand-in, not device memory, so the address is looked up with the device current
+// (cudaGetSymbolAddress) and passed to the kernels.  The lookup is cached per device and keyed
+// by the current context's id: after a device reset the module is loaded again, possibly at
+// another address, and the new context's id forces a fresh lookup.
 constexpr int kMaxDevices = 64;
-static void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;
+  void* ptr = nullptr;
+};
+static ScratchSlot g_slot[kMaxDevices];
+static std::mutex g_slot_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Id of the context current on this thread (0 if none or unknown).
+unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 hq_status scratch_for_current_device(uint8_t** out) {
   int dev = -1;
   HQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
-  void* p = __atomic_load_n(&g_scratch_ptr[dev], __ATOMIC_ACQUIRE);
-  if (p == nullptr) {
+  unsigned long long id = current_context_id();
+  if (id == 0) {  // the runtime has not made this device's context current on this thread yet
+    HQ_CUDA_TRY(cudaSetDevice(dev));
+    id = current_context_id();
+  }
+  std::lock_guard<std::mutex> lock(g_slot_mu);
+  ScratchSlot& slot = g_slot[dev];
+  if (slot.ptr == nullptr || id == 0 || slot.ctx_id != id) {
+    void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_rtn_scratch) != cudaSuccess || p == nullptr) {
       (void)cudaGetLastError();
       return HQ_ERR_CUDA;
     }
-    __atomic_store_n(&g_scratch_ptr[dev], p, __ATOMIC_RELEASE);
+    slot.ptr = p;
+    slot.ctx_id = id;
   }
-  *out = static_cast<uint8_t*>(p);
+  *out = static_cast<uint8_t*>(slot.ptr);
   return HQ_OK;
 }
 

@@ -168,6 +168,9 @@ struct SyrkArgs {
   int T;         // tokens
   int tiles;     // lower-triangle tiles
   int* status;
+  long long wait_limit;  // cycles a pipeline wait may take before the CTA gives up
+  int withhold_stage;    // -1, or a ring stage whose first release the MMA issuer skips (the
+                         // test of the timeout path: the producer's wait for it then expires)
 };
 
 __global__ void __launch_bounds__(kSyThreads, 1)
@@ -226,7 +229,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
       syrk_tile_coords(t, tiles_m, tiles_n, m0, n0);
       for (int k = 0; k < kiters; ++k, ++g) {
         const int s = g % kSyStages;
-        if (g >= kSyStages && !ptx::mbar_wait(&empty[s], ((g / kSyStages) - 1) & 1, abort_flag)) {
+        if (g >= kSyStages && !ptx::mbar_wait(&empty[s], ((g / kSyStages) - 1) & 1, abort_flag, args.wait_limit)) {
           ok = false;
           break;
         }
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
       int k = 0;
       for (int seg = 0; seg < nseg && ok; ++seg, ++sg) {
         const int acc = sg & 1;
-        if (sg >= 2 && !ptx::mbar_wait(&acce[acc], ((sg >> 1) - 1) & 1, abort_flag)) {
+        if (sg >= 2 && !ptx::mbar_wait(&acce[acc], ((sg >> 1) - 1) & 1, abort_flag, args.wait_limit)) {
           ok = false;
           break;
         }
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
         const int kend = (kiters < kbeg + kSySegIters) ? kiters : kbeg + kSySegIters;
         for (; k < kend; ++k, ++g) {
           const int s = g % kSyStages;
-          if (!ptx::mbar_wait(&full[s], (g / kSyStages) & 1, abort_flag)) {
+          if (!ptx::mbar_wait(&full[s], (g / kSyStages) & 1, abort_flag, args.wait_limit)) {
             ok = false;
             break;
           }
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
             const uint64_t bd = ptx::sdesc_sw128(sb + kk * 2048, 8192, 1024);
             ptx::mma_bf16(dacc, ad, bd, kIdesc, (k > kbeg || kk > 0) ? 1u : 0u);
           }
-          ptx::mma_commit(&empty[s]);
+          if (!(g == args.withhold_stage && g < kSyStages)) ptx::mma_commit(&empty[s]);
         }
         if (ok) ptx::mma_commit(&accf[acc]);
       }
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
       for (int i = 0; i < 128; ++i) sum[i] = 0.f;
       for (int seg = 0; seg < nseg; ++seg, ++sg) {
         const int acc = sg & 1;
-        if (!ptx::mbar_wait(&accf[acc], (sg >> 1) & 1, abort_flag)) {
+        if (!ptx::mbar_wait(&accf[acc], (sg >> 1) & 1, abort_flag, args.wait_limit)) {
           ok = false;
           break;
         }
@@ -356,7 +359,8 @@ bool syrk_tc_eligible(const void* X, int x_dtype, int64_t T, int64_t K) {
   return x_dtype == HQ_BF16 && (K % 8) == 0 && aligned(X, 16) && K <= (1 << 24) && T <= 0x7FFFFFFF;
 }
 
-hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev_status, cudaStream_t s) {
+hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev_status, cudaStream_t s,
+                         long long wait_limit, int withhold_stage) {
   CUtensorMap map;
   if (!make_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K), static_cast<uint64_t>(T),
                     static_cast<uint64_t>(K) * 2, 64, 64))
@@ -373,6 +377,8 @@ hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev
   a.T = static_cast<int>(T);
   a.tiles = static_cast<int>(tiles);
   a.status = dev_status;
+  a.wait_limit = wait_limit;
+  a.withhold_stage = withhold_stage;
   const int grid = static_cast<int>(tiles < kSySMs ? tiles : kSySMs);
   const int tm = timer_start(kTimeSyrk, s);
   syrk_tc_kernel<<<grid, kSyThreads, kSySmem, s>>>(map, a);

@@ -99,3 +99,15 @@ def test_invalid_arguments_refused_before_launch(hq):
     assert L.hq_imatrix(fake, 8, 0, fake, None) == hq.HQ_ERR_INVALID
     assert L.hq_qerr_terms(None, fake, None) == hq.HQ_ERR_INVALID
     assert L.hq_qerr_terms(fake, None, None) == hq.HQ_ERR_INVALID
+
+
+def test_header_constants_match_the_binding(hq):
+    """#define constants of hq.h that the binding repeats."""
+    src = open(os.path.join(ROOT, "include", "hq.h")).read()
+    m = re.search(r"#define\s+HQ_RTN_NOALLOC_MAX_GROUPS\s+(\d+)", src)
+    assert m and int(m.group(1)) == hq.HQ_RTN_NOALLOC_MAX_GROUPS
+    # refused on the host: one group more than the scratch holds, before anything is launched
+    fake = ctypes.c_void_p(256)
+    over = hq.HQ_RTN_NOALLOC_MAX_GROUPS // 2 + 1
+    assert hq.lib.hq_rtn_quantize_noalloc(fake, 0, over, 64, 32, None, fake, fake, None, None, None) == \
+        hq.HQ_ERR_UNSUPPORTED

@@ -102,6 +102,36 @@ def test_syrk_bf16_chunked_and_simt_agree(hq, cuda_device):
     _syrk_check(hq, X, impl=1, chunks=2)
 
 
+def test_syrk_wait_timeout_is_reported_and_the_stream_stays_usable(hq, cuda_device):
+    """The bounded-wait failure path, made to run: the MMA issuer never releases the first
+    operand stage, so the producer's wait to refill it runs out (limit 1e6 cycles, about half
+    a millisecond) before it issues another load.  The call reports HQ_ERR_TIMEOUT through its
+    status word, leaves H untouched (no tile finished) and returns; the next ordinary call on
+    the same stream then computes the right H."""
+    cfg = wl.small_config(wl.CONFIGS[1], N=1, K=128, T=512)
+    X = wl.make_activations(cfg, "cuda")
+    H = torch.zeros((128, 128), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hq.hq_debug_hessian_accumulate_timeout(H, X, status, wait_limit_cycles=1_000_000, withhold_stage=0)
+    torch.cuda.synchronize()
+    assert status.item() == hq.HQ_ERR_TIMEOUT
+    assert torch.count_nonzero(H).item() == 0
+    # the same kernel with the short limit and nothing withheld finishes normally
+    status.zero_()
+    hq.hq_debug_hessian_accumulate_timeout(H, X, status, wait_limit_cycles=1_000_000, withhold_stage=-1)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = oracle.hessian(to_np64(X))
+    lo = np.tril(np.ones((128, 128), bool))
+    assert rel_fro(to_np64(H)[lo], ref[lo]) <= H_REL_FRO
+    # an ordinary call after the failed one
+    H.zero_()
+    hq.hq_hessian_accumulate(H, X, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert rel_fro(to_np64(H)[lo], ref[lo]) <= H_REL_FRO
+
+
 # ----------------------------------------------------------------------------- factorisation
 
 def _spd(K, seed, corr=0.7):
@@ -124,9 +154,14 @@ def test_factor_upper_cholesky_of_inverse(hq, cuda_device, K):
     U = oracle.upper_factor_of_inverse(Hdamp)
     Ug = to_np64(Ut).T
     assert np.array_equal(Ug, np.triu(Ug))
-    assert rel_fro(Ug, U) < 2e-4
+    # fp64 factorisation, rounded once to fp32: the rounding alone gives about 2.5e-8 relative
+    # Frobenius on U and 1.2e-7 on U H' U^T - I on these Hessians (kappa 1e3-1e4)
+    assert rel_fro(Ug, U) < 1e-7
     I = Ug @ Hdamp @ Ug.T
-    assert np.abs(I - np.eye(K)).max() < 5e-3
+    assert np.abs(I - np.eye(K)).max() < 1e-6
+    # almost every entry is the correctly rounded fp32 value of the oracle's fp64 U
+    up = np.triu(np.ones((K, K), bool))
+    assert np.mean(Ug[up] == U[up].astype(np.float32).astype(np.float64)) >= 0.99
 
 
 def test_factor_not_positive_definite(hq, cuda_device):
@@ -295,6 +330,97 @@ def test_gptq_not_pd_reported(hq, cuda_device):
     W = torch.ones((N, K), device="cuda")
     with pytest.raises(hq.HQError) as e:
         _run_gptq(hq, W, torch.from_numpy(H).cuda(), 32)
+    assert e.value.status == hq.HQ_ERR_NOT_PD
+
+
+# ----------------------------------------------------------------------------- GPTQ edge cases
+
+def _corr_layer(N, K, G, seed, wdt=torch.float32):
+    cfg = wl.correlated_config(N, K, T=2 * K, group=G, seed=seed)
+    X = wl.make_activations(cfg, "cpu")
+    H32 = oracle.hessian(X.double().numpy()).astype(np.float32)
+    W = wl.make_weights(cfg, "cpu", N=N, K=K).to(wdt)
+    return W, H32
+
+
+def test_gptq_zero_rows_and_zero_groups(hq, cuda_device):
+    """An all-zero row gives codes 0 and scales 0 (absmax 0: s = 0, c = 0); a row whose first
+    groups are zero keeps them zero (no error to feed back), so their scales are 0 too; a zero
+    group after non-zero columns receives feedback and gets the oracle's non-zero scale."""
+    N, K, G = 48, 512, 64
+    W, H32 = _corr_layer(N, K, G, seed=21)
+    W[0] = 0.0
+    W[1, :2 * G] = 0.0
+    W[2, 3 * G:4 * G] = 0.0
+    W[3, K - G:] = 0.0
+    Wd = W.cuda()
+    codes, scales, q = _run_gptq(hq, Wd, torch.from_numpy(H32).cuda(), G)
+    r = _compare_gptq(Wd, H32.astype(np.float64), G, codes, scales, q, what="zero rows/groups")
+    assert np.all(codes[0] == 0) and np.all(scales[0] == 0.0)
+    assert np.all(codes[1, :2 * G] == 0) and np.all(scales[1, :2] == 0.0) and np.all(scales[1, 2:] > 0.0)
+    assert np.all(r["scales"][2, 3] > 0.0) and scales[2, 3] > 0.0
+    assert np.all(r["codes"][0] == 0) and np.all(r["scales"][0] == 0.0) and np.all(r["scales"][1, :2] == 0.0)
+
+
+def test_gptq_code_minus_eight_after_compensation(hq, cuda_device):
+    """The clamp after compensation: H block-diagonal in 2 x 2 blocks [[4, 1.5], [1.5, 1]], so
+    the first column of each pair feeds its error into the second with U'[0, 1] = -b/c (about
+    -1.46 after damping).  Each pair is (6.6 s, -7 s) with s = absmax / 7: the first rounds up
+    to 7 (residual -0.4 s) and pushes the second to about -7.59 s, which rounds to -8.  Negated
+    rows push it to +7.59 s, which is clamped to +7."""
+    N, K, G = 64, 256, 32
+    H = np.zeros((K, K), np.float32)
+    for p in range(0, K, 2):
+        H[p:p + 2, p:p + 2] = [[4.0, 1.5], [1.5, 1.0]]
+    rng = np.random.default_rng(8)
+    amp = np.exp(rng.standard_normal((N, 1))) * 0.02
+    pair = np.tile(np.array([6.6 / 7.0, -1.0]), K // 2)
+    sign = np.where(np.arange(N) % 2 == 0, 1.0, -1.0)[:, None]
+    W = torch.from_numpy((amp * sign * pair).astype(np.float32)).cuda()
+    codes, scales, q = _run_gptq(hq, W, torch.from_numpy(H).cuda(), G)
+    r = _compare_gptq(W, H.astype(np.float64), G, codes, scales, q, what="clamp")
+    assert np.array_equal(codes, r["codes"]) and np.array_equal(scales, r["scales"])
+    assert np.all(codes[0::2, 1::2] == -8) and np.all(codes[0::2, 0::2] == 7)
+    assert np.all(codes[1::2, 1::2] == 7) and np.all(codes[1::2, 0::2] == -7)
+
+
+@pytest.mark.parametrize("N,K,G,wdt", [(40, 128, 128, torch.float32), (24, 1024, 1024, torch.bfloat16),
+                                      (1, 128, 32, torch.float32), (1, 128, 128, torch.bfloat16)])
+def test_gptq_group_equals_k_and_single_row(hq, cuda_device, N, K, G, wdt):
+    """One group spanning the whole row (a single scale per row, including a panel as wide as
+    the group), and the smallest layer: one row of 128 columns."""
+    W, H32 = _corr_layer(N, K, G, seed=N + K + G, wdt=wdt)
+    Wd = W.cuda()
+    codes, scales, q = _run_gptq(hq, Wd, torch.from_numpy(H32).cuda(), G)
+    assert scales.shape == (N, K // G)
+    _compare_gptq(Wd, H32.astype(np.float64), G, codes, scales, q, what=f"N={N} K={K} G={G}")
+
+
+def test_gptq_non_finite_inputs(hq, cuda_device):
+    """Non-finite inputs: a NaN weight leaves every other row's codes and scales exactly as
+    without it (rows are independent); a Hessian with an infinite diagonal entry is refused as
+    HQ_ERR_INVALID (mean(diag H) not finite); a NaN below the diagonal is reported as
+    HQ_ERR_NOT_PD (the Cholesky pivot it reaches is not a positive number)."""
+    N, K, G = 32, 256, 64
+    W, H32 = _corr_layer(N, K, G, seed=31)
+    Hd = torch.from_numpy(H32).cuda()
+    Wd = W.cuda()
+    c0, s0, _ = _run_gptq(hq, Wd, Hd, G)
+    Wn = Wd.clone()
+    Wn[5, 70] = float("nan")
+    c1, s1, q1 = _run_gptq(hq, Wn, Hd, G)
+    keep = np.arange(N) != 5
+    assert np.array_equal(c0[keep], c1[keep]) and np.array_equal(s0[keep], s1[keep])
+    assert np.isnan(q1)
+    Hinf = Hd.clone()
+    Hinf[7, 7] = float("inf")
+    with pytest.raises(hq.HQError) as e:
+        _run_gptq(hq, Wd, Hinf, G)
+    assert e.value.status == hq.HQ_ERR_INVALID
+    Hnan = Hd.clone()
+    Hnan[100, 3] = float("nan")
+    with pytest.raises(hq.HQError) as e:
+        _run_gptq(hq, Wd, Hnan, G)
     assert e.value.status == hq.HQ_ERR_NOT_PD
 
 

@@ -3,8 +3,10 @@ benchmark times (one hq_hessian_accumulate over the layer's tokens, then hq_gptq
 
 GPTQ rows are independent given U, so the oracle sweeps a seeded sample of rows exactly; the
 oracle's H and U are its own fp64 computations from the same X.  For the Hessian at scale
-(4.19 M tokens) the oracle computes sampled entries of H as exact dot products.  The oracle
-never takes the CUDA path's output as an input."""
+(4.19 M tokens) the oracle computes sampled entries of H as exact dot products.  Codes, and the
+scales of every group up to a row's first differing code, are compared with the plain oracle,
+which never takes the CUDA path's output as an input; only the scales after that point are
+compared on the GPU's own code trajectory (the oracle replaying the GPU's codes)."""
 
 import numpy as np
 import pytest

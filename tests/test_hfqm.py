@@ -71,31 +71,36 @@ def test_malformed_packages_are_refused():
 
 @pytest.mark.gpu
 def test_package_of_hessians_through_the_codec(tmp_path, cuda_device):
+    """Hessians from the oracle (fp64 X^T X of seeded activations, rounded to fp32) are written
+    into a package through the library's encoder and read back through its decoder: every
+    .hessian payload is the oracle's Bf16TrilDiagF32 encoding of the same matrix byte for byte,
+    load_hessian returns the oracle's decoding bit for bit, and the .imatrix payload is the
+    importance vector written."""
+    import oracle
     import post_weight_quantization_tcgen05_b200 as hq
     import workloads as wl
-    tensors = []
+    tensors, ref_H = [], []
     for i, K in enumerate((256, 384)):
         cfg = wl.small_config(wl.CONFIGS[1], N=8, K=K, T=1024, seed=i + 1)
-        X = wl.make_activations(cfg, "cuda")
-        H = torch.zeros((K, K), device="cuda")
-        hq.hq_hessian_accumulate(H, X)
-        imp = torch.empty(K, device="cuda")
-        hq.hq_imatrix(H, cfg.T, imp)
-        tensors.append((f"layers.{i}.mlp", H, imp))
+        X = wl.make_activations(cfg, "cpu")
+        H32 = oracle.hessian(X.double().numpy()).astype(np.float32)
+        imp32 = oracle.imatrix(H32.astype(np.float64), cfg.T).astype(np.float32)
+        tensors.append((f"layers.{i}.mlp", torch.from_numpy(H32).cuda(), torch.from_numpy(imp32).cuda()))
+        ref_H.append(H32)
     path = str(tmp_path / "m.calib.hfq")
     hfqm.write_package(hq, path, 42, {"tokens": 1024}, tensors)
     arch, meta, entries, buf = hfqm.read_package(path)
     assert arch == 42 and meta == {"tokens": 1024} and len(entries) == 4
-    for (name, H, imp), eh, ei in zip(tensors, entries[0::2], entries[1::2]):
+    for (name, H, imp), H32, eh, ei in zip(tensors, ref_H, entries[0::2], entries[1::2]):
         K = H.shape[0]
-        assert eh.name == name + ".hessian" and eh.shape == (K, K)
-        ref = torch.empty((K, K), device="cuda")
-        tril = torch.empty(hq.hq_bf16tril_bytes(K), dtype=torch.uint8, device="cuda")
-        hq.hq_hessian_pack_bf16tril(H, tril)
-        hq.hq_hessian_unpack_bf16tril(tril, K, ref)
+        assert eh.name == name + ".hessian" and eh.shape == (K, K) and eh.quant_type == 130
+        enc = oracle.bf16tril_encode(H32)
+        assert bytes(buf[eh.offset:eh.offset + eh.data_size]) == enc
         got = hfqm.load_hessian(hq, buf, eh)
         torch.cuda.synchronize()
-        assert torch.equal(got, ref)
+        assert np.array_equal(got.cpu().numpy().view(np.uint32), oracle.bf16tril_decode(enc, K).view(np.uint32))
         assert torch.equal(hfqm.load_imatrix(buf, ei), imp)
         proj = hfqm.load_hessian(hq, buf, eh, project=True)
-        assert float(torch.linalg.norm(proj - ref) / torch.linalg.norm(ref)) < 1e-3
+        ref_proj = oracle.project_psd(oracle.bf16tril_decode(enc, K).astype(np.float64))
+        err = np.linalg.norm(proj.double().cpu().numpy() - ref_proj) / np.linalg.norm(ref_proj)
+        assert err < 1e-5, err

@@ -77,13 +77,13 @@ def test_bench_line_carries_the_contract_keys():
     import workloads as wl
     cfg = wl.CONFIGS[1]
     args = types.SimpleNamespace(steps=10, warmup=3)
-    peaks = bench._peaks()
+    peaks = dict(bench._peaks(), tf32_tflops=800.0, fp64_tflops=37.0)
     kernels = {"syrk": {"achieved": 1000.0, "ms_per_step": 0.2, "launches_per_step": 1.0},
                "tf32_gemm": {"achieved": 120.0, "ms_per_step": 1.1, "launches_per_step": 39.0}}
     e2e = {"value": 2.0e9, "unit": "weights/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
     clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
     line = bench.build_line(args, cfg, 1, 2.8e9, 9.3, [0.2], [9.0], [0.03], [0.03], 900.0, 7.9e7, 1.3e8,
-                            peaks, e2e, 394, clocks, (33.0, 6.7e11, 40), kernels, 37.0)
+                            peaks, e2e, 394, clocks, (33.0, 6.7e11, 40), kernels, {"fp64_tflops": 37.0})
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
         assert key in line, key
@@ -93,6 +93,28 @@ def test_bench_line_carries_the_contract_keys():
     for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
         assert key in roof, key
     assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    assert roof["peak"] == 37.0  # the fp64 rate measured in the run, not a nominal ratio
+    assert line["update_roofline"]["tf32_tflops"] == 800.0
     assert roof["traffic"] is None or roof["traffic"] > 0
     assert line["gpu_launches"] == 3940
     json.dumps(line)
+
+
+def test_reference_arm_times_what_it_reports():
+    """The oracle arm on the tiny layer: the steps it reports are the steps it timed (their
+    total fits inside the call's wall time), and its workload string is the GPU arm's."""
+    import time
+    import types
+
+    import bench
+    import workloads as wl
+    args = types.SimpleNamespace(steps=2, warmup=1, config=0)
+    t0 = time.perf_counter()
+    line = bench.run_reference(args)
+    wall = time.perf_counter() - t0
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["value"] > 0
+    assert line["ms_per_step"] * line["steps"] / 1e3 <= wall
+    assert line["config"]["workload"] == bench.workload_string(wl.CONFIGS[0])
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

@@ -45,11 +45,46 @@ def test_noalloc_matches_workspace_entry_point_twice(hq, cuda_device):
         assert abs(q - rq) <= 1e-12 * rq and qd.item() == q
 
 
+def test_noalloc_commits_no_memory_after_its_first_call(hq, cuda_device):
+    """The property the entry point exists for: once a first call on the device has loaded the
+    library's scratch array, later calls leave the device's free memory unchanged."""
+    N, K, G = 256, 1024, 64
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    W = torch.randn((N, K), generator=g, device="cuda")
+    codes, scales = hq.gptq_outputs(N, K, G)
+    qd = torch.zeros(1, dtype=torch.float64, device="cuda")
+    hq.hq_rtn_quantize_noalloc(W, G, codes, scales, qerr_dev=qd, want_qerr=False)  # warm-up
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(2):
+        hq.hq_rtn_quantize_noalloc(W, G, codes, scales, qerr_dev=qd, want_qerr=False)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+
+
+def test_noalloc_at_exactly_the_scratch_limit(hq, cuda_device):
+    """N * (K / group) equal to the scratch's capacity is accepted and matches the workspace
+    entry point."""
+    N, K, G = 8192, 2048, 16
+    assert N * (K // G) == hq.HQ_RTN_NOALLOC_MAX_GROUPS
+    g = torch.Generator(device="cuda")
+    g.manual_seed(9)
+    W = torch.rand((N, K), generator=g, device="cuda") * 2.0 - 1.0
+    codes, scales = hq.gptq_outputs(N, K, G)
+    q = hq.hq_rtn_quantize_noalloc(W, G, codes, scales)
+    torch.cuda.synchronize()
+    rc, rs, rq = _reference(hq, W, G, None)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(scales.cpu().numpy(), rs)
+    assert abs(q - rq) <= 1e-12 * rq
+
+
 def test_noalloc_refuses_more_groups_than_its_scratch(hq, cuda_device):
     W = torch.zeros((8, 64), device="cuda")
     codes, scales = hq.gptq_outputs(8, 64, 32)
     raw = hq.lib.hq_rtn_quantize_noalloc  # N * (K / group) beyond the scratch: refused, nothing launched
-    limit = 1048576
+    limit = hq.HQ_RTN_NOALLOC_MAX_GROUPS
     st = raw(W.data_ptr(), hq.HQ_F32, limit // 2 + 1, 64, 32, None, codes.data_ptr(), scales.data_ptr(),
                     None, None, None)
     assert st == hq.HQ_ERR_UNSUPPORTED
