@@ -95,6 +95,24 @@ hq_status hq_debug_f64_gemm(double* C, int64_t ldc, int M, int N, int Kred, cons
                             double* scratch, int64_t scratch_elems, hq_stream_t stream);
 
 /*
+ * The same product as hq_debug_f64_gemm, fp64-accurate on the int8 tensor cores: every operand
+ * row scaled by a power of two and cut into 7 signed 7-bit int8 slices (exact in fp64), the 28
+ * slice-pair products of anti-diagonals 0..6 accumulated exactly in int32 by tcgen05 kind::i8
+ * MMAs, recombined in fp64 (error-free slicing after Ozaki, Ogita, Oishi & Rump; no counterpart
+ * on the pages: a building block of the factorisation).  Relative error about 1e-14 of the
+ * product of the operands' row maxima per term.  `tri` as for hq_debug_f64_gemm, at 128-row
+ * granularity: the slices read only the 128-aligned band of each row where the declared
+ * triangular operand can be non-zero (entries outside it are never read, whatever they hold).
+ * Rows holding a NaN or an infinity give NaN products.  Kred <= 16384 (the int32 sums stay
+ * exact).  `scratch`: device, 256-byte aligned, hq_debug_i8x_scratch_bytes(M, N, Kred) bytes
+ * (the slices and the row exponents).  A, B 8-byte aligned.  C is not read when beta == 0.
+ */
+size_t hq_debug_i8x_scratch_bytes(int M, int N, int Kred);
+hq_status hq_debug_i8x_gemm(double* C, int64_t ldc, int M, int N, int Kred, const double* A, int64_t lda,
+                            const double* B, int64_t ldb, double alpha, double beta, int lower, int tri, void* scratch,
+                            size_t scratch_bytes, hq_stream_t stream);
+
+/*
  * out[i] = 1 / d[i] (fp64) by the reciprocal the factorisation's leaf kernel uses for its pivots
  * (hardware approximation refined by two Newton-Raphson steps), for d[i] positive, normal and
  * finite (other inputs give unspecified values).  n >= 0.  No counterpart on the pages.
@@ -107,7 +125,9 @@ hq_status hq_debug_rcp_f64(const double* d, double* out, int64_t n, hq_stream_t 
  * stream, with the launch's algorithmic work: 0 = fp64 GEMM, 128-wide tiles (flops);
  * 1 = fp64 GEMM, 64-wide tiles, including its split-K reduction (flops); 2 = factorisation
  * leaf (flops of a 128 x 128 Cholesky and triangular inverse); 3 = GPTQ block sweep (bytes);
- * 4 = tf32 lazy-update GEMM (flops of the product); 5 = tcgen05 SYRK (flops).
+ * 4 = tf32 lazy-update GEMM (flops of the product); 5 = tcgen05 SYRK (flops); 6 = int8-sliced
+ * fp64 GEMM product kernel (flops of the fp64 product it computes, triangular operands counted
+ * once); 7 = its slicing kernels (bytes: fp64 operands read, int8 slices written).
  * hq_debug_timing_start clears the records and sets the mask; hq_debug_timing_read
  * synchronises the recorded events and returns the sum of durations (ms), of work and the
  * number of launches of one class; hq_debug_timing_stop clears the mask.  Events are created

@@ -80,6 +80,9 @@ _SIGS = {
     "hq_debug_timing_read": (_int, [_int, _vp, _vp, _vp]),
     "hq_debug_f64_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _dbl, _dbl, _int, _int, _vp,
                                  _i64, _vp]),
+    "hq_debug_i8x_scratch_bytes": (_sz, [_int, _int, _int]),
+    "hq_debug_i8x_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _dbl, _dbl, _int, _int, _vp,
+                                 _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -274,7 +277,8 @@ def hq_debug_fp64_mma_rate(stream=None) -> float:
     return float(r)
 
 
-TIMING_CLASSES = {"f64_gemm_128": 0, "f64_gemm_64": 1, "leaf": 2, "sweep": 3, "tf32_gemm": 4, "syrk": 5}
+TIMING_CLASSES = {"f64_gemm_128": 0, "f64_gemm_64": 1, "leaf": 2, "sweep": 3, "tf32_gemm": 4, "syrk": 5,
+                  "i8x_gemm": 6, "i8x_slice": 7}
 
 
 def hq_debug_timing_start(classes) -> None:
@@ -317,6 +321,19 @@ def hq_debug_f64_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, tri=0, scratch=
     _check(lib.hq_debug_f64_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
                                  float(alpha), float(beta), int(bool(lower)), int(tri), _ptr(scratch),
                                  0 if scratch is None else scratch.numel(), _stream(stream)), "hq_debug_f64_gemm")
+
+
+def hq_debug_i8x_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, tri=0, scratch=None, stream=None) -> None:
+    """C = beta C + alpha A B^T (fp64) through the int8-sliced tensor-core GEMM (hq_debug.h)."""
+    M, Kred = A.shape
+    N = B.shape[0]
+    need = lib.hq_debug_i8x_scratch_bytes(M, N, Kred)
+    if scratch is None:
+        scratch = alloc_workspace(need, C.device)
+    st = lib.hq_debug_i8x_gemm(_ptr(C), C.shape[1], M, N, Kred, _ptr(A), A.shape[1], _ptr(B), B.shape[1],
+                               float(alpha), float(beta), int(bool(lower)), int(tri), _ptr(scratch),
+                               scratch.numel() * scratch.element_size(), _stream(stream))
+    _check(st, "hq_debug_i8x_gemm")
 
 
 def hq_bf16tril_bytes(K: int) -> int:

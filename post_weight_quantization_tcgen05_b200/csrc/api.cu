@@ -161,8 +161,8 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
   float* Ut = nullptr;
   float* U = nullptr;
   hq_status st = launch_factor(H, K, damp, reinterpret_cast<double*>(ws + L.a), reinterpret_cast<double*>(ws + L.x),
-                               reinterpret_cast<double*>(ws + L.xt), reinterpret_cast<double*>(ws + L.t), &hdr->lam,
-                               &hdr->info, &hdr->status, &Ut, &U, false, false, nullptr, nullptr, s);
+                               reinterpret_cast<double*>(ws + L.xt), reinterpret_cast<double*>(ws + L.t), ws + L.slices,
+                               &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, false, false, nullptr, nullptr, s);
   if (st != HQ_OK) return st;
   HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, Ut, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return finish_sync(s, hdr, nullptr);
@@ -199,6 +199,35 @@ hq_status hq_debug_f64_gemm(double* C, int64_t ldc, int M, int N, int Kred, cons
   g.scratch_elems = scratch == nullptr ? 0 : scratch_elems;
   g.skip = nullptr;
   return f64_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+size_t hq_debug_i8x_scratch_bytes(int M, int N, int Kred) {
+  if (M < 1 || N < 1 || Kred < 1) return 0;
+  return i8x_scratch_bytes(M, N, Kred);
+}
+
+hq_status hq_debug_i8x_gemm(double* C, int64_t ldc, int M, int N, int Kred, const double* A, int64_t lda,
+                            const double* B, int64_t ldb, double alpha, double beta, int lower, int tri, void* scratch,
+                            size_t scratch_bytes, hq_stream_t stream) {
+  if (C == nullptr || A == nullptr || B == nullptr || M < 0 || N < 0 || Kred < 1) return HQ_ERR_INVALID;
+  if (ldc < N || lda < Kred || ldb < Kred || tri < kTriNone || tri > kTriBLower) return HQ_ERR_INVALID;
+  if (lower && M != N) return HQ_ERR_UNSUPPORTED;
+  if (Kred > kI8xMaxKred) return HQ_ERR_UNSUPPORTED;
+  F64Gemm g{};
+  g.C = C;
+  g.ldc = ldc;
+  g.M = M;
+  g.N = N;
+  g.Kred = Kred;
+  g.A = A;
+  g.lda = lda;
+  g.B = B;
+  g.ldb = ldb;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.lower = lower ? 1 : 0;
+  g.tri = tri;
+  return i8x_gemm(g, static_cast<uint8_t*>(scratch), scratch_bytes, static_cast<cudaStream_t>(stream));
 }
 
 hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,

@@ -27,6 +27,7 @@
 //   4. U = J X J and U^T = J X^T J, both row-major (180-degree rotated copies)
 // A device flag `info` receives the first failing pivot (1-based, in M's order) and stops
 // every later kernel.
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -431,7 +432,26 @@ struct FactorCtx {
   int* status;
   cudaStream_t s;   // the caller's stream: the critical path
   SideStream* side;  // s2: Y^T products and transposes
+  uint8_t* slices[2];  // int8 slices of the large products' operands: [0] for s, [1] for s2
+  size_t slices_bytes;  // each
 };
+
+// Products with all three dimensions at least this large run on the int8 tensor cores
+// (gemm_i8x.cu), the rest on the fp64 tensor cores (gemm_f64.cu).
+constexpr int64_t kI8xMinDim = 1024;
+
+static bool use_i8x(int64_t M, int64_t N, int64_t Kred) {
+  return M >= kI8xMinDim && N >= kI8xMinDim && Kred >= kI8xMinDim && Kred <= kI8xMaxKred;
+}
+
+size_t factor_slice_bytes(int64_t K) {
+  const int64_t n1 = (K / kLeaf / 2) * kLeaf, n2 = K - n1;
+  const int64_t dims[4][3] = {{n2, n1, n1}, {n1, n2, n1}, {n2, n2, n1}, {n2, n1, n2}};
+  size_t b = 0;
+  for (const auto& d : dims)
+    if (use_i8x(d[0], d[1], d[2])) b = std::max(b, i8x_scratch_bytes(d[0], d[1], d[2]));
+  return b;
+}
 
 // `from` -> `to`: work enqueued on `to` from now on waits for everything enqueued on `from` so far.
 static hq_status stream_dep(SideStream* ss, cudaStream_t from, cudaStream_t to) {
@@ -467,6 +487,11 @@ static hq_status gemm(const FactorCtx& c, cudaStream_t s, double* scratch, doubl
   g.scratch = scratch;
   g.scratch_elems = scratch == nullptr ? 0 : c.tmp_end - scratch;
   g.skip = c.info;
+  g.status = c.status;
+  if (use_i8x(M, N, Kred)) {
+    uint8_t* sl = c.slices[s == c.s ? 0 : 1];
+    if (sl != nullptr && i8x_scratch_bytes(M, N, Kred) <= c.slices_bytes) return i8x_gemm(g, sl, c.slices_bytes, s);
+  }
   return f64_gemm(g, s);
 }
 
@@ -595,9 +620,8 @@ __global__ void sweep_pack_kernel(const double* __restrict__ X, int64_t K, float
 // ------------------------------------------------------------------------- driver
 
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form, bool split_ut,
-                        float** Ut_hi, float** Ut_lo, cudaStream_t s) {
-  (void)status;
+                        uint8_t* slices, double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form,
+                        bool split_ut, float** Ut_hi, float** Ut_lo, cudaStream_t s) {
   if (K % kLeaf != 0 || K % kSweepBlk != 0) return HQ_ERR_UNSUPPORTED;
   HQ_CUDA_TRY(cudaFuncSetAttribute(chol_inv_leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(kLeafSmem)));
@@ -620,7 +644,12 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   SideStream* side = nullptr;
   hq_status st = side_stream(&side);
   if (st != HQ_OK) return st;
-  FactorCtx c{A, X, XT, T + K * K, K, info, status, s, side};
+  const size_t sb = factor_slice_bytes(K);
+  FactorCtx c{A, X, XT, T + K * K, K, info, status, s, side, {nullptr, nullptr}, sb};
+  if (slices != nullptr && sb > 0) {
+    c.slices[0] = slices;
+    c.slices[1] = slices + sb;
+  }
   st = stream_dep(side, s, side->s2);  // the side stream starts after everything before this call
   if (st != HQ_OK) return st;
   st = chol_inv(c, 0, K, T);

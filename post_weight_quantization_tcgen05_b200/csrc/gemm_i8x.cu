@@ -1,0 +1,512 @@
+// fp64-accurate GEMM on the int8 tensor cores (tcgen05.mma kind::i8), by error-free slicing of
+// the fp64 operands (the Ozaki scheme: Ozaki, Ogita, Oishi & Rump 2012; run on integer matrix
+// units by Ootomo, Ozaki & Yokota 2024):
+//
+//   C[m, n] = beta * C[m, n] + alpha * sum_k A(m, k) B(n, k)      m < M, n < N
+//   A(m, k) = A[m * lda + k],  B(n, k) = B[n * ldb + k]           (both operands K-major)
+//
+// Slicing (i8x_slice_kernel, one warp per row).  Row r of an operand is scaled by 2^-e_r, e_r the
+// smallest exponent with max_k |x[r, k]| < 2^e_r, and cut into kSlices signed 7-bit integers:
+//   y_0 = x 2^-e_r;  d_s = trunc(128 y_s) in [-127, 127];  y_{s+1} = 128 y_s - d_s,
+// so x = 2^e_r sum_s d_s 2^(-7 (s + 1)) + 2^(e_r - 7 S) y_S with |y_S| < 1.  Every step is exact in
+// fp64 (a power-of-two scaling, a truncation, the subtraction of a value's own integer part).
+// Slice s of all rows is a plane [rows][Kpad] of int8 (K-major), zero outside the part of the
+// row the product reads (a declared triangular operand) and past Kred.
+//
+// Product.  x_a x_b = 2^(e_a + e_b) sum_{s,t} d_s d_t 2^(-7 (s + t + 2)): every slice product is
+// an exact integer, and the pairs of one anti-diagonal s + t = g share the scale 2^(-7 (g + 2)).
+// The pairs with g <= kSlices - 1 are kept (28 of the 49 for 7 slices); the dropped ones and the
+// slicing remainders are below about (kSlices + 2) 2^(-7 kSlices) = 1.6e-14 of |x_a| |x_b|
+// relative to each operand's row maximum.  Per 128 x 64 output tile the kernel accumulates each
+// anti-diagonal in its own int32 TMEM accumulator (7 x 64 columns); the sums are exact while
+// 7 * 127^2 * Kred < 2^31 (Kred <= 16384).  The epilogue converts each accumulator to fp64,
+// scales it by its power of two, adds the diagonals smallest first, scales by 2^(e_a + e_b) and
+// alpha and adds beta C (C is not read when beta == 0).
+//
+// Kernel (i8x_gemm_kernel, persistent, one CTA per SM, 192 threads): warp 0 issues TMA loads of
+// the slices ([rows][32 bytes of k] boxes, 32-byte swizzle; one 3-D box holds all 7 planes of an
+// operand) into a 4-stage ring; warp 1 issues the 28 kind::i8 MMAs (M = 128, N = 64, K = 32) of
+// each stage from one thread; warps 2-5 drain the accumulators of a finished tile (TMEM lane
+// quadrant = 32 tile rows each), stage 16-column chunks of the fp64 result in shared memory and
+// update C with coalesced 16-byte accesses.  A declared triangular operand shortens each tile's
+// contraction to the part where it can be non-zero; tiles run longest first.  Every wait is
+// bounded; on expiry the CTA records HQ_ERR_TIMEOUT, waits for what it issued and returns.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace hq {
+namespace {
+
+constexpr int kSlices = kI8xSlices;
+constexpr int kBM = 128, kBN = 64, kBK = 32;       // tile rows, tile columns, contraction bytes per stage
+constexpr int kStages = 4;
+constexpr int kASlice = kBM * kBK;                  // 4 KB per plane
+constexpr int kBSlice = kBN * kBK;                  // 2 KB per plane
+constexpr int kStageBytes = kSlices * (kASlice + kBSlice);
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kChunk = 16;                          // epilogue columns per round
+constexpr int kStLd = kChunk + 1;                   // staging row stride (doubles)
+constexpr int kEpiBytes = kEpiWarps * 32 * kStLd * 8;
+constexpr int kSmem = kStages * kStageBytes + kEpiBytes + 1024 + 256;
+constexpr int kTmemCols = 512;                      // kSlices * kBN = 448 used
+constexpr int kSMs = 148;
+static_assert(kSlices * kBN <= kTmemCols, "accumulators do not fit in TMEM");
+static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+
+constexpr int kNonFiniteRow = -0x7FFFFFFF;  // exponent marking a row with a NaN or an infinity
+
+// Part of row r (in units of 128 columns) where a declared triangular operand can be non-zero:
+// [klo, khi).  `which` 0 = operand A, 1 = operand B.
+__host__ __device__ inline void tri_row_range(int tri, int which, int64_t r, int64_t Kred, int64_t& klo,
+                                              int64_t& khi) {
+  klo = 0;
+  khi = Kred;
+  const int64_t blk = (r / 128) * 128;
+  if (which == 0 && tri == kTriAUpper) klo = blk < Kred ? blk : Kred;
+  if (which == 0 && tri == kTriALower) khi = blk + 128 < Kred ? blk + 128 : Kred;
+  if (which == 1 && tri == kTriBLower) khi = blk + 128 < Kred ? blk + 128 : Kred;
+}
+
+// ------------------------------------------------------------------------- slicing
+
+// One warp per row: e_r, then kSlices int8 planes of the row (16 columns per lane per round).
+__global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict__ X, int64_t ldx, int64_t rows,
+                                                        int64_t Kred, int64_t Kpad, int tri, int which,
+                                                        int8_t* __restrict__ planes, int* __restrict__ exps,
+                                                        const int* __restrict__ skip) {
+  if (skip != nullptr && *skip != 0) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  int64_t klo, khi;
+  tri_row_range(tri, which, r, Kred, klo, khi);
+  const double* xr = X + r * ldx;
+  double mx = 0.0;
+  bool bad = false;
+  for (int64_t k = klo + lane; k < khi; k += 32) {
+    const double v = xr[k];
+    bad |= !isfinite(v);
+    mx = fmax(mx, fabs(v));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  bad = __any_sync(0xffffffffu, bad);
+  // a row holding a NaN or an infinity is marked, and its products come out NaN
+  const int e = bad ? kNonFiniteRow : (mx > 0.0 ? ilogb(mx) + 1 : 0);
+  if (lane == 0) exps[r] = e;
+  const double sc = bad ? 0.0 : ldexp(1.0, -e);
+  const int64_t plane = rows * Kpad;
+  int8_t* out = planes + r * Kpad;
+  for (int64_t k0 = 16 * lane; k0 < Kpad; k0 += 16 * 32) {
+    uint32_t w[kSlices][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int s = 0; s < kSlices; ++s) w[s][q] = 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int64_t k = k0 + 4 * q + b;
+        double y = (k >= klo && k < khi && !bad) ? xr[k] * sc : 0.0;
+#pragma unroll
+        for (int s = 0; s < kSlices; ++s) {
+          y *= 128.0;
+          const double t = trunc(y);
+          y -= t;
+          w[s][q] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu) << (8 * b);
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < kSlices; ++s)
+      *reinterpret_cast<uint4*>(out + s * plane + k0) = make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
+  }
+}
+
+// ------------------------------------------------------------------------- product
+
+struct I8xArgs {
+  double* C;
+  int64_t ldc;
+  int M, N, Kpad;
+  int tiles_m, tiles_n, tiles;
+  double alpha, beta;
+  int lower, tri;
+  const int* eA;
+  const int* eB;
+  const int* skip;
+  int* status;
+};
+
+// Tile t in execution order -> (m0, n0, first and last contraction stage).  Longest contraction
+// first: with A upper the low tile rows, with A lower the high ones, with B lower the high tile
+// columns.  With `lower`, only tiles holding an element m >= n are enumerated.
+__device__ inline void i8x_tile(const I8xArgs& a, int t, int& m0, int& n0, int& kb0, int& kb1) {
+  int tm, tn;
+  if (a.lower) {
+    // tile row tm holds column tiles 0 .. min(2 tm + 1, tiles_n - 1); rows walked from the last
+    int rem = t;
+    tm = a.tiles_m - 1;
+    for (;; --tm) {
+      const int cnt = (2 * tm + 2 < a.tiles_n) ? 2 * tm + 2 : a.tiles_n;
+      if (rem < cnt || tm == 0) {
+        tn = rem;
+        break;
+      }
+      rem -= cnt;
+    }
+  } else if (a.tri == kTriBLower) {
+    tn = a.tiles_n - 1 - t / a.tiles_m;
+    tm = t % a.tiles_m;
+  } else if (a.tri == kTriALower) {
+    tm = a.tiles_m - 1 - t / a.tiles_n;
+    tn = t % a.tiles_n;
+  } else {
+    tm = t / a.tiles_n;
+    tn = t % a.tiles_n;
+  }
+  m0 = tm * kBM;
+  n0 = tn * kBN;
+  int64_t lo = 0, hi = a.Kpad;
+  if (a.tri == kTriAUpper) lo = m0;
+  if (a.tri == kTriALower) hi = m0 + kBM;
+  if (a.tri == kTriBLower) hi = (n0 / 128) * 128 + 128;
+  if (hi > a.Kpad) hi = a.Kpad;
+  if (lo > hi) lo = hi;
+  kb0 = static_cast<int>(lo / kBK);
+  kb1 = static_cast<int>((hi + kBK - 1) / kBK);
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// K-major operand tile with 32-byte rows and the 32-byte swizzle (layout type 6): 8-row atoms
+// of 256 bytes.
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16 >> 4) << 16;
+  d |= static_cast<uint64_t>(256 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(6) << 61;
+  return d;
+}
+
+// kind::i8 instruction descriptor: s32 accumulator (bits 4-5 = 2), signed A and B (bits 7-9,
+// 10-12 = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kBN) >> 3) << 17) |
+                              ((static_cast<uint32_t>(kBM) >> 4) << 24);
+
+// 32 lanes x 16 consecutive 32-bit TMEM columns, no wait.
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    i8x_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB, I8xArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  double* stage_c = reinterpret_cast<double*>(smem + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kEpiBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* accf = empty + kStages;  // accumulators filled (one tile's MMAs done)
+  uint64_t* acce = accf + 1;         // accumulators drained
+  uint64_t* drain = acce + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (args.skip != nullptr && *args.skip != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(accf, 1);
+    ptx::mbar_init(acce, kEpiWarps);
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    record_status(args.status, HQ_ERR_TIMEOUT);
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    ptx::prefetch_tensormap(&mA);
+    ptx::prefetch_tensormap(&mB);
+    int g = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
+      int m0, n0, kb0, kb1;
+      i8x_tile(args, t, m0, n0, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++g) {
+        const int s = g % kStages;
+        if (g >= kStages && !ptx::mbar_wait(&empty[s], ((g / kStages) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * kStageBytes;
+        ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+            "[%5];" ::"r"(ptx::smem_u32(st)),
+            "l"(reinterpret_cast<uint64_t>(&mA)), "r"(kb * kBK), "r"(m0), "r"(0), "r"(ptx::smem_u32(&full[s]))
+            : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+            "[%5];" ::"r"(ptx::smem_u32(st + kSlices * kASlice)),
+            "l"(reinterpret_cast<uint64_t>(&mB)), "r"(kb * kBK), "r"(n0), "r"(0), "r"(ptx::smem_u32(&full[s]))
+            : "memory");
+      }
+    }
+    if (!ok) {
+      fail();
+      const int first = g > kStages ? g - kStages : 0;
+      for (int k = first; k < g; ++k) ptx::mbar_wait(&full[k % kStages], (k / kStages) & 1, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    int g = 0, i = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x, ++i) {
+      int m0, n0, kb0, kb1;
+      i8x_tile(args, t, m0, n0, kb0, kb1);
+      if (i >= 1 && !ptx::mbar_wait(acce, (i - 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      for (int kb = kb0; kb < kb1; ++kb, ++g) {
+        const int s = g % kStages;
+        if (!ptx::mbar_wait(&full[s], (g / kStages) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t sa = ptx::smem_u32(smem + s * kStageBytes);
+        const uint32_t sb = sa + kSlices * kASlice;
+#pragma unroll
+        for (int p = 0; p < kSlices; ++p) {
+          const uint64_t ad = sdesc_sw32(sa + p * kASlice);
+#pragma unroll
+          for (int q = 0; q + p < kSlices; ++q) {
+            const uint64_t bd = sdesc_sw32(sb + q * kBSlice);
+            mma_i8(tmem + static_cast<uint32_t>((p + q) * kBN), ad, bd, kIdescI8, (kb > kb0 || p > 0) ? 1u : 0u);
+          }
+        }
+        ptx::mma_commit(&empty[s]);
+      }
+      if (!ok) break;
+      ptx::mma_commit(accf);  // (a tile with an empty contraction issues no MMA: its result is 0)
+    }
+    if (!ok) {
+      fail();
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, nullptr);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant: tile rows 32 q .. 32 q + 31
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    double* st = stage_c + (warp - 2) * 32 * kStLd;
+    bool ok = true;
+    int i = 0;
+    for (int t = blockIdx.x; t < args.tiles; t += gridDim.x, ++i) {
+      int m0, n0, kb0, kb1;
+      i8x_tile(args, t, m0, n0, kb0, kb1);
+      if (ok) {
+        ok = ptx::mbar_wait(accf, i & 1, abort_flag);
+        ptx::tc_fence_after();
+      }
+      if (!ok) break;
+      const int row = m0 + q * 32 + lane;
+      const int er = (row < args.M) ? args.eA[row] : 0;
+      const bool empty_k = kb1 <= kb0;
+      for (int c = 0; c < kBN / kChunk; ++c) {
+        double v[kChunk];
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) v[j] = 0.0;
+        if (!empty_k) {
+          uint32_t r[kSlices][16];
+#pragma unroll
+          for (int d = 0; d < kSlices; ++d)
+            tmem_ld16_nowait(tmem + lane_off + static_cast<uint32_t>(d * kBN + c * kChunk), r[d]);
+          ptx::tmem_wait_ld();
+          // smallest diagonal first: sum_d acc_d 2^(-7 (d + 2)), then 2^e_row
+#pragma unroll
+          for (int d = kSlices - 1; d >= 0; --d) {
+            const double sc = ldexp(1.0, -7 * (d + 2));
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j) v[j] = fma(static_cast<double>(static_cast<int>(r[d][j])), sc, v[j]);
+          }
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) v[j] = er == kNonFiniteRow ? __longlong_as_double(0x7FF8000000000000LL)
+                                                                       : ldexp(v[j], er);
+        }
+        if (c == kBN / kChunk - 1) {  // every accumulator column of this tile has been read
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(acce);
+        }
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) st[lane * kStLd + j] = v[j];
+        __syncwarp();
+        // the warp's 32 rows x 16 columns: 4 rows per instruction, 8 lanes x 2 columns per row
+        const int cl = 2 * (lane & 7);
+        const int col = n0 + c * kChunk + cl;
+        const int ec0 = (col < args.N) ? args.eB[col] : 0;
+        const int ec1 = (col + 1 < args.N) ? args.eB[col + 1] : 0;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int rl = 4 * it + (lane >> 3);
+          const int m = m0 + q * 32 + rl;
+          if (m >= args.M) continue;
+          double* crow = args.C + static_cast<int64_t>(m) * args.ldc;
+          const double nan = __longlong_as_double(0x7FF8000000000000LL);
+          const double p0 = ec0 == kNonFiniteRow ? nan : args.alpha * ldexp(st[rl * kStLd + cl], ec0);
+          const double p1 = ec1 == kNonFiniteRow ? nan : args.alpha * ldexp(st[rl * kStLd + cl + 1], ec1);
+          const bool w0 = col < args.N && (!args.lower || m >= col);
+          const bool w1 = col + 1 < args.N && (!args.lower || m >= col + 1);
+          if (w0) crow[col] = args.beta == 0.0 ? p0 : fma(args.beta, crow[col], p0);
+          if (w1) crow[col + 1] = args.beta == 0.0 ? p1 : fma(args.beta, crow[col + 1], p1);
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok) fail();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// 3-D tensor map over kSlices planes [rows][Kpad] int8 with a [box_rows][32] box spanning all
+// planes (32-byte swizzle).
+bool make_slice_map(CUtensorMap* map, const int8_t* planes, int64_t rows, int64_t Kpad, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kpad), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(kSlices)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kpad), static_cast<cuuint64_t>(rows * Kpad)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box_rows, static_cast<cuuint32_t>(kSlices)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(planes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+hq_status slice(const double* X, int64_t ldx, int64_t rows, int64_t Kred, int64_t Kpad, int tri, int which,
+                int8_t* planes, int* exps, const int* skip, cudaStream_t s) {
+  const int64_t grid = ceil_div(rows, 8);
+  i8x_slice_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, ldx, rows, Kred, Kpad, tri, which, planes, exps,
+                                                              skip);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
+}
+
+}  // namespace
+
+int64_t i8x_kpad(int64_t Kred) { return (Kred + kBK - 1) / kBK * kBK; }
+
+size_t i8x_scratch_bytes(int64_t M, int64_t N, int64_t Kred) {
+  const size_t kp = static_cast<size_t>(i8x_kpad(Kred));
+  const size_t a = round_up(static_cast<size_t>(kSlices) * M * kp, 256);
+  const size_t b = round_up(static_cast<size_t>(kSlices) * N * kp, 256);
+  return a + b + round_up(static_cast<size_t>(M) * 4, 256) + round_up(static_cast<size_t>(N) * 4, 256);
+}
+
+bool i8x_eligible(const F64Gemm& g) {
+  return g.Kred >= 1 && g.Kred <= kI8xMaxKred && g.M >= 1 && g.N >= 1 && (!g.lower || g.M == g.N);
+}
+
+hq_status i8x_gemm(const F64Gemm& g, uint8_t* scratch, size_t scratch_bytes, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0) return HQ_OK;
+  if (!i8x_eligible(g)) return HQ_ERR_UNSUPPORTED;
+  if (scratch == nullptr || !aligned(scratch, 256) || scratch_bytes < i8x_scratch_bytes(g.M, g.N, g.Kred))
+    return HQ_ERR_WORKSPACE;
+  const int64_t kp = i8x_kpad(g.Kred);
+  int8_t* pa = reinterpret_cast<int8_t*>(scratch);
+  const bool same = g.A == g.B && g.lda == g.ldb && g.M == g.N && g.tri == kTriNone;
+  int8_t* pb = same ? pa : pa + round_up(static_cast<size_t>(kSlices) * g.M * kp, 256);
+  int* ea = reinterpret_cast<int*>(pa + round_up(static_cast<size_t>(kSlices) * g.M * kp, 256) +
+                                   round_up(static_cast<size_t>(kSlices) * g.N * kp, 256));
+  int* eb = same ? ea : ea + round_up(static_cast<size_t>(g.M) * 4, 256) / 4;
+  const int ts = timer_start(kTimeI8xSlice, s);
+  hq_status st = slice(g.A, g.lda, g.M, g.Kred, kp, g.tri, 0, pa, ea, g.skip, s);
+  if (st != HQ_OK) return st;
+  if (!same) {
+    st = slice(g.B, g.ldb, g.N, g.Kred, kp, g.tri, 1, pb, eb, g.skip, s);
+    if (st != HQ_OK) return st;
+  }
+  // bytes: each operand's rows read once in fp64, kSlices planes written
+  timer_stop(ts, (same ? 1.0 : 2.0) * 0.5 * (g.M + g.N) * (8.0 * g.Kred + kSlices * static_cast<double>(kp)), s);
+  CUtensorMap mA, mB;
+  if (!make_slice_map(&mA, pa, g.M, kp, kBM) || !make_slice_map(&mB, pb, g.N, kp, kBN)) return HQ_ERR_CUDA;
+  I8xArgs a{};
+  a.C = g.C;
+  a.ldc = g.ldc;
+  a.M = g.M;
+  a.N = g.N;
+  a.Kpad = static_cast<int>(kp);
+  a.tiles_m = static_cast<int>(ceil_div(g.M, kBM));
+  a.tiles_n = static_cast<int>(ceil_div(g.N, kBN));
+  int64_t tiles = 0;
+  if (g.lower) {
+    for (int tmi = 0; tmi < a.tiles_m; ++tmi) tiles += (2 * tmi + 2 < a.tiles_n) ? 2 * tmi + 2 : a.tiles_n;
+  } else {
+    tiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+  }
+  if (tiles > 0x7FFFFFFF) return HQ_ERR_UNSUPPORTED;
+  a.tiles = static_cast<int>(tiles);
+  a.alpha = g.alpha;
+  a.beta = g.beta;
+  a.lower = g.lower;
+  a.tri = g.tri;
+  a.eA = ea;
+  a.eB = eb;
+  a.skip = g.skip;
+  a.status = g.status;
+  HQ_CUDA_TRY(cudaFuncSetAttribute(i8x_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+  const int grid = static_cast<int>(tiles < kSMs ? tiles : kSMs);
+  const int tm = timer_start(kTimeI8xGemm, s);
+  i8x_gemm_kernel<<<grid, kThreads, kSmem, s>>>(mA, mB, a);
+  HQ_LAUNCH_CHECK();
+  // work: 2 flops per multiply-add a declared triangular operand leaves non-zero (the fp64
+  // product's own count, as for the fp64 kernel)
+  double flops = 2.0 * g.M * g.N * static_cast<double>(g.Kred);
+  if (g.tri != kTriNone || g.lower) flops *= 0.5;
+  timer_stop(tm, flops, s);
+  return HQ_OK;
+}
+
+}  // namespace hq

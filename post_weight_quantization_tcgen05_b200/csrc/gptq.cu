@@ -372,7 +372,8 @@ __global__ void __launch_bounds__(256) qerr_finalize_kernel(const double* __rest
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    const double q = rd[0] > 0.0 ? sqrt(rn[0] / rd[0]) : 0.0;
+    // an all-zero layer has qerr 0; non-finite sums (a NaN or infinite weight) stay non-finite
+    const double q = rd[0] == 0.0 ? 0.0 : sqrt(rn[0] / rd[0]);
     hdr->num = rn[0];
     hdr->den = rd[0];
     hdr->qerr = q;
@@ -429,6 +430,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
   L.t = off;
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
+  L.slices = off;  // int8 slices of the factorisation's large products (two streams)
+  off = round_up(off + 2 * factor_slice_bytes(K), al);
   L.total = off;
   return L;
 }
@@ -458,8 +461,8 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   float* Ut_hi = nullptr;
   float* Ut_lo = nullptr;
   const bool split = (update_impl == 0);  // 3xTF32 updates take pre-split operands
-  hq_status st = launch_factor(H, K, damp, A, X, XT, T, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, true, split,
-                               &Ut_hi, &Ut_lo, s);
+  hq_status st = launch_factor(H, K, damp, A, X, XT, T, ws + L.slices, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U,
+                               true, split, &Ut_hi, &Ut_lo, s);
   if (st != HQ_OK) return st;
 
   {

@@ -79,6 +79,8 @@ enum TimerClass {
   kTimeSweep = 3,       // sweep_block_kernel (bytes)
   kTimeTf32Gemm = 4,    // tf32_gemm_kernel (flops of the product, not of its 3 passes)
   kTimeSyrk = 5,        // tcgen05 SYRK (flops)
+  kTimeI8xGemm = 6,     // i8x_gemm_kernel (flops of the fp64 product it emulates)
+  kTimeI8xSlice = 7,    // i8x_slice_kernel (bytes: fp64 operand read, int8 slices written)
 };
 int timer_start(int cls, cudaStream_t s);
 void timer_stop(int idx, double work, cudaStream_t s);
@@ -99,8 +101,20 @@ struct F64Gemm {
   double* scratch;  // room for split-K partial tiles (may be NULL: no split)
   int64_t scratch_elems;
   const int* skip;
+  int* status;      // device status word for bounded-wait timeouts (may be NULL)
 };
 hq_status f64_gemm(const F64Gemm& g, cudaStream_t s);
+
+// gemm_i8x.cu: the same product, fp64-accurate, on the int8 tensor cores (tcgen05 kind::i8) from
+// kI8xSlices int8 slices per operand row.  `scratch` (256-byte aligned) holds the slices and the
+// row exponents: i8x_scratch_bytes(M, N, Kred) bytes.  Kred <= kI8xMaxKred keeps the int32 sums
+// exact.
+constexpr int kI8xSlices = 7;
+constexpr int64_t kI8xMaxKred = 16384;
+int64_t i8x_kpad(int64_t Kred);
+size_t i8x_scratch_bytes(int64_t M, int64_t N, int64_t Kred);
+bool i8x_eligible(const F64Gemm& g);
+hq_status i8x_gemm(const F64Gemm& g, uint8_t* scratch, size_t scratch_bytes, cudaStream_t s);
 
 // factor.cu: out[i] = 1 / d[i] by the leaf's Newton-Raphson reciprocal (for tests)
 hq_status launch_rcp_nr(const double* d, double* out, int64_t n, cudaStream_t s);
@@ -126,13 +140,16 @@ __host__ __device__ __forceinline__ int sweep_upack_offset(int j, int l, int m) 
 // With split_ut, also the strict lower triangle of *Ut split into a tf32 part and the fp32
 // remainder (Ut = Ut_hi + Ut_lo there), in T's storage; the upper parts of Ut_hi and Ut_lo are
 // not written.
+// `slices` (NULL: every product on the fp64 tensor cores) holds 2 * factor_slice_bytes(K) bytes,
+// 256-byte aligned: the int8 slices of the large products' operands, one half per stream.
+size_t factor_slice_bytes(int64_t K);
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form, bool split_ut,
-                        float** Ut_hi, float** Ut_lo, cudaStream_t s);
+                        uint8_t* slices, double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form,
+                        bool split_ut, float** Ut_hi, float** Ut_lo, cudaStream_t s);
 
 // gptq.cu
 struct GptqLayout {
-  size_t header, partials, wf, err, err_lo, a, x, xt, t, total;
+  size_t header, partials, wf, err, err_lo, a, x, xt, t, slices, total;
   int sweep_rows, sweep_grid;  // rows per sweep CTA, sweep CTAs
 };
 // Device-side header at the start of the GPTQ / RTN workspace.
