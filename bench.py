@@ -189,9 +189,13 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     for w in range(args.warmup):
-        if w == args.warmup - 1:  # creates the timing events of the dominant kernel before the timed region
-            hq.hq_debug_timing_start([DOMINANT])
         layer.step()
+    torch.cuda.synchronize()
+    # the kernel class with the largest share of a step, from one step with every launch timed
+    # (outside the timed region); its launches are then timed live inside the timed region
+    dominant = dominant_class(kernel_breakdown(hq, layer, flush, steps=1))
+    hq.hq_debug_timing_start([dominant])  # creates its events before the timed region
+    layer.step()
     torch.cuda.synchronize()
 
     # ---- timed region: K steps, each bracketed by events, L2 flushed between steps; the library
@@ -201,14 +205,14 @@ def run_ours(args, rank, world, local_rank):
     launches0 = hq.hq_debug_launch_count()
     _barrier(world)
     torch.cuda.synchronize()
-    hq.hq_debug_timing_start([DOMINANT])
+    hq.hq_debug_timing_start([dominant])
     with ClockSampler(local_rank) as clk:
         for k in range(args.steps):
             flush.fill_(k & 0xFF)
             layer.step(stage_events=evs[k])
         torch.cuda.synchronize()
     hq.hq_debug_timing_stop()
-    dom = hq.hq_debug_timing_read(DOMINANT)
+    dom = (dominant,) + tuple(hq.hq_debug_timing_read(dominant))
     _barrier(world)
     launches = (hq.hq_debug_launch_count() - launches0) // max(args.steps, 1)
     step_ms = [e[0].elapsed_time(e[4]) for e in evs]
@@ -320,11 +324,13 @@ def time_layer(hq, cfg, dev, flush, steps: int = 2, warmup: int = 1, peaks=None)
            "steps": steps, "ms_per_step": step_ms, "weights_per_s": cfg.N * cfg.K / (step_ms / 1e3),
            "gptq_quantize_ms": gptq_ms, "gptq_weights_per_s": cfg.N * cfg.K / (gptq_ms / 1e3),
            "syrk_ms": syrk_ms, "xtx_tflops": cfg.T * cfg.K * (cfg.K + 1) / (syrk_ms / 1e3) / 1e12}
-    if peaks is not None:  # kernel-level rooflines of the two tensor-core stages (one more step)
+    if peaks is not None:  # kernel-level rooflines (one more step, every launch timed)
         kernels = kernel_breakdown(hq, layer, flush, steps=1)
         out["syrk_roofline"] = syrk_line(kernels, out["xtx_tflops"], peaks)
         out["update_roofline"] = update_line(cfg, kernels, peaks)
         out["kernels_ms"] = {k: v["ms_per_step"] for k, v in kernels.items()}
+        out["rooflines"] = {k: class_roofline(k, v["ms_total"], v["work_total"], v["launches_total"], 1, peaks, cfg)
+                            for k, v in kernels.items()}
     del layer
     torch.cuda.empty_cache()
     return out
@@ -410,20 +416,89 @@ def other_configs(hq, dev, flush, peaks):
     return out
 
 
-# The kernel with the largest share of a step (ncu launch list of this benchmark) and the others
-# reported in the breakdown, with the unit of their algorithmic work.
-DOMINANT = "f64_gemm_128"
+# Kernel classes the library times (hq_debug_timing_*), with the unit of their algorithmic work.
 KERNEL_NAMES = {"f64_gemm_128": ("f64_gemm_kernel<128>", "TFLOP/s"),
                 "f64_gemm_64": ("f64_gemm_kernel<64> + split-K reduce", "TFLOP/s"),
+                "i8x_gemm": ("i8x_gemm_kernel (fp64 products from int8 slices on tcgen05 kind::i8)", "TFLOP/s"),
+                "i8x_slice": ("i8x_slice_kernel (fp64 operands cut into int8 slices)", "GB/s"),
                 "leaf": ("chol_inv_leaf_kernel", "TFLOP/s"),
                 "sweep": ("sweep_block_kernel", "GB/s"),
                 "tf32_gemm": ("upd_gemm_kernel<BN> (3xTF32 lazy updates)", "TFLOP/s"),
                 "syrk": ("syrk_tc_kernel (persistent tcgen05 SYRK)", "TFLOP/s")}
-# fp64 tensor-core peak: no measured figure exists for fp64, so the measured bf16 burst is scaled
-# by NVIDIA's nominal dense ratio for B200 (fp64 tensor 37 TFLOP/s : bf16 2250 TFLOP/s)
+# int8 slice-pair products per fp64 product in the int8-sliced GEMM (7 slices, anti-diagonals 0-6)
+I8X_PAIRS = 28
+# fp64 tensor-core peak when no fp64 rate was measured: the measured bf16 burst scaled by NVIDIA's
+# nominal dense ratio for B200 (fp64 tensor 37 TFLOP/s : bf16 2250 TFLOP/s)
 FP64_OVER_BF16 = 37.0 / 2250.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "f64_gemm_kernel_128_q_proj.md")
-KERNEL_SOURCE = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "csrc", "gemm_f64.cu")
+# committed ncu summaries (DRAM traffic per launch) and the source each was taken from
+PROFILES = {"f64_gemm_128": ("f64_gemm_kernel_128_q_proj.md", "gemm_f64.cu"),
+            "f64_gemm_64": ("f64_gemm_kernel_64_q_proj.md", "gemm_f64.cu"),
+            "i8x_gemm": ("i8x_gemm_kernel_down_proj.md", "gemm_i8x.cu"),
+            "leaf": ("chol_inv_leaf_kernel_q_proj.md", "factor.cu"),
+            "sweep": ("sweep_block_kernel_q_proj.md", "gptq.cu"),
+            "tf32_gemm": ("upd_gemm_kernel_q_proj.md", "gemm_upd.cu"),
+            "syrk": ("syrk_tc_kernel_q_proj.md", "syrk.cu")}
+
+
+def dominant_class(kernels) -> str:
+    """The timed kernel class with the most device time per step."""
+    return max(kernels, key=lambda c: kernels[c]["ms_per_step"]) if kernels else "f64_gemm_64"
+
+
+def class_roofline(cls: str, ms: float, work: float, launches: int, steps: int, peaks, cfg) -> dict:
+    """Roofline of one kernel class from its summed launch time `ms` and algorithmic `work`
+    (the library's per-launch figure) over `steps` steps: the bound, achieved rate, peak and
+    fraction, in the unit of the bound."""
+    s = ms / 1e3
+    out = {"kernel": KERNEL_NAMES[cls][0], "class": cls, "launches_per_step": launches / max(steps, 1),
+           "ms_per_step": ms / max(steps, 1)}
+    fp64 = peaks.get("fp64_tflops") or peaks["bf16_tflops"] * FP64_OVER_BF16
+    if cls in ("f64_gemm_128", "f64_gemm_64", "leaf"):
+        out.update(bound="tensor", unit="TFLOP/s", achieved=work / s / 1e12 if s > 0 else None, peak=fp64,
+                   peak_source="fp64 dense rate measured in this run: the larger of the fp64 torch.matmul (cuBLAS) "
+                               "rate and the library's fp64 MMA rate")
+    elif cls == "i8x_gemm":
+        out.update(bound="tensor", unit="TOP/s", achieved=I8X_PAIRS * work / s / 1e12 if s > 0 else None,
+                   peak=peaks.get("int8_tops"), fp64_equivalent_tflops=work / s / 1e12 if s > 0 else None,
+                   peak_source="int8 dense rate measured in this run (torch._int_mm); work = 28 exact int8 "
+                               "slice-pair products per fp64 multiply-add pair (2 ops each)")
+    elif cls in ("sweep", "i8x_slice"):
+        out.update(bound="hbm", unit="GB/s", achieved=work / s / 1e9 if s > 0 else None, peak=peaks["hbm_gbs"],
+                   peak_source=peaks["source"] + " HBM copy")
+    elif cls == "syrk":
+        out.update(bound="tensor", unit="TFLOP/s", achieved=work / s / 1e12 if s > 0 else None,
+                   peak=peaks["bf16_tflops"], peak_source=peaks["source"] + " bf16 dense burst")
+    elif cls == "tf32_gemm":
+        roof = update_roofline_ms(cfg, peaks) * max(steps, 1)
+        out.update(bound="tensor / hbm per launch", unit="ms", achieved=roof, peak=ms,
+                   peak_source="per-launch roofline time (tf32 measured in this run, HBM copy) against the measured "
+                               "time: frac = roofline / measured")
+    a, p = out.get("achieved"), out.get("peak")
+    out["frac"] = (a / p) if (a is not None and p) else None
+    return out
+
+
+def profiled_traffic(cls: str):
+    """DRAM bytes per launch of kernel class `cls` from its committed ncu summary, or None when
+    there is none or the kernel's source has changed since that capture."""
+    import hashlib
+    if cls not in PROFILES:
+        return None
+    summary = os.path.join(ROOT, "profiles", PROFILES[cls][0])
+    source = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "csrc", PROFILES[cls][1])
+    if not os.path.exists(summary):
+        return None
+    with open(source, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    vals = {}
+    with open(summary) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha256")):
+                k, v = line.strip().split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != sha or "traffic_bytes_per_launch" not in vals:
+        return None
+    return float(vals["traffic_bytes_per_launch"])
 
 
 def update_roofline_ms(cfg, peaks, tf32_tflops=None) -> float:
@@ -469,7 +544,8 @@ def kernel_breakdown(hq, layer, flush, steps: int = 2):
             continue
         scale = 1e12 if unit == "TFLOP/s" else 1e9
         out[cls] = {"kernel": name, "ms_per_step": ms / steps, "launches_per_step": n / steps,
-                    "achieved": work / (ms / 1e3) / scale, "unit": unit}
+                    "achieved": work / (ms / 1e3) / scale, "unit": unit, "ms_total": ms, "work_total": work,
+                    "launches_total": n}
     return out
 
 
@@ -610,25 +686,6 @@ def measure_dense_peaks(hq, dev, n: int = 8192):
     return out
 
 
-def profiled_traffic():
-    """dram bytes per launch of the dominant kernel from the committed ncu summary, or None when
-    the kernel's source has changed since that capture."""
-    import hashlib
-    if not os.path.exists(PROFILE_SUMMARY):
-        return None
-    with open(KERNEL_SOURCE, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    vals = {}
-    with open(PROFILE_SUMMARY) as f:
-        for line in f:
-            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha256")):
-                k, v = line.strip().split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_sha256") != sha or "traffic_bytes_per_launch" not in vals:
-        return None
-    return float(vals["traffic_bytes_per_launch"])
-
-
 def measure_e2e(args, layer, flush, world):
     cfg = layer.cfg
     weights = cfg.N * cfg.K
@@ -730,17 +787,12 @@ def update_line(cfg, kernels, peaks):
 
 def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops, enc_bytes,
                dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense):
-    dom_ms, dom_flop, dom_n = dom
-    achieved = dom_flop / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
-    peak = peaks.get("fp64_tflops") or peaks["bf16_tflops"] * FP64_OVER_BF16
-    roofline = {"kernel": KERNEL_NAMES[DOMINANT][0] + " (fp64 MMA, factorisation products)", "bound": "tensor",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak if achieved is not None else None, "traffic": profiled_traffic(),
-                "launches_per_step": dom_n / max(args.steps, 1), "ms_per_step": dom_ms / max(args.steps, 1),
-                "peak_source": ("fp64 dense rate measured in this run: the larger of the fp64 torch.matmul "
-                                "(cuBLAS) rate and the library's fp64 MMA rate" if peaks.get("fp64_tflops") else
-                                f"{peaks['source']} bf16 dense burst x nominal fp64-tensor/bf16 ratio 37/2250"),
-                "dense_peaks_measured": dense}
+    cls, dom_ms, dom_work, dom_n = dom
+    roofline = class_roofline(cls, dom_ms, dom_work, dom_n, args.steps, peaks, cfg)
+    roofline["traffic"] = profiled_traffic(cls)
+    roofline["timing"] = ("every launch of the class timed by CUDA events on its own stream inside the timed "
+                          "region; the class with the largest share of a step, from a breakdown taken before it")
+    roofline["dense_peaks_measured"] = dense
     line = {
         "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
         "value": value,
@@ -763,6 +815,9 @@ def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, d
                       "decode": dec_bytes / (statistics.mean(dec_ms) / 1e3) / 1e9},
         "roofline": roofline,
         "kernels": kernels,
+        "rooflines": ({k: class_roofline(k, v["ms_total"], v["work_total"], v["launches_total"],
+                                         round(v["launches_total"] / v["launches_per_step"]) if v["launches_per_step"]
+                                         else 1, peaks, cfg) for k, v in kernels.items()} if kernels else None),
         "syrk_roofline": syrk_line(kernels, syrk_tflops, peaks),
         "update_roofline": update_line(cfg, kernels, peaks),
         "e2e": e2e,

@@ -121,6 +121,43 @@ hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, con
                            size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * hq_gptq_quantize in two stages, for a layer whose rows are quantised on several devices
+ * against one factorisation: given U, the sweep's feedback stays inside each row ([gptq]
+ * experiment summary: the error-feedback sweep runs row by row over the columns), so one device
+ * factorises, the factor buffer is broadcast (it is plain bytes), and every device sweeps its own
+ * rows.  hq_gptq_factorize + hq_gptq_sweep give the same codes, scales and qerr as
+ * hq_gptq_quantize on the same rows.
+ *
+ * hq_gptq_factor_bytes(K): size of the factor buffer: a small header (factorisation status and
+ *   lambda), the 128 x 128 diagonal blocks of U' = diag(U)^-1 U in the sweep's packed order, and
+ *   the strict lower triangle of U'^T split into a tf32 part and its fp32 remainder (about
+ *   8 K^2 bytes).  0 for an unsupported K (K a multiple of 128, at most 65536).
+ * hq_gptq_factor_workspace_bytes(K): scratch of hq_gptq_factorize (the fp64 factorisation).
+ * hq_gptq_sweep_workspace_bytes(N, K, group): scratch of hq_gptq_sweep (no fp64 matrices).
+ *
+ * hq_gptq_factorize: lambda = damp * mean(diag H), U'^T of (H + lambda I)^-1 into `factor`
+ *   (device, 256-byte aligned, at least hq_gptq_factor_bytes(K) bytes; HQ_ERR_INVALID otherwise).
+ *   H, damp, K as for hq_gptq_quantize.  Synchronises `stream` and returns HQ_ERR_NOT_PD or
+ *   HQ_ERR_INVALID like hq_gptq_quantize; the factor's header then records the failure, so a
+ *   buffer broadcast after a failed factorisation makes every hq_gptq_sweep on it return the
+ *   same status.
+ * hq_gptq_sweep: the sweep of W [N, K] against a factor buffer (device, 256-byte aligned, read
+ *   only, made by hq_gptq_factorize for the same K); W, group, imp, codes, scales, qerr_out,
+ *   qerr_dev as for hq_gptq_quantize; workspace at least hq_gptq_sweep_workspace_bytes(N, K,
+ *   group).  Synchronises `stream` once at the end; HQ_ERR_NOT_PD / HQ_ERR_INVALID when the
+ *   factor records a failed factorisation.  hq_qerr_terms reads this workspace too.
+ */
+size_t hq_gptq_factor_bytes(int64_t K);
+size_t hq_gptq_factor_workspace_bytes(int64_t K);
+size_t hq_gptq_sweep_workspace_bytes(int64_t N, int64_t K, int64_t group);
+hq_status hq_gptq_factorize(const float* H, int64_t K, float damp, void* factor, size_t factor_bytes,
+                            void* workspace, size_t workspace_bytes, hq_stream_t stream);
+hq_status hq_gptq_sweep(const void* W, int w_dtype, int64_t N, int64_t K, const void* factor,
+                        int64_t group, const float* imp, uint8_t* codes, float* scales,
+                        double* qerr_out, double* qerr_dev, void* workspace, size_t workspace_bytes,
+                        hq_stream_t stream);
+
+/*
  * The two fp64 sums behind the qerr of the last hq_gptq_quantize or hq_rtn_quantize that ran
  * with this workspace ([gptq] qerr definition): terms_dev[0] = sum imp[k] (W[n,k] - q[n,k])^2,
  * terms_dev[1] = sum imp[k] W[n,k]^2, so that qerr = sqrt(terms[0] / terms[1]).  For callers that
@@ -133,6 +170,14 @@ hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, con
  * finished call's results).
  */
 hq_status hq_qerr_terms(const void* workspace, double* terms_dev, hq_stream_t stream);
+
+/*
+ * qerr from its two sums ([gptq] qerr definition): *qerr_dev = sqrt(terms_dev[0] / terms_dev[1]),
+ * 0 when terms_dev[1] == 0 (an all-zero layer); non-finite sums give a non-finite qerr.  For
+ * callers that added the sums of a layer's row shards (e.g. by an all-reduce).  Device pointers;
+ * asynchronous.
+ */
+hq_status hq_qerr_from_terms(const double* terms_dev, double* qerr_dev, hq_stream_t stream);
 
 /* Bytes of workspace hq_rtn_quantize needs (0 if the shape is invalid). */
 size_t hq_rtn_workspace_bytes(int64_t N, int64_t K, int64_t group);
@@ -220,6 +265,21 @@ hq_status hq_hadamard_rotate_weights(const void* W, int w_dtype, int64_t N, int6
                                      const float* signs, float* W_out, hq_stream_t stream);
 hq_status hq_hadamard_rotate_hessian(const float* H, int64_t K, int64_t block, const float* signs, float* H_out,
                                      hq_stream_t stream);
+
+/*
+ * The lower triangle of an fp32 Hessian packed row by row without gaps, element (i, j), j <= i,
+ * at i (i + 1) / 2 + j: hq_tril32_count(K) = K (K + 1) / 2 values.  The exchange format of a
+ * Hessian accumulated over token chunks on several devices ([calib] "Hessian storage": H is a
+ * sum over chunks; [imat]: partial statistics merge by addition): the packed partial sums are
+ * added (an all-reduce) and unpacked, moving about half the bytes of the full matrix.  Exact
+ * copies.
+ * hq_hessian_pack_lower: H fp32 [K, K] (lower triangle incl. diagonal read) -> packed.
+ * hq_hessian_unpack_lower: packed -> H's lower triangle incl. diagonal (the strict upper
+ *   triangle is not written).  Device pointers, K >= 1, asynchronous.
+ */
+size_t hq_tril32_count(int64_t K);
+hq_status hq_hessian_pack_lower(const float* H, int64_t K, float* packed, hq_stream_t stream);
+hq_status hq_hessian_unpack_lower(const float* packed, int64_t K, float* H, hq_stream_t stream);
 
 /* Bf16TrilDiagF32 payload size: K*4 + K*(K-1)/2*2 bytes ([calib] "Hessian storage"). */
 size_t hq_bf16tril_bytes(int64_t K);

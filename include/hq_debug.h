@@ -17,7 +17,8 @@ extern "C" {
  * The damping + factorisation stage of hq_gptq_quantize alone: writes U^T (fp32 [K, K],
  * row-major; U^T[c, j] = U[j, c] for c >= j, zero above the diagonal) where U is the upper
  * Cholesky factor of (H + damp * mean(diag H) I)^-1 ([gptq] experiment summary, "Cholesky-
- * based Hessian inverse").  Uses hq_gptq_workspace_bytes(1, K, 128) bytes of workspace.
+ * based Hessian inverse").  Uses hq_gptq_factor_workspace_bytes(K) bytes of workspace (which
+ * hq_gptq_workspace_bytes(N, K, group) always exceeds).
  * Synchronises `stream` and returns HQ_ERR_NOT_PD / HQ_ERR_INVALID like hq_gptq_quantize.
  */
 hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, void* workspace,
@@ -26,7 +27,7 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
 /*
  * hq_gptq_quantize with an explicit choice of the lazy-update kernel:
  * update_impl 0 = tcgen05 tensor cores in 3xTF32 (the default path), 1 = fp32 CUDA cores
- * (reference for the tensor-core one), 2 = tcgen05 tensor cores in plain tf32.
+ * (reference for the tensor-core one).
  */
 hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
                                       int64_t group, float damp, const float* imp, uint8_t* codes,
@@ -57,17 +58,6 @@ hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype,
  */
 hq_status hq_debug_hessian_accumulate_timeout(float* H, const void* X, int64_t T, int64_t K, int* dev_status,
                                               int64_t wait_limit_cycles, int withhold_stage, hq_stream_t stream);
-
-/*
- * The tensor-core fp32 GEMM used by the GPTQ lazy updates:
- *   C[m, n] = beta * C[m, n] + alpha * sum_k A[m * lda + k] * B[n * ldb + k]
- * for m < M, n < N (if `lower`, only elements with m >= n are written).  split3 = 1 selects
- * 3xTF32 (about fp32 accuracy), 0 plain tf32.  A and B 16-byte aligned, lda and ldb
- * multiples of 4.  No counterpart on the pages: a building block of the path.
- */
-hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
-                             const float* B, int64_t ldb, float alpha, float beta, int lower, int split3,
-                             hq_stream_t stream);
 
 /*
  * The GPTQ lazy-update product (persistent tcgen05 kernel, 3xTF32 from pre-split operands):

@@ -58,6 +58,15 @@ _SIGS = {
     "hq_rtn_quantize": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hq_rtn_quantize_noalloc": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "hq_qerr_terms": (_int, [_vp, _vp, _vp]),
+    "hq_qerr_from_terms": (_int, [_vp, _vp, _vp]),
+    "hq_gptq_factor_bytes": (_sz, [_i64]),
+    "hq_gptq_factor_workspace_bytes": (_sz, [_i64]),
+    "hq_gptq_sweep_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "hq_gptq_factorize": (_int, [_vp, _i64, _f, _vp, _sz, _vp, _sz, _vp]),
+    "hq_gptq_sweep": (_int, [_vp, _int, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hq_tril32_count": (_sz, [_i64]),
+    "hq_hessian_pack_lower": (_int, [_vp, _i64, _vp, _vp]),
+    "hq_hessian_unpack_lower": (_int, [_vp, _i64, _vp, _vp]),
     "hq_hadamard_rotate_weights": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp]),
     "hq_hadamard_rotate_hessian": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "hq_psd_workspace_bytes": (_sz, [_i64]),
@@ -71,7 +80,6 @@ _SIGS = {
     "hq_debug_hessian_accumulate_impl": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _int, _vp]),
     "hq_debug_hessian_accumulate_timeout": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _int, _vp]),
     "hq_debug_launch_count": (ctypes.c_uint64, []),
-    "hq_debug_tf32_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _f, _f, _int, _int, _vp]),
     "hq_debug_rcp_f64": (_int, [_vp, _vp, _i64, _vp]),
     "hq_debug_upd_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _i64, _vp, _vp, _i64, _vp]),
     "hq_debug_fp64_mma_rate": (ctypes.c_double, [_vp, _i64, _vp]),
@@ -185,6 +193,63 @@ def hq_gptq_quantize(W, H, group: int, damp: float, codes, scales, workspace, im
     return q.value if want_qerr else None
 
 
+def hq_gptq_factor_bytes(K: int) -> int:
+    return int(lib.hq_gptq_factor_bytes(K))
+
+
+def hq_gptq_factor_workspace_bytes(K: int) -> int:
+    return int(lib.hq_gptq_factor_workspace_bytes(K))
+
+
+def hq_gptq_sweep_workspace_bytes(N: int, K: int, group: int) -> int:
+    return int(lib.hq_gptq_sweep_workspace_bytes(N, K, group))
+
+
+def hq_gptq_factorize(H, damp: float, factor, workspace, stream=None) -> None:
+    """Damping and factorisation of the undamped fp32 H [K, K] into the factor buffer (uint8)."""
+    K = H.shape[0]
+    st = lib.hq_gptq_factorize(_ptr(H), K, float(damp), _ptr(factor), factor.numel() * factor.element_size(),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hq_gptq_factorize")
+
+
+def hq_gptq_sweep(W, factor, group: int, codes, scales, workspace, imp=None, want_qerr: bool = True, qerr_dev=None,
+                  stream=None):
+    """The GPTQ sweep of W [N, K] against a factor buffer; returns qerr (host) if requested."""
+    N, K = W.shape
+    q = ctypes.c_double(float("nan"))
+    st = lib.hq_gptq_sweep(_ptr(W), _dtype(W), N, K, _ptr(factor), int(group), _ptr(imp), _ptr(codes), _ptr(scales),
+                           ctypes.byref(q) if want_qerr else None, _ptr(qerr_dev), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hq_gptq_sweep")
+    return q.value if want_qerr else None
+
+
+def hq_qerr_from_terms(terms_dev, qerr_dev, stream=None) -> None:
+    _check(lib.hq_qerr_from_terms(_ptr(terms_dev), _ptr(qerr_dev), _stream(stream)), "hq_qerr_from_terms")
+
+
+def hq_tril32_count(K: int) -> int:
+    return int(lib.hq_tril32_count(K))
+
+
+def _need_f32(*ts) -> None:
+    for t in ts:
+        if t.dtype != torch.float32:
+            raise ValueError("expected an fp32 tensor")
+
+
+def hq_hessian_pack_lower(H, packed, stream=None) -> None:
+    _need_f32(H, packed)
+    K = H.shape[0]
+    _check(lib.hq_hessian_pack_lower(_ptr(H), K, _ptr(packed), _stream(stream)), "hq_hessian_pack_lower")
+
+
+def hq_hessian_unpack_lower(packed, K: int, H, stream=None) -> None:
+    _need_f32(H, packed)
+    _check(lib.hq_hessian_unpack_lower(_ptr(packed), K, _ptr(H), _stream(stream)), "hq_hessian_unpack_lower")
+
+
 def hq_debug_gptq_quantize_impl(W, H, group: int, damp: float, codes, scales, workspace, update_impl: int, imp=None,
                                 want_qerr: bool = True, qerr_dev=None, stream=None):
     N, K = W.shape
@@ -257,15 +322,6 @@ def hq_debug_factor(H, damp: float, Ut_out, workspace, stream=None) -> None:
     K = H.shape[0]
     _check(lib.hq_debug_factor(_ptr(H), K, float(damp), _ptr(Ut_out), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)), "hq_debug_factor")
-
-
-def hq_debug_tf32_gemm(C, A, B, alpha=1.0, beta=0.0, lower=False, split3=True, stream=None) -> None:
-    """C = beta C + alpha A B^T (fp32 row-major views, tensor cores)."""
-    M, Kred = A.shape
-    N = B.shape[0]
-    _check(lib.hq_debug_tf32_gemm(_ptr(C), C.stride(0), M, N, Kred, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
-                                  float(alpha), float(beta), int(bool(lower)), int(bool(split3)), _stream(stream)),
-           "hq_debug_tf32_gemm")
 
 
 def hq_debug_fp64_mma_rate(stream=None) -> float:

@@ -59,6 +59,12 @@ hq_status gptq_common(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   return finish_sync(s, reinterpret_cast<const WsHeader*>(ws + L.header), qerr_out);
 }
 
+// qerr = sqrt(num / den) from the two sums, 0 for an all-zero layer (the qerr finaliser's rule).
+__global__ void qerr_from_terms_kernel(const double* __restrict__ terms, double* __restrict__ q) {
+  const double num = terms[0], den = terms[1];
+  *q = den == 0.0 ? 0.0 : sqrt(num / den);
+}
+
 // Both the GPTQ and the RTN workspace start with the status header (layout offset 0).
 __global__ void qerr_terms_kernel(const WsHeader* __restrict__ hdr, double* __restrict__ out) {
   out[0] = hdr->num;
@@ -138,11 +144,68 @@ hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, con
                      workspace_bytes, 0, static_cast<cudaStream_t>(stream));
 }
 
+size_t hq_gptq_factor_bytes(int64_t K) {
+  if (!gptq_shape_ok(1, K, 128)) return 0;
+  return factor_layout(K).total;
+}
+
+size_t hq_gptq_factor_workspace_bytes(int64_t K) {
+  if (!gptq_shape_ok(1, K, 128)) return 0;
+  return factor_ws_layout(K).total;
+}
+
+size_t hq_gptq_sweep_workspace_bytes(int64_t N, int64_t K, int64_t group) {
+  if (!gptq_shape_ok(N, K, group)) return 0;
+  return gptq_layout(N, K, group).sweep_total;
+}
+
+hq_status hq_gptq_factorize(const float* H, int64_t K, float damp, void* factor, size_t factor_bytes, void* workspace,
+                            size_t workspace_bytes, hq_stream_t stream) {
+  if (H == nullptr || factor == nullptr) return HQ_ERR_INVALID;
+  if (!(damp > 0.f) || !isfinite(damp)) return HQ_ERR_INVALID;
+  if (!gptq_shape_ok(1, K, 128)) return HQ_ERR_UNSUPPORTED;
+  if (!aligned(factor, 256) || factor_bytes < factor_layout(K).total) return HQ_ERR_INVALID;
+  const GptqLayout L = factor_ws_layout(K);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.total) return HQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
+  hq_status st = launch_factorize(H, K, damp, ws, L, static_cast<uint8_t*>(factor), false, s);
+  if (st != HQ_OK) return st;
+  return finish_sync(s, hdr, nullptr);
+}
+
+hq_status hq_gptq_sweep(const void* W, int w_dtype, int64_t N, int64_t K, const void* factor, int64_t group,
+                        const float* imp, uint8_t* codes, float* scales, double* qerr_out, double* qerr_dev,
+                        void* workspace, size_t workspace_bytes, hq_stream_t stream) {
+  if (W == nullptr || factor == nullptr || codes == nullptr || scales == nullptr || !valid_dtype(w_dtype))
+    return HQ_ERR_INVALID;
+  if (N < 1 || K < 1 || group < 1 || K % group != 0) return HQ_ERR_INVALID;
+  if (!gptq_shape_ok(N, K, group)) return HQ_ERR_UNSUPPORTED;
+  if (!aligned(factor, 256)) return HQ_ERR_INVALID;
+  const GptqLayout L = gptq_layout(N, K, group);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.sweep_total) return HQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  hq_status st = launch_sweep(W, w_dtype, N, K, group, imp, codes, scales, qerr_dev, ws,
+                              static_cast<const uint8_t*>(factor), 0, true, s);
+  if (st != HQ_OK) return st;
+  return finish_sync(s, reinterpret_cast<const WsHeader*>(ws + L.header), qerr_out);
+}
+
+hq_status hq_qerr_from_terms(const double* terms_dev, double* qerr_dev, hq_stream_t stream) {
+  if (terms_dev == nullptr || qerr_dev == nullptr) return HQ_ERR_INVALID;
+  qerr_from_terms_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(terms_dev, qerr_dev);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
+}
+
 hq_status hq_debug_gptq_quantize_impl(const void* W, int w_dtype, int64_t N, int64_t K, const float* H,
                                       int64_t group, float damp, const float* imp, uint8_t* codes, float* scales,
                                       double* qerr_out, double* qerr_dev, void* workspace, size_t workspace_bytes,
                                       int update_impl, hq_stream_t stream) {
-  if (update_impl < 0 || update_impl > 2) return HQ_ERR_INVALID;
+  if (update_impl < 0 || update_impl > 1) return HQ_ERR_INVALID;
   return gptq_common(W, w_dtype, N, K, H, group, damp, imp, codes, scales, qerr_out, qerr_dev, workspace,
                      workspace_bytes, update_impl, static_cast<cudaStream_t>(stream));
 }
@@ -152,19 +215,16 @@ hq_status hq_debug_factor(const float* H, int64_t K, float damp, float* Ut_out, 
   if (H == nullptr || Ut_out == nullptr) return HQ_ERR_INVALID;
   if (!(damp > 0.f) || !isfinite(damp)) return HQ_ERR_INVALID;
   if (!gptq_shape_ok(1, K, 128)) return HQ_ERR_UNSUPPORTED;
-  const GptqLayout L = gptq_layout(1, K, 128);
+  const GptqLayout L = factor_ws_layout(K);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.total) return HQ_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
-  float* Ut = nullptr;
-  float* U = nullptr;
   hq_status st = launch_factor(H, K, damp, reinterpret_cast<double*>(ws + L.a), reinterpret_cast<double*>(ws + L.x),
                                reinterpret_cast<double*>(ws + L.xt), reinterpret_cast<double*>(ws + L.t), ws + L.slices,
-                               &hdr->lam, &hdr->info, &hdr->status, &Ut, &U, false, false, nullptr, nullptr, s);
+                               &hdr->lam, &hdr->info, &hdr->status, false, Ut_out, nullptr, nullptr, nullptr, s);
   if (st != HQ_OK) return st;
-  HQ_CUDA_TRY(cudaMemcpyAsync(Ut_out, Ut, static_cast<size_t>(K) * K * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return finish_sync(s, hdr, nullptr);
 }
 
@@ -228,28 +288,6 @@ hq_status hq_debug_i8x_gemm(double* C, int64_t ldc, int M, int N, int Kred, cons
   g.lower = lower ? 1 : 0;
   g.tri = tri;
   return i8x_gemm(g, static_cast<uint8_t*>(scratch), scratch_bytes, static_cast<cudaStream_t>(stream));
-}
-
-hq_status hq_debug_tf32_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A, int64_t lda,
-                             const float* B, int64_t ldb, float alpha, float beta, int lower, int split3,
-                             hq_stream_t stream) {
-  if (C == nullptr || A == nullptr || B == nullptr || M < 0 || N < 0 || Kred < 1) return HQ_ERR_INVALID;
-  if (ldc < N || lda < Kred || ldb < Kred) return HQ_ERR_INVALID;
-  Tf32Gemm g{};
-  g.C = C;
-  g.ldc = ldc;
-  g.M = M;
-  g.N = N;
-  g.Kred = Kred;
-  g.A = A;
-  g.lda = lda;
-  g.B = B;
-  g.ldb = ldb;
-  g.alpha = alpha;
-  g.beta = beta;
-  g.lower = lower ? 1 : 0;
-  g.split3 = split3 != 0;
-  return tf32_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
 hq_status hq_debug_upd_gemm(float* C, int64_t ldc, int M, int N, int Kred, const float* A_hi, const float* A_lo,

@@ -620,8 +620,8 @@ __global__ void sweep_pack_kernel(const double* __restrict__ X, int64_t K, float
 // ------------------------------------------------------------------------- driver
 
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        uint8_t* slices, double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form,
-                        bool split_ut, float** Ut_hi, float** Ut_lo, cudaStream_t s) {
+                        uint8_t* slices, double* lam, int* info, int* status, bool sweep_form, float* Ut, float* U,
+                        float* Ut_hi, float* Ut_lo, cudaStream_t s) {
   if (K % kLeaf != 0 || K % kSweepBlk != 0) return HQ_ERR_UNSUPPORTED;
   HQ_CUDA_TRY(cudaFuncSetAttribute(chol_inv_leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(kLeafSmem)));
@@ -632,7 +632,8 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
     reverse_damp_kernel<<<static_cast<unsigned>(nb * (nb + 1) / 2), 256, 0, s>>>(H, K, lam, A, info);
     HQ_LAUNCH_CHECK();
   }
-  if (sweep_form && split_ut) {
+  const bool split_only = sweep_form && Ut == nullptr;
+  if (split_only) {
     // the products' triangular tiles and the leaves read zeros only inside the diagonal leaf
     // blocks, and nothing downstream reads X or X^T outside their triangles
     zero_diag_blocks_kernel<<<static_cast<unsigned>(K / kLeaf), 256, 0, s>>>(X, XT, K);
@@ -657,23 +658,14 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   const hq_status st_join = stream_dep(side, side->s2, s);
   if (st != HQ_OK) return st;
   if (st_join != HQ_OK) return st_join;
-  // A is dead now: the fp32 results go into its storage
-  *Ut = reinterpret_cast<float*>(A);
-  *U = reinterpret_cast<float*>(A) + K * K;
+  // A and the temporaries are dead now: the outputs may overlay them
   const int64_t grid = ceil_div(K * K, 4 * 256) < 148 * 32 ? ceil_div(K * K, 4 * 256) : 148 * 32;
-  // the temporaries are dead too: the split U^T goes into their storage
-  float* hi = split_ut ? reinterpret_cast<float*>(T) : nullptr;
-  float* lo = split_ut ? reinterpret_cast<float*>(T) + K * K : nullptr;
-  if (Ut_hi != nullptr) *Ut_hi = hi;
-  if (Ut_lo != nullptr) *Ut_lo = lo;
-  // the 3xTF32 updates of the sweep read only the split strict lower part of U'^T
-  float* ut_plain = (sweep_form && split_ut) ? nullptr : *Ut;
-  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, sweep_form ? nullptr : *U, ut_plain, hi, lo,
+  rotate_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, XT, K, sweep_form ? nullptr : U, Ut, Ut_hi, Ut_lo,
                                                             sweep_form, info);
   HQ_LAUNCH_CHECK();
-  if (sweep_form) {
+  if (sweep_form && U != nullptr) {
     const int64_t pg = ceil_div(K * kSweepBlk, 256) < 148 * 16 ? ceil_div(K * kSweepBlk, 256) : 148 * 16;
-    sweep_pack_kernel<<<static_cast<unsigned>(pg), 256, 0, s>>>(X, K, *U, info);
+    sweep_pack_kernel<<<static_cast<unsigned>(pg), 256, 0, s>>>(X, K, U, info);
     HQ_LAUNCH_CHECK();
   }
   return HQ_OK;

@@ -354,7 +354,8 @@ __global__ void w_prep_kernel(const void* __restrict__ W, int dt, int64_t n, flo
 }
 
 __global__ void __launch_bounds__(256) qerr_finalize_kernel(const double* __restrict__ partials, int64_t count,
-                                                            WsHeader* hdr, double* qerr_dev) {
+                                                            WsHeader* hdr, double* qerr_dev,
+                                                            const int* __restrict__ finfo) {
   __shared__ double rn[256], rd[256];
   double n = 0.0, d = 0.0;
   for (int64_t i = threadIdx.x; i < count; i += blockDim.x) {
@@ -377,13 +378,14 @@ __global__ void __launch_bounds__(256) qerr_finalize_kernel(const double* __rest
     hdr->num = rn[0];
     hdr->den = rd[0];
     hdr->qerr = q;
+    if (finfo != nullptr) hdr->info = *finfo;  // the factorisation's status, for the host
     if (qerr_dev != nullptr) *qerr_dev = q;
   }
 }
 
 hq_status launch_qerr_finalize(const double* partials, int64_t count, WsHeader* hdr, double* qerr_dev,
-                               cudaStream_t s) {
-  qerr_finalize_kernel<<<1, 256, 0, s>>>(partials, count, hdr, qerr_dev);
+                               cudaStream_t s, const int* finfo) {
+  qerr_finalize_kernel<<<1, 256, 0, s>>>(partials, count, hdr, qerr_dev, finfo);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
 }
@@ -405,6 +407,41 @@ static int64_t panel_width(int64_t K, int64_t group) {
   return P < K ? P : K;
 }
 
+FactorLayout factor_layout(int64_t K) {
+  FactorLayout F{};
+  const size_t al = 256;
+  size_t off = 0;
+  F.hdr = off;
+  off = round_up(off + sizeof(FactorHeader), al);
+  F.upack = off;  // packed diagonal blocks of U'
+  off = round_up(off + static_cast<size_t>(K) * kBlk * sizeof(float), al);
+  F.hi = off;     // U'^T strict lower triangle: tf32 part (or, for the CUDA-core updates, U'^T itself)
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  F.lo = off;     // its fp32 remainder
+  off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
+  F.total = off;
+  return F;
+}
+
+// The factorisation's scratch from offset `off` on: the recursion's temporaries T and the matrix A
+// side by side (a factor buffer produced in place overlays both once they are dead), X = L^-1,
+// X^T, and the int8 slices of the large products.
+static void factor_scratch_layout(int64_t K, size_t off, GptqLayout& L) {
+  const size_t al = 256;
+  const size_t kk = static_cast<size_t>(K) * K * sizeof(double);
+  L.t = off;
+  off = round_up(off + kk, al);
+  L.a = off;
+  off = round_up(off + kk, al);
+  L.x = off;
+  off = round_up(off + kk, al);
+  L.xt = off;
+  off = round_up(off + kk, al);
+  L.slices = off;
+  off = round_up(off + 2 * factor_slice_bytes(K), al);
+  L.total = off;
+}
+
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   GptqLayout L{};
   const size_t al = 256;
@@ -422,48 +459,62 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group) {
   off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
   L.err_lo = off;  // remainder part of the errors for the 3xTF32 updates
   off = round_up(off + static_cast<size_t>(N) * P * sizeof(float), al);
-  L.a = off;  // fp64 A, later U'^T and the packed diagonal blocks of U' in fp32
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
-  L.x = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
-  L.xt = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
-  L.t = off;
-  off = round_up(off + static_cast<size_t>(K) * K * sizeof(double), al);
-  L.slices = off;  // int8 slices of the factorisation's large products (two streams)
-  off = round_up(off + 2 * factor_slice_bytes(K), al);
-  L.total = off;
+  L.sweep_total = off;
+  factor_scratch_layout(K, off, L);
   return L;
+}
+
+GptqLayout factor_ws_layout(int64_t K) {
+  GptqLayout L{};
+  L.header = 0;
+  factor_scratch_layout(K, round_up(sizeof(WsHeader), 256), L);
+  return L;
+}
+
+__global__ void factor_header_kernel(const WsHeader* __restrict__ hdr, FactorHeader* __restrict__ fh) {
+  fh->info = hdr->info;
+  fh->lam = hdr->lam;
+}
+
+hq_status launch_factorize(const float* H, int64_t K, float damp, uint8_t* ws, const GptqLayout& L, uint8_t* factor,
+                           bool plain_ut, cudaStream_t s) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  const FactorLayout F = factor_layout(K);
+  float* hi = reinterpret_cast<float*>(factor + F.hi);
+  float* lo = reinterpret_cast<float*>(factor + F.lo);
+  hq_status st = launch_factor(H, K, damp, reinterpret_cast<double*>(ws + L.a), reinterpret_cast<double*>(ws + L.x),
+                               reinterpret_cast<double*>(ws + L.xt), reinterpret_cast<double*>(ws + L.t),
+                               ws + L.slices, &hdr->lam, &hdr->info, &hdr->status, true, plain_ut ? hi : nullptr,
+                               reinterpret_cast<float*>(factor + F.upack), plain_ut ? nullptr : hi,
+                               plain_ut ? nullptr : lo, s);
+  if (st != HQ_OK) return st;
+  factor_header_kernel<<<1, 1, 0, s>>>(hdr, reinterpret_cast<FactorHeader*>(factor + F.hdr));
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
 }
 
 // W[:, c0 : c0+ncols] -= D[:, 0:kred] * U'[k0 : k0+kred, c0 : c0+ncols]   (residuals D, row stride lde)
 static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
-                              const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut,
-                              const float* Ut_hi, const float* Ut_lo, const int* info, int* status, cudaStream_t s);
+                              const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut_hi,
+                              const float* Ut_lo, const int* info, int* status, cudaStream_t s);
 
-hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
-                      const float* imp, uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws,
-                      int update_impl, cudaStream_t s) {
+hq_status launch_sweep(const void* W, int w_dtype, int64_t N, int64_t K, int64_t group, const float* imp,
+                       uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws, const uint8_t* factor,
+                       int update_impl, bool reset_header, cudaStream_t s) {
   const GptqLayout L = gptq_layout(N, K, group);
+  const FactorLayout F = factor_layout(K);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   double* partials = reinterpret_cast<double*>(ws + L.partials);
   float* Wf = reinterpret_cast<float*>(ws + L.wf);
   float* Err = reinterpret_cast<float*>(ws + L.err);
   float* Err_lo = reinterpret_cast<float*>(ws + L.err_lo);
-  double* A = reinterpret_cast<double*>(ws + L.a);
-  double* X = reinterpret_cast<double*>(ws + L.x);
-  double* XT = reinterpret_cast<double*>(ws + L.xt);
-  double* T = reinterpret_cast<double*>(ws + L.t);
-  HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
-
-  float* Ut = nullptr;
-  float* U = nullptr;
-  float* Ut_hi = nullptr;
-  float* Ut_lo = nullptr;
+  const FactorHeader* fh = reinterpret_cast<const FactorHeader*>(factor + F.hdr);
+  const float* Upack = reinterpret_cast<const float*>(factor + F.upack);
+  const float* Ut_hi = reinterpret_cast<const float*>(factor + F.hi);
+  const float* Ut_lo = reinterpret_cast<const float*>(factor + F.lo);
+  const int* info = &fh->info;
+  if (reset_header) HQ_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s));
   const bool split = (update_impl == 0);  // 3xTF32 updates take pre-split operands
-  hq_status st = launch_factor(H, K, damp, A, X, XT, T, ws + L.slices, &hdr->lam, &hdr->info, &hdr->status, &Ut, &U,
-                               true, split, &Ut_hi, &Ut_lo, s);
-  if (st != HQ_OK) return st;
 
   {
     const int64_t n = N * K;
@@ -477,7 +528,7 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   a.Wf = Wf;
   a.N = N;
   a.K = K;
-  a.Upack = U;
+  a.Upack = Upack;
   a.group = static_cast<int>(group);
   a.Err = Err;
   a.Err_lo = split ? Err_lo : nullptr;
@@ -488,7 +539,7 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   a.w_dtype = w_dtype;
   a.imp = imp;
   a.partials = partials;
-  a.info = &hdr->info;
+  a.info = info;
 
   void (*kern)(SweepArgs, int) = nullptr;
   switch (group) {
@@ -501,6 +552,7 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
   const int threads = L.sweep_rows / kRowsPerWarp * 32;
   HQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
 
+  hq_status st = HQ_OK;
   for (int64_t p0 = 0; p0 < K; p0 += P) {
     const int64_t p1 = (p0 + P < K) ? p0 + P : K;
     for (int64_t j0 = p0; j0 < p1; j0 += kBlk) {
@@ -514,18 +566,31 @@ hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const fl
                          N * (static_cast<double>(kBlk) / group) * 4.0, s);
       const int64_t j1 = j0 + kBlk;
       if (j1 < p1) {  // inner update of the rest of the panel
-        st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), Err_lo + (j0 - p0), P, j0, kBlk, Ut,
-                          Ut_hi, Ut_lo, &hdr->info, &hdr->status, s);
+        st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), Err_lo + (j0 - p0), P, j0, kBlk,
+                          Ut_hi, Ut_lo, info, &hdr->status, s);
         if (st != HQ_OK) return st;
       }
     }
     if (p1 < K) {  // outer update of everything right of the panel
-      st = sweep_update(update_impl, Wf, N, K, p1, K - p1, Err, Err_lo, P, p0, p1 - p0, Ut, Ut_hi, Ut_lo, &hdr->info,
+      st = sweep_update(update_impl, Wf, N, K, p1, K - p1, Err, Err_lo, P, p0, p1 - p0, Ut_hi, Ut_lo, info,
                         &hdr->status, s);
       if (st != HQ_OK) return st;
     }
   }
-  return launch_qerr_finalize(partials, static_cast<int64_t>(K / kBlk) * L.sweep_grid, hdr, qerr_dev, s);
+  return launch_qerr_finalize(partials, static_cast<int64_t>(K / kBlk) * L.sweep_grid, hdr, qerr_dev, s, info);
+}
+
+hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
+                      const float* imp, uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws,
+                      int update_impl, cudaStream_t s) {
+  const GptqLayout L = gptq_layout(N, K, group);
+  HQ_CUDA_TRY(cudaMemsetAsync(ws + L.header, 0, sizeof(WsHeader), s));
+  // the factor buffer overlays the recursion's temporaries and A, both dead once it is written
+  uint8_t* factor = ws + L.t;
+  static_assert(sizeof(FactorHeader) <= 256, "factor header");
+  hq_status st = launch_factorize(H, K, damp, ws, L, factor, update_impl != 0, s);
+  if (st != HQ_OK) return st;
+  return launch_sweep(W, w_dtype, N, K, group, imp, codes, scales, qerr_dev, ws, factor, update_impl, false, s);
 }
 
 // CUDA-core fp32 version of the lazy update (cross-check of the tensor-core kernel).
@@ -570,9 +635,8 @@ __global__ void __launch_bounds__(256) update_simt_kernel(float* __restrict__ C,
 }
 
 static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t c0, int64_t ncols, const float* E,
-                              const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut,
-                              const float* Ut_hi, const float* Ut_lo, const int* info, int* status, cudaStream_t s) {
-  const float* B = Ut + c0 * K + k0;  // B(n, k) = U^T[c0 + n][k0 + k] = U[k0 + k][c0 + n]
+                              const float* E_lo, int64_t lde, int64_t k0, int64_t kred, const float* Ut_hi,
+                              const float* Ut_lo, const int* info, int* status, cudaStream_t s) {
   if (impl == 0) {  // 3xTF32 from the pre-split operands (E, E_lo from the sweep; U^T split once)
     UpdGemm g{};
     g.C = Wf + c0;
@@ -590,28 +654,13 @@ static hq_status sweep_update(int impl, float* Wf, int64_t N, int64_t K, int64_t
     g.status = status;
     return upd_gemm(g, s);
   }
-  if (impl == 1) {
-    const int64_t ctas = ceil_div(N, 64) * ceil_div(ncols, 64);
-    update_simt_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(Wf + c0, K, N, ncols, E, lde, B, K, kred, info);
-    HQ_LAUNCH_CHECK();
-    return HQ_OK;
-  }
-  Tf32Gemm g{};
-  g.C = Wf + c0;
-  g.ldc = K;
-  g.M = static_cast<int>(N);
-  g.N = static_cast<int>(ncols);
-  g.Kred = static_cast<int>(kred);
-  g.A = E;
-  g.lda = lde;
-  g.B = B;
-  g.ldb = K;
-  g.alpha = -1.f;
-  g.beta = 1.f;
-  g.split3 = (impl == 0);
-  g.skip = info;
-  g.status = status;
-  return tf32_gemm(g, s);
+  // fp32 CUDA cores, with U'^T itself in the place of its tf32 part:
+  // B(n, k) = U'^T[c0 + n][k0 + k] = U'[k0 + k][c0 + n]
+  const int64_t ctas = ceil_div(N, 64) * ceil_div(ncols, 64);
+  update_simt_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(Wf + c0, K, N, ncols, E, lde, Ut_hi + c0 * K + k0,
+                                                                  K, kred, info);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
 }
 
 }  // namespace hq

@@ -17,26 +17,13 @@ hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev
                          long long wait_limit = kWaitLimitCycles, int withhold_stage = -1);
 hq_status launch_syrk_simt(float* H, const void* X, int x_dtype, int64_t T, int64_t K, cudaStream_t s);
 
+// tril32.cu: the lower triangle of H packed row by row (pack: H -> packed; else packed -> H's
+// lower triangle)
+hq_status launch_tril32(const float* src, float* dst, int64_t K, bool pack, cudaStream_t s);
+
 // codec.cu
 hq_status launch_tril_encode(const float* H, int64_t K, uint8_t* out, cudaStream_t s);
 hq_status launch_tril_decode(const uint8_t* in, int64_t K, float* H, cudaStream_t s);
-
-// gemm_tf32.cu: C = beta C + alpha A B^T on the tensor cores (kind::tf32)
-struct Tf32Gemm {
-  float* C;
-  int64_t ldc;
-  int M, N, Kred;
-  const float* A;  // A(m, k) = A[m * lda + k]
-  int64_t lda;
-  const float* B;  // B(n, k) = B[n * ldb + k]
-  int64_t ldb;
-  float alpha, beta;
-  int lower, row0, col0;  // write only row0 + m >= col0 + n when lower
-  bool split3;            // 3xTF32 (about fp32 accuracy) instead of 1xTF32
-  const int* skip;
-  int* status;
-};
-hq_status tf32_gemm(const Tf32Gemm& g, cudaStream_t s);
 
 // gemm_upd.cu: C -= (A_hi + A_lo) (B_hi + B_lo)^T in 3xTF32 on tcgen05 (the GPTQ lazy updates),
 // operands pre-split into tf32 and remainder parts, K-major, 16-byte aligned rows.
@@ -77,7 +64,7 @@ enum TimerClass {
   kTimeF64Gemm64 = 1,   // f64_gemm_kernel, 64-wide tiles, with its split-K reduction (flops)
   kTimeLeaf = 2,        // chol_inv_leaf_kernel (flops of Cholesky + triangular inverse)
   kTimeSweep = 3,       // sweep_block_kernel (bytes)
-  kTimeTf32Gemm = 4,    // tf32_gemm_kernel (flops of the product, not of its 3 passes)
+  kTimeTf32Gemm = 4,    // upd_gemm_kernel (flops of the product, not of its 3 tf32 passes)
   kTimeSyrk = 5,        // tcgen05 SYRK (flops)
   kTimeI8xGemm = 6,     // i8x_gemm_kernel (flops of the fp64 product it emulates)
   kTimeI8xSlice = 7,    // i8x_slice_kernel (bytes: fp64 operand read, int8 slices written)
@@ -131,25 +118,39 @@ __host__ __device__ __forceinline__ int sweep_upack_offset(int j, int l, int m) 
 }
 
 // factor.cu: the upper Cholesky factor U of the inverse of the damped Hessian, in fp32, from an
-// fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; the fp32 results are written into
-// A's storage once A is no longer needed: *Ut (first half) and *U (second half).
-//   sweep_form == false: *Ut = U^T (row-major, lower), *U = U (row-major, upper).
-//   sweep_form == true:  *Ut = U'^T with U' = diag(U)^-1 U (row-major, lower, unit diagonal),
-//                        *U = the packed diagonal blocks of U' (K / kSweepBlk blocks, see
-//                        sweep_upack_offset; K must be a multiple of kSweepBlk).
-// With split_ut, also the strict lower triangle of *Ut split into a tf32 part and the fp32
-// remainder (Ut = Ut_hi + Ut_lo there), in T's storage; the upper parts of Ut_hi and Ut_lo are
-// not written.
-// `slices` (NULL: every product on the fp64 tensor cores) holds 2 * factor_slice_bytes(K) bytes,
-// 256-byte aligned: the int8 slices of the large products' operands, one half per stream.
+// fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; `slices` (NULL: every product on the
+// fp64 tensor cores) holds 2 * factor_slice_bytes(K) bytes, 256-byte aligned: the int8 slices of
+// the large products' operands, one half per stream.  Outputs (each may be NULL; they must not
+// overlap X or XT; they may overlap A and T, which are dead by then):
+//   sweep_form == false: U (row-major, upper) and Ut = U^T (row-major, lower).
+//   sweep_form == true:  U receives the packed diagonal blocks of U' = diag(U)^-1 U (K / kSweepBlk
+//                        blocks, see sweep_upack_offset; K a multiple of kSweepBlk) and Ut = U'^T
+//                        (row-major, lower, unit diagonal).
+//   Ut_hi, Ut_lo: the strict lower triangle of the same Ut split into a tf32 part and the fp32
+//                 remainder (their upper parts are not written).
+// With Ut == NULL and sweep_form, only the strict lower triangle of Ut is ever formed.
 size_t factor_slice_bytes(int64_t K);
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
-                        uint8_t* slices, double* lam, int* info, int* status, float** Ut, float** U, bool sweep_form,
-                        bool split_ut, float** Ut_hi, float** Ut_lo, cudaStream_t s);
+                        uint8_t* slices, double* lam, int* info, int* status, bool sweep_form, float* Ut, float* U,
+                        float* Ut_hi, float* Ut_lo, cudaStream_t s);
+
+// The factor buffer: everything the GPTQ sweep needs from the factorisation, in one block that
+// ranks sharing a layer's rows can broadcast.  Header, packed diagonal blocks of U', and the
+// strict lower triangle of U'^T split into its tf32 part (hi) and fp32 remainder (lo); for the
+// CUDA-core updates hi holds U'^T itself.
+struct FactorHeader {
+  int info;  // factorisation status: 0 ok, k > 0 first failing pivot, -1 mean(diag) <= 0
+  int pad;
+  double lam;
+};
+struct FactorLayout {
+  size_t hdr, upack, hi, lo, total;
+};
+FactorLayout factor_layout(int64_t K);
 
 // gptq.cu
 struct GptqLayout {
-  size_t header, partials, wf, err, err_lo, a, x, xt, t, slices, total;
+  size_t header, partials, wf, err, err_lo, sweep_total, t, a, x, xt, slices, total;
   int sweep_rows, sweep_grid;  // rows per sweep CTA, sweep CTAs
 };
 // Device-side header at the start of the GPTQ / RTN workspace.
@@ -162,6 +163,18 @@ struct WsHeader {
 };
 bool gptq_shape_ok(int64_t N, int64_t K, int64_t group);
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t group);
+// The workspace of the factorisation alone: the header at 0, then its scratch (t .. slices).
+GptqLayout factor_ws_layout(int64_t K);
+// Damping and factorisation into `factor` (factor_layout(K).total bytes); `ws` laid out as L.
+// plain_ut: U'^T unsplit in the hi slot (the CUDA-core updates) instead of the split.
+hq_status launch_factorize(const float* H, int64_t K, float damp, uint8_t* ws, const GptqLayout& L, uint8_t* factor,
+                           bool plain_ut, cudaStream_t s);
+// The sweep of W's N rows against a factor buffer, in a workspace whose first L.sweep_total bytes
+// follow gptq_layout(N, K, group).  update_impl 0: 3xTF32 tensor cores, 1: fp32 CUDA cores (the
+// factor then holds U'^T unsplit).
+hq_status launch_sweep(const void* W, int w_dtype, int64_t N, int64_t K, int64_t group, const float* imp,
+                       uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws, const uint8_t* factor,
+                       int update_impl, bool reset_header, cudaStream_t s);
 hq_status launch_gptq(const void* W, int w_dtype, int64_t N, int64_t K, const float* H, int64_t group, float damp,
                       const float* imp, uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws,
                       int update_impl, cudaStream_t s);
@@ -172,7 +185,8 @@ hq_status launch_rtn(const void* W, int w_dtype, int64_t N, int64_t K, int64_t g
                      uint8_t* codes, float* scales, double* qerr_dev, uint8_t* ws, cudaStream_t s);
 
 // gptq.cu: qerr reduction shared by GPTQ and RTN
+// (finfo: optional device int copied into hdr->info, the factorisation's status)
 hq_status launch_qerr_finalize(const double* partials, int64_t count, WsHeader* hdr, double* qerr_dev,
-                               cudaStream_t s);
+                               cudaStream_t s, const int* finfo = nullptr);
 
 }  // namespace hq

@@ -78,12 +78,15 @@ def test_bench_line_carries_the_contract_keys():
     cfg = wl.CONFIGS[1]
     args = types.SimpleNamespace(steps=10, warmup=3)
     peaks = dict(bench._peaks(), tf32_tflops=800.0, fp64_tflops=37.0)
-    kernels = {"syrk": {"achieved": 1000.0, "ms_per_step": 0.2, "launches_per_step": 1.0},
-               "tf32_gemm": {"achieved": 120.0, "ms_per_step": 1.1, "launches_per_step": 39.0}}
+    kernels = {"syrk": {"achieved": 1000.0, "ms_per_step": 0.2, "launches_per_step": 1.0, "ms_total": 0.4,
+                        "work_total": 4.3e11, "launches_total": 2},
+               "tf32_gemm": {"achieved": 120.0, "ms_per_step": 1.1, "launches_per_step": 39.0, "ms_total": 2.2,
+                             "work_total": 2.6e11, "launches_total": 78}}
     e2e = {"value": 2.0e9, "unit": "weights/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
     clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
     line = bench.build_line(args, cfg, 1, 2.8e9, 9.3, [0.2], [9.0], [0.03], [0.03], 900.0, 7.9e7, 1.3e8,
-                            peaks, e2e, 394, clocks, (33.0, 6.7e11, 40), kernels, {"fp64_tflops": 37.0})
+                            peaks, e2e, 394, clocks, ("f64_gemm_64", 33.0, 6.7e11, 40), kernels,
+                            {"fp64_tflops": 37.0})
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
         assert key in line, key
@@ -94,6 +97,10 @@ def test_bench_line_carries_the_contract_keys():
         assert key in roof, key
     assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
     assert roof["peak"] == 37.0  # the fp64 rate measured in the run, not a nominal ratio
+    assert roof["achieved"] == pytest.approx(6.7e11 / 0.033 / 1e12)
+    i8 = bench.class_roofline("i8x_gemm", 10.0, 1e12, 4, 10, dict(peaks, int8_tops=3000.0), cfg)
+    assert i8["unit"] == "TOP/s" and i8["achieved"] == pytest.approx(28 * 1e12 / 0.01 / 1e12)
+    assert i8["frac"] == pytest.approx(i8["achieved"] / 3000.0)
     assert line["update_roofline"]["tf32_tflops"] == 800.0
     assert roof["traffic"] is None or roof["traffic"] > 0
     assert line["gpu_launches"] == 3940
