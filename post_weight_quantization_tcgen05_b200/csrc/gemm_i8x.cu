@@ -8,8 +8,9 @@
 // Slicing (i8x_slice_kernel, one warp per row).  Row r of an operand is scaled by 2^-e_r, e_r the
 // smallest exponent with max_k |x[r, k]| < 2^e_r, and cut into kSlices signed 7-bit integers:
 //   y_0 = x 2^-e_r;  d_s = trunc(128 y_s) in [-127, 127];  y_{s+1} = 128 y_s - d_s,
-// so x = 2^e_r sum_s d_s 2^(-7 (s + 1)) + 2^(e_r - 7 S) y_S with |y_S| < 1.  Every step is exact in
-// fp64 (a power-of-two scaling, a truncation, the subtraction of a value's own integer part).
+// so x = 2^e_r sum_s d_s 2^(-7 (s + 1)) + 2^(e_r - 7 S) y_S with |y_S| < 1: the base-128 digits of
+// |x| 2^-e_r, signed like x.  The kernel reads them off the fp64 bit pattern with integer shifts
+// (slice_digits), which gives the same digits as the fp64 steps above.
 // Slice s of all rows is a plane [rows][Kpad] of int8 (K-major), zero outside the part of the
 // row the product reads (a declared triangular operand) and past Kred.
 //
@@ -72,7 +73,33 @@ __host__ __device__ inline void tri_row_range(int tri, int which, int64_t r, int
 
 // ------------------------------------------------------------------------- slicing
 
-// One warp per row: e_r, then kSlices int8 planes of the row (16 columns per lane per round).
+// Slices of one fp64 value x with |x| < 2^e (e the row exponent), from its bit pattern: with
+// x = m 2^(q - 52) (m the 53-bit significand, q the unbiased exponent), the integer
+// X = trunc(|x| 2^(7 kSlices - e)) = m >> (52 - 7 kSlices + e - q) has at most 7 kSlices bits, and
+// its base-128 digits, most significant first and signed like x, are the slices.  Exactly the
+// digits of the sequential construction: truncating toward zero keeps every remainder's sign.
+// Packs digit s of x into byte b of w[s].
+__device__ __forceinline__ void slice_digits(double x, int e, int b, uint32_t (&w)[kSlices]) {
+  const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(x));
+  const int be = static_cast<int>((bits >> 52) & 0x7FF);
+  const unsigned long long m = (bits & 0xFFFFFFFFFFFFFull) | (be != 0 ? (1ull << 52) : 0ull);
+  const int q = (be != 0 ? be : 1) - 1023;
+  // q < e for normal x, so sh > 0; a subnormal x has fewer significant bits than q says and
+  // can need a left shift (X stays below 2^(7 kSlices) since |x| < 2^e)
+  const int sh = 52 - 7 * kSlices + e - q;
+  const unsigned long long X = sh >= 64 ? 0ull : (sh >= 0 ? (m >> sh) : (m << (-sh)));
+  const bool neg = (bits >> 63) != 0;
+#pragma unroll
+  for (int s = 0; s < kSlices; ++s) {
+    int d = static_cast<int>((X >> (7 * (kSlices - 1 - s))) & 127ull);
+    d = neg ? -d : d;
+    w[s] |= (static_cast<uint32_t>(d) & 0xFFu) << (8 * b);
+  }
+}
+
+// One warp per row: the row maximum over the part the product reads, e_r, then the kSlices int8
+// planes of the row, 128 columns per warp round (each lane 4 consecutive values: two 16-byte
+// loads, one 4-byte store per plane).
 __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict__ X, int64_t ldx, int64_t rows,
                                                         int64_t Kred, int64_t Kpad, int tri, int which,
                                                         int8_t* __restrict__ planes, int* __restrict__ exps,
@@ -84,6 +111,8 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
   int64_t klo, khi;
   tri_row_range(tri, which, r, Kred, klo, khi);
   const double* xr = X + r * ldx;
+  // 16-byte loads need an even row start and ldx; otherwise scalar loads
+  const bool vec = ((reinterpret_cast<uintptr_t>(xr) & 15) == 0);
   double mx = 0.0;
   bool bad = false;
   for (int64_t k = klo + lane; k < khi; k += 32) {
@@ -97,31 +126,30 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
   // a row holding a NaN or an infinity is marked, and its products come out NaN
   const int e = bad ? kNonFiniteRow : (mx > 0.0 ? ilogb(mx) + 1 : 0);
   if (lane == 0) exps[r] = e;
-  const double sc = bad ? 0.0 : ldexp(1.0, -e);
   const int64_t plane = rows * Kpad;
   int8_t* out = planes + r * Kpad;
-  for (int64_t k0 = 16 * lane; k0 < Kpad; k0 += 16 * 32) {
-    uint32_t w[kSlices][4];
+  for (int64_t k0 = 4 * lane; k0 < Kpad; k0 += 4 * 32) {
+    double v[4];
+    if (vec && k0 >= klo && k0 + 4 <= khi) {
+      const double2 a = *reinterpret_cast<const double2*>(xr + k0);
+      const double2 b = *reinterpret_cast<const double2*>(xr + k0 + 2);
+      v[0] = a.x;
+      v[1] = a.y;
+      v[2] = b.x;
+      v[3] = b.y;
+    } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+      for (int b = 0; b < 4; ++b) v[b] = (k0 + b >= klo && k0 + b < khi) ? xr[k0 + b] : 0.0;
+    }
+    uint32_t w[kSlices];
 #pragma unroll
-      for (int s = 0; s < kSlices; ++s) w[s][q] = 0u;
+    for (int s2 = 0; s2 < kSlices; ++s2) w[s2] = 0u;
+    if (!bad) {
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int64_t k = k0 + 4 * q + b;
-        double y = (k >= klo && k < khi && !bad) ? xr[k] * sc : 0.0;
-#pragma unroll
-        for (int s = 0; s < kSlices; ++s) {
-          y *= 128.0;
-          const double t = trunc(y);
-          y -= t;
-          w[s][q] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu) << (8 * b);
-        }
-      }
+      for (int b = 0; b < 4; ++b) slice_digits(v[b], e, b, w);
     }
 #pragma unroll
-    for (int s = 0; s < kSlices; ++s)
-      *reinterpret_cast<uint4*>(out + s * plane + k0) = make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
+    for (int s2 = 0; s2 < kSlices; ++s2) *reinterpret_cast<uint32_t*>(out + s2 * plane + k0) = w[s2];
   }
 }
 
@@ -179,16 +207,6 @@ __device__ inline void i8x_tile(const I8xArgs& a, int t, int& m0, int& n0, int& 
   kb1 = static_cast<int>((hi + kBK - 1) / kBK);
 }
 
-__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // K-major operand tile with 32-byte rows and the 32-byte swizzle (layout type 6): 8-row atoms
 // of 256 bytes.
 __device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
@@ -205,6 +223,49 @@ __device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
 // 10-12 = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
 constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kBN) >> 3) << 17) |
                               ((static_cast<uint32_t>(kBM) >> 4) << 24);
+
+// kind::i8 MMA, D[tmem] (+)= A[smem] B[smem]^T.  Use selects what happens to the A operand in
+// the tensor core's collector buffer: 0 read from shared memory and dropped (the default), 1 read
+// and kept (fill), 2 taken from the buffer and kept (use), 3 taken from the buffer and dropped
+// (lastuse).  Consecutive MMAs on the same A slice then read it from shared memory once.
+template <int Use>
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+#define HQ_I8_MMA(Q)                                                                              \
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"                               \
+               "tcgen05.mma.cta_group::1.kind::i8" Q " [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d), \
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)                                \
+               : "memory")
+  if constexpr (Use == 1)
+    HQ_I8_MMA(".collector::a::fill");
+  else if constexpr (Use == 2)
+    HQ_I8_MMA(".collector::a::use");
+  else if constexpr (Use == 3)
+    HQ_I8_MMA(".collector::a::lastuse");
+  else
+    HQ_I8_MMA("");
+#undef HQ_I8_MMA
+}
+
+// The MMAs of one stage for A slice P: with B slices 0 .. kSlices - 1 - P into the accumulators
+// of anti-diagonals P .. kSlices - 1, A read from shared memory once (collector buffer).
+template <int P, int Q>
+__device__ __forceinline__ void mma_row(uint32_t tmem, uint64_t ad, uint32_t sb, uint32_t first) {
+  if constexpr (Q + P < kSlices) {
+    constexpr int n = kSlices - P;
+    constexpr int use = (n == 1) ? 0 : (Q == 0 ? 1 : (Q == n - 1 ? 3 : 2));
+    const uint64_t bd = sdesc_sw32(sb + Q * kBSlice);
+    mma_i8<use>(tmem + static_cast<uint32_t>((P + Q) * kBN), ad, bd, kIdescI8, (first && P == 0) ? 0u : 1u);
+    mma_row<P, Q + 1>(tmem, ad, sb, first);
+  }
+}
+template <int P>
+__device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t sa, uint32_t sb, uint32_t first) {
+  if constexpr (P < kSlices) {
+    mma_row<P, 0>(tmem, sdesc_sw32(sa + P * kASlice), sb, first);
+    mma_stage<P + 1>(tmem, sa, sb, first);
+  }
+}
 
 // 32 lanes x 16 consecutive 32-bit TMEM columns, no wait.
 __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
@@ -311,15 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const uint32_t sa = ptx::smem_u32(smem + s * kStageBytes);
         const uint32_t sb = sa + kSlices * kASlice;
-#pragma unroll
-        for (int p = 0; p < kSlices; ++p) {
-          const uint64_t ad = sdesc_sw32(sa + p * kASlice);
-#pragma unroll
-          for (int q = 0; q + p < kSlices; ++q) {
-            const uint64_t bd = sdesc_sw32(sb + q * kBSlice);
-            mma_i8(tmem + static_cast<uint32_t>((p + q) * kBN), ad, bd, kIdescI8, (kb > kb0 || p > 0) ? 1u : 0u);
-          }
-        }
+        // the first stage of a tile overwrites each accumulator with its first product (P == 0)
+        mma_stage<0>(tmem, sa, sb, kb == kb0 ? 1u : 0u);
         ptx::mma_commit(&empty[s]);
       }
       if (!ok) break;
