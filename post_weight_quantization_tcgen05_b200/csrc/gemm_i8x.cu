@@ -26,8 +26,10 @@
 //
 // Kernel (i8x_gemm_kernel, persistent, one CTA per SM, 192 threads): warp 0 issues TMA loads of
 // the slices ([rows][32 bytes of k] boxes, 32-byte swizzle; one 3-D box holds all 7 planes of an
-// operand) into a 4-stage ring; warp 1 issues the 28 kind::i8 MMAs (M = 128, N = 64, K = 32) of
-// each stage from one thread; warps 2-5 drain the accumulators of a finished tile (TMEM lane
+// operand) into a 4-stage ring; warp 1 issues the kind::i8 MMAs of each stage from one thread
+// (M = 128, K = 32; A slice s against the band of B slices 0 .. 6 - s as one operand, N = 64 (7 - s)
+// split at 256: 10 MMAs doing the 28 slice-pair products); warps 2-5 drain the accumulators of a
+// finished tile (TMEM lane
 // quadrant = 32 tile rows each), stage 16-column chunks of the fp64 result in shared memory and
 // update C with coalesced 16-byte accesses.  A declared triangular operand shortens each tile's
 // contraction to the part where it can be non-zero; tiles run longest first.  Every wait is
@@ -219,15 +221,10 @@ __device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
   return d;
 }
 
-// kind::i8 instruction descriptor: s32 accumulator (bits 4-5 = 2), signed A and B (bits 7-9,
-// 10-12 = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kBN) >> 3) << 17) |
-                              ((static_cast<uint32_t>(kBM) >> 4) << 24);
-
 // kind::i8 MMA, D[tmem] (+)= A[smem] B[smem]^T.  Use selects what happens to the A operand in
 // the tensor core's collector buffer: 0 read from shared memory and dropped (the default), 1 read
 // and kept (fill), 2 taken from the buffer and kept (use), 3 taken from the buffer and dropped
-// (lastuse).  Consecutive MMAs on the same A slice then read it from shared memory once.
+// (lastuse).
 template <int Use>
 __device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -247,22 +244,30 @@ __device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t
 #undef HQ_I8_MMA
 }
 
-// The MMAs of one stage for A slice P: with B slices 0 .. kSlices - 1 - P into the accumulators
-// of anti-diagonals P .. kSlices - 1, A read from shared memory once (collector buffer).
-template <int P, int Q>
-__device__ __forceinline__ void mma_row(uint32_t tmem, uint64_t ad, uint32_t sb, uint32_t first) {
-  if constexpr (Q + P < kSlices) {
-    constexpr int n = kSlices - P;
-    constexpr int use = (n == 1) ? 0 : (Q == 0 ? 1 : (Q == n - 1 ? 3 : 2));
-    const uint64_t bd = sdesc_sw32(sb + Q * kBSlice);
-    mma_i8<use>(tmem + static_cast<uint32_t>((P + Q) * kBN), ad, bd, kIdescI8, (first && P == 0) ? 0u : 1u);
-    mma_row<P, Q + 1>(tmem, ad, sb, first);
+// The MMAs of one stage.  The B slices of a stage lie one after another in shared memory, so B
+// slices 0 .. kSlices - 1 - P form a single K-major matrix of kBN (kSlices - P) rows, and
+// A slice P times that band lands slice pair (P, t) in columns kBN (P + t) .. of the accumulator:
+// exactly the columns of anti-diagonal P + t.  One wide MMA per A slice (split at 256 columns)
+// instead of one narrow MMA per slice pair: the tensor core's time per instruction hardly
+// depends on N, so wide instructions keep it busy.  10 MMAs per stage for 7 slices.
+template <int P, int C>
+__device__ __forceinline__ void mma_band(uint32_t tmem, uint64_t ad, uint32_t sb, uint32_t first) {
+  constexpr int total = kBN * (kSlices - P);
+  constexpr int n0 = 256 * C;
+  if constexpr (n0 < total) {
+    constexpr int n = (total - n0) < 256 ? (total - n0) : 256;
+    static_assert(n % 16 == 0 && n >= 16, "MMA width");
+    constexpr uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(n) >> 3) << 17) |
+                               ((static_cast<uint32_t>(kBM) >> 4) << 24);
+    mma_i8<0>(tmem + static_cast<uint32_t>(P * kBN + n0), ad, sdesc_sw32(sb + n0 * kBK), idesc,
+              (first && P == 0) ? 0u : 1u);
+    mma_band<P, C + 1>(tmem, ad, sb, first);
   }
 }
 template <int P>
 __device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t sa, uint32_t sb, uint32_t first) {
   if constexpr (P < kSlices) {
-    mma_row<P, 0>(tmem, sdesc_sw32(sa + P * kASlice), sb, first);
+    mma_band<P, 0>(tmem, sdesc_sw32(sa + P * kASlice), sb, first);
     mma_stage<P + 1>(tmem, sa, sb, first);
   }
 }
