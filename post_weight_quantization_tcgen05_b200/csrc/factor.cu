@@ -16,9 +16,10 @@
 //                                X21 = -X22 Y
 //
 // Every product takes both operands K-major (row-major [rows, contraction]), so X^T is kept
-// next to X (leaves write both, X21^T is copied by a tiled transpose).  Everything runs in fp64
-// (gemm_f64.cu for the products; each declares its triangular operand so that tiles skip the
-// zero part of the contraction).  Leaves are 128 x 128 blocks factored and inverted by one CTA
+// next to X (leaves write both; the product that forms X21 also writes X21^T).  Everything is
+// fp64-accurate: products with all dimensions >= kI8xMinDim run on the int8 tensor cores from
+// exact int8 slices (gemm_i8x.cu), the others on the fp64 tensor cores (gemm_f64.cu); each
+// declares its triangular operand so that tiles skip the zero part of the contraction.  Leaves are 128 x 128 blocks factored and inverted by one CTA
 // (chol_inv_leaf_kernel).  Steps:
 //   1. lambda = damp * mean(diag H)            (fp64 reduction, one CTA)
 //   2. A = J (H + lambda I) J in fp64, lower triangle (tiled transpose of H's lower triangle)
@@ -469,7 +470,7 @@ static hq_status stream_dep(SideStream* ss, cudaStream_t from, cudaStream_t to) 
 // `scratch` (up to the end of the temporaries; NULL: no split) receives split-K partial tiles.
 static hq_status gemm(const FactorCtx& c, cudaStream_t s, double* scratch, double* C, int64_t ldc, int M, int N,
                       int Kred, const double* A, int64_t lda, const double* B, int64_t ldb, double alpha,
-                      double beta, bool lower, int tri) {
+                      double beta, bool lower, int tri, double* Ct = nullptr, int64_t ldct = 0) {
   F64Gemm g{};
   g.C = C;
   g.ldc = ldc;
@@ -488,6 +489,8 @@ static hq_status gemm(const FactorCtx& c, cudaStream_t s, double* scratch, doubl
   g.scratch_elems = scratch == nullptr ? 0 : c.tmp_end - scratch;
   g.skip = c.info;
   g.status = c.status;
+  g.Ct = Ct;
+  g.ldct = ldct;
   if (use_i8x(M, N, Kred)) {
     uint8_t* sl = c.slices[s == c.s ? 0 : 1];
     if (sl != nullptr && i8x_scratch_bytes(M, N, Kred) <= c.slices_bytes) return i8x_gemm(g, sl, c.slices_bytes, s);
@@ -495,28 +498,12 @@ static hq_status gemm(const FactorCtx& c, cudaStream_t s, double* scratch, doubl
   return f64_gemm(g, s);
 }
 
-// dst[j][i] = src[i][j] for an R x C block (32 x 32 tiles through shared memory).
-__global__ void __launch_bounds__(256) transpose_kernel(const double* __restrict__ src, int64_t lds, int64_t R,
-                                                        int64_t C, double* __restrict__ dst, int64_t ldd,
-                                                        const int* __restrict__ info) {
-  if (*info != 0) return;
-  __shared__ double t[32][33];
-  const int64_t tiles_c = (C + 31) / 32;
-  const int64_t r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
-  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
-  for (int i = ty; i < 32; i += 8)
-    if (r0 + i < R && c0 + tx < C) t[i][tx] = src[(r0 + i) * lds + c0 + tx];
-  __syncthreads();
-  for (int j = ty; j < 32; j += 8)
-    if (c0 + j < C && r0 + tx < R) dst[(c0 + j) * ldd + r0 + tx] = t[tx][j];
-}
-
 // X = L^-1 and X^T for the n x n block of A at (off, off); `tmp` has room for the temporaries
 // of this level and all levels below (2 * n2 * n1 here, about a quarter of that per level below).
-// Critical path on c.s: left half, T, the Schur update, right half, X21.  Y^T (needs only T and
-// the left half) and the transpose of X21 run on the side stream, overlapping the right half's
-// leaves and small products; they take no split-K scratch (the region beyond this level's
-// temporaries belongs to the right half meanwhile).
+// Critical path on c.s: left half, T, the Schur update, right half, X21 (with X21^T).  Y^T (needs
+// only T and the left half) runs on the side stream, overlapping the right half's leaves and
+// small products; it takes no split-K scratch (the region beyond this level's temporaries
+// belongs to the right half meanwhile).
 static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tmp) {
   const int64_t K = c.K;
   if (n == kLeaf) {
@@ -554,14 +541,8 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
   if (st != HQ_OK) return st;
   st = stream_dep(c.side, s2, c.s);  // Y^T
   if (st != HQ_OK) return st;
-  st = gemm(c, c.s, rest, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false, kTriALower);  // X21 = -X22 Y
-  if (st != HQ_OK) return st;
-  st = stream_dep(c.side, c.s, s2);
-  if (st != HQ_OK) return st;
-  const int64_t tiles = ceil_div(n2, 32) * ceil_div(n1, 32);
-  transpose_kernel<<<static_cast<unsigned>(tiles), 256, 0, s2>>>(X21, K, n2, n1, XT12, K, c.info);
-  HQ_LAUNCH_CHECK();
-  return HQ_OK;
+  // X21 = -X22 Y, and its transpose into X^T
+  return gemm(c, c.s, rest, X21, K, in2, in1, in2, X22, K, YT, n2, -1.0, 0.0, false, kTriALower, XT12, K);
 }
 
 // ------------------------------------------------------------------------- 4. U, U^T

@@ -17,7 +17,9 @@
 // Tiles are launched most expensive first (their contraction length depends on the triangular
 // operand).  When a problem has too few tiles to fill the GPU, the contraction is split over
 // CTAs that write partial tiles to scratch, and a second kernel adds the partials in a fixed
-// order (so results do not depend on scheduling).
+// order (so results do not depend on scheduling).  (Letting the last CTA of each tile add them
+// instead was measured slower: one CTA then reads every partial of its tile.)  The written C
+// can also be stored transposed (Ct).
 #include <algorithm>
 
 #include "common.cuh"
@@ -183,7 +185,9 @@ __global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm 
           P[static_cast<int64_t>(m) * g.N + n] = acc[i][j][h];
         } else if (!(g.lower && m < n)) {
           double* cp = g.C + static_cast<int64_t>(m) * g.ldc + n;
-          *cp = (g.beta != 0.0 ? g.beta * *cp : 0.0) + g.alpha * acc[i][j][h];
+          const double v = (g.beta != 0.0 ? g.beta * *cp : 0.0) + g.alpha * acc[i][j][h];
+          *cp = v;
+          if (g.Ct != nullptr) g.Ct[static_cast<int64_t>(n) * g.ldct + m] = v;
         }
       }
     }
@@ -201,7 +205,9 @@ __global__ void __launch_bounds__(256) f64_splitk_reduce_kernel(F64Gemm g, int s
     double sum = 0.0;
     for (int s = 0; s < splits; ++s) sum += g.scratch[s * MN + e];
     double* c = g.C + static_cast<int64_t>(m) * g.ldc + n;
-    *c = (g.beta != 0.0 ? g.beta * *c : 0.0) + g.alpha * sum;
+    const double v = (g.beta != 0.0 ? g.beta * *c : 0.0) + g.alpha * sum;
+    *c = v;
+    if (g.Ct != nullptr) g.Ct[static_cast<int64_t>(n) * g.ldct + m] = v;
   }
 }
 

@@ -22,7 +22,8 @@
 // anti-diagonal in its own int32 TMEM accumulator (7 x 64 columns); the sums are exact while
 // 7 * 127^2 * Kred < 2^31 (Kred <= 16384).  The epilogue converts each accumulator to fp64,
 // scales it by its power of two, adds the diagonals smallest first, scales by 2^(e_a + e_b) and
-// alpha and adds beta C (C is not read when beta == 0).
+// alpha and adds beta C (C is not read when beta == 0); optionally it also stores the result
+// transposed (Ct), from the staged chunk, one coalesced row of Ct per column.
 //
 // Kernel (i8x_gemm_kernel, persistent, one CTA per SM, 192 threads): warp 0 issues TMA loads of
 // the slices ([rows][32 bytes of k] boxes, 32-byte swizzle; one 3-D box holds all 7 planes of an
@@ -160,6 +161,8 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
 struct I8xArgs {
   double* C;
   int64_t ldc;
+  double* Ct;  // optional transposed copy of what is written
+  int64_t ldct;
   int M, N, Kpad;
   int tiles_m, tiles_n, tiles;
   double alpha, beta;
@@ -452,8 +455,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           const double p1 = ec1 == kNonFiniteRow ? nan : args.alpha * ldexp(st[rl * kStLd + cl + 1], ec1);
           const bool w0 = col < args.N && (!args.lower || m >= col);
           const bool w1 = col + 1 < args.N && (!args.lower || m >= col + 1);
-          if (w0) crow[col] = args.beta == 0.0 ? p0 : fma(args.beta, crow[col], p0);
-          if (w1) crow[col + 1] = args.beta == 0.0 ? p1 : fma(args.beta, crow[col + 1], p1);
+          if (w0) {
+            const double v = args.beta == 0.0 ? p0 : fma(args.beta, crow[col], p0);
+            crow[col] = v;
+            st[rl * kStLd + cl] = v;
+          }
+          if (w1) {
+            const double v = args.beta == 0.0 ? p1 : fma(args.beta, crow[col + 1], p1);
+            crow[col + 1] = v;
+            st[rl * kStLd + cl + 1] = v;
+          }
+        }
+        __syncwarp();
+        if (args.Ct != nullptr) {  // the transpose: row n of Ct takes the warp's 32 rows, one per lane
+          const int m = m0 + q * 32 + lane;
+#pragma unroll 4
+          for (int j = 0; j < kChunk; ++j) {
+            const int n = n0 + c * kChunk + j;
+            if (m < args.M && n < args.N && (!args.lower || m >= n))
+              args.Ct[static_cast<int64_t>(n) * args.ldct + m] = st[lane * kStLd + j];
+          }
         }
         __syncwarp();
       }
@@ -534,6 +555,8 @@ hq_status i8x_gemm(const F64Gemm& g, uint8_t* scratch, size_t scratch_bytes, cud
   I8xArgs a{};
   a.C = g.C;
   a.ldc = g.ldc;
+  a.Ct = g.Ct;
+  a.ldct = g.ldct;
   a.M = g.M;
   a.N = g.N;
   a.Kpad = static_cast<int>(kp);

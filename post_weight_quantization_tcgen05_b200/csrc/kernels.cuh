@@ -89,6 +89,8 @@ struct F64Gemm {
   int64_t scratch_elems;
   const int* skip;
   int* status;      // device status word for bounded-wait timeouts (may be NULL)
+  double* Ct;       // optional: every written C[m][n] also stored at Ct[n * ldct + m]
+  int64_t ldct;
 };
 hq_status f64_gemm(const F64Gemm& g, cudaStream_t s);
 
