@@ -163,24 +163,30 @@ __device__ __forceinline__ void ldl4_inverse(const double (&s)[16], double (&d)[
   w[12] = w30; w[13] = w31; w[14] = w32; w[15] = w33;
 }
 
-// X = L^-1 and X^T for the 128 x 128 lower block at A, where A = L L^T (Cholesky), by blocked
-// right-looking elimination with 4 x 4 pivot blocks, in one CTA of 16 warps.  fp64.  The Schur
-// complement S and Y (the block elimination of the identity) live in shared memory as the 136
-// lower 8 x 8 tiles of each; warp I owns tile row I of both.  Block step kt (pivot block
-// B = rows/columns 4kt .. 4kt+3), with the panel P = S[:, B] read with zeros at rows <= 4kt+3
-// and W = S_BB^-1 = L_B^-T D_B^-1 L_B^-1 (computed in the previous step):
-//   warp I computes G_I = P_I W (one fp64 MMA) and then updates its tiles, one fp64 MMA
-//   (m8n8k4) per 8 x 8 tile:  S[I][J] -= G_I P_J^T (right of B),  Y[I][J] -= G_I Y[B][J] (left);
-//   the warp owning the next pivot block's diagonal tile updates that tile first and computes
-//   the next W (and keeps D_B, L_B^-1) while the others go on; one barrier per block step.
-// Rows of Y in block B are final once B is eliminated, up to L_B^-1 and D_B^-1/2:
-// X[B][j] = D_B^-1/2 L_B^-1 Y[B][j], applied at the end.  Pivots (the entries of D) are checked
-// at the end (a bad pivot only produces values that are then discarded).
+// X = L^-1 and X^T for the 128 x 128 lower block at A, where A = L L^T (Cholesky), in one CTA of
+// 16 warps, fp64, in three phases.  With 4 x 4 pivot blocks B, A = M S M^T where M is block unit
+// lower triangular (off-diagonal blocks the multipliers N = M - I) and S block diagonal (the
+// pivot blocks S_BB = L_B D_B L_B^T); so L = M diag(L_B D_B^1/2) and
+// X = diag(D_B^-1/2 L_B^-1) M^-1.  The Schur complement S and the multipliers N live in shared
+// memory as the 136 lower 8 x 8 tiles of each.
+//   1. Block right-looking elimination, warp I owning tile row I.  Block step kt (B = rows and
+//      columns 4kt .. 4kt+3), with the panel P = S[:, B] read with zeros at rows <= 4kt+3 and
+//      W = S_BB^-1 = L_B^-T D_B^-1 L_B^-1 (computed in the previous step): warp I computes
+//      G_I = P_I W (one fp64 MMA), stores it as N's block, and updates its tiles right of B,
+//      S[I][J] -= G_I P_J^T (one fp64 MMA m8n8k4 per 8 x 8 tile); the warp owning the next pivot
+//      block's diagonal tile updates that tile first and computes the next W (and keeps D_B,
+//      L_B^-1) while the others go on; one barrier per block step.
+//   2. Z = M^-1 by block forward substitution, warp J computing tile column J alone (no
+//      barriers): Z_JJ = I - N_JJ, Z_IJ = -(I - N_II) sum_{K=J..I-1} N_IK Z_KJ; Z takes S's tiles.
+//   3. X = diag(D_B^-1/2 L_B^-1) Z, written to X and X^T.
+// Pivots (the entries of D) are checked after phase 1 (a bad pivot only produces values that
+// are then discarded).  Updating the inverse alongside the elimination instead (the identity
+// eliminated with S) costs twice the barrier-synchronised tile work per step.
 constexpr int kLB = kLeaf;                    // 128
 constexpr int kLT = kLB / 8;                  // 16 tile rows, one per warp
 constexpr int kLTiles = kLT * (kLT + 1) / 2;  // 136
 constexpr int kLeafThreads = 32 * kLT;
-constexpr size_t kLeafSmem = (2 * kLTiles * 64 + 2 * 16 + kLB + (kLB / 4) * 6) * sizeof(double);
+constexpr size_t kLeafSmem = (2 * kLTiles * 64 + 2 * 16 + kLB + (kLB / 4) * 6 + 2 * kLB * 4) * sizeof(double);
 
 // Element (r, c) of lower tile (I, J): tiles row by row, 64 doubles each, the two 4-column
 // halves of rows 2, 3, 6, 7 swapped (fragment loads of 8 rows x 4 columns and of 4 rows x 8
@@ -197,16 +203,15 @@ __device__ __forceinline__ void dmma_leaf(double& d0, double& d1, double a, doub
       : "d"(a), "d"(b));
 }
 
-// W, D, L^-1 of pivot block `blk` (rows 4 blk .. 4 blk + 3) from S in shared memory (every lane
+// W, D, L^-1 of pivot block `blk` from its 4 x 4 block `pb` (row-major, lower part read; every lane
 // of the calling warp computes them; lane 0 stores).
-__device__ __forceinline__ void leaf_block_inverse(const double* Ssm, int blk, double* wdst, double* dsm,
-                                                   double* msm, int lane) {
-  const int JB = blk >> 1, h = blk & 1;
+__device__ __forceinline__ void leaf_block_inverse(const double* pb, int blk, double* wdst, double* dsm, double* msm,
+                                                   int lane) {
   double sd[16], d[4], m[6], w[16];
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) sd[r * 4 + c] = (c <= r) ? Ssm[lt_idx(JB, JB, 4 * h + r, 4 * h + c)] : 0.0;
+    for (int c = 0; c < 4; ++c) sd[r * 4 + c] = (c <= r) ? pb[r * 4 + c] : 0.0;
   ldl4_inverse(sd, d, m, w);
   if (lane == 0) {
 #pragma unroll
@@ -224,8 +229,8 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
                                                                          int* __restrict__ info, int diag_off) {
   if (*info != 0) return;
   extern __shared__ __align__(16) double lsm[];
-  double* Ssm = lsm;                 // S tiles (later X)
-  double* Ysm = Ssm + kLTiles * 64;  // Y tiles
+  double* Ssm = lsm;                 // S tiles (later Z = M^-1)
+  double* Ysm = Ssm + kLTiles * 64;  // multiplier tiles N (later the output coefficients)
   double* wsm = Ysm + kLTiles * 64;  // W of the current and of the next block, 4 x 4 each
   double* dsm = wsm + 2 * 16;        // pivots
   double* msm = dsm + kLB;           // strict lower part of L_B^-1 per block (6 each)
@@ -233,39 +238,41 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
   const int fg = lane / 4, ft = lane % 4;
 
-  // S = lower part of A, Y = I (all loads of a thread in flight together)
-#pragma unroll 1
-  for (int u0 = 0; u0 < kLB * kLB / kLeafThreads; u0 += 16) {
-    double vals[16];
+  double* pan = msm + (kLB / 4) * 6;  // [2][kLB][4]: the panel of the current and the next block
+  const int I = warp;
+  // N = 0 (the multipliers' tiles), S: tile row I in registers, lane (g = fg, t = ft) holding
+  // elements (g, 2t) and (g, 2t + 1) of each tile (I, J), J <= I (zero above the diagonal)
+  for (int e = tid; e < kLTiles * 64 / 2; e += kLeafThreads)
+    reinterpret_cast<double2*>(Ysm)[e] = make_double2(0.0, 0.0);
+  double2 sreg[kLT];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int e = tid + kLeafThreads * (u0 + u), i = e / kLB, j = e % kLB;
-      vals[u] = (j <= i) ? A[static_cast<int64_t>(i) * lda + j] : 0.0;
-    }
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int e = tid + kLeafThreads * (u0 + u), i = e / kLB, j = e % kLB;
-      if (j / 8 > i / 8) continue;  // tile above the diagonal: not stored
-      Ssm[lt_idx(i / 8, j / 8, i % 8, j % 8)] = vals[u];
-      Ysm[lt_idx(i / 8, j / 8, i % 8, j % 8)] = (i == j) ? 1.0 : 0.0;
+  for (int J = 0; J < kLT; ++J) {
+    sreg[J] = make_double2(0.0, 0.0);
+    if (J <= I) {
+      const int r = 8 * I + fg, c = 8 * J + 2 * ft;
+      const double2 v = *reinterpret_cast<const double2*>(A + static_cast<int64_t>(r) * lda + c);
+      sreg[J] = make_double2(c <= r ? v.x : 0.0, c + 1 <= r ? v.y : 0.0);
     }
   }
+  // the panel of pivot block 0 (tile column 0, columns 0..3): lanes t < 2 hold it
+  if (ft < 2) *reinterpret_cast<double2*>(&pan[(8 * I + fg) * 4 + 2 * ft]) = sreg[0];
   if (tid == 0) bad = kLB;
   __syncthreads();
-  if (warp == 0) leaf_block_inverse(Ssm, 0, wsm, dsm, msm, lane);
+  if (warp == 0) leaf_block_inverse(pan, 0, wsm, dsm, msm, lane);
   __syncthreads();
 
-  const int I = warp;
+  // block steps, fully unrolled (tile indices are then compile-time register indices)
+#pragma unroll
   for (int kt = 0; kt < kLB / 4; ++kt) {
     const int JB = kt >> 1, h = kt & 1;
     const int J0 = JB + h;        // first tile row / column with an element beyond the pivot block
     const int lim = 4 * kt + 3;   // rows <= lim have no part in the update
-    const int JBn = (kt + 1) >> 1;  // diagonal tile of the next pivot block
+    const double* pc = pan + (kt & 1) * kLB * 4;  // this block's panel P (rows x its 4 columns)
     if (I >= J0) {
       // -G_I = -P_I W: A = P_I (8 x 4, zero at rows <= lim), B = W padded to 4 x 8
       double a;
       {
-        const double p = (8 * I + fg > lim) ? Ssm[lt_idx(I, JB, fg, 4 * h + ft)] : 0.0;
+        const double p = (8 * I + fg > lim) ? pc[(8 * I + fg) * 4 + ft] : 0.0;
         const double wv = (fg < 4) ? wsm[(kt & 1) * 16 + ft * 4 + fg] : 0.0;  // W[t][g]
         double g0 = 0.0, g1 = 0.0;
         dmma_leaf(g0, g1, p, wv);
@@ -273,56 +280,29 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
         const double x0 = __shfl_sync(0xffffffffu, g0, src), x1 = __shfl_sync(0xffffffffu, g1, src);
         a = -((ft & 1) ? x1 : x0);
       }
-      // S[I][J] -= G_I P_J^T for J0 <= J <= I.  The next pivot block's diagonal tile is
-      // (J0, J0) (J0 == JBn): its warp has no other S tile and computes the next W right after.
-      // Tiles go four at a time: loads, then MMAs, then stores.
-      const bool next_w = (I == JBn) && (kt + 1 < kLB / 4);
-      for (int J1 = J0; J1 <= I; J1 += 4) {
-        double b[4];
-        double2 cv[4];
+      // the multiplier block G_I (rows of tile I, the pivot block's 4 columns) -> N
+      Ysm[lt_idx(I, JB, fg, 4 * h + ft)] = -a;
+      // S[I][J] -= G_I P_J^T for J0 <= J <= I, in registers; the pivot block's own columns stay
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int J = J1 + u;
-          b[u] = 0.0;
-          cv[u] = make_double2(0.0, 0.0);
-          if (J > I) continue;
-          b[u] = (8 * J + fg > lim) ? Ssm[lt_idx(J, JB, fg, 4 * h + ft)] : 0.0;  // P_J[g][t]
-          cv[u] = *reinterpret_cast<const double2*>(&Ssm[lt_idx(I, J, fg, 2 * ft)]);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dmma_leaf(cv[u].x, cv[u].y, a, b[u]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int J = J1 + u;
-          if (J <= I && !(J == JB && h == 0 && ft < 2))  // B's own columns stay
-            *reinterpret_cast<double2*>(&Ssm[lt_idx(I, J, fg, 2 * ft)]) = cv[u];
+      for (int J = J0; J < kLT; ++J) {
+        if (J <= I) {
+          const double b = (8 * J + fg > lim) ? pc[(8 * J + fg) * 4 + ft] : 0.0;  // P_J[g][t]
+          double2 cv = sreg[J];
+          dmma_leaf(cv.x, cv.y, a, b);
+          if (!(J == JB && h == 0 && ft < 2)) sreg[J] = cv;
         }
       }
-      if (next_w) {
+    }
+    if (kt + 1 < kLB / 4) {
+      // publish the next block's panel (tile column JBn, columns 4 hn .. 4 hn + 3), then the warp
+      // owning its diagonal tile computes its W while the others go on
+      const int JBn = (kt + 1) >> 1, hn = (kt + 1) & 1;
+      double* pn = pan + ((kt + 1) & 1) * kLB * 4;
+      if (I >= JBn && (ft >> 1) == hn)
+        *reinterpret_cast<double2*>(&pn[(8 * I + fg) * 4 + 2 * (ft - 2 * hn)]) = sreg[JBn];
+      if (I == JBn) {
         __syncwarp();
-        leaf_block_inverse(Ssm, kt + 1, wsm + ((kt + 1) & 1) * 16, dsm, msm, lane);
-      }
-      // Y[I][J] -= G_I Y[B][J] for J <= JB
-      for (int J1 = 0; J1 <= JB; J1 += 4) {
-        double b[4];
-        double2 cv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int J = J1 + u;
-          b[u] = 0.0;
-          cv[u] = make_double2(0.0, 0.0);
-          if (J > JB) continue;
-          b[u] = Ysm[lt_idx(JB, J, 4 * h + ft, fg)];  // Y[B][8J + g], row t
-          cv[u] = *reinterpret_cast<const double2*>(&Ysm[lt_idx(I, J, fg, 2 * ft)]);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dmma_leaf(cv[u].x, cv[u].y, a, b[u]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int J = J1 + u;
-          if (J <= JB && !(I == JB && h == 0 && fg < 4))  // B's own rows stay
-            *reinterpret_cast<double2*>(&Ysm[lt_idx(I, J, fg, 2 * ft)]) = cv[u];
-        }
+        leaf_block_inverse(pn + (8 * JBn + 4 * hn) * 4, kt + 1, wsm + ((kt + 1) & 1) * 16, dsm, msm, lane);
       }
     }
     __syncthreads();
@@ -337,11 +317,50 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
     if (tid == 0) atomicCAS(info, 0, diag_off + bad + 1);
     return;
   }
-  // X tile (I, J) = C_I Y tile (I, J), with C_I = diag(D_b^-1/2 L_b^-1, D_b'^-1/2 L_b'^-1) the
+  // Z = (I + N)^-1, the inverse of the block unit lower triangular factor (tile by tile, warp J
+  // computes tile column J, no barriers; S is no longer needed and takes Z):
+  //   Z_JJ = I - N_JJ   (N_JJ is the diagonal tile's lower-left 4 x 4 block, N_JJ^2 = 0)
+  //   Z_IJ = (I - N_II) (-Acc),  Acc = sum_{K = J .. I-1} N_IK Z_KJ   for I > J
+  {
+    const int J = warp;
+    {
+      double2 z;
+      const int c0 = 2 * ft;
+      const double n0 = (fg >= 4 && c0 < 4) ? Ysm[lt_idx(J, J, fg, c0)] : 0.0;
+      const double n1 = (fg >= 4 && c0 + 1 < 4) ? Ysm[lt_idx(J, J, fg, c0 + 1)] : 0.0;
+      z.x = (fg == c0 ? 1.0 : 0.0) - n0;
+      z.y = (fg == c0 + 1 ? 1.0 : 0.0) - n1;
+      *reinterpret_cast<double2*>(&Ssm[lt_idx(J, J, fg, c0)]) = z;
+    }
+    __syncwarp();
+    for (int Ir = J + 1; Ir < kLT; ++Ir) {
+      double acc0 = 0.0, acc1 = 0.0;
+      for (int Kc = J; Kc < Ir; ++Kc) {
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+          const double av = Ysm[lt_idx(Ir, Kc, fg, 4 * kh + ft)];  // N_IK[g][4 kh + t]
+          const double bv = Ssm[lt_idx(Kc, J, 4 * kh + ft, fg)];   // Z_KJ[4 kh + t][g]
+          dmma_leaf(acc0, acc1, av, bv);
+        }
+      }
+      *reinterpret_cast<double2*>(&Ssm[lt_idx(Ir, J, fg, 2 * ft)]) = make_double2(acc0, acc1);
+      __syncwarp();
+      // (I - N_II)(-Acc) = -Acc + N_II Acc, N_II nonzero in rows 4..7, columns 0..3 only
+      const double av = (fg >= 4) ? Ysm[lt_idx(Ir, Ir, fg, ft)] : 0.0;  // N_II[g][t]
+      const double bv = Ssm[lt_idx(Ir, J, ft, fg)];                     // Acc[t][g]
+      double z0 = -acc0, z1 = -acc1;
+      dmma_leaf(z0, z1, av, bv);
+      __syncwarp();
+      *reinterpret_cast<double2*>(&Ssm[lt_idx(Ir, J, fg, 2 * ft)]) = make_double2(z0, z1);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // X tile (I, J) = C_I Z tile (I, J), with C_I = diag(D_b^-1/2 L_b^-1, D_b'^-1/2 L_b'^-1) the
   // block-diagonal 8 x 8 matrix of tile row I's two pivot blocks (two fp64 MMAs per tile);
   // written to X (row-major) and X^T straight from the fragments.  Elements above the diagonal
   // come out zero, as X and X^T already hold there.
-  double* csm = Ssm;  // (S is no longer needed) row i: the 4 coefficients of its block's row
+  double* csm = Ysm;  // (N is no longer needed) row i: the 4 coefficients of its block's row
   {
     const int i = tid;  // row i of the leaf, block i / 4, row r = i % 4 of that block
     if (i < kLB) {
@@ -371,8 +390,8 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
     // k = 0..3 (rows 0..3 of the Y tile) feed output rows 0..3; k = 4..7 feed rows 4..7
     const double a0 = (fg < 4) ? csm[(8 * TI + fg) * 4 + ft] : 0.0;
     const double a1 = (fg >= 4) ? csm[(8 * TI + fg) * 4 + ft] : 0.0;
-    const double b0 = Ysm[lt_idx(TI, TJ, ft, fg)];      // Y[8TI + t][8TJ + g]
-    const double b1 = Ysm[lt_idx(TI, TJ, 4 + ft, fg)];  // Y[8TI + 4 + t][8TJ + g]
+    const double b0 = Ssm[lt_idx(TI, TJ, ft, fg)];      // Z[8TI + t][8TJ + g]
+    const double b1 = Ssm[lt_idx(TI, TJ, 4 + ft, fg)];  // Z[8TI + 4 + t][8TJ + g]
     double x0 = 0.0, x1 = 0.0;
     dmma_leaf(x0, x1, a0, b0);
     dmma_leaf(x0, x1, a1, b1);

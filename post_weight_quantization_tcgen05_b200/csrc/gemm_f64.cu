@@ -10,7 +10,8 @@
 // changes GPTQ codes).  The fp64 MMA rounds like an fp64 FMA chain; on B200 it sustains about
 // 37 TFLOP/s against about 33 for CUDA-core DFMA, with a fraction of the issue slots.
 //
-// Design: BT x BT output tiles (BT = 128: 8 warps of 32 x 64; BT = 64: 4 warps of 32 x 32).
+// Design: BT x BT output tiles (BT = 128: 8 warps of 32 x 64; BT = 64: 4 warps of 32 x 32;
+// BT = 32: 4 warps of 16 x 16).
 // Operands stream through a 4-stage cp.async ring of [BT rows][16 k] slices; element (r, k) of a
 // slice sits at r * 16 + (k ^ ((r & 3) << 2)), so that a fragment load (8 rows x 4 consecutive
 // k) touches distinct banks in each half-warp, and 16-byte pairs stay contiguous for cp.async.
@@ -275,11 +276,15 @@ hq_status f64_gemm(const F64Gemm& g, cudaStream_t s) {
       g.ldb % 2 != 0)
     return HQ_ERR_UNSUPPORTED;
   // 128-wide tiles (one CTA per SM) when they fill the SMs at least once, else 64-wide (up to
-  // three per SM), split along the contraction when even those are too few
+  // three per SM, split along the contraction when fewer than two per SM), and for the small
+  // products of the recursion's lower levels 32-wide tiles without a split: they finish in about
+  // one kernel's latency, where a split costs a second launch (measured: the K = 5120
+  // factorisation 5.24 ms against 5.92 with 64-wide split tiles)
   const int64_t t128 = tile_count<128>(g);
   if (t128 >= kSMs) return launch_f64<128>(g, t128, 1, s);
   const int64_t t64 = tile_count<64>(g);
-  return launch_f64<64>(g, t64, choose_splits(g, t64, 2 * kSMs), s);
+  if (t64 >= kSMs) return launch_f64<64>(g, t64, choose_splits(g, t64, 2 * kSMs), s);
+  return launch_f64<32>(g, tile_count<32>(g), 1, s);
 }
 
 // fp64 MMA issue rate with nothing else in the way: each warp runs 8 independent accumulator
