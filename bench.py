@@ -418,7 +418,7 @@ def other_configs(hq, dev, flush, peaks):
 
 # Kernel classes the library times (hq_debug_timing_*), with the unit of their algorithmic work.
 KERNEL_NAMES = {"f64_gemm_128": ("f64_gemm_kernel<128>", "TFLOP/s"),
-                "f64_gemm_64": ("f64_gemm_kernel<64> + split-K reduce", "TFLOP/s"),
+                "f64_gemm_64": ("f64_gemm_kernel<64>, <32> (+ split-K reduce)", "TFLOP/s"),
                 "i8x_gemm": ("i8x_gemm_kernel (fp64 products from int8 slices on tcgen05 kind::i8)", "TFLOP/s"),
                 "i8x_slice": ("i8x_slice_kernel (fp64 operands cut into int8 slices)", "GB/s"),
                 "leaf": ("chol_inv_leaf_kernel", "TFLOP/s"),
