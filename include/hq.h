@@ -129,9 +129,9 @@ hq_status hq_gptq_quantize(const void* W, int w_dtype, int64_t N, int64_t K, con
  * hq_gptq_quantize on the same rows.
  *
  * hq_gptq_factor_bytes(K): size of the factor buffer: a small header (factorisation status and
- *   lambda), the 128 x 128 diagonal blocks of U' = diag(U)^-1 U in the sweep's packed order, and
- *   the strict lower triangle of U'^T split into a tf32 part and its fp32 remainder (about
- *   8 K^2 bytes).  0 for an unsupported K (K a multiple of 128, at most 65536).
+ *   lambda), the 128 x 128 diagonal blocks of U' = diag(U)^-1 U in the sweep's packed order, the
+ *   384 columns of U' right of each diagonal block (the in-panel updates), and the strict lower
+ *   triangle of U'^T split into a tf32 part and its fp32 remainder (about 8 K^2 bytes).  0 for an unsupported K (K a multiple of 128, at most 65536).
  * hq_gptq_factor_workspace_bytes(K): scratch of hq_gptq_factorize (the fp64 factorisation).
  * hq_gptq_sweep_workspace_bytes(N, K, group): scratch of hq_gptq_sweep (no fp64 matrices).
  *

@@ -617,6 +617,24 @@ __global__ void sweep_pack_kernel(const double* __restrict__ X, int64_t K, float
   }
 }
 
+// The bands of U' (kSweepBand): Ub[b][k][c] = U'[b B + k][(b + 1) B + c], the same fp64 quotient
+// rounded once as in the packed blocks and in U'^T; 0 past column K - 1.
+__global__ void sweep_band_kernel(const double* __restrict__ X, int64_t K, float* __restrict__ Ub,
+                                  const int* __restrict__ info) {
+  if (*info != 0) return;
+  constexpr int B = kSweepBlk;
+  const int64_t total = K * kSweepBand;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = e / (static_cast<int64_t>(B) * kSweepBand);
+    const int r = static_cast<int>(e % (static_cast<int64_t>(B) * kSweepBand));
+    const int64_t gj = b * B + r / kSweepBand, gc = (b + 1) * B + r % kSweepBand;
+    float v = 0.f;
+    if (gc < K) v = static_cast<float>(X[(K - 1 - gj) * K + (K - 1 - gc)] / X[(K - 1 - gj) * (K + 1)]);
+    Ub[e] = v;
+  }
+}
+
 // ------------------------------------------------------------------------- driver
 
 hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double* X, double* XT, double* T,
@@ -666,6 +684,9 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
   if (sweep_form && U != nullptr) {
     const int64_t pg = ceil_div(K * kSweepBlk, 256) < 148 * 16 ? ceil_div(K * kSweepBlk, 256) : 148 * 16;
     sweep_pack_kernel<<<static_cast<unsigned>(pg), 256, 0, s>>>(X, K, U, info);
+    HQ_LAUNCH_CHECK();
+    const int64_t bg = ceil_div(K * kSweepBand, 256) < 148 * 16 ? ceil_div(K * kSweepBand, 256) : 148 * 16;
+    sweep_band_kernel<<<static_cast<unsigned>(bg), 256, 0, s>>>(X, K, U + K * kSweepBlk, info);
     HQ_LAUNCH_CHECK();
   }
   return HQ_OK;

@@ -53,20 +53,29 @@ static int sweep_rows_per_cta(int64_t N) {
   return static_cast<int>(r);
 }
 
-static size_t sweep_smem_bytes(int rows) {
-  return (static_cast<size_t>(kBlk) * kBlk + static_cast<size_t>(rows) * (kBlk + 1) + rows * 4 + kBlk) * sizeof(float) +
-         static_cast<size_t>(rows) * kBlk;
+// Rows per CTA up to which the updates inside a panel run in the sweep kernel itself (one launch
+// per panel; fp32 FMAs on the CUDA cores from the band of U'); with more rows they run as
+// tensor-core GEMM launches between the blocks.
+constexpr int kFusedMaxRows = 64;
+constexpr int kUsK = 32;       // band rows per staged chunk
+constexpr int kLD = kBlk + 4;  // row of the residual stage, 16-byte aligned
+
+static size_t sweep_smem_bytes(int rows, bool fused) {
+  size_t floats = static_cast<size_t>(kBlk) * kBlk + static_cast<size_t>(rows) * kLD + rows * 4 + kBlk;
+  if (fused) floats += 2 * static_cast<size_t>(kUsK) * kBlk;
+  return floats * sizeof(float) + static_cast<size_t>(rows) * kBlk;
 }
 
 struct SweepArgs {
   float* Wf;
   int64_t N, K;
   const float* Upack;  // packed diagonal blocks of U' (sweep_upack_offset order), kBlk^2 floats each
+  const float* band;   // the bands of U' (kSweepBand), read by the in-kernel panel updates
   int group;
   float* Err;        // panel residual buffer [N, P] (the tf32 part when Err_lo is set)
   float* Err_lo;     // NULL, or the fp32 remainder of each residual (Err + Err_lo = residual)
   int64_t err_ld;    // P
-  int err_col;       // column of this block inside the panel buffer
+  int err_col;       // column of the launch's first block inside the panel buffer
   uint8_t* codes;
   float* scales;
   const void* W;
@@ -105,19 +114,113 @@ __device__ __forceinline__ void quant_pair(float wa, float sa, float rsa, float 
 
 __device__ __forceinline__ float recip_or_zero(float s) { return s > 0.f ? __frcp_rn(s) : 0.f; }
 
+// The updates a block owes the later blocks of its panel, for this CTA's rows:
+//   W[r, j0 + kBlk : p1) -= D[r, :] U'[j0 : j0 + kBlk, j0 + kBlk : p1)
+// D the block's residuals (the stage `dst`), U' read from the block's band, fp32 FMAs in k order.
+// Warp w takes rows 4w .. 4w + 3 (the CTA has exactly rows / 4 warps) and lane l the columns
+// 4l .. 4l + 3 of each 128-column chunk; the band passes through shared memory in 32 x 128
+// chunks by cp.async, the next chunk in flight while one is used.  Called by all threads with
+// the caller's cp.async groups possibly pending; returns with none pending, after a barrier.
+__device__ __forceinline__ void panel_update(const SweepArgs& a, int j0, int p1, int64_t r0, const float* dst,
+                                             float* Us) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t K = a.K;
+  const int j1 = j0 + kBlk;
+  constexpr int kKC = kBlk / kUsK;  // band chunks per 128 columns
+  const int nunits = (p1 - j1) / kBlk * kKC;
+  const float* band = a.band + static_cast<int64_t>(j0 / kBlk) * kBlk * kSweepBand;
+  const uint32_t us0 = static_cast<uint32_t>(__cvta_generic_to_shared(Us));
+  auto stage = [&](int u) {  // chunk u: band rows 32 (u % 4) .., columns 128 (u / 4) ..
+    const float* src = band + static_cast<int64_t>((u % kKC) * kUsK) * kSweepBand + (u / kKC) * kBlk;
+    const uint32_t d0 = us0 + static_cast<uint32_t>((u & 1) * kUsK * kBlk * 4);
+    for (int e = tid; e < kUsK * kBlk / 4; e += blockDim.x) {
+      const int k = e / (kBlk / 4), q = e % (kBlk / 4);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d0 + 16u * e), "l"(src + k * kSweepBand + 4 * q)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  stage(0);
+  float acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 1
+  for (int u = 0; u < nunits; ++u) {
+    if (u + 1 < nunits) {
+      stage(u + 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const int kc = u % kKC;
+    const float* ub = Us + (u & 1) * kUsK * kBlk + 4 * lane;
+    const float* db = dst + (4 * warp) * kLD + kc * kUsK;
+#pragma unroll
+    for (int k = 0; k < kUsK; k += 4) {
+      float dv[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 d4 = *reinterpret_cast<const float4*>(db + r * kLD + k);
+        dv[r][0] = d4.x;
+        dv[r][1] = d4.y;
+        dv[r][2] = d4.z;
+        dv[r][3] = d4.w;
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const float4 u4 = *reinterpret_cast<const float4*>(ub + (k + kk) * kBlk);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          acc[r][0] = fmaf(dv[r][kk], u4.x, acc[r][0]);
+          acc[r][1] = fmaf(dv[r][kk], u4.y, acc[r][1]);
+          acc[r][2] = fmaf(dv[r][kk], u4.z, acc[r][2]);
+          acc[r][3] = fmaf(dv[r][kk], u4.w, acc[r][3]);
+        }
+      }
+    }
+    if (kc == kKC - 1) {  // this 128-column chunk is complete: W -= acc
+      const int64_t col = j1 + (u / kKC) * kBlk + 4 * lane;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int64_t row = r0 + 4 * warp + r;
+        if (row < a.N) {
+          float4* wp = reinterpret_cast<float4*>(a.Wf + row * K + col);
+          float4 w = *wp;
+          w.x -= acc[r][0];
+          w.y -= acc[r][1];
+          w.z -= acc[r][2];
+          w.w -= acc[r][3];
+          *wp = w;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+      }
+    }
+    __syncthreads();  // this chunk's buffer is refilled two chunks later
+  }
+}
+
+
 // GS: group size when it is 32, 64 or 128 (scales computed inside the block), or 0 when the
 // group spans several blocks (scale computed at the group's first block from Wf).
-template <int GS>
-__global__ void __launch_bounds__(kMaxSweepThreads) sweep_block_kernel(SweepArgs a, int j0) {
+// The CTA sweeps the blocks j0 = p0, p0 + kBlk, .. < p1 of its rows.  With kFused the updates that
+// each block owes the later blocks of the panel [p0, p1) run here as well (panel_update), between
+// the blocks; otherwise a launch covers one block and the host runs those updates as GEMMs.
+template <int GS, bool kFused>
+__global__ void __launch_bounds__(kFused ? kFusedMaxRows / kRowsPerWarp * 32 : kMaxSweepThreads)
+    sweep_block_kernel(SweepArgs a, int p0, int p1) {
   if (*a.info != 0) return;
-  constexpr int LD = kBlk + 1;  // padded row of the residual stage
   extern __shared__ float4 sm4[];
   float* Ur = reinterpret_cast<float*>(sm4);      // packed U' block
   const int rows = static_cast<int>(blockDim.x / 32) * kRowsPerWarp;
-  float* dst = Ur + kBlk * kBlk;                   // [rows][LD]: residuals
-  float* scl_s = dst + rows * LD;                  // [rows][4]
+  float* dst = Ur + kBlk * kBlk;                   // [rows][kLD]: residuals
+  float* scl_s = dst + rows * kLD;                 // [rows][4]
   float* sup_s = scl_s + rows * 4;                 // [kBlk]: U'[j][j + 1], 0 for the last j
-  int8_t* code_s = reinterpret_cast<int8_t*>(sup_s + kBlk);  // [rows][kBlk]
+  float* Us = sup_s + kBlk;                        // kFused: [2][kUsK][kBlk], chunks of the band
+  int8_t* code_s = reinterpret_cast<int8_t*>(Us + (kFused ? 2 * kUsK * kBlk : 0));  // [rows][kBlk]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, l = lane & (kLanesPerRow - 1);
@@ -127,12 +230,18 @@ __global__ void __launch_bounds__(kMaxSweepThreads) sweep_block_kernel(SweepArgs
   const bool vA = rowA < a.N, vB = rowB < a.N;
   const int64_t K = a.K;
 
-  {  // packed U' block -> shared memory, all copies in flight at once
-    const float4* src = reinterpret_cast<const float4*>(a.Upack + static_cast<int64_t>(j0 / kBlk) * (kBlk * kBlk));
+  // packed U' block of the columns from jb on -> shared memory, all copies in flight at once
+  auto load_upack = [&](int jb) {
+    const float4* src = reinterpret_cast<const float4*>(a.Upack + static_cast<int64_t>(jb / kBlk) * (kBlk * kBlk));
     const uint32_t dst0 = static_cast<uint32_t>(__cvta_generic_to_shared(sm4));
     for (int e = tid; e < kBlk * kBlk / 4; e += blockDim.x)
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst0 + 16u * e), "l"(src + e) : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  load_upack(p0);
+#pragma unroll 1
+  for (int j0 = p0;; j0 += kBlk) {  // up to the last block (`more` false; always after one without kFused)
+  {
     for (int t = tid; t < kBlk; t += blockDim.x) {
       const int c = t + 1;
       sup_s[t] = c < kBlk ? a.Upack[static_cast<int64_t>(j0 / kBlk) * (kBlk * kBlk) +
@@ -248,8 +357,8 @@ __global__ void __launch_bounds__(kMaxSweepThreads) sweep_block_kernel(SweepArgs
       const int col = kLanesPerRow * R + l;
       float cA, cB;
       quant_pair(w0[0], sA, rsA, w1[0], sB, rsB, cA, cB);
-      dst[rlA * LD + col] = fmaf(-cA, sA, w0[0]);
-      dst[rlB * LD + col] = fmaf(-cB, sB, w1[0]);
+      dst[rlA * kLD + col] = fmaf(-cA, sA, w0[0]);
+      dst[rlB * kLD + col] = fmaf(-cB, sB, w1[0]);
       code_s[rlA * kBlk + col] = static_cast<int8_t>(cA);
       code_s[rlB * kBlk + col] = static_cast<int8_t>(cB);
     }
@@ -266,22 +375,25 @@ __global__ void __launch_bounds__(kMaxSweepThreads) sweep_block_kernel(SweepArgs
     scl_s[rlB * 4] = sB;
   }
   __syncthreads();
+  const bool more = kFused && j0 + kBlk < p1;
+  if (more) load_upack(j0 + kBlk);  // Ur is free: the next block's U' arrives during the epilogue
 
   // residuals -> panel buffer (coalesced rows), codes -> packed bytes, scales, qerr partials
+  const int err_col = a.err_col + (j0 - p0);
   const int nwarps = static_cast<int>(blockDim.x / 32);
   for (int r = warp; r < rows; r += nwarps) {
     if (r0 + r >= a.N) break;
-    const float* srcr = dst + r * LD + 4 * lane;
+    const float* srcr = dst + r * kLD + 4 * lane;
     const float4 e4 = make_float4(srcr[0], srcr[1], srcr[2], srcr[3]);
     if (a.Err_lo == nullptr) {
-      reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = e4;
+      reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + err_col)[lane] = e4;
     } else {  // split for the 3xTF32 updates: tf32 part (low 13 mantissa bits cleared) + remainder
       const float4 h4 = make_float4(__uint_as_float(__float_as_uint(e4.x) & 0xFFFFE000u),
                                     __uint_as_float(__float_as_uint(e4.y) & 0xFFFFE000u),
                                     __uint_as_float(__float_as_uint(e4.z) & 0xFFFFE000u),
                                     __uint_as_float(__float_as_uint(e4.w) & 0xFFFFE000u));
-      reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + a.err_col)[lane] = h4;
-      reinterpret_cast<float4*>(a.Err_lo + (r0 + r) * a.err_ld + a.err_col)[lane] =
+      reinterpret_cast<float4*>(a.Err + (r0 + r) * a.err_ld + err_col)[lane] = h4;
+      reinterpret_cast<float4*>(a.Err_lo + (r0 + r) * a.err_ld + err_col)[lane] =
           make_float4(e4.x - h4.x, e4.y - h4.y, e4.z - h4.z, e4.w - h4.w);
     }
     // lane writes bytes 2*lane, 2*lane+1 of the row's 64 code bytes
@@ -344,6 +456,9 @@ __global__ void __launch_bounds__(kMaxSweepThreads) sweep_block_kernel(SweepArgs
     double* p = a.partials + (static_cast<int64_t>(j0 / kBlk) * gridDim.x + blockIdx.x) * 2;
     p[0] = sn;
     p[1] = sd;
+  }
+  if (!more) break;
+  panel_update(a, j0, p1, r0, dst, Us);
   }
 }
 
@@ -413,8 +528,9 @@ FactorLayout factor_layout(int64_t K) {
   size_t off = 0;
   F.hdr = off;
   off = round_up(off + sizeof(FactorHeader), al);
-  F.upack = off;  // packed diagonal blocks of U'
-  off = round_up(off + static_cast<size_t>(K) * kBlk * sizeof(float), al);
+  F.upack = off;  // packed diagonal blocks of U', then its bands (contiguous: one output of the factorisation)
+  F.band = off + static_cast<size_t>(K) * kBlk * sizeof(float);
+  off = round_up(off + static_cast<size_t>(K) * (kBlk + kSweepBand) * sizeof(float), al);
   F.hi = off;     // U'^T strict lower triangle: tf32 part (or, for the CUDA-core updates, U'^T itself)
   off = round_up(off + static_cast<size_t>(K) * K * sizeof(float), al);
   F.lo = off;     // its fp32 remainder
@@ -433,6 +549,9 @@ static void factor_scratch_layout(int64_t K, size_t off, GptqLayout& L) {
   off = round_up(off + kk, al);
   L.a = off;
   off = round_up(off + kk, al);
+  // a factor buffer made in place (launch_gptq) must end before X, which its producers read
+  const size_t fend = round_up(L.t + factor_layout(K).total, al);
+  if (off < fend) off = fend;
   L.x = off;
   off = round_up(off + kk, al);
   L.xt = off;
@@ -510,6 +629,7 @@ hq_status launch_sweep(const void* W, int w_dtype, int64_t N, int64_t K, int64_t
   float* Err_lo = reinterpret_cast<float*>(ws + L.err_lo);
   const FactorHeader* fh = reinterpret_cast<const FactorHeader*>(factor + F.hdr);
   const float* Upack = reinterpret_cast<const float*>(factor + F.upack);
+  const float* band = reinterpret_cast<const float*>(factor + F.band);
   const float* Ut_hi = reinterpret_cast<const float*>(factor + F.hi);
   const float* Ut_lo = reinterpret_cast<const float*>(factor + F.lo);
   const int* info = &fh->info;
@@ -529,6 +649,7 @@ hq_status launch_sweep(const void* W, int w_dtype, int64_t N, int64_t K, int64_t
   a.N = N;
   a.K = K;
   a.Upack = Upack;
+  a.band = band;
   a.group = static_cast<int>(group);
   a.Err = Err;
   a.Err_lo = split ? Err_lo : nullptr;
@@ -541,34 +662,50 @@ hq_status launch_sweep(const void* W, int w_dtype, int64_t N, int64_t K, int64_t
   a.partials = partials;
   a.info = info;
 
-  void (*kern)(SweepArgs, int) = nullptr;
+  // the updates inside a panel run in the sweep kernel when a CTA's rows are few and the panel
+  // lies inside the bands of U'
+  const bool fused = L.sweep_rows <= kFusedMaxRows && P <= kBlk + kSweepBand;
+  void (*kern)(SweepArgs, int, int) = nullptr;
   switch (group) {
-    case 32: kern = sweep_block_kernel<32>; break;
-    case 64: kern = sweep_block_kernel<64>; break;
-    case 128: kern = sweep_block_kernel<128>; break;
-    default: kern = sweep_block_kernel<0>; break;
+    case 32: kern = fused ? sweep_block_kernel<32, true> : sweep_block_kernel<32, false>; break;
+    case 64: kern = fused ? sweep_block_kernel<64, true> : sweep_block_kernel<64, false>; break;
+    case 128: kern = fused ? sweep_block_kernel<128, true> : sweep_block_kernel<128, false>; break;
+    default: kern = fused ? sweep_block_kernel<0, true> : sweep_block_kernel<0, false>; break;
   }
-  const size_t smem = sweep_smem_bytes(L.sweep_rows);
+  const size_t smem = sweep_smem_bytes(L.sweep_rows, fused);
   const int threads = L.sweep_rows / kRowsPerWarp * 32;
   HQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  // bytes of one block: its working weights in, its residuals out (fp32), its block of U', packed
+  // codes and scales out
+  const double block_bytes = static_cast<double>(N) * kBlk * 8.0 + kBlk * kBlk * 4.0 + N * (kBlk / 2.0) +
+                             N * (static_cast<double>(kBlk) / group) * 4.0;
 
   hq_status st = HQ_OK;
   for (int64_t p0 = 0; p0 < K; p0 += P) {
     const int64_t p1 = (p0 + P < K) ? p0 + P : K;
-    for (int64_t j0 = p0; j0 < p1; j0 += kBlk) {
-      a.err_col = static_cast<int>(j0 - p0);
+    if (fused) {
+      a.err_col = 0;
       const int tm = timer_start(kTimeSweep, s);
-      kern<<<L.sweep_grid, threads, smem, s>>>(a, static_cast<int>(j0));
+      kern<<<L.sweep_grid, threads, smem, s>>>(a, static_cast<int>(p0), static_cast<int>(p1));
       HQ_LAUNCH_CHECK();
-      // bytes: the block of working weights in, its residuals out (fp32), the block of U', packed
-      // codes and the block's scales out
-      timer_stop(tm, static_cast<double>(N) * kBlk * 8.0 + kBlk * kBlk * 4.0 + N * (kBlk / 2.0) +
-                         N * (static_cast<double>(kBlk) / group) * 4.0, s);
-      const int64_t j1 = j0 + kBlk;
-      if (j1 < p1) {  // inner update of the rest of the panel
-        st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), Err_lo + (j0 - p0), P, j0, kBlk,
-                          Ut_hi, Ut_lo, info, &hdr->status, s);
-        if (st != HQ_OK) return st;
+      // plus, for the updates inside the panel, the later columns' weights in and out and the band
+      double bytes = 0.0;
+      for (int64_t j1 = p0 + kBlk; j1 <= p1; j1 += kBlk)
+        bytes += block_bytes + (static_cast<double>(N) * 8.0 + kBlk * 4.0) * static_cast<double>(p1 - j1);
+      timer_stop(tm, bytes, s);
+    } else {
+      for (int64_t j0 = p0; j0 < p1; j0 += kBlk) {
+        a.err_col = static_cast<int>(j0 - p0);
+        const int tm = timer_start(kTimeSweep, s);
+        kern<<<L.sweep_grid, threads, smem, s>>>(a, static_cast<int>(j0), static_cast<int>(j0 + kBlk));
+        HQ_LAUNCH_CHECK();
+        timer_stop(tm, block_bytes, s);
+        const int64_t j1 = j0 + kBlk;
+        if (j1 < p1) {  // inner update of the rest of the panel
+          st = sweep_update(update_impl, Wf, N, K, j1, p1 - j1, Err + (j0 - p0), Err_lo + (j0 - p0), P, j0, kBlk,
+                            Ut_hi, Ut_lo, info, &hdr->status, s);
+          if (st != HQ_OK) return st;
+        }
       }
     }
     if (p1 < K) {  // outer update of everything right of the panel

@@ -118,6 +118,10 @@ constexpr int kSweepBlk = 128;
 __host__ __device__ __forceinline__ int sweep_upack_offset(int j, int l, int m) {
   return ((j * 16 + l) * 2 + ((m >> 2) ^ ((l >> 2) & 1))) * 4 + (m & 3);
 }
+// The band of U' right of each diagonal block, for the updates inside a 512-column panel:
+// band b (kSweepBlk x kSweepBand floats, row-major) holds U'[b kSweepBlk + k][(b + 1) kSweepBlk + c]
+// for k < kSweepBlk, c < kSweepBand (0 past column K - 1).
+constexpr int kSweepBand = 384;
 
 // factor.cu: the upper Cholesky factor U of the inverse of the damped Hessian, in fp32, from an
 // fp64 factorisation.  A, X, XT, T are K x K fp64 scratch; `slices` (NULL: every product on the
@@ -126,7 +130,8 @@ __host__ __device__ __forceinline__ int sweep_upack_offset(int j, int l, int m) 
 // overlap X or XT; they may overlap A and T, which are dead by then):
 //   sweep_form == false: U (row-major, upper) and Ut = U^T (row-major, lower).
 //   sweep_form == true:  U receives the packed diagonal blocks of U' = diag(U)^-1 U (K / kSweepBlk
-//                        blocks, see sweep_upack_offset; K a multiple of kSweepBlk) and Ut = U'^T
+//                        blocks, see sweep_upack_offset; K a multiple of kSweepBlk) followed by
+//                        its bands (K kSweepBand floats, see kSweepBand), and Ut = U'^T
 //                        (row-major, lower, unit diagonal).
 //   Ut_hi, Ut_lo: the strict lower triangle of the same Ut split into a tf32 part and the fp32
 //                 remainder (their upper parts are not written).
@@ -137,7 +142,7 @@ hq_status launch_factor(const float* H, int64_t K, float damp, double* A, double
                         float* Ut_hi, float* Ut_lo, cudaStream_t s);
 
 // The factor buffer: everything the GPTQ sweep needs from the factorisation, in one block that
-// ranks sharing a layer's rows can broadcast.  Header, packed diagonal blocks of U', and the
+// ranks sharing a layer's rows can broadcast.  Header, packed diagonal blocks of U', its bands, and the
 // strict lower triangle of U'^T split into its tf32 part (hi) and fp32 remainder (lo); for the
 // CUDA-core updates hi holds U'^T itself.
 struct FactorHeader {
@@ -146,7 +151,7 @@ struct FactorHeader {
   double lam;
 };
 struct FactorLayout {
-  size_t hdr, upack, hi, lo, total;
+  size_t hdr, upack, band, hi, lo, total;
 };
 FactorLayout factor_layout(int64_t K);
 
