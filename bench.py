@@ -527,16 +527,23 @@ def update_roofline_ms(cfg, peaks, tf32_tflops=None) -> float:
 
 
 def kernel_breakdown(hq, layer, flush, steps: int = 2):
-    """Per kernel class: device time and achieved rate over `steps` steps, every launch timed."""
-    hq.hq_debug_timing_start(list(KERNEL_NAMES))
-    layer.step()  # creates the events
-    torch.cuda.synchronize()
-    hq.hq_debug_timing_start(list(KERNEL_NAMES))
-    for k in range(steps):
-        flush.fill_(k & 0xFF)
-        layer.step()
-    torch.cuda.synchronize()
-    hq.hq_debug_timing_stop()
+    """Per kernel class: device time and achieved rate over `steps` steps, every launch timed.
+    The factorisation's second stream is folded into the caller's stream meanwhile, so that each
+    launch's events bracket that launch alone and the shares compare with ncu's serialised
+    launch list (the timed region itself keeps both streams)."""
+    hq.hq_debug_timing_serialize(True)
+    try:
+        hq.hq_debug_timing_start(list(KERNEL_NAMES))
+        layer.step()  # creates the events
+        torch.cuda.synchronize()
+        hq.hq_debug_timing_start(list(KERNEL_NAMES))
+        for k in range(steps):
+            flush.fill_(k & 0xFF)
+            layer.step()
+        torch.cuda.synchronize()
+        hq.hq_debug_timing_stop()
+    finally:
+        hq.hq_debug_timing_serialize(False)
     out = {}
     for cls, (name, unit) in KERNEL_NAMES.items():
         ms, work, n = hq.hq_debug_timing_read(cls)

@@ -121,10 +121,15 @@ hq_status hq_debug_rcp_f64(const double* d, double* out, int64_t n, hq_stream_t 
  * hq_debug_timing_start clears the records and sets the mask; hq_debug_timing_read
  * synchronises the recorded events and returns the sum of durations (ms), of work and the
  * number of launches of one class; hq_debug_timing_stop clears the mask.  Events are created
- * on first use and kept.  One process-wide record: not for concurrent use.  No counterpart
+ * on first use and kept.  One process-wide record: not for concurrent use.
+ * hq_debug_timing_serialize(1): from then on (until hq_debug_timing_serialize(0)) the
+ * factorisation runs its off-critical-path products on the caller's stream instead of a second
+ * stream, so that every recorded duration covers its own launch alone (shares then compare with
+ * a serialised profiler launch list); results are unchanged.  Off by default.  No counterpart
  * on the pages.
  */
 hq_status hq_debug_timing_start(int class_mask);
+hq_status hq_debug_timing_serialize(int on);
 hq_status hq_debug_timing_stop(void);
 hq_status hq_debug_timing_read(int kernel_class, double* ms_total, double* work_total, int64_t* launches);
 

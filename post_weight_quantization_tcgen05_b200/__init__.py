@@ -84,6 +84,7 @@ _SIGS = {
     "hq_debug_upd_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _i64, _vp, _vp, _i64, _vp]),
     "hq_debug_fp64_mma_rate": (ctypes.c_double, [_vp, _i64, _vp]),
     "hq_debug_timing_start": (_int, [_int]),
+    "hq_debug_timing_serialize": (_int, [_int]),
     "hq_debug_timing_stop": (_int, []),
     "hq_debug_timing_read": (_int, [_int, _vp, _vp, _vp]),
     "hq_debug_f64_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _i64, _vp, _i64, _dbl, _dbl, _int, _int, _vp,
@@ -343,6 +344,11 @@ def hq_debug_timing_start(classes) -> None:
     for c in classes:
         mask |= 1 << TIMING_CLASSES[c]
     _check(lib.hq_debug_timing_start(mask), "hq_debug_timing_start")
+
+
+def hq_debug_timing_serialize(on: bool) -> None:
+    """Run the factorisation's second-stream work on the caller's stream (on) or not (off)."""
+    _check(lib.hq_debug_timing_serialize(1 if on else 0), "hq_debug_timing_serialize")
 
 
 def hq_debug_timing_stop() -> None:

@@ -545,7 +545,7 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
   const double* X22 = c.X + (off + n1) * K + off + n1;
   double* XT12 = c.XT + off * K + off + n1;
   const int in1 = static_cast<int>(n1), in2 = static_cast<int>(n2);
-  cudaStream_t s2 = c.side->s2;
+  cudaStream_t s2 = timing_serialized() ? c.s : c.side->s2;
   hq_status st = chol_inv(c, off, n1, rest);
   if (st != HQ_OK) return st;
   st = gemm(c, c.s, rest, T, n1, in2, in1, in1, A21, K, X11, K, 1.0, 0.0, false, kTriBLower);  // T = A21 X11^T

@@ -71,6 +71,10 @@ enum TimerClass {
 };
 int timer_start(int cls, cudaStream_t s);
 void timer_stop(int idx, double work, cudaStream_t s);
+// True after hq_debug_timing_serialize(1): work that would overlap on a second stream then runs
+// on the caller's stream, so that each launch's events bracket that launch alone (as in a
+// serialised profiler launch list).
+bool timing_serialized();
 
 // gemm_f64.cu: C = beta C + alpha A B^T in fp64 on the fp64 tensor cores
 enum F64Tri { kTriNone = 0, kTriAUpper = 1, kTriALower = 2, kTriBLower = 3 };

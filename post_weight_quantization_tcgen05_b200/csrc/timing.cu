@@ -18,6 +18,7 @@ struct TimedLaunch {
 
 std::mutex g_mu;
 int g_mask = 0;                     // classes being timed (bit per TimerClass)
+int g_serialize = 0;                // hq_debug_timing_serialize
 std::vector<TimedLaunch> g_pool;    // events are created once and reused
 size_t g_used = 0;
 
@@ -44,6 +45,8 @@ int timer_start(int cls, cudaStream_t s) {
   return static_cast<int>(g_used++);
 }
 
+bool timing_serialized() { return __atomic_load_n(&g_serialize, __ATOMIC_RELAXED) != 0; }
+
 void timer_stop(int idx, double work, cudaStream_t s) {
   if (idx < 0) return;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -60,6 +63,11 @@ extern "C" hq_status hq_debug_timing_start(int class_mask) {
   std::lock_guard<std::mutex> lk(g_mu);
   g_used = 0;
   __atomic_store_n(&g_mask, class_mask, __ATOMIC_RELAXED);
+  return HQ_OK;
+}
+
+extern "C" hq_status hq_debug_timing_serialize(int on) {
+  __atomic_store_n(&g_serialize, on != 0 ? 1 : 0, __ATOMIC_RELAXED);
   return HQ_OK;
 }
 

@@ -622,3 +622,22 @@ def test_kernel_timing_records_every_launch(hq, cuda_device):
     # nothing is recorded once timing is stopped
     hq.hq_debug_factor(H, 0.01, Ut, ws)
     assert hq.hq_debug_timing_read("leaf")[2] == n
+
+
+def test_serialized_timing_gives_the_same_bits(hq, cuda_device):
+    """hq_debug_timing_serialize only moves the factorisation's second-stream products onto the
+    caller's stream: codes, scales and qerr are bit-identical (K = 4096 reaches the int8-sliced
+    products on both streams)."""
+    N, K, G = 256, 4096, 128
+    cfg = wl.correlated_config(N, K, T=K, group=G, seed=11)
+    X = wl.make_activations(cfg, "cuda")
+    H = torch.zeros((K, K), device="cuda")
+    hq.hq_hessian_accumulate(H, X)
+    W = wl.make_weights(cfg, "cuda", N=N, K=K)
+    base = _run_gptq(hq, W, H, G)
+    hq.hq_debug_timing_serialize(True)
+    try:
+        ser = _run_gptq(hq, W, H, G)
+    finally:
+        hq.hq_debug_timing_serialize(False)
+    assert np.array_equal(base[0], ser[0]) and np.array_equal(base[1], ser[1]) and base[2] == ser[2]
