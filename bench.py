@@ -380,8 +380,9 @@ def time_hessian_at_scale(hq, cfg, dev, flush, peaks, distinct: int = 8):
 
 def time_psd_projection(hq, Hstored, peaks, steps: int = 40):
     """hq_hessian_project_psd on a copy of a decoded Hessian (one untimed call first): its time
-    and its rate against the tensor roofline of its products (three tf32 MMAs per product, tf32
-    peak taken as half the measured bf16 burst, NVIDIA's nominal dense ratio)."""
+    and its rate against the tensor roofline of its products (three tf32 MMAs per product at the
+    tf32 rate measured in this run; half the bf16 burst, NVIDIA's nominal dense ratio, when there
+    is none)."""
     K = Hstored.shape[0]
     ws = hq.alloc_workspace(hq.hq_psd_workspace_bytes(K), Hstored.device)
     P = Hstored.clone()
@@ -396,13 +397,15 @@ def time_psd_projection(hq, Hstored, peaks, steps: int = 40):
     ms = a.elapsed_time(b)
     flops = 4.0 * (steps + 0.5) * float(K) ** 3
     useful = flops / (ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops"] / 2.0 / 3.0
+    tf32 = peaks.get("tf32_tflops")
+    peak = (tf32 if tf32 else peaks["bf16_tflops"] / 2.0) / 3.0
     moved = float(torch.linalg.norm(P - Hstored) / torch.linalg.norm(Hstored))
     del ws, P
     return {"kernels": "upd_gemm_kernel<BN> (3xTF32 Newton-Schulz products) + elementwise", "K": K,
             "steps": steps, "ms": ms, "achieved_useful_tflops": useful, "peak_useful_tflops": peak,
             "frac": useful / peak, "relative_change": moved,
-            "peak_source": peaks["source"] + " bf16 dense burst / 2 (nominal tf32 ratio) / 3 MMAs per product"}
+            "peak_source": ("tf32 dense rate measured in this run" if tf32 else
+                            peaks["source"] + " bf16 dense burst / 2 (nominal tf32 ratio)") + " / 3 MMAs per product"}
 
 
 def other_configs(hq, dev, flush, peaks):
@@ -431,9 +434,8 @@ I8X_PAIRS = 28
 # nominal dense ratio for B200 (fp64 tensor 37 TFLOP/s : bf16 2250 TFLOP/s)
 FP64_OVER_BF16 = 37.0 / 2250.0
 # committed ncu summaries (DRAM traffic per launch) and the source each was taken from
-PROFILES = {"f64_gemm_128": ("f64_gemm_kernel_128_q_proj.md", "gemm_f64.cu"),
-            "f64_gemm_64": ("f64_gemm_kernel_64_q_proj.md", "gemm_f64.cu"),
-            "i8x_gemm": ("i8x_gemm_kernel_down_proj.md", "gemm_i8x.cu"),
+PROFILES = {"f64_gemm_64": ("f64_gemm_kernel_32_q_proj.md", "gemm_f64.cu"),
+            "i8x_gemm": ("i8x_gemm_kernel_q_proj.md", "gemm_i8x.cu"),
             "leaf": ("chol_inv_leaf_kernel_q_proj.md", "factor.cu"),
             "sweep": ("sweep_block_kernel_q_proj.md", "gptq.cu"),
             "tf32_gemm": ("upd_gemm_kernel_q_proj.md", "gemm_upd.cu"),
