@@ -146,6 +146,23 @@ double hq_debug_fp64_mma_rate(void* scratch, int64_t scratch_bytes, hq_stream_t 
  * threads).  A statistic for profiling; never reset. */
 uint64_t hq_debug_launch_count(void);
 
+/*
+ * The bounds-checking build.  libhq_bounds.so is the same library compiled with HQ_DEBUG_BOUNDS:
+ * the kernels check their computed global indices against the extents they were given, and the
+ * first failing check (a tag of the source file's name in bits 16-30, the source line in bits
+ * 0-15) is recorded in a device word while the access it guards is skipped.  It stands in for a
+ * memory checker on machines where none can run.  No counterpart on the pages.
+ *
+ * hq_debug_bounds_status: *enabled = 1 in the bounds-checking build (0 in libhq.so, where
+ *   *violation is always 0); *violation = the recorded failure, 0 if none; the word is then
+ *   cleared.  Synchronises the current device (a blocking copy from a device symbol).
+ * hq_debug_bounds_selftest: launches one check that fails by construction (an index equal to
+ *   the range's length; nothing is accessed), so that the next hq_debug_bounds_status reports
+ *   it.  HQ_ERR_UNSUPPORTED in libhq.so, which launches nothing.
+ */
+hq_status hq_debug_bounds_status(int* enabled, int* violation);
+hq_status hq_debug_bounds_selftest(hq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,7 +15,12 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhq.so")
+# HQ_LIBRARY=libhq_bounds.so selects the bounds-checking build of the same library (hq_debug.h);
+# no other name is accepted.
+_LIB_NAME = os.environ.get("HQ_LIBRARY", "libhq.so")
+if _LIB_NAME not in ("libhq.so", "libhq_bounds.so"):
+    raise ImportError(f"HQ_LIBRARY must be libhq.so or libhq_bounds.so, not {_LIB_NAME!r}")
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), _LIB_NAME)
 
 HQ_OK = 0
 HQ_ERR_INVALID = 1
@@ -39,7 +44,7 @@ class HQError(RuntimeError):
 
 
 if not os.path.exists(_LIB_PATH):
-    raise ImportError(f"libhq.so not found at {_LIB_PATH}; build it with "
+    raise ImportError(f"{_LIB_NAME} not found at {_LIB_PATH}; build it with "
                       "`python post_weight_quantization_tcgen05_b200/build.py`")
 
 lib = ctypes.CDLL(_LIB_PATH)
@@ -80,6 +85,8 @@ _SIGS = {
     "hq_debug_hessian_accumulate_impl": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _int, _vp]),
     "hq_debug_hessian_accumulate_timeout": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _int, _vp]),
     "hq_debug_launch_count": (ctypes.c_uint64, []),
+    "hq_debug_bounds_status": (_int, [_vp, _vp]),
+    "hq_debug_bounds_selftest": (_int, [_vp]),
     "hq_debug_rcp_f64": (_int, [_vp, _vp, _i64, _vp]),
     "hq_debug_upd_gemm": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _i64, _vp, _vp, _i64, _vp]),
     "hq_debug_fp64_mma_rate": (ctypes.c_double, [_vp, _i64, _vp]),
@@ -140,6 +147,27 @@ def hq_abi_version() -> int:
 
 def hq_debug_launch_count() -> int:
     return int(lib.hq_debug_launch_count())
+
+
+def hq_debug_bounds_status():
+    """(enabled, violation): whether this is the bounds-checking build, and the first recorded
+    failing index check (0 if none; cleared by the call)."""
+    en, v = ctypes.c_int(), ctypes.c_int()
+    _check(lib.hq_debug_bounds_status(ctypes.byref(en), ctypes.byref(v)), "hq_debug_bounds_status")
+    return bool(en.value), int(v.value)
+
+
+def hq_debug_bounds_selftest(stream=None) -> None:
+    """Launch one index check that fails by construction (bounds-checking build only)."""
+    _check(lib.hq_debug_bounds_selftest(_stream(stream)), "hq_debug_bounds_selftest")
+
+
+def bounds_file_tag(name: str) -> int:
+    """The tag the bounds-checking build records for source file `name` (bits 16-30)."""
+    h = 0
+    for c in name.encode():
+        h = (h * 31 + c) & 0x7FFF
+    return h | 1
 
 
 def hq_hessian_accumulate(H, X, dev_status=None, stream=None) -> None:

@@ -1,6 +1,8 @@
-"""Builds libhq.so (sm_100a) in-tree with nvcc.
+"""Builds libhq.so (sm_100a) in-tree with nvcc, and its bounds-checking build libhq_bounds.so
+(the same sources with HQ_DEBUG_BOUNDS and relocatable device code, for the device word the
+index checks share).
 
-    python post_weight_quantization_tcgen05_b200/build.py [--force]
+    python post_weight_quantization_tcgen05_b200/build.py [--force] [--bounds | --all]
 
 (Run it as a script, or load it by path: importing it through the package would first import
 the binding, which needs the library this script builds.)
@@ -22,6 +24,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libhq.so")
+LIB_BOUNDS = os.path.join(PKG, "libhq_bounds.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -45,10 +48,10 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
@@ -64,26 +67,38 @@ def _run(cmd: list[str], verbose: bool) -> None:
         sys.stderr.write(r.stdout + r.stderr)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compiles every translation unit to an object (in parallel), then links the library."""
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, bounds: bool = False) -> str:
+    """Compiles every translation unit to an object (in parallel), then links the library
+    (libhq.so, or libhq_bounds.so with `bounds`)."""
+    lib = LIB_BOUNDS if bounds else LIB
+    if not force and not _stale(lib):
+        return lib
     from concurrent.futures import ThreadPoolExecutor
-    os.makedirs(OBJ_DIR, exist_ok=True)
-    objs = [os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o") for src in sources()]
-    cmds = [[_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-c", "-o", obj, src] for src, obj in zip(sources(), objs)]
+    obj_dir = os.path.join(OBJ_DIR, "bounds") if bounds else OBJ_DIR
+    extra = ["-DHQ_DEBUG_BOUNDS", "-rdc=true"] if bounds else []
+    os.makedirs(obj_dir, exist_ok=True)
+    objs = [os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o") for src in sources()]
+    cmds = [[_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", "-o", obj, src] for src, obj in zip(sources(), objs)]
     with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
         for f in [ex.submit(_run, c, verbose) for c in cmds]:
             f.result()
-    tmp = LIB + ".tmp"
-    _run([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs], verbose)
-    os.replace(tmp, LIB)
-    return LIB
+    tmp = lib + ".tmp"
+    link = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared"]
+    if bounds:
+        link.append("-rdc=true")
+    _run([*link, "-o", tmp, *objs], verbose)
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--bounds", action="store_true", help="build libhq_bounds.so only")
+    ap.add_argument("--all", action="store_true", help="build libhq.so and libhq_bounds.so")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose))
+    if args.bounds or args.all:
+        print(build(force=args.force, verbose=args.verbose, bounds=True))
+    if not args.bounds:
+        print(build(force=args.force, verbose=args.verbose))

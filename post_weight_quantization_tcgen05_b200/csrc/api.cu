@@ -73,6 +73,18 @@ __global__ void qerr_terms_kernel(const WsHeader* __restrict__ hdr, double* __re
 
 }  // namespace
 
+#ifdef HQ_DEBUG_BOUNDS
+namespace hq {
+__device__ int g_hq_bounds_violation = 0;
+
+// One check that fails by construction (index n of an n-element range); nothing is accessed.
+__global__ void bounds_selftest_kernel(int n) {
+  const int idx = n;
+  if (HQ_IN_BOUNDS(idx < n)) return;
+}
+}  // namespace hq
+#endif
+
 extern "C" {
 
 const char* hq_status_string(int status) {
@@ -91,6 +103,33 @@ const char* hq_status_string(int status) {
 int hq_abi_version(void) { return kAbiVersion; }
 
 uint64_t hq_debug_launch_count(void) { return __atomic_load_n(&launch_counter(), __ATOMIC_RELAXED); }
+
+hq_status hq_debug_bounds_status(int* enabled, int* violation) {
+  if (enabled == nullptr || violation == nullptr) return HQ_ERR_INVALID;
+#ifdef HQ_DEBUG_BOUNDS
+  int v = 0;
+  HQ_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_hq_bounds_violation, sizeof(int)));
+  const int zero = 0;
+  HQ_CUDA_TRY(cudaMemcpyToSymbol(g_hq_bounds_violation, &zero, sizeof(int)));
+  *enabled = 1;
+  *violation = v;
+#else
+  *enabled = 0;
+  *violation = 0;
+#endif
+  return HQ_OK;
+}
+
+hq_status hq_debug_bounds_selftest(hq_stream_t stream) {
+#ifdef HQ_DEBUG_BOUNDS
+  bounds_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(4);
+  HQ_LAUNCH_CHECK();
+  return HQ_OK;
+#else
+  (void)stream;
+  return HQ_ERR_UNSUPPORTED;
+#endif
+}
 
 hq_status hq_debug_hessian_accumulate_impl(float* H, const void* X, int x_dtype, int64_t T, int64_t K,
                                            int* dev_status, int impl, hq_stream_t stream) {

@@ -95,16 +95,19 @@ __global__ void __launch_bounds__(kEncPairThreads) tril_encode_pair_kernel(const
       const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (c + q < len) my[d + q] = static_cast<uint16_t>(__float_as_uint(f[q]) >> 16);
+        if (c + q < len && HQ_IN_BOUNDS(d + q < kEncStrip)) my[d + q] = static_cast<uint16_t>(__float_as_uint(f[q]) >> 16);
     }
     __syncwarp();
     const int P1 = P0 + len;
     const int A0 = (P0 + 7) & ~7, A1 = P1 & ~7;
-    for (int a = A0 + 8 * lane; a + 8 <= A1; a += 256) pay4[a / 8] = *reinterpret_cast<const uint4*>(my + (a - base));
+    const int npay = K * (K - 1) / 2;
+    for (int a = A0 + 8 * lane; a + 8 <= A1; a += 256)
+      if (HQ_IN_BOUNDS(a + 8 <= npay && a - base + 8 <= kEncStrip))
+        pay4[a / 8] = *reinterpret_cast<const uint4*>(my + (a - base));
     const int h1 = min(A0, P1);
-    if (P0 + lane < h1) pay[P0 + lane] = my[P0 + lane - base];
+    if (P0 + lane < h1 && HQ_IN_BOUNDS(P0 + lane < npay)) pay[P0 + lane] = my[P0 + lane - base];
     const int t0 = max(A1, A0);
-    if (t0 + lane < P1) pay[t0 + lane] = my[t0 + lane - base];
+    if (t0 + lane < P1 && HQ_IN_BOUNDS(t0 + lane < npay)) pay[t0 + lane] = my[t0 + lane - base];
     __syncwarp();
   }
   if (4 * p < K) {  // diagonal entries 4p .. 4p + 3 (K % 4 == 0)
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(256) tril_decode_vec_kernel(const uint8_t* __r
   for (int k = 0; k < kDecTile / 16; ++k) {
     const int r = threadIdx.x / 16 + 16 * k;
     const int64_t i = i0 + r, j = j0 + c4;
-    if (i >= K || j >= K) continue;  // K % 4 == 0: a row's 4 columns are all in range or all out
+    if (i >= K || j >= K || !HQ_IN_BOUNDS(j + 3 < K)) continue;  // K % 4 == 0: a row's 4 columns are all in range or all out
     float4 o;
     if (bi == bj) {
       o.x = (c4 + 0 <= r) ? tile[r][c4 + 0] : tile[c4 + 0][r];
@@ -271,7 +274,7 @@ __global__ void __launch_bounds__(256) tril_decode_vec_kernel(const uint8_t* __r
     for (int k = 0; k < kDecTile / 16; ++k) {
       const int c = threadIdx.x / 16 + 16 * k, r4 = c4;
       const int64_t j = j0 + c, i = i0 + r4;
-      if (i >= K || j >= K) continue;
+      if (i >= K || j >= K || !HQ_IN_BOUNDS(i + 3 < K)) continue;
       *reinterpret_cast<float4*>(H + j * K + i) = make_float4(tile[r4][c], tile[r4 + 1][c], tile[r4 + 2][c], tile[r4 + 3][c]);
     }
   }

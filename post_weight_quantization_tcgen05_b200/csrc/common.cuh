@@ -42,4 +42,34 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Index checks of the bounds-checking build (HQ_DEBUG_BOUNDS, built as libhq_bounds.so; the
+// stand-in for a memory checker).  HQ_IN_BOUNDS(cond) guards one computed global access: in
+// that build a false condition records where it failed (first failure wins: a tag of the source
+// file's name in the high 16 bits, the line in the low 16) in a device word that
+// hq_debug_bounds_status reads, and the guarded access is skipped.  In the regular build the
+// condition is not evaluated and the macro is true.
+constexpr int bounds_file_tag(const char* path) {
+  const char* base = path;
+  for (const char* c = path; *c != 0; ++c)
+    if (*c == '/') base = c + 1;
+  int h = 0;
+  for (const char* c = base; *c != 0; ++c) h = (h * 31 + static_cast<unsigned char>(*c)) & 0x7FFF;
+  return h | 1;
+}
+template <int V>
+struct BoundsTag {
+  static constexpr int value = V;
+};
+#ifdef HQ_DEBUG_BOUNDS
+extern __device__ int g_hq_bounds_violation;
+__device__ __forceinline__ bool bounds_check(bool ok, int where) {
+  if (!ok) atomicCAS(&g_hq_bounds_violation, 0, where);
+  return ok;
+}
+#define HQ_IN_BOUNDS(cond) \
+  (::hq::bounds_check((cond), (::hq::BoundsTag<::hq::bounds_file_tag(__FILE__)>::value << 16) | __LINE__))
+#else
+#define HQ_IN_BOUNDS(cond) true
+#endif
+
 }  // namespace hq

@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
                                                                          double* __restrict__ XT, int64_t ldx,
                                                                          int* __restrict__ info, int diag_off) {
   if (*info != 0) return;
+  // the block lies inside the matrix (uniform over the CTA: no thread is left at a barrier)
+  if (!HQ_IN_BOUNDS(diag_off >= 0 && diag_off + kLB <= ldx && kLB <= lda)) return;
   extern __shared__ __align__(16) double lsm[];
   double* Ssm = lsm;                 // S tiles (later Z = M^-1)
   double* Ysm = Ssm + kLTiles * 64;  // multiplier tiles N (later the output coefficients)
@@ -613,7 +615,7 @@ __global__ void sweep_pack_kernel(const double* __restrict__ X, int64_t K, float
       const int64_t gj = b * B + j, gc = b * B + c;
       v = static_cast<float>(X[(K - 1 - gj) * K + (K - 1 - gc)] / X[(K - 1 - gj) * (K + 1)]);
     }
-    Up[b * B * B + sweep_upack_offset(j, l, m)] = v;
+    if (HQ_IN_BOUNDS(b < K / B)) Up[b * B * B + sweep_upack_offset(j, l, m)] = v;
   }
 }
 

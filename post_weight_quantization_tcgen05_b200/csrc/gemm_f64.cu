@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm 
       const int p = tid + Cfg::kThreads * u;
       const int r = p / 8, k = 2 * (p % 8);
       const int dst = swz(r, k);
-      const bool va = m0 + r < g.M, vb = n0 + r < g.N;
+      const bool kin = HQ_IN_BOUNDS(k0 + k + 1 < g.Kred);
+      const bool va = m0 + r < g.M && kin, vb = n0 + r < g.N && kin;
       cp_async16(As + dst, g.A + static_cast<int64_t>(va ? m0 + r : m0) * g.lda + k0 + k, va);
       cp_async16(Bs + dst, g.B + static_cast<int64_t>(vb ? n0 + r : n0) * g.ldb + k0 + k, vb);
     }
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm 
         if (n >= g.N) continue;
         if (P != nullptr) {
           P[static_cast<int64_t>(m) * g.N + n] = acc[i][j][h];
-        } else if (!(g.lower && m < n)) {
+        } else if (!(g.lower && m < n) && HQ_IN_BOUNDS(n < g.ldc && (g.Ct == nullptr || m < g.ldct))) {
           double* cp = g.C + static_cast<int64_t>(m) * g.ldc + n;
           const double v = (g.beta != 0.0 ? g.beta * *cp : 0.0) + g.alpha * acc[i][j][h];
           *cp = v;
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(256) f64_splitk_reduce_kernel(F64Gemm g, int s
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < MN;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int m = static_cast<int>(e / g.N), n = static_cast<int>(e % g.N);
-    if (g.lower && m < n) continue;
+    if ((g.lower && m < n) || !HQ_IN_BOUNDS(n < g.ldc && (g.Ct == nullptr || m < g.ldct))) continue;
     double sum = 0.0;
     for (int s = 0; s < splits; ++s) sum += g.scratch[s * MN + e];
     double* c = g.C + static_cast<int64_t>(m) * g.ldc + n;

@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
       for (int b = 0; b < 4; ++b) slice_digits(v[b], e, b, w);
     }
 #pragma unroll
-    for (int s2 = 0; s2 < kSlices; ++s2) *reinterpret_cast<uint32_t*>(out + s2 * plane + k0) = w[s2];
+    if (HQ_IN_BOUNDS(k0 + 4 <= Kpad && khi <= Kred))
+      for (int s2 = 0; s2 < kSlices; ++s2) *reinterpret_cast<uint32_t*>(out + s2 * plane + k0) = w[s2];
   }
 }
 
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < 8; ++it) {
           const int rl = 4 * it + (lane >> 3);
           const int m = m0 + q * 32 + rl;
-          if (m >= args.M) continue;
+          if (m >= args.M || !HQ_IN_BOUNDS(col < args.ldc)) continue;
           double* crow = args.C + static_cast<int64_t>(m) * args.ldc;
           const double nan = __longlong_as_double(0x7FF8000000000000LL);
           const double p0 = ec0 == kNonFiniteRow ? nan : args.alpha * ldexp(st[rl * kStLd + cl], ec0);
@@ -472,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 4
           for (int j = 0; j < kChunk; ++j) {
             const int n = n0 + c * kChunk + j;
-            if (m < args.M && n < args.N && (!args.lower || m >= n))
+            if (m < args.M && n < args.N && (!args.lower || m >= n) && HQ_IN_BOUNDS(m < args.ldct))
               args.Ct[static_cast<int64_t>(n) * args.ldct + m] = st[lane * kStLd + j];
           }
         }

@@ -129,6 +129,11 @@ __device__ __forceinline__ void panel_update(const SweepArgs& a, int j0, int p1,
   constexpr int kKC = kBlk / kUsK;  // band chunks per 128 columns
   const int nunits = (p1 - j1) / kBlk * kKC;
   const float* band = a.band + static_cast<int64_t>(j0 / kBlk) * kBlk * kSweepBand;
+  if (!HQ_IN_BOUNDS(p1 <= K && p1 - j1 > 0 && p1 - j1 <= kSweepBand && (p1 - j1) % kBlk == 0)) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    return;  // uniform over the CTA
+  }
   const uint32_t us0 = static_cast<uint32_t>(__cvta_generic_to_shared(Us));
   auto stage = [&](int u) {  // chunk u: band rows 32 (u % 4) .., columns 128 (u / 4) ..
     const float* src = band + static_cast<int64_t>((u % kKC) * kUsK) * kSweepBand + (u / kKC) * kBlk;
@@ -186,7 +191,7 @@ __device__ __forceinline__ void panel_update(const SweepArgs& a, int j0, int p1,
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int64_t row = r0 + 4 * warp + r;
-        if (row < a.N) {
+        if (row < a.N && HQ_IN_BOUNDS(col + 3 < K)) {
           float4* wp = reinterpret_cast<float4*>(a.Wf + row * K + col);
           float4 w = *wp;
           w.x -= acc[r][0];
@@ -234,13 +239,18 @@ __global__ void __launch_bounds__(kFused ? kFusedMaxRows / kRowsPerWarp * 32 : k
   auto load_upack = [&](int jb) {
     const float4* src = reinterpret_cast<const float4*>(a.Upack + static_cast<int64_t>(jb / kBlk) * (kBlk * kBlk));
     const uint32_t dst0 = static_cast<uint32_t>(__cvta_generic_to_shared(sm4));
-    for (int e = tid; e < kBlk * kBlk / 4; e += blockDim.x)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst0 + 16u * e), "l"(src + e) : "memory");
+    if (HQ_IN_BOUNDS(jb >= 0 && jb + kBlk <= a.K))
+      for (int e = tid; e < kBlk * kBlk / 4; e += blockDim.x)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst0 + 16u * e), "l"(src + e) : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
   load_upack(p0);
 #pragma unroll 1
   for (int j0 = p0;; j0 += kBlk) {  // up to the last block (`more` false; always after one without kFused)
+  if (!HQ_IN_BOUNDS(j0 >= 0 && j0 + kBlk <= a.K && a.err_col + (j0 - p0) + kBlk <= a.err_ld)) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    return;  // uniform over the CTA
+  }
   {
     for (int t = tid; t < kBlk; t += blockDim.x) {
       const int c = t + 1;

@@ -207,7 +207,8 @@ __global__ void __launch_bounds__(32 * W) hadamard_cols_lower_kernel(const float
   reg_fwht<32>(v);
   if constexpr (W == 1) {
 #pragma unroll
-    for (int m = 0; m < 32; ++m) G[(r0 + m) * K + c0 + lane] = v[m] * scale;
+    for (int m = 0; m < 32; ++m)
+      if (HQ_IN_BOUNDS(r0 + m < K && c0 + lane < K)) G[(r0 + m) * K + c0 + lane] = v[m] * scale;
   } else {
 #pragma unroll
     for (int m = 0; m < 32; ++m) t[(32 * w + m) * LD + lane] = v[m];  // the elements this thread read
@@ -220,7 +221,8 @@ __global__ void __launch_bounds__(32 * W) hadamard_cols_lower_kernel(const float
       for (int w2 = 0; w2 < W; ++w2) u[w2] = t[(32 * w2 + m) * LD + lane];
       reg_fwht<W>(u);
 #pragma unroll
-      for (int w2 = 0; w2 < W; ++w2) G[(r0 + 32 * w2 + m) * K + c0 + lane] = u[w2] * scale;
+      for (int w2 = 0; w2 < W; ++w2)
+        if (HQ_IN_BOUNDS(r0 + 32 * w2 + m < K && c0 + lane < K)) G[(r0 + 32 * w2 + m) * K + c0 + lane] = u[w2] * scale;
     }
   }
 }
@@ -271,7 +273,7 @@ __global__ void __launch_bounds__(256) hadamard_rows_mirror_kernel(float* G, int
   __syncthreads();
   for (int e = threadIdx.x; e < 32 * B; e += blockDim.x) {
     const int j = e >> 5, rl = e & 31;
-    G[(cb + j) * K + r0 + rl] = t[rl * LD + j + (j >> 5)];
+    if (HQ_IN_BOUNDS(cb + j < K && r0 + rl < K)) G[(cb + j) * K + r0 + rl] = t[rl * LD + j + (j >> 5)];
   }
 }
 

@@ -34,7 +34,8 @@ __global__ void __launch_bounds__(128) rtn_kernel(const void* __restrict__ W, in
       c0 = fminf(fmaxf(rintf(__fdiv_rn(w0, s)), -8.f), 7.f);
       c1 = fminf(fmaxf(rintf(__fdiv_rn(w1, s)), -8.f), 7.f);
     }
-    codes[row * (K / 2) + (g * G) / 2 + p] =
+    if (HQ_IN_BOUNDS((g * G) / 2 + p < K / 2))
+      codes[row * (K / 2) + (g * G) / 2 + p] =
         static_cast<uint8_t>((static_cast<int>(c0) & 0xF) | ((static_cast<int>(c1) & 0xF) << 4));
     const double i0 = imp != nullptr ? static_cast<double>(imp[g * G + 2 * p]) : 1.0;
     const double i1 = imp != nullptr ? static_cast<double>(imp[g * G + 2 * p + 1]) : 1.0;

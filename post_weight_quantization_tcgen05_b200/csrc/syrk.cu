@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256) syrk_simt_kernel(float* __restrict__ H, c
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int64_t j = j0 + tx + 16 * v;
-      if (j <= i) H[i * K + j] += acc[u][v];
+      if (j <= i && HQ_IN_BOUNDS(j < K)) H[i * K + j] += acc[u][v];
     }
   }
 }
@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(kSyThreads, 1)
         uint8_t* sa = smem + s * kSyStageBytes;
         uint8_t* sb = sa + 16384;
         const int t0 = k * kSyBK;
+        // record only: a tile's loads are never skipped (the stage's byte count is already
+        // announced), and the copy engine fills coordinates past the tensor with zeros
+        (void)HQ_IN_BOUNDS(m0 < args.K && n0 < args.K && t0 < args.T);
         ptx::mbar_arrive_expect_tx(&full[s], kSyStageBytes);
         ptx::tma_load_2d(sa, &mapX, m0, t0, &full[s]);
         ptx::tma_load_2d(sa + 8192, &mapX, m0 + 64, t0, &full[s]);
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kSyThreads, 1)
       if (!ok) break;
       // row `row`, columns c0 .. c0 + 127 of H += sum (lower part only)
       const int row = m0 + q * 32 + lane;
-      if (row < args.K) {
+      if (row < args.K && HQ_IN_BOUNDS(n0 + h * 128 < args.K)) {
         float* hrow = args.H + static_cast<int64_t>(row) * args.K;
         const int c0 = n0 + h * 128;
 #pragma unroll

@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(256) tril32_kernel(const float* __restrict__ s
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); i < K; i += warps) {
     const int64_t p = i * (i + 1) / 2;
     const int64_t r = i * K;
-    for (int64_t j = lane; j <= i; j += 32) {
+    for (int64_t j = lane; j <= i && HQ_IN_BOUNDS(p + j < K * (K + 1) / 2); j += 32) {
       if (kPack)
         dst[p + j] = src[r + j];
       else

@@ -111,3 +111,41 @@ def test_header_constants_match_the_binding(hq):
     over = hq.HQ_RTN_NOALLOC_MAX_GROUPS // 2 + 1
     assert hq.lib.hq_rtn_quantize_noalloc(fake, 0, over, 64, 32, None, fake, fake, None, None, None) == \
         hq.HQ_ERR_UNSUPPORTED
+
+
+def test_bounds_build_exports_the_same_symbols():
+    """libhq_bounds.so (the HQ_DEBUG_BOUNDS build) is built beside libhq.so and exports every
+    declared function too."""
+    path = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "libhq_bounds.so")
+    if not os.path.exists(path):
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(
+            "hq_build", os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "build.py"))
+        b = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(b)
+        b.build(bounds=True)
+    blib = ctypes.CDLL(path)
+    for n in sorted(_declared_functions()):
+        assert hasattr(blib, n), n
+
+
+def test_regular_build_reports_no_bounds_checks(hq):
+    """In libhq.so the checks compile away: the status says so and the self-test is refused
+    without launching anything."""
+    assert hq.hq_debug_bounds_status() == (False, 0)
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_debug_bounds_selftest(stream=0)
+    assert e.value.status == hq.HQ_ERR_UNSUPPORTED
+
+
+def test_bounds_file_tag_matches_the_device_side_hash(hq):
+    """The tag the binding computes for a file name follows the same hash as the device macro
+    (31-multiplier rolling hash of the bytes, 15 bits, low bit set): fixed values."""
+    def ref(name):
+        h = 0
+        for c in name.encode():
+            h = (h * 31 + c) % 32768
+        return h | 1
+    for n in ("api.cu", "gptq.cu", "syrk.cu", "codec.cu", "factor.cu"):
+        assert hq.bounds_file_tag(n) == ref(n)
+        assert 1 <= hq.bounds_file_tag(n) < 32768
