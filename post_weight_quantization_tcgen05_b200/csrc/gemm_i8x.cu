@@ -100,25 +100,32 @@ __device__ __forceinline__ void slice_digits(double x, int e, int b, uint32_t (&
   }
 }
 
-// One warp per row: the row maximum over the part the product reads, e_r, then the kSlices int8
-// planes of the row, 128 columns per warp round (each lane 4 consecutive values: two 16-byte
-// loads, one 4-byte store per plane).
+// kSliceWarps warps per row (two rows per 256-thread CTA): the row maximum over the part the
+// product reads (a strided pass, then a warp and a CTA reduction), e_r, then the kSlices int8
+// planes of the row, 512 columns per round (each thread 4 consecutive values: two 16-byte loads,
+// one 4-byte store per plane).  The maximum does not depend on the order of the reduction.
+constexpr int kSliceWarps = 4;
+constexpr int kSliceRowThreads = 32 * kSliceWarps;
+
 __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict__ X, int64_t ldx, int64_t rows,
                                                         int64_t Kred, int64_t Kpad, int tri, int which,
                                                         int8_t* __restrict__ planes, int* __restrict__ exps,
                                                         const int* __restrict__ skip) {
   if (skip != nullptr && *skip != 0) return;
-  const int lane = threadIdx.x & 31;
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (r >= rows) return;
-  int64_t klo, khi;
-  tri_row_range(tri, which, r, Kred, klo, khi);
-  const double* xr = X + r * ldx;
+  __shared__ double red_mx[256 / 32];
+  __shared__ int red_bad[256 / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = threadIdx.x % kSliceRowThreads;  // thread within the row's group
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (256 / kSliceRowThreads) + threadIdx.x / kSliceRowThreads;
+  const bool valid = r < rows;
+  int64_t klo = 0, khi = 0;
+  if (valid) tri_row_range(tri, which, r, Kred, klo, khi);
+  const double* xr = X + (valid ? r : 0) * ldx;
   // 16-byte loads need an even row start and ldx; otherwise scalar loads
   const bool vec = ((reinterpret_cast<uintptr_t>(xr) & 15) == 0);
   double mx = 0.0;
   bool bad = false;
-  for (int64_t k = klo + lane; k < khi; k += 32) {
+  for (int64_t k = klo + t; k < khi; k += kSliceRowThreads) {
     const double v = xr[k];
     bad |= !isfinite(v);
     mx = fmax(mx, fabs(v));
@@ -126,12 +133,26 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    red_mx[warp] = mx;
+    red_bad[warp] = bad ? 1 : 0;
+  }
+  __syncthreads();  // every thread of the CTA reaches it: the invalid rows only skip their work
+  const int w0 = (threadIdx.x / kSliceRowThreads) * kSliceWarps;
+  mx = red_mx[w0];
+  bad = red_bad[w0] != 0;
+#pragma unroll
+  for (int w = 1; w < kSliceWarps; ++w) {
+    mx = fmax(mx, red_mx[w0 + w]);
+    bad |= red_bad[w0 + w] != 0;
+  }
+  if (!valid) return;
   // a row holding a NaN or an infinity is marked, and its products come out NaN
   const int e = bad ? kNonFiniteRow : (mx > 0.0 ? ilogb(mx) + 1 : 0);
-  if (lane == 0) exps[r] = e;
+  if (t == 0) exps[r] = e;
   const int64_t plane = rows * Kpad;
   int8_t* out = planes + r * Kpad;
-  for (int64_t k0 = 4 * lane; k0 < Kpad; k0 += 4 * 32) {
+  for (int64_t k0 = 4 * t; k0 < Kpad; k0 += 4 * kSliceRowThreads) {
     double v[4];
     if (vec && k0 >= klo && k0 + 4 <= khi) {
       const double2 a = *reinterpret_cast<const double2*>(xr + k0);
@@ -151,7 +172,6 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
 #pragma unroll
       for (int b = 0; b < 4; ++b) slice_digits(v[b], e, b, w);
     }
-#pragma unroll
     if (HQ_IN_BOUNDS(k0 + 4 <= Kpad && khi <= Kred))
       for (int s2 = 0; s2 < kSlices; ++s2) *reinterpret_cast<uint32_t*>(out + s2 * plane + k0) = w[s2];
   }
@@ -508,7 +528,7 @@ bool make_slice_map(CUtensorMap* map, const int8_t* planes, int64_t rows, int64_
 
 hq_status slice(const double* X, int64_t ldx, int64_t rows, int64_t Kred, int64_t Kpad, int tri, int which,
                 int8_t* planes, int* exps, const int* skip, cudaStream_t s) {
-  const int64_t grid = ceil_div(rows, 8);
+  const int64_t grid = ceil_div(rows, 256 / kSliceRowThreads);
   i8x_slice_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, ldx, rows, Kred, Kpad, tri, which, planes, exps,
                                                               skip);
   HQ_LAUNCH_CHECK();

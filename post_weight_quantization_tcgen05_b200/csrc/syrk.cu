@@ -328,7 +328,9 @@ __global__ void __launch_bounds__(kSyThreads, 1)
       if (!ok) break;
       // row `row`, columns c0 .. c0 + 127 of H += sum (lower part only)
       const int row = m0 + q * 32 + lane;
-      if (row < args.K && HQ_IN_BOUNDS(n0 + h * 128 < args.K)) {
+      // a tile may overhang H (its upper half can start past column K - 1); each write below
+      // checks its own column
+      if (row < args.K && HQ_IN_BOUNDS(n0 < args.K)) {
         float* hrow = args.H + static_cast<int64_t>(row) * args.K;
         const int c0 = n0 + h * 128;
 #pragma unroll

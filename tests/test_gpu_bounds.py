@@ -16,6 +16,12 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+@pytest.fixture(scope="module")
+def hq():
+    import post_weight_quantization_tcgen05_b200 as m
+    return m
+
+
 def test_bounds_build_finds_no_violation_and_changes_no_bit(hq, cuda_device, tmp_path):
     lib = os.path.join(ROOT, "post_weight_quantization_tcgen05_b200", "libhq_bounds.so")
     assert os.path.exists(lib), "libhq_bounds.so not built (build.py --all)"
