@@ -100,14 +100,13 @@ __global__ void __launch_bounds__(kEncPairThreads) tril_encode_pair_kernel(const
     __syncwarp();
     const int P1 = P0 + len;
     const int A0 = (P0 + 7) & ~7, A1 = P1 & ~7;
-    const int npay = K * (K - 1) / 2;
     for (int a = A0 + 8 * lane; a + 8 <= A1; a += 256)
-      if (HQ_IN_BOUNDS(a + 8 <= npay && a - base + 8 <= kEncStrip))
+      if (HQ_IN_BOUNDS(a + 8 <= K * (K - 1) / 2 && a - base + 8 <= kEncStrip))
         pay4[a / 8] = *reinterpret_cast<const uint4*>(my + (a - base));
     const int h1 = min(A0, P1);
-    if (P0 + lane < h1 && HQ_IN_BOUNDS(P0 + lane < npay)) pay[P0 + lane] = my[P0 + lane - base];
+    if (P0 + lane < h1 && HQ_IN_BOUNDS(P0 + lane < K * (K - 1) / 2)) pay[P0 + lane] = my[P0 + lane - base];
     const int t0 = max(A1, A0);
-    if (t0 + lane < P1 && HQ_IN_BOUNDS(t0 + lane < npay)) pay[t0 + lane] = my[t0 + lane - base];
+    if (t0 + lane < P1 && HQ_IN_BOUNDS(t0 + lane < K * (K - 1) / 2)) pay[t0 + lane] = my[t0 + lane - base];
     __syncwarp();
   }
   if (4 * p < K) {  // diagonal entries 4p .. 4p + 3 (K % 4 == 0)

@@ -37,6 +37,43 @@ inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintp
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
+// Programmatic dependent launch along the factorisation's chain of short kernels (the small fp64
+// products, their split-K reduce, the leaves): a kernel launched by launch_chained may be
+// scheduled while its predecessor on the stream still runs.  It calls pdl_wait before touching
+// memory (it returns once the predecessor has completed and its writes are visible), and
+// pdl_launch_dependents near its end, so that its own successor is scheduled in turn without
+// holding SM slots for long (slots the second stream's work would otherwise use).  In a kernel
+// launched the ordinary way both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// A launch_chained call with the error handling and the launch count of HQ_LAUNCH_CHECK.
+#define HQ_LAUNCH_CHAINED(expr)                            \
+  do {                                                     \
+    cudaError_t _e = (expr);                               \
+    if (_e != cudaSuccess) {                               \
+      (void)cudaGetLastError();                            \
+      return HQ_ERR_CUDA;                                  \
+    }                                                      \
+    __atomic_fetch_add(&::hq::launch_counter(), 1, __ATOMIC_RELAXED); \
+  } while (0)
+
 // Records a device-side failure code in a caller-visible status word (first writer wins).
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);

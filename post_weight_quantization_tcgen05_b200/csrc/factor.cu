@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
                                                                          double* __restrict__ X,
                                                                          double* __restrict__ XT, int64_t ldx,
                                                                          int* __restrict__ info, int diag_off) {
+  pdl_wait();
   if (*info != 0) return;
   // the block lies inside the matrix (uniform over the CTA: no thread is left at a barrier)
   if (!HQ_IN_BOUNDS(diag_off >= 0 && diag_off + kLB <= ldx && kLB <= lda)) return;
@@ -362,6 +363,7 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
   // block-diagonal 8 x 8 matrix of tile row I's two pivot blocks (two fp64 MMAs per tile);
   // written to X (row-major) and X^T straight from the fragments.  Elements above the diagonal
   // come out zero, as X and X^T already hold there.
+  pdl_launch_dependents();  // the successor may be scheduled during the output phase
   double* csm = Ysm;  // (N is no longer needed) row i: the 4 coefficients of its block's row
   {
     const int i = tid;  // row i of the leaf, block i / 4, row r = i % 4 of that block
@@ -529,9 +531,9 @@ static hq_status chol_inv(const FactorCtx& c, int64_t off, int64_t n, double* tm
   const int64_t K = c.K;
   if (n == kLeaf) {
     const int tm = timer_start(kTimeLeaf, c.s);
-    chol_inv_leaf_kernel<<<1, kLeafThreads, kLeafSmem, c.s>>>(c.A + off * K + off, K, c.X + off * K + off,
-                                                      c.XT + off * K + off, K, c.info, static_cast<int>(off));
-    HQ_LAUNCH_CHECK();
+    HQ_LAUNCH_CHAINED(launch_chained(chol_inv_leaf_kernel, dim3(1), dim3(kLeafThreads), kLeafSmem, c.s,
+                                     c.A + off * K + off, K, c.X + off * K + off, c.XT + off * K + off, K, c.info,
+                                     static_cast<int>(off)));
     timer_stop(tm, 2.0 * kLeaf * kLeaf * kLeaf / 3.0, c.s);  // Cholesky n^3/3 + triangular inverse n^3/3
     return HQ_OK;
   }

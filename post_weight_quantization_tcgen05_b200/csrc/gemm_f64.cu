@@ -99,7 +99,11 @@ template <int BT>
 __global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm g, int splits) {
   using Cfg = F64Cfg<BT>;
   extern __shared__ __align__(16) double smem[];
-  if (g.skip != nullptr && *g.skip != 0) return;
+  pdl_wait();
+  if (g.skip != nullptr && *g.skip != 0) {
+    pdl_launch_dependents();
+    return;
+  }
   const int t = blockIdx.x / splits, sp = blockIdx.x % splits;
   int mt, nt;
   tile_of(g, BT, t, mt, nt);
@@ -169,6 +173,7 @@ __global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm 
     }
   }
   cp_async_wait<0>();
+  pdl_launch_dependents();  // the successor may be scheduled while this CTA writes its tile
 
   // lane holds C rows wm0 + 8 i + fg, columns wn0 + 8 j + 2 ft + {0, 1}
   const int64_t MN = static_cast<int64_t>(g.M) * g.N;
@@ -198,6 +203,8 @@ __global__ void __launch_bounds__(F64Cfg<BT>::kThreads) f64_gemm_kernel(F64Gemm 
 
 // C = beta C + alpha * (sum of the partial tiles, split 0 first).
 __global__ void __launch_bounds__(256) f64_splitk_reduce_kernel(F64Gemm g, int splits) {
+  pdl_wait();
+  pdl_launch_dependents();
   if (g.skip != nullptr && *g.skip != 0) return;
   const int64_t MN = static_cast<int64_t>(g.M) * g.N;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < MN;
@@ -243,13 +250,13 @@ hq_status launch_f64(const F64Gemm& g, int64_t tiles, int splits, cudaStream_t s
   HQ_CUDA_TRY(cudaFuncSetAttribute(f64_gemm_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    Cfg::kSmemBytes));
   const int tm = timer_start(BT == 128 ? kTimeF64Gemm128 : kTimeF64Gemm64, s);
-  f64_gemm_kernel<BT><<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmemBytes, s>>>(g, splits);
-  HQ_LAUNCH_CHECK();
+  HQ_LAUNCH_CHAINED(launch_chained(f64_gemm_kernel<BT>, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads),
+                                   Cfg::kSmemBytes, s, g, splits));
   if (splits > 1) {
     const int64_t MN = static_cast<int64_t>(g.M) * g.N;
     const int64_t grid = std::min<int64_t>(ceil_div(MN, 256), kSMs * 8);
-    f64_splitk_reduce_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(g, splits);
-    HQ_LAUNCH_CHECK();
+    HQ_LAUNCH_CHAINED(launch_chained(f64_splitk_reduce_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, g,
+                                     splits));
   }
   timer_stop(tm, f64_gemm_flops(g), s);
   return HQ_OK;
