@@ -31,6 +31,8 @@
 // fp32 in the workspace.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -305,8 +307,11 @@ __global__ void __launch_bounds__(kFused ? kFusedMaxRows / kRowsPerWarp * 32 : k
   // column-to-column dependency chain and the result is bit-identical to the owner's slot.
   float curA = __shfl_sync(0xffffffffu, w0[0], src_base);
   float curB = __shfl_sync(0xffffffffu, w1[0], src_base);
-#pragma unroll 1
-  for (int R = 0; R < kSlots; ++R) {
+  // One round of 16 columns with S live slots: in round R slot m holds column 16 (R + m) + l, so
+  // slots m >= 8 - R lie past the block (zero, and zero in U'); rounds 2r and 2r + 1 update the
+  // first 8 - 2r slots only (the skipped updates would add zero to zero).
+  auto sweep_round = [&](int R, auto slots) {
+    constexpr int S = decltype(slots)::value;
 #pragma unroll
     for (int jr = 0; jr < kLanesPerRow; ++jr) {
       const int j = kLanesPerRow * R + jr;
@@ -333,7 +338,9 @@ __global__ void __launch_bounds__(kFused ? kFusedMaxRows / kRowsPerWarp * 32 : k
         }
       }
       const float4 u0 = *reinterpret_cast<const float4*>(Ur + sweep_upack_offset(j, l, 0));
-      const float4 u1 = *reinterpret_cast<const float4*>(Ur + sweep_upack_offset(j, l, 4));
+      const float4 u1 = S > 4 ? *reinterpret_cast<const float4*>(Ur + sweep_upack_offset(j, l, 4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
       const float usup = sup_s[j];
       // column j + 1 before column j's feedback: slot 0 of lane jr + 1, or after the round's
       // last column slot 1 of lane 0
@@ -344,24 +351,22 @@ __global__ void __launch_bounds__(kFused ? kFusedMaxRows / kRowsPerWarp * 32 : k
       const float da = fmaf(-ca, sA, curA);
       const float db = fmaf(-cb, sB, curB);
       // U' is zero in the packed block on and left of column j: lanes l <= jr keep slot 0
-      w0[0] = fmaf(-da, u0.x, w0[0]);
-      w0[1] = fmaf(-da, u0.y, w0[1]);
-      w0[2] = fmaf(-da, u0.z, w0[2]);
-      w0[3] = fmaf(-da, u0.w, w0[3]);
-      w0[4] = fmaf(-da, u1.x, w0[4]);
-      w0[5] = fmaf(-da, u1.y, w0[5]);
-      w0[6] = fmaf(-da, u1.z, w0[6]);
-      w0[7] = fmaf(-da, u1.w, w0[7]);
-      w1[0] = fmaf(-db, u0.x, w1[0]);
-      w1[1] = fmaf(-db, u0.y, w1[1]);
-      w1[2] = fmaf(-db, u0.z, w1[2]);
-      w1[3] = fmaf(-db, u0.w, w1[3]);
-      w1[4] = fmaf(-db, u1.x, w1[4]);
-      w1[5] = fmaf(-db, u1.y, w1[5]);
-      w1[6] = fmaf(-db, u1.z, w1[6]);
-      w1[7] = fmaf(-db, u1.w, w1[7]);
+#pragma unroll
+      for (int m = 0; m < S; ++m) {
+        w0[m] = fmaf(-da, uu[m], w0[m]);
+        w1[m] = fmaf(-db, uu[m], w1[m]);
+      }
       curA = fmaf(-da, usup, preA);
       curB = fmaf(-db, usup, preB);
+    }
+  };
+#pragma unroll 1
+  for (int R = 0; R < kSlots; ++R) {
+    switch (R >> 1) {
+      case 0: sweep_round(R, std::integral_constant<int, 8>{}); break;
+      case 1: sweep_round(R, std::integral_constant<int, 6>{}); break;
+      case 2: sweep_round(R, std::integral_constant<int, 4>{}); break;
+      default: sweep_round(R, std::integral_constant<int, 2>{}); break;
     }
     {  // slot 0 of lane l now holds the final weight of column 16 R + l
       const int col = kLanesPerRow * R + l;
