@@ -65,7 +65,10 @@ int hq_abi_version(void);
  *   T >= 0 (T == 0 is a no-op), K >= 1.
  *   dev_status : optional device int; if non-NULL a kernel that hits a bounded-wait timeout
  *            stores HQ_ERR_TIMEOUT there (the caller zeroes it beforehand).
- * Asynchronous: returns after enqueueing.  H must not alias X.
+ * Asynchronous: returns after enqueueing.  H must not alias X.  Repeated calls give the same
+ * bits, except that on the tensor-core path a call whose tiles leave a short last round (at most
+ * half of the GPU's 148 SMs) splits those tiles by tokens, and their entries then receive
+ * partial sums in a run-dependent order (differences of the last bit of fp32).
  */
 hq_status hq_hessian_accumulate(float* H, const void* X, int x_dtype, int64_t T, int64_t K,
                                 int* dev_status, hq_stream_t stream);

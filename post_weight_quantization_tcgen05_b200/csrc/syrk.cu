@@ -5,7 +5,10 @@
 // which computes the same sum with exact products and fp32 accumulation.
 //
 // Tensor-core path: one CTA per SM walks 128 x 256 lower-triangle tiles of H (static round
-// robin; all tiles cost the same).  Warp 0 issues TMA loads of 64-token x 64-channel bf16 boxes
+// robin; all tiles cost the same).  When the last round would hold at most half the SMs' worth
+// of tiles (600 tiles on 148 SMs at K = 6144: 4 rounds and 8 tiles), those tiles are cut by
+// 1024-token segments into pieces spread over the idle SMs (the tensor core takes about the same
+// time per instruction at any N up to 256, so narrower tiles would not fill the gap).  Warp 0 issues TMA loads of 64-token x 64-channel bf16 boxes
 // into a 4-stage ring of 48 KB stages (A: channels m0..m0+127, B: n0..n0+255, both MN-major);
 // warp 1 allocates all 512 TMEM columns and issues kind::f16 MMAs from one thread; warps 2-9
 // drain the accumulators.  The tensor core's fp32 accumulation loses precision in proportion to
@@ -17,12 +20,16 @@
 // core fills the other accumulator.  After a tile's last segment each thread adds its row's 128
 // sums to H (lower part only) with 16-byte reductions performed in L2 (red.global.add.v4.f32):
 // nothing is read back, so the epilogue warps return at once to the next tile's segments (a
-// read-modify-write from the SM measured 2-12 % slower).  Every element of H receives one
-// addition per call, so the result does not depend on timing.
+// read-modify-write from the SM measured 2-12 % slower).  An element of a whole tile receives
+// one addition per call, so its result does not depend on timing; the pieces of a cut tile add
+// their partial sums in whatever order they finish, so those elements may differ in the last
+// bit from run to run.
 //
 // Every wait is bounded: on expiry the CTA records HQ_ERR_TIMEOUT, waits (bounded) for its
 // in-flight TMA and MMA work, frees TMEM and returns.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -169,11 +176,35 @@ struct SyrkArgs {
   int K;         // H is K x K, row-major
   int T;         // tokens
   int tiles;     // lower-triangle tiles
+  int full_rounds;  // tiles every CTA takes whole (round robin)
+  int left;         // tiles left after the full rounds
+  int pieces;       // pieces each left tile is cut into (by 1024-token segments)
   int* status;
   long long wait_limit;  // cycles a pipeline wait may take before the CTA gives up
   int withhold_stage;    // -1, or a ring stage whose first release the MMA issuer skips (the
                          // test of the timeout path: the producer's wait for it then expires)
 };
+
+// The work of CTA b: tiles b + i grid for i < full_rounds (all segments), then, if b < left
+// pieces, piece b % pieces of left tile full_rounds grid + b / pieces (a contiguous range of its
+// segments).  A launch whose last round would leave most SMs idle so spreads that round's few
+// tiles over them; the pieces of a tile add their partial sums into H on their own.
+__device__ inline int syrk_items(const SyrkArgs& a) {
+  return a.full_rounds + (static_cast<int>(blockIdx.x) < a.left * a.pieces ? 1 : 0);
+}
+__device__ inline void syrk_item(const SyrkArgs& a, int i, int nseg, int& t, int& s0, int& s1) {
+  const int b = blockIdx.x;
+  if (i < a.full_rounds) {
+    t = b + i * static_cast<int>(gridDim.x);
+    s0 = 0;
+    s1 = nseg;
+    return;
+  }
+  const int p = b % a.pieces;
+  t = a.full_rounds * static_cast<int>(gridDim.x) + b / a.pieces;
+  s0 = p * nseg / a.pieces;
+  s1 = (p + 1) * nseg / a.pieces;
+}
 
 __global__ void __launch_bounds__(kSyThreads, 1)
     syrk_tc_kernel(const __grid_constant__ CUtensorMap mapX, SyrkArgs args) {
@@ -226,10 +257,13 @@ __global__ void __launch_bounds__(kSyThreads, 1)
     ptx::prefetch_tensormap(&mapX);
     int g = 0;  // stages issued by this CTA
     bool ok = true;
-    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
-      int m0, n0;
+    const int nitems = syrk_items(args);
+    for (int it = 0; it < nitems && ok; ++it) {
+      int t, s0, s1, m0, n0;
+      syrk_item(args, it, nseg, t, s0, s1);
       syrk_tile_coords(t, tiles_m, tiles_n, m0, n0);
-      for (int k = 0; k < kiters; ++k, ++g) {
+      const int k1 = (kiters < s1 * kSySegIters) ? kiters : s1 * kSySegIters;
+      for (int k = s0 * kSySegIters; k < k1; ++k, ++g) {
         const int s = g % kSyStages;
         if (g >= kSyStages && !ptx::mbar_wait(&empty[s], ((g / kSyStages) - 1) & 1, abort_flag, args.wait_limit)) {
           ok = false;
@@ -260,9 +294,12 @@ __global__ void __launch_bounds__(kSyThreads, 1)
     bool ok = true;
     int g = 0;   // stages consumed
     int sg = 0;  // segments issued (accumulator = sg & 1)
-    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
-      int k = 0;
-      for (int seg = 0; seg < nseg && ok; ++seg, ++sg) {
+    const int nitems = syrk_items(args);
+    for (int it = 0; it < nitems && ok; ++it) {
+      int t, s0, s1;
+      syrk_item(args, it, nseg, t, s0, s1);
+      int k = s0 * kSySegIters;
+      for (int seg = s0; seg < s1 && ok; ++seg, ++sg) {
         const int acc = sg & 1;
         if (sg >= 2 && !ptx::mbar_wait(&acce[acc], ((sg >> 1) - 1) & 1, abort_flag, args.wait_limit)) {
           ok = false;
@@ -307,13 +344,15 @@ __global__ void __launch_bounds__(kSyThreads, 1)
     const bool vec = (reinterpret_cast<uintptr_t>(args.H) & 15) == 0 && (args.K % 4) == 0;
     bool ok = true;
     int sg = 0;
-    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
-      int m0, n0;
+    const int nitems = syrk_items(args);
+    for (int it = 0; it < nitems && ok; ++it) {
+      int t, s0, s1, m0, n0;
+      syrk_item(args, it, nseg, t, s0, s1);
       syrk_tile_coords(t, tiles_m, tiles_n, m0, n0);
       float sum[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) sum[i] = 0.f;
-      for (int seg = 0; seg < nseg; ++seg, ++sg) {
+      for (int seg = s0; seg < s1; ++seg, ++sg) {
         const int acc = sg & 1;
         if (!ptx::mbar_wait(&accf[acc], (sg >> 1) & 1, abort_flag, args.wait_limit)) {
           ok = false;
@@ -380,10 +419,24 @@ hq_status launch_syrk_tc(float* H, const void* X, int64_t T, int64_t K, int* dev
   a.K = static_cast<int>(K);
   a.T = static_cast<int>(T);
   a.tiles = static_cast<int>(tiles);
+  // whole tiles round robin; a last round of at most half the SMs' worth of tiles is cut into
+  // pieces of whole 1024-token segments and spread over the SMs it would leave idle
+  const int nseg = static_cast<int>(ceil_div(ceil_div(T, kSyBK), kSySegIters));
+  int grid = static_cast<int>(tiles < kSySMs ? tiles : kSySMs);
+  a.full_rounds = static_cast<int>(tiles / grid);
+  a.left = static_cast<int>(tiles - static_cast<int64_t>(a.full_rounds) * grid);
+  a.pieces = 1;
+  if (tiles < kSySMs) {  // one partial round only: cut every tile
+    a.full_rounds = 0;
+    a.left = static_cast<int>(tiles);
+    a.pieces = std::max(1, std::min(kSySMs / a.left, nseg));
+    grid = a.left * a.pieces;
+  } else if (a.left > 0) {
+    a.pieces = std::max(1, std::min(grid / a.left, nseg));
+  }
   a.status = dev_status;
   a.wait_limit = wait_limit;
   a.withhold_stage = withhold_stage;
-  const int grid = static_cast<int>(tiles < kSySMs ? tiles : kSySMs);
   const int tm = timer_start(kTimeSyrk, s);
   syrk_tc_kernel<<<grid, kSyThreads, kSySmem, s>>>(map, a);
   HQ_LAUNCH_CHECK();

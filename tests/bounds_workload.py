@@ -44,8 +44,10 @@ def run_all(hq) -> tuple[dict, dict]:
     out["H_f32"] = _hessian(hq, 300, 136, 2, dtype=torch.float32)
     mark("syrk_f32")
 
-    # int8-sliced products (K = 2048) and the fused panel sweep (200 rows: 4 per CTA)
-    H = _hessian(hq, 2304, 2048, 3)
+    # int8-sliced products (K = 2048) and the fused panel sweep (200 rows: 4 per CTA); at most
+    # 1024 tokens per SYRK call here, so that no call cuts tiles into pieces (whose partial sums
+    # arrive in a run-dependent order) and both builds see the same bits
+    H = _hessian(hq, 1024, 2048, 3)
     W = (torch.randn((200, 2048), device="cuda", generator=_gen(4)) * 0.02).to(torch.bfloat16)
     codes, scales = hq.gptq_outputs(200, 2048, 128)
     ws = hq.alloc_workspace(hq.hq_gptq_workspace_bytes(200, 2048, 128))
