@@ -474,7 +474,7 @@ size_t factor_slice_bytes(int64_t K) {
   size_t b = 0;
   for (const auto& d : dims)
     if (use_i8x(d[0], d[1], d[2])) b = std::max(b, i8x_scratch_bytes(d[0], d[1], d[2]));
-  return b;
+  return round_up(b, 256);  // the second stream's half starts right after the first
 }
 
 // `from` -> `to`: work enqueued on `to` from now on waits for everything enqueued on `from` so far.

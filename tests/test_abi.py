@@ -149,3 +149,10 @@ def test_bounds_file_tag_matches_the_device_side_hash(hq):
     for n in ("api.cu", "gptq.cu", "syrk.cu", "codec.cu", "factor.cu"):
         assert hq.bounds_file_tag(n) == ref(n)
         assert 1 <= hq.bounds_file_tag(n) < 32768
+
+
+def test_i8x_scratch_sizes_keep_256_byte_alignment(hq):
+    """The int8-sliced GEMM's scratch size is a multiple of 256 bytes (the factorisation places
+    one scratch per stream back to back, and the product requires a 256-byte aligned base)."""
+    for M, N, K in ((64, 64, 32), (1280, 1280, 1280), (2560, 2560, 2560), (8704, 8704, 8704), (1000, 600, 300)):
+        assert hq.lib.hq_debug_i8x_scratch_bytes(M, N, K) % 256 == 0
