@@ -135,6 +135,13 @@ def test_hessian_at_scale_sampled_and_codec(hq, cuda_device):
     jj = (rng.random(48) * (ii + 1)).astype(np.int64)
     ii = np.concatenate([ii, ii[:8]])
     jj = np.concatenate([jj, ii[:8]])
+    # and entries of the last 8 tiles in the SYRK's order (each 8192-token call has 600 tiles on
+    # 148 SMs: 4 whole rounds, then these 8 are cut by token segments over the idle SMs); they
+    # lie in rows 5888 .. 6143, columns 5376 .. the diagonal
+    ci = rng.integers(5888, K, 16)
+    cj = 5376 + (rng.random(16) * (ci - 5376 + 1)).astype(np.int64)
+    ii = np.concatenate([ii, ci])
+    jj = np.concatenate([jj, cj])
     cols = np.unique(np.concatenate([ii, jj]))
     cols_t = torch.from_numpy(cols).cuda()
     pos = {c: n for n, c in enumerate(cols)}
