@@ -250,7 +250,7 @@ def run_ours(args, rank, world, local_rank):
         "decode": {"achieved": codec["decode_gbs"], "frac": codec["decode_gbs"] / hbm, "us": codec["decode_us"]},
         "peak": hbm, "peak_source": f"{peaks['source']} HBM copy",
         "bytes": codec["bytes"],
-        "method": "each call alone after an L2 flush (write then read of 256 MiB), events around the call"}
+        "method": "each call alone after an L2 flush (write then read of 256 MiB), events around the call, the GPU rested 0.5 s first"}
     if world == 1 and not args.no_other_configs:
         return_line["hadamard_rotation"] = time_hadamard(hq, layer, flush, peaks)
         return_line["syrk_per_call"] = time_syrk_per_call(hq, layer, flush, peaks)
@@ -364,6 +364,7 @@ def time_hessian_at_scale(hq, cfg, dev, flush, peaks, distinct: int = 8):
     lay.cfg, lay.H = cfg, H
     lay.tril = torch.empty(hqm.hq_bf16tril_bytes(K), dtype=torch.uint8, device=dev)
     lay.Hfull = torch.empty((K, K), dtype=torch.float32, device=dev)
+    burst = codec_throughput(hq, lay, flush, rest_s=0.0)  # right after the SYRK's power-capped burst
     codec = codec_throughput(hq, lay, flush)
     hbm = peaks["hbm_gbs"]
     psd = time_psd_projection(hq, lay.Hfull, peaks)  # the decoded (stored) H, as a reader gets it
@@ -371,7 +372,10 @@ def time_hessian_at_scale(hq, cfg, dev, flush, peaks, distinct: int = 8):
            "syrk_ms": ms, "xtx_tflops": cfg.T * K * (K + 1) / (ms / 1e3) / 1e12,
            "xtx_frac_of_bf16_peak": cfg.T * K * (K + 1) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
            "codec": {"encode_gbs": codec["encode_gbs"], "encode_frac": codec["encode_gbs"] / hbm,
-                     "decode_gbs": codec["decode_gbs"], "decode_frac": codec["decode_gbs"] / hbm},
+                     "decode_gbs": codec["decode_gbs"], "decode_frac": codec["decode_gbs"] / hbm,
+                     "method": "each call alone after an L2 flush, the GPU rested 0.5 s first",
+                     "right_after_syrk_burst": {"encode_frac": burst["encode_gbs"] / hbm,
+                                                "decode_frac": burst["decode_gbs"] / hbm}},
            "psd_projection": psd}
     del chunks, H, lay
     torch.cuda.empty_cache()
@@ -601,11 +605,18 @@ def time_syrk_per_call(hq, layer, flush, peaks, tokens: int = 512, reps: int = 3
         return {"error": str(e)}
 
 
-def codec_throughput(hq, layer, flush, reps: int = 5):
+def codec_throughput(hq, layer, flush, reps: int = 5, rest_s: float = 0.5):
     """Encode and decode of the step's H, each launched right after an L2 flush and timed by
     events around the call alone (in the step, the encode follows hq_gptq_quantize's host
     synchronisation, so its stage time also holds the host's launch latency).  The flush ends
-    with a read so that no dirty lines are written back during the timed call."""
+    with a read so that no dirty lines are written back during the timed call.  The GPU first
+    idles for `rest_s` seconds: for a few hundred ms after a power-capped burst (the chunked
+    SYRK at scale runs at the 1 kW cap) the clocks recover, and in that window a plain fill of
+    the same buffer moves about a quarter fewer bytes per second; the rested figure is the
+    kernel's, the other the transient's (reported beside it where a burst precedes)."""
+    if rest_s > 0:
+        torch.cuda.synchronize()
+        time.sleep(rest_s)
     K = layer.cfg.K
     enc_ms, dec_ms = [], []
     # a write then a read of buffers larger than L2: the L2 holds clean lines of neither input
