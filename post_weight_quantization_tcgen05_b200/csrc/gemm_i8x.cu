@@ -5,14 +5,15 @@
 //   C[m, n] = beta * C[m, n] + alpha * sum_k A(m, k) B(n, k)      m < M, n < N
 //   A(m, k) = A[m * lda + k],  B(n, k) = B[n * ldb + k]           (both operands K-major)
 //
-// Slicing (i8x_slice_kernel, one warp per row).  Row r of an operand is scaled by 2^-e_r, e_r the
+// Slicing (i8x_slice_kernel, four warps per row).  Row r of an operand is scaled by 2^-e_r, e_r the
 // smallest exponent with max_k |x[r, k]| < 2^e_r, and cut into kSlices signed 7-bit integers:
 //   y_0 = x 2^-e_r;  d_s = trunc(128 y_s) in [-127, 127];  y_{s+1} = 128 y_s - d_s,
 // so x = 2^e_r sum_s d_s 2^(-7 (s + 1)) + 2^(e_r - 7 S) y_S with |y_S| < 1: the base-128 digits of
 // |x| 2^-e_r, signed like x.  The kernel reads them off the fp64 bit pattern with integer shifts
 // (slice_digits), which gives the same digits as the fp64 steps above.
-// Slice s of all rows is a plane [rows][Kpad] of int8 (K-major), zero outside the part of the
-// row the product reads (a declared triangular operand) and past Kred.
+// The slices are int8, zero outside the part of the row the product reads (a declared triangular
+// operand) and past Kred, stored in the shared-memory image of the product's pipeline stages
+// (layouts A and B at slice_atom_a / slice_atom_b below).
 //
 // Product.  x_a x_b = 2^(e_a + e_b) sum_{s,t} d_s d_t 2^(-7 (s + t + 2)): every slice product is
 // an exact integer, and the pairs of one anti-diagonal s + t = g share the scale 2^(-7 (g + 2)).
@@ -25,20 +26,20 @@
 // alpha and adds beta C (C is not read when beta == 0); optionally it also stores the result
 // transposed (Ct), from the staged chunk, one coalesced row of Ct per column.
 //
-// Kernel (i8x_gemm_kernel, persistent, one CTA per SM, 192 threads): warp 0 issues TMA loads of
-// the slices ([rows][32 bytes of k] boxes, 32-byte swizzle; one 3-D box holds all 7 planes of an
-// operand) into a 4-stage ring; warp 1 issues the kind::i8 MMAs of each stage from one thread
+// Kernel (i8x_gemm_kernel, persistent, one CTA per SM, 192 threads): warp 0 copies each stage
+// of the A and the B tile (all 7 slices, 32 bytes of k) with one bulk copy each, 28 KB and 14 KB
+// contiguous, into a 4-stage ring; warp 1 issues the kind::i8 MMAs of each stage from one thread
 // (M = 128, K = 32; A slice s against the band of B slices 0 .. 6 - s as one operand, N = 64 (7 - s)
 // split at 256: 10 MMAs doing the 28 slice-pair products); warps 2-5 drain the accumulators of a
 // finished tile (TMEM lane
 // quadrant = 32 tile rows each), stage 16-column chunks of the fp64 result in shared memory and
 // update C with coalesced 16-byte accesses.  A declared triangular operand shortens each tile's
-// contraction to the part where it can be non-zero; tiles run longest first.  Every wait is
+// contraction to the part where it can be non-zero; tiles are enumerated longest first and dealt
+// to the CTAs in waves walked alternately forward and backward.  Every wait is
 // bounded; on expiry the CTA records HQ_ERR_TIMEOUT, waits for what it issued and returns.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
-#include "tmap.cuh"
 
 namespace hq {
 namespace {
@@ -49,6 +50,8 @@ constexpr int kStages = 4;
 constexpr int kASlice = kBM * kBK;                  // 4 KB per plane
 constexpr int kBSlice = kBN * kBK;                  // 2 KB per plane
 constexpr int kStageBytes = kSlices * (kASlice + kBSlice);
+constexpr int kABlockBytes = kSlices * kASlice;     // one stage of an A tile: 28 KB, one bulk copy
+constexpr int kBBlockBytes = kSlices * kBSlice;     // one stage of a B tile: 14 KB, one bulk copy
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kChunk = 16;                          // epilogue columns per round
@@ -100,17 +103,39 @@ __device__ __forceinline__ void slice_digits(double x, int e, int b, uint32_t (&
   }
 }
 
+// Slice layouts in global memory: the exact shared-memory image of one pipeline stage, so that a
+// stage of a tile is one contiguous bulk copy.  An operand's rows are cut into blocks of the tile
+// height (kBM rows for A, kBN for B; the last block padded, its padding rows never written and
+// read only into outputs that are not stored), its contraction into 32-byte chunks; the unit is
+// the 256-byte atom of 8 rows x 32 bytes in the 32-byte swizzle (the two 16-byte halves of rows
+// 4-7 swapped), and the atoms of (chunk, block) lie together:
+//   A: [chunk][block][8-row group][slice][atom]   slice s of the tile = 16 atoms 7 x 256 bytes apart
+//   B: [chunk][block][slice][8-row group][atom]   the slices stacked along N, as one K-major band
+__device__ __forceinline__ int64_t slice_atom_a(int64_t kc, int64_t r, int s, int64_t nblk) {
+  return ((kc * nblk + r / kBM) * (kBM / 8) + (r % kBM) / 8) * kSlices + s;
+}
+__device__ __forceinline__ int64_t slice_atom_b(int64_t kc, int64_t r, int s, int64_t nblk) {
+  return ((kc * nblk + r / kBN) * kSlices + s) * (kBN / 8) + (r % kBN) / 8;
+}
+// byte of (row r, contraction byte c of its 32-byte chunk) inside the atom
+__device__ __forceinline__ int slice_in_atom(int64_t r, int c) {
+  const int rr = static_cast<int>(r & 7);
+  return (rr << 5) | (c ^ (((rr >> 2) & 1) << 4));
+}
+
 // kSliceWarps warps per row (two rows per 256-thread CTA): the row maximum over the part the
 // product reads (a strided pass, then a warp and a CTA reduction), e_r, then the kSlices int8
-// planes of the row, 512 columns per round (each thread 4 consecutive values: two 16-byte loads,
-// one 4-byte store per plane).  The maximum does not depend on the order of the reduction.
+// slices of the row, 512 columns per round (each thread 4 consecutive values: two 16-byte loads,
+// one 4-byte store per slice and layout written: A, B or both).  The maximum does not depend on
+// the order of the reduction.
 constexpr int kSliceWarps = 4;
 constexpr int kSliceRowThreads = 32 * kSliceWarps;
 
 __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict__ X, int64_t ldx, int64_t rows,
                                                         int64_t Kred, int64_t Kpad, int tri, int which,
-                                                        int8_t* __restrict__ planes, int* __restrict__ exps,
-                                                        const int* __restrict__ skip) {
+                                                        int8_t* __restrict__ out_a, int64_t nblk_a,
+                                                        int8_t* __restrict__ out_b, int64_t nblk_b,
+                                                        int* __restrict__ exps, const int* __restrict__ skip) {
   if (skip != nullptr && *skip != 0) return;
   __shared__ double red_mx[256 / 32];
   __shared__ int red_bad[256 / 32];
@@ -150,8 +175,6 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
   // a row holding a NaN or an infinity is marked, and its products come out NaN
   const int e = bad ? kNonFiniteRow : (mx > 0.0 ? ilogb(mx) + 1 : 0);
   if (t == 0) exps[r] = e;
-  const int64_t plane = rows * Kpad;
-  int8_t* out = planes + r * Kpad;
   for (int64_t k0 = 4 * t; k0 < Kpad; k0 += 4 * kSliceRowThreads) {
     double v[4];
     if (vec && k0 >= klo && k0 + 4 <= khi) {
@@ -172,14 +195,24 @@ __global__ void __launch_bounds__(256) i8x_slice_kernel(const double* __restrict
 #pragma unroll
       for (int b = 0; b < 4; ++b) slice_digits(v[b], e, b, w);
     }
-    if (HQ_IN_BOUNDS(k0 + 4 <= Kpad && khi <= Kred))
-      for (int s2 = 0; s2 < kSlices; ++s2) *reinterpret_cast<uint32_t*>(out + s2 * plane + k0) = w[s2];
+    if (!HQ_IN_BOUNDS(k0 + 4 <= Kpad && khi <= Kred)) continue;
+    const int64_t kc = k0 / kBK;
+    const int in_atom = slice_in_atom(r, static_cast<int>(k0 % kBK));
+    if (out_a != nullptr && HQ_IN_BOUNDS(r / kBM < nblk_a))
+      for (int s2 = 0; s2 < kSlices; ++s2)
+        *reinterpret_cast<uint32_t*>(out_a + (slice_atom_a(kc, r, s2, nblk_a) << 8) + in_atom) = w[s2];
+    if (out_b != nullptr && HQ_IN_BOUNDS(r / kBN < nblk_b))
+      for (int s2 = 0; s2 < kSlices; ++s2)
+        *reinterpret_cast<uint32_t*>(out_b + (slice_atom_b(kc, r, s2, nblk_b) << 8) + in_atom) = w[s2];
   }
 }
 
 // ------------------------------------------------------------------------- product
 
 struct I8xArgs {
+  const int8_t* pa;  // A slices, layout A (one stage of a tile = kABlockBytes contiguous bytes)
+  const int8_t* pb;  // B slices, layout B (kBBlockBytes per stage of a tile)
+  int nblk_a, nblk_b;
   double* C;
   int64_t ldc;
   double* Ct;  // optional transposed copy of what is written
@@ -233,13 +266,19 @@ __device__ inline void i8x_tile(const I8xArgs& a, int t, int& m0, int& n0, int& 
   kb1 = static_cast<int>((hi + kBK - 1) / kBK);
 }
 
+// The i-th tile of persistent CTA b of G: waves of G tiles walked alternately forward and backward.
+// Tiles are enumerated longest contraction first, so a CTA that takes a wave's longest tile takes
+// the next wave's shortest; on the factorisation's triangular products (tile lengths falling
+// linearly) this brings the busiest CTA from about 1.18 to 1.02 times the mean work.
+__device__ __forceinline__ int i8x_cta_tile(int i, int b, int G) { return i * G + ((i & 1) ? G - 1 - b : b); }
+
 // K-major operand tile with 32-byte rows and the 32-byte swizzle (layout type 6): 8-row atoms
-// of 256 bytes.
-__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+// of 256 bytes, consecutive atoms (8 rows further along M or N) `sbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr, uint32_t sbo = 256) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>(16 >> 4) << 16;
-  d |= static_cast<uint64_t>(256 >> 4) << 32;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(6) << 61;
   return d;
@@ -291,7 +330,7 @@ __device__ __forceinline__ void mma_band(uint32_t tmem, uint64_t ad, uint32_t sb
 template <int P>
 __device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t sa, uint32_t sb, uint32_t first) {
   if constexpr (P < kSlices) {
-    mma_band<P, 0>(tmem, sdesc_sw32(sa + P * kASlice), sb, first);
+    mma_band<P, 0>(tmem, sdesc_sw32(sa + P * 256, 256 * kSlices), sb, first);
     mma_stage<P + 1>(tmem, sa, sb, first);
   }
 }
@@ -307,7 +346,7 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[1
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    i8x_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB, I8xArgs args) {
+    i8x_gemm_kernel(const __grid_constant__ I8xArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   double* stage_c = reinterpret_cast<double*>(smem + kStages * kStageBytes);
@@ -348,11 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
-    ptx::prefetch_tensormap(&mA);
-    ptx::prefetch_tensormap(&mB);
     int g = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x) {
+    for (int j = 0, t = i8x_cta_tile(0, blockIdx.x, gridDim.x); t < args.tiles && ok;
+         t = i8x_cta_tile(++j, blockIdx.x, gridDim.x)) {
       int m0, n0, kb0, kb1;
       i8x_tile(args, t, m0, n0, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++g) {
@@ -363,15 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* st = smem + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
+        // the stage of the A tile and of the B tile: one contiguous copy each
+        const bool in = HQ_IN_BOUNDS(kb < args.Kpad / kBK && m0 / kBM < args.nblk_a && n0 / kBN < args.nblk_b);
+        const int8_t* srca = args.pa + (in ? (static_cast<int64_t>(kb) * args.nblk_a + m0 / kBM) * kABlockBytes : 0);
+        const int8_t* srcb = args.pb + (in ? (static_cast<int64_t>(kb) * args.nblk_b + n0 / kBN) * kBBlockBytes : 0);
         asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-            "[%5];" ::"r"(ptx::smem_u32(st)),
-            "l"(reinterpret_cast<uint64_t>(&mA)), "r"(kb * kBK), "r"(m0), "r"(0), "r"(ptx::smem_u32(&full[s]))
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                ptx::smem_u32(st)),
+            "l"(srca), "r"(kABlockBytes), "r"(ptx::smem_u32(&full[s]))
             : "memory");
         asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-            "[%5];" ::"r"(ptx::smem_u32(st + kSlices * kASlice)),
-            "l"(reinterpret_cast<uint64_t>(&mB)), "r"(kb * kBK), "r"(n0), "r"(0), "r"(ptx::smem_u32(&full[s]))
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                ptx::smem_u32(st + kABlockBytes)),
+            "l"(srcb), "r"(kBBlockBytes), "r"(ptx::smem_u32(&full[s]))
             : "memory");
       }
     }
@@ -384,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     int g = 0, i = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < args.tiles && ok; t += gridDim.x, ++i) {
+    for (int t = i8x_cta_tile(0, blockIdx.x, gridDim.x); t < args.tiles && ok; t = i8x_cta_tile(++i, blockIdx.x, gridDim.x)) {
       int m0, n0, kb0, kb1;
       i8x_tile(args, t, m0, n0, kb0, kb1);
       if (i >= 1 && !ptx::mbar_wait(acce, (i - 1) & 1, abort_flag)) {
@@ -420,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     double* st = stage_c + (warp - 2) * 32 * kStLd;
     bool ok = true;
     int i = 0;
-    for (int t = blockIdx.x; t < args.tiles; t += gridDim.x, ++i) {
+    for (int t = i8x_cta_tile(0, blockIdx.x, gridDim.x); t < args.tiles; t = i8x_cta_tile(++i, blockIdx.x, gridDim.x)) {
       int m0, n0, kb0, kb1;
       i8x_tile(args, t, m0, n0, kb0, kb1);
       if (ok) {
@@ -513,24 +555,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // 3-D tensor map over kSlices planes [rows][Kpad] int8 with a [box_rows][32] box spanning all
 // planes (32-byte swizzle).
-bool make_slice_map(CUtensorMap* map, const int8_t* planes, int64_t rows, int64_t Kpad, uint32_t box_rows) {
-  auto enc = tensor_map_encoder();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(Kpad), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(kSlices)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(Kpad), static_cast<cuuint64_t>(rows * Kpad)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box_rows, static_cast<cuuint32_t>(kSlices)};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(planes), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 hq_status slice(const double* X, int64_t ldx, int64_t rows, int64_t Kred, int64_t Kpad, int tri, int which,
-                int8_t* planes, int* exps, const int* skip, cudaStream_t s) {
+                int8_t* out_a, int8_t* out_b, int* exps, const int* skip, cudaStream_t s) {
   const int64_t grid = ceil_div(rows, 256 / kSliceRowThreads);
-  i8x_slice_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, ldx, rows, Kred, Kpad, tri, which, planes, exps,
-                                                              skip);
+  i8x_slice_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(X, ldx, rows, Kred, Kpad, tri, which, out_a,
+                                                              ceil_div(rows, kBM), out_b, ceil_div(rows, kBN),
+                                                              exps, skip);
   HQ_LAUNCH_CHECK();
   return HQ_OK;
 }
@@ -539,10 +569,18 @@ hq_status slice(const double* X, int64_t ldx, int64_t rows, int64_t Kred, int64_
 
 int64_t i8x_kpad(int64_t Kred) { return (Kred + kBK - 1) / kBK * kBK; }
 
+// Slices of A (rows padded to whole kBM blocks) and of B (whole kBN blocks), then the row exponents.
+size_t i8x_slices_a_bytes(int64_t M, int64_t kp) {
+  return round_up(static_cast<size_t>(kSlices) * round_up(static_cast<size_t>(M), kBM) * kp, 256);
+}
+size_t i8x_slices_b_bytes(int64_t N, int64_t kp) {
+  return round_up(static_cast<size_t>(kSlices) * round_up(static_cast<size_t>(N), kBN) * kp, 256);
+}
+
 size_t i8x_scratch_bytes(int64_t M, int64_t N, int64_t Kred) {
   const size_t kp = static_cast<size_t>(i8x_kpad(Kred));
-  const size_t a = round_up(static_cast<size_t>(kSlices) * M * kp, 256);
-  const size_t b = round_up(static_cast<size_t>(kSlices) * N * kp, 256);
+  const size_t a = i8x_slices_a_bytes(M, kp);
+  const size_t b = i8x_slices_b_bytes(N, kp);
   return a + b + round_up(static_cast<size_t>(M) * 4, 256) + round_up(static_cast<size_t>(N) * 4, 256);
 }
 
@@ -557,23 +595,25 @@ hq_status i8x_gemm(const F64Gemm& g, uint8_t* scratch, size_t scratch_bytes, cud
     return HQ_ERR_WORKSPACE;
   const int64_t kp = i8x_kpad(g.Kred);
   int8_t* pa = reinterpret_cast<int8_t*>(scratch);
+  // the same matrix as both operands (A22 -= T T^T): read and sliced once, written in both layouts
   const bool same = g.A == g.B && g.lda == g.ldb && g.M == g.N && g.tri == kTriNone;
-  int8_t* pb = same ? pa : pa + round_up(static_cast<size_t>(kSlices) * g.M * kp, 256);
-  int* ea = reinterpret_cast<int*>(pa + round_up(static_cast<size_t>(kSlices) * g.M * kp, 256) +
-                                   round_up(static_cast<size_t>(kSlices) * g.N * kp, 256));
+  int8_t* pb = pa + i8x_slices_a_bytes(g.M, kp);
+  int* ea = reinterpret_cast<int*>(pb + i8x_slices_b_bytes(g.N, kp));
   int* eb = same ? ea : ea + round_up(static_cast<size_t>(g.M) * 4, 256) / 4;
   const int ts = timer_start(kTimeI8xSlice, s);
-  hq_status st = slice(g.A, g.lda, g.M, g.Kred, kp, g.tri, 0, pa, ea, g.skip, s);
+  hq_status st = slice(g.A, g.lda, g.M, g.Kred, kp, g.tri, 0, pa, same ? pb : nullptr, ea, g.skip, s);
   if (st != HQ_OK) return st;
   if (!same) {
-    st = slice(g.B, g.ldb, g.N, g.Kred, kp, g.tri, 1, pb, eb, g.skip, s);
+    st = slice(g.B, g.ldb, g.N, g.Kred, kp, g.tri, 1, nullptr, pb, eb, g.skip, s);
     if (st != HQ_OK) return st;
   }
   // bytes: each operand's rows read once in fp64, kSlices planes written
   timer_stop(ts, (same ? 1.0 : 2.0) * 0.5 * (g.M + g.N) * (8.0 * g.Kred + kSlices * static_cast<double>(kp)), s);
-  CUtensorMap mA, mB;
-  if (!make_slice_map(&mA, pa, g.M, kp, kBM) || !make_slice_map(&mB, pb, g.N, kp, kBN)) return HQ_ERR_CUDA;
   I8xArgs a{};
+  a.pa = pa;
+  a.pb = pb;
+  a.nblk_a = static_cast<int>(ceil_div(g.M, kBM));
+  a.nblk_b = static_cast<int>(ceil_div(g.N, kBN));
   a.C = g.C;
   a.ldc = g.ldc;
   a.Ct = g.Ct;
@@ -602,7 +642,7 @@ hq_status i8x_gemm(const F64Gemm& g, uint8_t* scratch, size_t scratch_bytes, cud
   HQ_CUDA_TRY(cudaFuncSetAttribute(i8x_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
   const int grid = static_cast<int>(tiles < kSMs ? tiles : kSMs);
   const int tm = timer_start(kTimeI8xGemm, s);
-  i8x_gemm_kernel<<<grid, kThreads, kSmem, s>>>(mA, mB, a);
+  i8x_gemm_kernel<<<grid, kThreads, kSmem, s>>>(a);
   HQ_LAUNCH_CHECK();
   // work: 2 flops per multiply-add a declared triangular operand leaves non-zero (the fp64
   // product's own count, as for the fp64 kernel)

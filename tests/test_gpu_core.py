@@ -557,6 +557,29 @@ def test_i8x_gemm_against_fp64(hq, cuda_device, M, N, Kred, lower, tri, garbage)
     assert err0 < 1e-12, err0
 
 
+@pytest.mark.parametrize("n,Kred,lower", [(1000, 700, True), (1000, 700, False), (136, 2048, True)])
+def test_i8x_gemm_same_operand(hq, cuda_device, n, Kred, lower):
+    """C -= T T^T with one tensor as both operands (the factorisation's A22 update): T is read and
+    sliced once into both slice layouts; the result is bit-identical to the product with a copy
+    of T as the second operand (sliced on its own) and within 1e-12 of torch's fp64 product.
+    Sizes ragged against the 128-row and 64-row tile blocks."""
+    g = _gen(n + Kred)
+    T = torch.randn((n, Kred), generator=g, device="cuda", dtype=torch.float64)
+    C0 = torch.randn((n, n), generator=g, device="cuda", dtype=torch.float64)
+    C1, C2 = C0.clone(), C0.clone()
+    hq.hq_debug_i8x_gemm(C1, T, T, alpha=-1.0, beta=1.0, lower=lower)
+    hq.hq_debug_i8x_gemm(C2, T, T.clone(), alpha=-1.0, beta=1.0, lower=lower)
+    torch.cuda.synchronize()
+    assert torch.equal(C1, C2)
+    prod = T @ T.T
+    ref = C0 - prod
+    if lower:
+        mask = torch.ones((n, n), dtype=torch.bool, device="cuda").tril()
+        assert torch.equal(C1[~mask], C0[~mask])
+        C1, ref, prod = C1[mask], ref[mask], prod[mask]
+    assert ((C1 - ref).norm() / prod.norm()).item() < 1e-12
+
+
 def test_i8x_gemm_non_finite_rows_give_nan(hq, cuda_device):
     """A row with a NaN or an infinity gives a NaN row (A) or column (B) of the product, so that
     non-finite values still reach the factorisation's pivot check; every other entry is
