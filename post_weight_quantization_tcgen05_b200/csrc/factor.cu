@@ -223,6 +223,68 @@ __device__ __forceinline__ void leaf_block_inverse(const double* pb, int blk, do
   }
 }
 
+// One level of the leaf's triangular inverse by recursive doubling: with Z = M^-1 known on the
+// diagonal blocks of S tiles, every pair of them (tile rows b0 .. b0 + 2S - 1) gets its
+// off-diagonal block from the inverse of a 2 x 2 block lower triangular matrix,
+//   Z21 = -Z22 (M21 Z11),  M21 = N21,
+// as 8 x 8 tile products (two fp64 MMAs each, the two k halves in separate accumulators).  The
+// 8 S tiles of the level go to the 16 warps, their columns rotated so that every warp gets long
+// and short sums alike.  T = M21 Z11 is stored in Z21's tiles, and Z21 is held in registers until
+// every warp has read T.  Ends with a CTA barrier.
+template <int S>
+__device__ __forceinline__ void leaf_inverse_level(double* Zs, const double* Ns, int warp, int fg, int ft) {
+  constexpr int kTiles = 8 * S;
+  constexpr int kPer = (kTiles + kLT - 1) / kLT;
+  auto tile = [&](int u, int& I, int& J, int& b0) {
+    const int q = warp + kLT * u;
+    const int p = q / (S * S), i = (q % (S * S)) / S, j = (q + 3 * u) % S;
+    b0 = 2 * S * p;
+    I = b0 + S + i;
+    J = b0 + j;
+    return q < kTiles;
+  };
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    int I, J, b0;
+    if (!tile(u, I, J, b0)) continue;
+    double c0 = 0.0, c1 = 0.0, e0 = 0.0, e1 = 0.0;
+#pragma unroll
+    for (int k = 0; k < S; ++k) {
+      const int K = b0 + k;  // T_IJ = sum_{K >= J} N_IK Z_KJ over the first block
+      if (K >= J) {
+        dmma_leaf(c0, c1, Ns[lt_idx(I, K, fg, ft)], Zs[lt_idx(K, J, ft, fg)]);
+        dmma_leaf(e0, e1, Ns[lt_idx(I, K, fg, 4 + ft)], Zs[lt_idx(K, J, 4 + ft, fg)]);
+      }
+    }
+    *reinterpret_cast<double2*>(&Zs[lt_idx(I, J, fg, 2 * ft)]) = make_double2(c0 + e0, c1 + e1);
+  }
+  __syncthreads();
+  double2 z[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    int I, J, b0;
+    z[u] = make_double2(0.0, 0.0);
+    if (!tile(u, I, J, b0)) continue;
+    double c0 = 0.0, c1 = 0.0, e0 = 0.0, e1 = 0.0;
+#pragma unroll
+    for (int k = 0; k < S; ++k) {
+      const int K = b0 + S + k;  // Z21_IJ = -sum_{K <= I} Z_IK T_KJ over the second block
+      if (K <= I) {
+        dmma_leaf(c0, c1, Zs[lt_idx(I, K, fg, ft)], Zs[lt_idx(K, J, ft, fg)]);
+        dmma_leaf(e0, e1, Zs[lt_idx(I, K, fg, 4 + ft)], Zs[lt_idx(K, J, 4 + ft, fg)]);
+      }
+    }
+    z[u] = make_double2(-(c0 + e0), -(c1 + e1));
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    int I, J, b0;
+    if (tile(u, I, J, b0)) *reinterpret_cast<double2*>(&Zs[lt_idx(I, J, fg, 2 * ft)]) = z[u];
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const double* __restrict__ A, int64_t lda,
                                                                          double* __restrict__ X,
                                                                          double* __restrict__ XT, int64_t ldx,
@@ -320,10 +382,10 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
     if (tid == 0) atomicCAS(info, 0, diag_off + bad + 1);
     return;
   }
-  // Z = (I + N)^-1, the inverse of the block unit lower triangular factor (tile by tile, warp J
-  // computes tile column J, no barriers; S is no longer needed and takes Z):
-  //   Z_JJ = I - N_JJ   (N_JJ is the diagonal tile's lower-left 4 x 4 block, N_JJ^2 = 0)
-  //   Z_IJ = (I - N_II) (-Acc),  Acc = sum_{K = J .. I-1} N_IK Z_KJ   for I > J
+  // Z = (I + N)^-1, the inverse of the block unit lower triangular factor (S is no longer needed
+  // and takes Z): the diagonal tiles Z_JJ = I - N_JJ (N_JJ is the diagonal tile's lower-left
+  // 4 x 4 block, N_JJ^2 = 0), then the off-diagonal blocks by recursive doubling over blocks of
+  // 1, 2, 4 and 8 tile rows.
   {
     const int J = warp;
     {
@@ -335,30 +397,12 @@ __global__ void __launch_bounds__(kLeafThreads, 1) chol_inv_leaf_kernel(const do
       z.y = (fg == c0 + 1 ? 1.0 : 0.0) - n1;
       *reinterpret_cast<double2*>(&Ssm[lt_idx(J, J, fg, c0)]) = z;
     }
-    __syncwarp();
-    for (int Ir = J + 1; Ir < kLT; ++Ir) {
-      double acc0 = 0.0, acc1 = 0.0;
-      for (int Kc = J; Kc < Ir; ++Kc) {
-#pragma unroll
-        for (int kh = 0; kh < 2; ++kh) {
-          const double av = Ysm[lt_idx(Ir, Kc, fg, 4 * kh + ft)];  // N_IK[g][4 kh + t]
-          const double bv = Ssm[lt_idx(Kc, J, 4 * kh + ft, fg)];   // Z_KJ[4 kh + t][g]
-          dmma_leaf(acc0, acc1, av, bv);
-        }
-      }
-      *reinterpret_cast<double2*>(&Ssm[lt_idx(Ir, J, fg, 2 * ft)]) = make_double2(acc0, acc1);
-      __syncwarp();
-      // (I - N_II)(-Acc) = -Acc + N_II Acc, N_II nonzero in rows 4..7, columns 0..3 only
-      const double av = (fg >= 4) ? Ysm[lt_idx(Ir, Ir, fg, ft)] : 0.0;  // N_II[g][t]
-      const double bv = Ssm[lt_idx(Ir, J, ft, fg)];                     // Acc[t][g]
-      double z0 = -acc0, z1 = -acc1;
-      dmma_leaf(z0, z1, av, bv);
-      __syncwarp();
-      *reinterpret_cast<double2*>(&Ssm[lt_idx(Ir, J, fg, 2 * ft)]) = make_double2(z0, z1);
-      __syncwarp();
-    }
   }
   __syncthreads();
+  leaf_inverse_level<1>(Ssm, Ysm, warp, fg, ft);
+  leaf_inverse_level<2>(Ssm, Ysm, warp, fg, ft);
+  leaf_inverse_level<4>(Ssm, Ysm, warp, fg, ft);
+  leaf_inverse_level<8>(Ssm, Ysm, warp, fg, ft);
   // X tile (I, J) = C_I Z tile (I, J), with C_I = diag(D_b^-1/2 L_b^-1, D_b'^-1/2 L_b'^-1) the
   // block-diagonal 8 x 8 matrix of tile row I's two pivot blocks (two fp64 MMAs per tile);
   // written to X (row-major) and X^T straight from the fragments.  Elements above the diagonal
