@@ -192,11 +192,15 @@ def run_ours(args, rank, world, local_rank):
         layer.step()
     torch.cuda.synchronize()
     # the kernel class with the largest share of a step, from one step with every launch timed
-    # (outside the timed region); its launches are then timed live inside the timed region
-    dominant = dominant_class(kernel_breakdown(hq, layer, flush, steps=1))
+    # (outside the timed region), net of the launch processing each launch's event pair holds;
+    # its launches are then timed live, inside the timed region when they are few
+    overhead_us = launch_overhead_us()
+    dominant = dominant_class(kernel_breakdown(hq, layer, flush, steps=1, overhead_us=overhead_us))
     hq.hq_debug_timing_start([dominant])  # creates its events before the timed region
     layer.step()
     torch.cuda.synchronize()
+    dom_lps = hq.hq_debug_timing_read(dominant)[2]  # launches in one step
+    inline = dom_lps <= MAX_INLINE_TIMED_LAUNCHES
 
     # ---- timed region: K steps, each bracketed by events, L2 flushed between steps; the library
     #      records events around every launch of the dominant kernel on its own stream
@@ -205,14 +209,26 @@ def run_ours(args, rank, world, local_rank):
     launches0 = hq.hq_debug_launch_count()
     _barrier(world)
     torch.cuda.synchronize()
-    hq.hq_debug_timing_start([dominant])
+    if inline:
+        hq.hq_debug_timing_start([dominant])
+    else:
+        hq.hq_debug_timing_stop()
     with ClockSampler(local_rank) as clk:
         for k in range(args.steps):
             flush.fill_(k & 0xFF)
             layer.step(stage_events=evs[k])
         torch.cuda.synchronize()
     hq.hq_debug_timing_stop()
-    dom = (dominant,) + tuple(hq.hq_debug_timing_read(dominant))
+    if inline:
+        dom = (dominant,) + tuple(hq.hq_debug_timing_read(dominant))
+    else:  # the same steps again, every launch of the dominant class timed
+        hq.hq_debug_timing_start([dominant])
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            layer.step()
+        torch.cuda.synchronize()
+        hq.hq_debug_timing_stop()
+        dom = (dominant,) + tuple(hq.hq_debug_timing_read(dominant))
     _barrier(world)
     launches = (hq.hq_debug_launch_count() - launches0) // max(args.steps, 1)
     step_ms = [e[0].elapsed_time(e[4]) for e in evs]
@@ -228,7 +244,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- e2e: same calls, inputs from pinned host memory, results copied back
     e2e = None if args.no_e2e else measure_e2e(args, layer, flush, world)
     # ---- per-kernel breakdown (outside the timed region: events around every launch)
-    kernels = kernel_breakdown(hq, layer, flush)
+    kernels = kernel_breakdown(hq, layer, flush, overhead_us=overhead_us)
     codec = codec_throughput(hq, layer, flush)
     peaks = _peaks()
     dense = measure_dense_peaks(hq, dev)
@@ -242,7 +258,8 @@ def run_ours(args, rank, world, local_rank):
     dec_bytes = hq.hq_bf16tril_bytes(cfg.K) + 4 * cfg.K * cfg.K
     clocks = clk.summary()
     return_line = build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops,
-                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense)
+                             enc_bytes, dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense,
+                             inline, overhead_us)
     hbm = peaks["hbm_gbs"]
     return_line["codec_roofline"] = {
         "kernels": "tril_encode_pair_kernel / tril_decode_vec_kernel", "bound": "hbm", "unit": "GB/s",
@@ -447,8 +464,17 @@ PROFILES = {"f64_gemm_64": ("f64_gemm_kernel_32_q_proj.md", "gemm_f64.cu"),
 
 
 def dominant_class(kernels) -> str:
-    """The timed kernel class with the most device time per step."""
-    return max(kernels, key=lambda c: kernels[c]["ms_per_step"]) if kernels else "f64_gemm_64"
+    """The timed kernel class with the most device time per step (net of launch processing where
+    the breakdown has it)."""
+    if not kernels:
+        return "f64_gemm_64"
+    return max(kernels, key=lambda c: kernels[c].get("ms_net_per_step", kernels[c]["ms_per_step"]))
+
+
+# A dominant class with more launches per step than this is timed in a second pass of the same
+# steps: an event pair around each of its launches would break the chained launches of the
+# factorisation and slow the headline steps down.
+MAX_INLINE_TIMED_LAUNCHES = 16
 
 
 def class_roofline(cls: str, ms: float, work: float, launches: int, steps: int, peaks, cfg) -> dict:
@@ -532,11 +558,30 @@ def update_roofline_ms(cfg, peaks, tf32_tflops=None) -> float:
     return total * 1e3
 
 
-def kernel_breakdown(hq, layer, flush, steps: int = 2):
+def launch_overhead_us(reps: int = 50) -> float:
+    """Median time of an event pair around an empty kernel launched right behind a busy one on
+    the same stream (µs): the GPU's processing of a launch, which every per-launch event pair of
+    the breakdown also holds.  (In the step itself the chained launches overlap it with their
+    predecessor.)"""
+    pairs = []
+    for _ in range(reps):
+        torch.cuda._sleep(200000)  # keeps the GPU busy until the host has queued the pair
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        torch.cuda._sleep(0)
+        b.record()
+        pairs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in pairs) * 1e3
+
+
+def kernel_breakdown(hq, layer, flush, steps: int = 2, overhead_us: float | None = None):
     """Per kernel class: device time and achieved rate over `steps` steps, every launch timed.
     The factorisation's second stream is folded into the caller's stream meanwhile, so that each
     launch's events bracket that launch alone and the shares compare with ncu's serialised
-    launch list (the timed region itself keeps both streams)."""
+    launch list (the timed region itself keeps both streams).  With `overhead_us` (see
+    launch_overhead_us) each class also gets its time net of one launch processing per launch,
+    `ms_net_per_step`, the figure that compares with a profiler's kernel durations."""
     hq.hq_debug_timing_serialize(True)
     try:
         hq.hq_debug_timing_start(list(KERNEL_NAMES))
@@ -559,6 +604,8 @@ def kernel_breakdown(hq, layer, flush, steps: int = 2):
         out[cls] = {"kernel": name, "ms_per_step": ms / steps, "launches_per_step": n / steps,
                     "achieved": work / (ms / 1e3) / scale, "unit": unit, "ms_total": ms, "work_total": work,
                     "launches_total": n}
+        if overhead_us is not None:
+            out[cls]["ms_net_per_step"] = max(ms - n * overhead_us / 1e3, 0.0) / steps
     return out
 
 
@@ -806,12 +853,17 @@ def update_line(cfg, kernels, peaks):
 
 
 def build_line(args, cfg, world, value, ms_per_step, syrk_ms, gptq_ms, enc_ms, dec_ms, syrk_tflops, enc_bytes,
-               dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense):
+               dec_bytes, peaks, e2e, launches, clocks, dom, kernels, dense, inline=True, overhead_us=None):
     cls, dom_ms, dom_work, dom_n = dom
     roofline = class_roofline(cls, dom_ms, dom_work, dom_n, args.steps, peaks, cfg)
     roofline["traffic"] = profiled_traffic(cls)
-    roofline["timing"] = ("every launch of the class timed by CUDA events on its own stream inside the timed "
-                          "region; the class with the largest share of a step, from a breakdown taken before it")
+    where = ("inside the timed region" if inline else
+             f"in a second pass of the same {args.steps} steps right after the timed region (more than "
+             f"{MAX_INLINE_TIMED_LAUNCHES} launches per step: their event pairs would slow the timed steps)")
+    roofline["timing"] = (f"every launch of the class timed by CUDA events on its own stream {where}; the class "
+                          "with the largest share of a step, net of the launch processing each launch's event "
+                          "pair holds, from a breakdown taken before the timed region")
+    roofline["launch_overhead_us"] = overhead_us
     roofline["dense_peaks_measured"] = dense
     line = {
         "metric": "GPTQ-int4 weights/s (whole path: SYRK + factorisation + sweep + codec)",
