@@ -176,8 +176,9 @@ __device__ __forceinline__ void ldl4_inverse(const double (&s)[16], double (&d)[
 //      S[I][J] -= G_I P_J^T (one fp64 MMA m8n8k4 per 8 x 8 tile); the warp owning the next pivot
 //      block's diagonal tile updates that tile first and computes the next W (and keeps D_B,
 //      L_B^-1) while the others go on; one barrier per block step.
-//   2. Z = M^-1 by block forward substitution, warp J computing tile column J alone (no
-//      barriers): Z_JJ = I - N_JJ, Z_IJ = -(I - N_II) sum_{K=J..I-1} N_IK Z_KJ; Z takes S's tiles.
+//   2. Z = M^-1: the diagonal tiles Z_JJ = I - N_JJ, then the off-diagonal blocks by recursive
+//      doubling over blocks of 1, 2, 4 and 8 tile rows, Z21 = -Z22 (N21 Z11), the tiles of each
+//      level spread over all 16 warps (leaf_inverse_level); Z takes S's tiles.
 //   3. X = diag(D_B^-1/2 L_B^-1) Z, written to X and X^T.
 // Pivots (the entries of D) are checked after phase 1 (a bad pivot only produces values that
 // are then discarded).  Updating the inverse alongside the elimination instead (the identity
