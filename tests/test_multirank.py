@@ -107,6 +107,35 @@ def test_bench_line_carries_the_contract_keys():
     json.dumps(line)
 
 
+def test_dominant_class_is_ranked_net_of_launch_processing():
+    """A class of many short launches does not outrank a class of few long ones on the launch
+    processing its per-launch event pairs hold; without the net figure the raw time decides; a
+    dominant class with many launches per step is timed outside the headline steps, and the line
+    says where it was timed."""
+    import types
+
+    import bench
+    import workloads as wl
+    kernels = {"f64_gemm_64": {"ms_per_step": 1.83, "ms_net_per_step": 0.94, "launches_per_step": 144.0},
+               "i8x_gemm": {"ms_per_step": 1.52, "ms_net_per_step": 1.45, "launches_per_step": 12.0},
+               "leaf": {"ms_per_step": 1.54, "ms_net_per_step": 1.29, "launches_per_step": 40.0}}
+    assert bench.dominant_class(kernels) == "i8x_gemm"
+    raw = {k: {kk: vv for kk, vv in v.items() if kk != "ms_net_per_step"} for k, v in kernels.items()}
+    assert bench.dominant_class(raw) == "f64_gemm_64"
+    assert bench.dominant_class({}) == "f64_gemm_64"
+    assert 12 <= bench.MAX_INLINE_TIMED_LAUNCHES < 40
+    cfg = wl.CONFIGS[1]
+    args = types.SimpleNamespace(steps=10, warmup=3)
+    peaks = dict(bench._peaks(), tf32_tflops=800.0, fp64_tflops=37.0, int8_tops=3000.0)
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    e2e = {"value": 2.0e9, "unit": "weights/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
+    for inline, where in ((True, "inside the timed region"), (False, "second pass")):
+        line = bench.build_line(args, cfg, 1, 2.8e9, 9.3, [0.2], [9.0], [0.03], [0.03], 900.0, 7.9e7, 1.3e8,
+                                peaks, e2e, 249, clocks, ("leaf", 15.0, 1e9, 400), {}, {}, inline, 6.1)
+        assert where in line["roofline"]["timing"]
+        assert line["roofline"]["launch_overhead_us"] == 6.1
+
+
 def test_reference_arm_times_what_it_reports():
     """The oracle arm on the tiny layer: the steps it reports are the steps it timed (their
     total fits inside the call's wall time), and its workload string is the GPU arm's."""
