@@ -47,8 +47,8 @@ namespace {
 constexpr int kSlices = kI8xSlices;
 constexpr int kBM = 128, kBN = 64, kBK = 32;       // tile rows, tile columns, contraction bytes per stage
 constexpr int kStages = 4;
-constexpr int kASlice = kBM * kBK;                  // 4 KB per plane
-constexpr int kBSlice = kBN * kBK;                  // 2 KB per plane
+constexpr int kASlice = kBM * kBK;                  // 4 KB: one slice of an A tile's stage
+constexpr int kBSlice = kBN * kBK;                  // 2 KB: one slice of a B tile's stage
 constexpr int kStageBytes = kSlices * (kASlice + kBSlice);
 constexpr int kABlockBytes = kSlices * kASlice;     // one stage of an A tile: 28 KB, one bulk copy
 constexpr int kBBlockBytes = kSlices * kBSlice;     // one stage of a B tile: 14 KB, one bulk copy
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ bulk-copy producer
     int g = 0;
     bool ok = true;
     for (int j = 0, t = i8x_cta_tile(0, blockIdx.x, gridDim.x); t < args.tiles && ok;
@@ -553,8 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// 3-D tensor map over kSlices planes [rows][Kpad] int8 with a [box_rows][32] box spanning all
-// planes (32-byte swizzle).
+// Slices of X's rows into layout A (out_a) and/or layout B (out_b); either may be null.
 hq_status slice(const double* X, int64_t ldx, int64_t rows, int64_t Kred, int64_t Kpad, int tri, int which,
                 int8_t* out_a, int8_t* out_b, int* exps, const int* skip, cudaStream_t s) {
   const int64_t grid = ceil_div(rows, 256 / kSliceRowThreads);
@@ -607,7 +606,7 @@ hq_status i8x_gemm(const F64Gemm& g, uint8_t* scratch, size_t scratch_bytes, cud
     st = slice(g.B, g.ldb, g.N, g.Kred, kp, g.tri, 1, nullptr, pb, eb, g.skip, s);
     if (st != HQ_OK) return st;
   }
-  // bytes: each operand's rows read once in fp64, kSlices planes written
+  // bytes: each operand's rows read once in fp64, kSlices slices written
   timer_stop(ts, (same ? 1.0 : 2.0) * 0.5 * (g.M + g.N) * (8.0 * g.Kred + kSlices * static_cast<double>(kp)), s);
   I8xArgs a{};
   a.pa = pa;
