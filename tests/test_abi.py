@@ -156,3 +156,16 @@ def test_i8x_scratch_sizes_keep_256_byte_alignment(hq):
     one scratch per stream back to back, and the product requires a 256-byte aligned base)."""
     for M, N, K in ((64, 64, 32), (1280, 1280, 1280), (2560, 2560, 2560), (8704, 8704, 8704), (1000, 600, 300)):
         assert hq.lib.hq_debug_i8x_scratch_bytes(M, N, K) % 256 == 0
+
+
+def test_i8x_scratch_covers_whole_tile_blocks(hq):
+    """The slices are stored in whole tile blocks (A rows in blocks of 128, B rows in blocks of
+    64, the contraction in 32-byte chunks, 7 slices), and every pipeline stage of the product is
+    one bulk copy of a whole block; the scratch therefore holds the padded blocks of both
+    operands plus the row exponents, so that the last block's copies stay inside it."""
+    def up(x, m):
+        return (x + m - 1) // m * m
+    for M, N, K in ((1, 1, 1), (64, 64, 32), (129, 65, 33), (1000, 600, 300), (2560, 1280, 2560)):
+        kp = up(K, 32)
+        need = up(7 * up(M, 128) * kp, 256) + up(7 * up(N, 64) * kp, 256) + up(4 * M, 256) + up(4 * N, 256)
+        assert hq.lib.hq_debug_i8x_scratch_bytes(M, N, K) >= need, (M, N, K)
